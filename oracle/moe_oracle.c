@@ -1,0 +1,311 @@
+/*
+ * moe_oracle.c -- plain, slow CPU statement of the MoE expert layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  The CUDA library never includes, links or calls
+ * this file, and this file shares no code, header, table or helper with it.
+ * Only the test suite, the smoke check and the benchmark's CPU-baseline leg
+ * use it.
+ *
+ * Sources (web pages on the subject; cited by title and section):
+ *  [MoE-latency]  "MoE 少算 FLOPs,延迟反而涨了:慢在搬 token 的路上"
+ *                 sections "dense 和 MoE 的差别" (router scores every expert,
+ *                 picks top-2, emits two routing weights; only the picked
+ *                 experts process the token) and "router 之后还有一串动作"
+ *                 (k assignments per token, grouped by expert = dispatch, rows
+ *                 sorted by expert = permutation, one matrix per expert in a
+ *                 grouped GEMM, inverse mapping back to token order, multiply
+ *                 by routing weight, sum = combine / unpermutation).
+ *  [FinDEP]       "FinDEP: Efficient MoE Inference with Fine-Grained
+ *                 Scheduling of Disaggregated Expert Parallelism", section
+ *                 "核心公式", MoE-layer formula: three GEMMs per expert
+ *                 (here the SwiGLU form W1, W3, W2); section "问题定义":
+ *                 shared experts are always-on experts.
+ *  [MegaScale]    "MegaScale-Infer: Serving Mixture-of-Experts at Scale with
+ *                 Disaggregated Expert Parallelism", section "核心问题"
+ *                 (Mixtral 8x22B: 156 tokens over 8 experts at top-2 gives
+ *                 39 rows per expert on average).
+ *
+ * Readings where the pages are silent (each one is a choice, documented in the
+ * design notes):
+ *  - logits: fp32 W_gate, bf16 x; the oracle sums in fp64 and rounds the logit
+ *    to fp32, because the expert choice (an integer decided by floating point)
+ *    is taken in the kernel's precision, fp32;
+ *  - top-k: larger fp32 logit first; on equal values the lower expert index
+ *    wins; picks are listed in that order;
+ *  - routing weights: softmax over all E renormalised over the k picks, which
+ *    equals a softmax over the k picked logits: w_j = e^(l_j-l_0)/sum_i e^(l_i-l_0);
+ *  - dispatch is stable: inside an expert's group, rows follow assignment id
+ *    a = t*k + j;
+ *  - expert FFN is SwiGLU: h = silu(x W1^T) * (x W3^T), y = h W2^T,
+ *    silu(z) = z / (1 + e^-z); all sums in fp64; bf16 rounding (to nearest,
+ *    ties to even) at h, at y, at the shared-expert output s and at out;
+ *  - combine: out[t] = bf16( sum_j w_j * y[row(t,j)] + s[t] ), j in pick order;
+ *  - shared experts (optional, Is > 0): one SwiGLU FFN of width Is over every
+ *    token, weight 1, added after the routed sum.
+ *
+ * Layouts: x [N,H] bf16 (uint16 storage); W_gate [H,E] fp32; bias [E] fp32 or
+ * NULL; W1, W3 [E,I,H] bf16; W2 [E,H,I] bf16; Ws1, Ws3 [Is,H] bf16;
+ * Ws2 [H,Is] bf16; all row-major.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- bf16 ---- */
+
+/* bf16 keeps the top 16 bits of an IEEE binary32. */
+double oracle_bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double straight to bf16 (8 significant bits, binary32 exponent
+ * range), to nearest with ties to even, overflow to infinity.  No detour
+ * through fp32, so there is no double rounding. */
+uint16_t oracle_round_to_bf16(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v)) return 0x7FC0u;
+    if (isinf(v)) return (uint16_t)(sign | 0x7F80u);
+    double a = fabs(v), q;
+    if (a < 0x1p-126) {
+        /* subnormal range: the spacing is 2^-133 */
+        q = rint(a * 0x1p133) * 0x1p-133;
+    } else {
+        int ex;
+        double m = frexp(a, &ex); /* a = m * 2^ex, 0.5 <= m < 1 */
+        q = ldexp(rint(ldexp(m, 8)), ex - 8);
+    }
+    if (q >= 0x1p128) return (uint16_t)(sign | 0x7F80u);
+    float f = (float)q; /* exact: q has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
+}
+
+/* -------------------------------------------------------------- router ---- */
+
+/* [MoE-latency] "dense 和 MoE 的差别": the router reads a token's hidden state
+ * and scores every expert.  logits[t,e] = sum_h x[t,h] * W_gate[h,e] + bias[e],
+ * in fp64. */
+void oracle_router_logits(const uint16_t *x, const float *W_gate, const float *bias,
+                          int64_t N, int H, int E, double *logits)
+{
+    for (int64_t t = 0; t < N; ++t)
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int h = 0; h < H; ++h)
+                s += oracle_bf16_to_double(x[t * H + h]) * (double)W_gate[(int64_t)h * E + e];
+            if (bias) s += (double)bias[e];
+            logits[t * E + e] = s;
+        }
+}
+
+/* [MoE-latency] "dense 和 MoE 的差别": pick the top-k experts and give k
+ * routing weights.  Selection compares fp32 values; ties go to the lower
+ * index.  w is the softmax over the k picked logits (equal to the full softmax
+ * renormalised over the picks).  Returns 0, or -1 on bad sizes. */
+int oracle_topk(const float *logits, int64_t N, int E, int k, int32_t *idx, double *w)
+{
+    if (E < 1 || k < 1 || k > E) return -1;
+    char *taken = (char *)malloc((size_t)E);
+    if (!taken) return -1;
+    for (int64_t t = 0; t < N; ++t) {
+        const float *l = logits + t * E;
+        memset(taken, 0, (size_t)E);
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e; /* strict: lower index keeps a tie */
+            }
+            taken[best] = 1;
+            idx[t * k + j] = best;
+        }
+        double l0 = (double)l[idx[t * k]], den = 0.0;
+        for (int j = 0; j < k; ++j) den += exp((double)l[idx[t * k + j]] - l0);
+        for (int j = 0; j < k; ++j) w[t * k + j] = exp((double)l[idx[t * k + j]] - l0) / den;
+    }
+    free(taken);
+    return 0;
+}
+
+/* ------------------------------------------------------------ dispatch ---- */
+
+/* [MoE-latency] "router 之后还有一串动作": N tokens give N*k assignments;
+ * grouping them by expert is dispatch, sorting token rows by expert is the
+ * permutation.  counts[e] = #assignments to e; offsets = exclusive scan with
+ * offsets[E] = N*k; assignment a = t*k+j lands at row offsets[e] + (number of
+ * earlier assignments to e).  Returns 0, or -1 on an index outside [0,E). */
+int oracle_dispatch(const int32_t *idx, int64_t N, int E, int k, int32_t *counts,
+                    int32_t *offsets, int32_t *row_to_token, int32_t *token_to_row)
+{
+    if (E < 1 || k < 1 || N < 0) return -1;
+    int64_t R = N * k;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t a = 0; a < R; ++a) {
+        if (idx[a] < 0 || idx[a] >= E) return -1;
+        counts[idx[a]] += 1;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *fill = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    if (!fill) return -1;
+    for (int64_t a = 0; a < R; ++a) {
+        int e = idx[a];
+        int32_t row = offsets[e] + fill[e]++;
+        row_to_token[row] = (int32_t)(a / k);
+        token_to_row[a] = row;
+    }
+    free(fill);
+    return 0;
+}
+
+/* x_perm[row] = x[row_to_token[row]] (the permuted copy of token rows). */
+void oracle_permute_rows(const uint16_t *x, const int32_t *row_to_token, int64_t R, int H,
+                         uint16_t *x_perm)
+{
+    for (int64_t r = 0; r < R; ++r)
+        memcpy(x_perm + r * H, x + (int64_t)row_to_token[r] * H, (size_t)H * sizeof(uint16_t));
+}
+
+/* ---------------------------------------------------------- expert FFN ---- */
+
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* [FinDEP] "核心公式": an expert is three GEMMs; here the SwiGLU expert
+ * y = W2 (silu(W1 x) * (W3 x)).  One row, one expert: W1, W3 [I,H], W2 [H,I].
+ * fp64 sums; h and y rounded to bf16. */
+void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t *W3,
+                       const uint16_t *W2, int H, int I, uint16_t *yrow)
+{
+    double *xd = (double *)malloc((size_t)H * sizeof(double));
+    double *hd = (double *)malloc((size_t)I * sizeof(double));
+    for (int c = 0; c < H; ++c) xd[c] = oracle_bf16_to_double(xrow[c]);
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int c = 0; c < H; ++c) {
+            g += xd[c] * oracle_bf16_to_double(W1[(int64_t)i * H + c]);
+            u += xd[c] * oracle_bf16_to_double(W3[(int64_t)i * H + c]);
+        }
+        hd[i] = oracle_bf16_to_double(oracle_round_to_bf16(silu(g) * u));
+    }
+    for (int o = 0; o < H; ++o) {
+        double y = 0.0;
+        for (int i = 0; i < I; ++i) y += hd[i] * oracle_bf16_to_double(W2[(int64_t)o * I + i]);
+        yrow[o] = oracle_round_to_bf16(y);
+    }
+    free(xd);
+    free(hd);
+}
+
+/* [MoE-latency] "router 之后还有一串动作": each expert runs its own rows.
+ * Rows offsets[e] .. offsets[e+1]-1 of x_perm go through expert e. */
+void oracle_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
+                       const uint16_t *W3, const uint16_t *W2, int E, int H, int I,
+                       uint16_t *y_perm)
+{
+    int64_t we = (int64_t)I * H;
+    for (int e = 0; e < E; ++e)
+        for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r)
+            oracle_swiglu_ffn(x_perm + r * H, W1 + e * we, W3 + e * we, W2 + e * we, H, I,
+                              y_perm + r * H);
+}
+
+/* ------------------------------------------------------------- combine ---- */
+
+/* [MoE-latency] "router 之后还有一串动作": inverse mapping back to token
+ * order, multiply by the routing weight, add.  out[t] = bf16(sum_j w[t,j] *
+ * y_perm[token_to_row[t,j]] + s[t]) in fp64, j in pick order; s may be NULL. */
+void oracle_combine(const uint16_t *y_perm, const int32_t *token_to_row, const double *w,
+                    const uint16_t *s, int64_t N, int H, int k, uint16_t *out)
+{
+    for (int64_t t = 0; t < N; ++t)
+        for (int o = 0; o < H; ++o) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j)
+                acc += w[t * k + j] *
+                       oracle_bf16_to_double(y_perm[(int64_t)token_to_row[t * k + j] * H + o]);
+            if (s) acc += oracle_bf16_to_double(s[t * H + o]);
+            out[t * H + o] = oracle_round_to_bf16(acc);
+        }
+}
+
+/* --------------------------------------------------------------- layer ---- */
+
+/* The whole sparse path from given fp32 logits: top-k, dispatch, permuted
+ * rows, per-expert SwiGLU, optional shared experts ([FinDEP] "问题定义"),
+ * combine.  Optional outputs (may be NULL): idx [N,k], w [N,k], counts [E],
+ * offsets [E+1], row_to_token [N*k], token_to_row [N*k], y_perm [N*k,H].
+ * Returns 0, or -1 on bad arguments / allocation failure. */
+int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint16_t *W1,
+                              const uint16_t *W3, const uint16_t *W2, const uint16_t *Ws1,
+                              const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
+                              int E, int k, int Is, uint16_t *out, int32_t *idx_out,
+                              double *w_out, int32_t *counts_out, int32_t *offsets_out,
+                              int32_t *r2t_out, int32_t *t2r_out, uint16_t *y_perm_out)
+{
+    if (N < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E || Is < 0) return -1;
+    int64_t R = N * k;
+    int rc = -1;
+    int32_t *idx = (int32_t *)malloc((size_t)(R ? R : 1) * sizeof(int32_t));
+    double *w = (double *)malloc((size_t)(R ? R : 1) * sizeof(double));
+    int32_t *counts = (int32_t *)malloc((size_t)E * sizeof(int32_t));
+    int32_t *offsets = (int32_t *)malloc((size_t)(E + 1) * sizeof(int32_t));
+    int32_t *r2t = (int32_t *)malloc((size_t)(R ? R : 1) * sizeof(int32_t));
+    int32_t *t2r = (int32_t *)malloc((size_t)(R ? R : 1) * sizeof(int32_t));
+    uint16_t *xp = (uint16_t *)malloc((size_t)(R ? R : 1) * H * sizeof(uint16_t));
+    uint16_t *yp = (uint16_t *)malloc((size_t)(R ? R : 1) * H * sizeof(uint16_t));
+    uint16_t *s = NULL;
+    if (!idx || !w || !counts || !offsets || !r2t || !t2r || !xp || !yp) goto done;
+    if (oracle_topk(logits, N, E, k, idx, w)) goto done;
+    if (oracle_dispatch(idx, N, E, k, counts, offsets, r2t, t2r)) goto done;
+    oracle_permute_rows(x, r2t, R, H, xp);
+    oracle_expert_ffn(xp, offsets, W1, W3, W2, E, H, I, yp);
+    if (Is > 0) {
+        s = (uint16_t *)malloc((size_t)(N ? N : 1) * H * sizeof(uint16_t));
+        if (!s) goto done;
+        for (int64_t t = 0; t < N; ++t) oracle_swiglu_ffn(x + t * H, Ws1, Ws3, Ws2, H, Is, s + t * H);
+    }
+    oracle_combine(yp, t2r, w, s, N, H, k, out);
+    if (idx_out) memcpy(idx_out, idx, (size_t)R * sizeof(int32_t));
+    if (w_out) memcpy(w_out, w, (size_t)R * sizeof(double));
+    if (counts_out) memcpy(counts_out, counts, (size_t)E * sizeof(int32_t));
+    if (offsets_out) memcpy(offsets_out, offsets, (size_t)(E + 1) * sizeof(int32_t));
+    if (r2t_out) memcpy(r2t_out, r2t, (size_t)R * sizeof(int32_t));
+    if (t2r_out) memcpy(t2r_out, t2r, (size_t)R * sizeof(int32_t));
+    if (y_perm_out) memcpy(y_perm_out, yp, (size_t)R * H * sizeof(uint16_t));
+    rc = 0;
+done:
+    free(idx); free(w); free(counts); free(offsets); free(r2t); free(t2r); free(xp); free(yp);
+    free(s);
+    return rc;
+}
+
+/* The whole layer from x: fp64 logits rounded to fp32 (the precision the
+ * expert choice is taken in), then the path above.  logits_out [N,E] may be
+ * NULL. */
+int oracle_layer(const uint16_t *x, const float *W_gate, const float *bias, const uint16_t *W1,
+                 const uint16_t *W3, const uint16_t *W2, const uint16_t *Ws1, const uint16_t *Ws3,
+                 const uint16_t *Ws2, int64_t N, int H, int I, int E, int k, int Is,
+                 uint16_t *out, float *logits_out)
+{
+    if (N < 0 || H < 1 || E < 1) return -1;
+    double *l64 = (double *)malloc((size_t)(N ? N : 1) * E * sizeof(double));
+    float *l32 = (float *)malloc((size_t)(N ? N : 1) * E * sizeof(float));
+    int rc = -1;
+    if (l64 && l32) {
+        oracle_router_logits(x, W_gate, bias, N, H, E, l64);
+        for (int64_t i = 0; i < N * E; ++i) l32[i] = (float)l64[i];
+        rc = oracle_layer_given_logits(x, l32, W1, W3, W2, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out,
+                                       NULL, NULL, NULL, NULL, NULL, NULL, NULL);
+        if (rc == 0 && logits_out) memcpy(logits_out, l32, (size_t)N * E * sizeof(float));
+    }
+    free(l64);
+    free(l32);
+    return rc;
+}

@@ -1,0 +1,296 @@
+"""Pins for the CPU oracle, each against something other than the oracle itself.
+
+CPU only.  Sources of truth used here: hand-worked fixtures under
+tests/golden/ (each cites the page and section it follows), torch's own bf16
+conversion, float64 BLAS products, full sorts, numpy's stable argsort, dense
+evaluation of every expert on every token, and invariants of the method.
+"""
+import math
+from pathlib import Path
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from expert_ffn_layer_moe_b200.inputs import CONFIGS, MoEConfig, make_inputs
+from tests._bf16 import dec, enc, to_u16, ulp_diff
+
+GOLD = Path(__file__).parent / "golden"
+
+
+def _rows(name):
+    for line in (GOLD / name).read_text().splitlines():
+        line = line.strip()
+        if line and not line.startswith("#"):
+            yield line
+
+
+def small_layer(N=24, H=64, I=32, E=4, k=2, Is=0, seed=3):
+    cfg = MoEConfig("pin", N=N, H=H, I=I, E=E, k=k, Is=Is)
+    t = make_inputs(cfg, seed=seed)
+    return cfg, {n: (to_u16(v) if v is not None and v.dtype == torch.bfloat16 else
+                     (None if v is None else v.numpy())) for n, v in t.items()}
+
+
+def dense_swiglu(xd, W1d, W3d, W2d):
+    """Dense SwiGLU FFN in float64 with torch's silu and BLAS products,
+    rounding to bf16 where the layer does (h and y)."""
+    x = torch.from_numpy(xd)
+    g = x @ torch.from_numpy(W1d).T
+    u = x @ torch.from_numpy(W3d).T
+    h = dec(enc((F.silu(g) * u).numpy()))
+    return enc((torch.from_numpy(h) @ torch.from_numpy(W2d).T).numpy())
+
+
+# ------------------------------------------------------------------ bf16 ----
+
+def test_bf16_rounding_golden():
+    for line in _rows("bf16_rounding.txt"):
+        val, bits = line.split()[:2]
+        assert oracle.round_to_bf16(float.fromhex(val)) == int(bits, 16), line
+
+
+def test_bf16_rounding_matches_torch_on_fp32_values():
+    g = torch.Generator().manual_seed(11)
+    mant = torch.rand(20000, generator=g, dtype=torch.float64) + 1.0
+    ex = torch.randint(-140, 128, (20000,), generator=g)
+    v = (mant * torch.pow(2.0, ex.to(torch.float64))).to(torch.float32)
+    v[::2] *= -1
+    # exact midpoints between bf16 neighbours, where ties-to-even decides
+    mid = (torch.randint(0, 2 ** 15, (4000,), generator=g, dtype=torch.int32) << 16) | 0x8000
+    v = torch.cat([v, mid.view(torch.float32)])
+    v = v[torch.isfinite(v)]
+    want = to_u16(v.to(torch.bfloat16))
+    got = oracle.round_to_bf16(v.to(torch.float64).numpy())
+    assert np.array_equal(got, want)
+
+
+def test_bf16_decode_all_patterns():
+    u = np.arange(0, 65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.bf16_to_f64(u)
+    want = dec(u)
+    finite = np.isfinite(want)
+    assert np.array_equal(got[finite], want[finite])
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+
+
+# ---------------------------------------------------------------- router ----
+
+def test_logits_match_float64_product():
+    cfg = CONFIGS["tiny"]
+    t = make_inputs(cfg, seed=0, weights=False)
+    bias = torch.linspace(-1, 1, cfg.E, dtype=torch.float32)
+    got = oracle.router_logits(to_u16(t["x"]), t["W_gate"].numpy(), bias.numpy())
+    xd = t["x"].to(torch.float64)
+    want = (xd @ t["W_gate"].to(torch.float64) + bias.to(torch.float64)).numpy()
+    scale = (xd.abs() @ t["W_gate"].to(torch.float64).abs()).numpy() + 1.0
+    assert np.all(np.abs(got - want) <= 1e-13 * scale)
+
+
+def test_topk_golden_ties():
+    for line in _rows("topk_ties.txt"):
+        k, logits, want = [p.strip() for p in line.split("|")]
+        l = np.array([[float(v) for v in logits.split()]], dtype=np.float32)
+        idx, w = oracle.topk(l, int(k))
+        assert idx[0].tolist() == [int(v) for v in want.split()], line
+
+
+def test_topk_matches_full_sort():
+    g = np.random.default_rng(5)
+    N, E = 200, 37
+    # coarse values force many exact ties
+    l = (g.integers(-6, 6, size=(N, E)) * 0.5).astype(np.float32)
+    for k in (1, 2, 5, E):
+        idx, _ = oracle.topk(l, k)
+        for t in range(N):
+            order = sorted(range(E), key=lambda e: (-float(l[t, e]), e))
+            assert idx[t].tolist() == order[:k]
+
+
+def test_topk_weights_closed_forms():
+    g = np.random.default_rng(6)
+    l = g.standard_normal((64, 16)).astype(np.float32)
+    _, w1 = oracle.topk(l, 1)
+    assert np.all(w1 == 1.0)
+    idx, w2 = oracle.topk(l, 2)
+    l0 = l[np.arange(64), idx[:, 0]].astype(np.float64)
+    l1 = l[np.arange(64), idx[:, 1]].astype(np.float64)
+    assert np.allclose(w2[:, 0], 1.0 / (1.0 + np.exp(l1 - l0)), rtol=1e-15, atol=0)
+    # softmax over all E renormalised over the picks equals the stated form
+    idx, w6 = oracle.topk(l, 6)
+    p = np.exp(l.astype(np.float64) - l.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    pk = np.take_along_axis(p, idx.astype(np.int64), 1)
+    assert np.allclose(w6, pk / pk.sum(1, keepdims=True), rtol=1e-13, atol=0)
+    assert np.allclose(w6.sum(1), 1.0, rtol=0, atol=1e-15)
+    assert np.all(np.diff(w6, axis=1) <= 0)
+    # the golden two-expert weights (hand-worked layer)
+    rows = dict(r.split(maxsplit=1) for r in _rows("tiny_layer_by_hand.txt"))
+    _, w = oracle.topk(np.array([[1.0, -1.0]], np.float32), 2)
+    assert np.allclose(w[0], [float(v) for v in rows["w"].split()], rtol=1e-15, atol=0)
+
+
+# -------------------------------------------------------------- dispatch ----
+
+def test_dispatch_matches_stable_argsort():
+    g = np.random.default_rng(7)
+    N, E, k = 300, 9, 3
+    idx = np.stack([g.permutation(E)[:k] for _ in range(N)]).astype(np.int32)
+    idx[:40] = [0, 1, 2]                              # a hot expert group
+    counts, offsets, r2t, t2r = oracle.dispatch(idx, E)
+    order = np.argsort(idx.ravel(), kind="stable")    # assignment ids sorted by expert
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
+    assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    assert np.array_equal(r2t, order // k)
+    inv = np.empty_like(order)
+    inv[order] = np.arange(N * k)
+    assert np.array_equal(t2r.ravel(), inv)
+
+
+def test_dispatch_invariants_and_empty_experts():
+    g = np.random.default_rng(8)
+    N, E, k = 50, 12, 2
+    idx = np.stack([g.choice([1, 4, 7, 9], size=k, replace=False) for _ in range(N)]).astype(np.int32)
+    counts, offsets, r2t, t2r = oracle.dispatch(idx, E)
+    assert counts.sum() == N * k and offsets[-1] == N * k
+    assert all(counts[e] == 0 for e in range(E) if e not in (1, 4, 7, 9))
+    assert np.all(np.diff(offsets) >= 0)
+    assert sorted(t2r.ravel().tolist()) == list(range(N * k))      # bijection
+    assert np.array_equal(r2t[t2r], np.repeat(np.arange(N)[:, None], k, 1))
+    for e in range(E):
+        seg = r2t[offsets[e]:offsets[e + 1]]
+        assert np.all(np.diff(seg) > 0)                            # stable, ascending token
+
+
+def test_dispatch_rejects_bad_index():
+    with pytest.raises(ValueError):
+        oracle.dispatch(np.array([[0, 5]], np.int32), 4)
+    with pytest.raises(ValueError):
+        oracle.dispatch(np.array([[0, -1]], np.int32), 4)
+
+
+def test_mixtral_worked_example_mean_rows():
+    """156 tokens, 8 experts, top-2: 312 assignments, 39 rows per expert on
+    average (MegaScale-Infer summary, section "核心问题")."""
+    fx = dict(r.split() for r in _rows("mixtral_worked_example.txt"))
+    cfg = CONFIGS["mixtral_8x22b_decode"]
+    assert (cfg.N, cfg.E, cfg.k) == (int(fx["tokens"]), int(fx["experts"]), int(fx["top_k"]))
+    t = make_inputs(cfg, seed=0, weights=False)
+    l64 = oracle.router_logits(to_u16(t["x"]), t["W_gate"].numpy())
+    idx, _ = oracle.topk(l64.astype(np.float32), cfg.k)
+    counts, offsets, _, _ = oracle.dispatch(idx, cfg.E)
+    assert counts.sum() == int(fx["assignments"])
+    assert counts.sum() / cfg.E == float(fx["mean_rows_per_expert"])
+    assert float(fx["ffn_mfu"]) == cfg.k / cfg.E
+
+
+def test_permute_rows_copies_bits():
+    cfg, t = small_layer()
+    idx, _ = oracle.topk(oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32), cfg.k)
+    _, _, r2t, _ = oracle.dispatch(idx, cfg.E)
+    assert np.array_equal(oracle.permute_rows(t["x"], r2t), t["x"][r2t])
+
+
+# ------------------------------------------------------------ expert FFN ----
+
+def test_swiglu_ffn_matches_dense_float64():
+    cfg, t = small_layer(N=8, H=96, I=48, E=2)
+    W1, W3, W2 = t["W1"][1], t["W3"][1], t["W2"][1]
+    want = dense_swiglu(dec(t["x"]), dec(W1), dec(W3), dec(W2))
+    got = np.stack([oracle.swiglu_ffn(t["x"][i], W1, W3, W2) for i in range(cfg.N)])
+    d = ulp_diff(got, want)
+    assert d.max() <= 1 and (d == 0).mean() > 0.99
+
+
+def test_layer_by_hand():
+    rows = dict(r.split(maxsplit=1) for r in _rows("tiny_layer_by_hand.txt"))
+    b = lambda *v: np.array(v, np.float32).astype(np.float64)
+    x = enc(np.array([[1.0, 0.0]]))
+    Wg = np.array([[1.0, -1.0], [0.0, 0.0]], np.float32)
+    W1 = enc(np.array([[[2.0, 0.0]], [[-1.0, 0.0]]]))
+    W3 = enc(np.array([[[1.0, 0.0]], [[4.0, 0.0]]]))
+    W2 = enc(np.array([[[1.0], [-0.5]], [[1.0], [2.0]]]))
+    out, logits = oracle.layer(x, Wg, W1, W3, W2, k=2)
+    assert logits.tolist() == [[1.0, -1.0]]
+    res = oracle.layer_given_logits(x, logits, W1, W3, W2, 2, extras=True)
+    assert res["idx"][0].tolist() == [int(v) for v in rows["idx"].split()]
+    r0, r1 = res["token_to_row"][0]
+    assert res["y_perm"][r0].tolist() == [int(v, 16) for v in rows["y0"].split()]
+    assert res["y_perm"][r1].tolist() == [int(v, 16) for v in rows["y1"].split()]
+    assert out[0].tolist() == [int(v, 16) for v in rows["out"].split()]
+    Ws1 = enc(np.array([[1.0, 0.0]])); Ws3 = enc(np.array([[1.0, 0.0]]))
+    Ws2 = enc(np.array([[1.0], [1.0]]))
+    out_s, _ = oracle.layer(x, Wg, W1, W3, W2, k=2, Ws1=Ws1, Ws3=Ws3, Ws2=Ws2)
+    assert out_s[0].tolist() == [int(v, 16) for v in rows["out_shared"].split()]
+
+
+def test_layer_equals_dense_masked_evaluation():
+    """Run every expert on every token, weight by the routing mask and sum in
+    pick order: the sparse dispatch/permute/combine path must agree."""
+    cfg, t = small_layer(N=20, H=64, I=32, E=5, k=3)
+    l32 = oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32)
+    out = oracle.layer_given_logits(t["x"], l32, t["W1"], t["W3"], t["W2"], cfg.k)
+    idx, w = oracle.topk(l32, cfg.k)
+    xd = dec(t["x"])
+    Y = np.stack([dec(dense_swiglu(xd, dec(t["W1"][e]), dec(t["W3"][e]), dec(t["W2"][e])))
+                  for e in range(cfg.E)])                         # [E, N, H]
+    acc = np.zeros((cfg.N, cfg.H))
+    for j in range(cfg.k):
+        acc += w[:, j:j + 1] * Y[idx[:, j], np.arange(cfg.N)]
+    d = ulp_diff(out, enc(acc))
+    assert d.max() <= 1 and (d == 0).mean() > 0.99
+
+
+def test_single_expert_top1_is_dense_swiglu():
+    cfg, t = small_layer(N=16, H=64, I=96, E=1, k=1)
+    out, _ = oracle.layer(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], k=1)
+    want = dense_swiglu(dec(t["x"]), dec(t["W1"][0]), dec(t["W3"][0]), dec(t["W2"][0]))
+    d = ulp_diff(out, want)
+    assert d.max() <= 1 and (d == 0).mean() > 0.99
+
+
+def test_shared_expert_alone_is_dense_swiglu():
+    cfg, t = small_layer(N=12, H=64, I=32, E=3, k=2, Is=48)
+    W2zero = np.zeros_like(t["W2"])
+    out, _ = oracle.layer(t["x"], t["W_gate"], t["W1"], t["W3"], W2zero, k=2,
+                          Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"])
+    want = dense_swiglu(dec(t["x"]), dec(t["Ws1"]), dec(t["Ws3"]), dec(t["Ws2"]))
+    d = ulp_diff(out, want)
+    assert d.max() <= 1 and (d == 0).mean() > 0.99
+
+
+def test_expert_relabelling_is_invisible():
+    cfg, t = small_layer(N=16, H=64, I=32, E=6, k=2)
+    out, _ = oracle.layer(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], k=2)
+    pi = np.array([3, 5, 0, 2, 1, 4])
+    out_p, _ = oracle.layer(t["x"], t["W_gate"][:, pi], t["W1"][pi], t["W3"][pi], t["W2"][pi], k=2)
+    assert np.array_equal(out, out_p)
+
+
+def test_w2_scaling_by_two_is_exact():
+    cfg, t = small_layer(N=10, H=64, I=32, E=4, k=2)
+    l32 = oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32)
+    out = oracle.layer_given_logits(t["x"], l32, t["W1"], t["W3"], t["W2"], 2)
+    out2 = oracle.layer_given_logits(t["x"], l32, t["W1"], t["W3"], enc(2.0 * dec(t["W2"])), 2)
+    assert np.array_equal(dec(out2), 2.0 * dec(out))
+
+
+def test_layer_routes_with_its_own_fp32_logits():
+    cfg, t = small_layer(N=10, H=64, I=32, E=4, k=2)
+    out, l32 = oracle.layer(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], k=2)
+    assert np.array_equal(l32, oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32))
+    assert np.array_equal(out, oracle.layer_given_logits(t["x"], l32, t["W1"], t["W3"], t["W2"], 2))
+
+
+def test_qwen3_30b_shape_matches_parameter_arithmetic():
+    """The MoE-latency article, section "内存按总参数算": Qwen3-30B-A3B holds
+    30.5B parameters, 8 of 128 experts per token, 48 layers, about 61 GB at
+    2 bytes per parameter.  The expert stacks of the Qwen3-30B-shaped layer
+    must fit inside that total."""
+    c = CONFIGS["qwen3_30b_a3b"]
+    expert_params = c.E * 3 * c.H * c.I * 48
+    assert c.E == 128 and c.k == 8
+    assert 0.9 * 30.5e9 < expert_params < 30.5e9
+    assert abs(30.5e9 * 2 / 1e9 - 61) < 0.5
