@@ -1,0 +1,384 @@
+"""Benchmark of the MoE expert layer on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+A step is one pass of the whole layer -- router, dispatch/permutation, W1/W3
+grouped GEMM + SwiGLU, W2 grouped GEMM, shared experts when the workload has
+them, combine -- over one batch of N synthetic tokens (seeded, inputs resident
+in HBM before timing).  Under torchrun every rank runs its own batch against its
+own copy of the weights (the layer shards by tokens with no exchange step:
+weak scaling); time is the max over ranks of CUDA-event time.
+
+`--impl reference` times the plain CPU oracle (test infrastructure, never tuned)
+on rank 0 on a bounded sample of tokens of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from expert_ffn_layer_moe_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PHASES = ("route", "permute", "gemm13", "gemm2", "shared", "combine")
+LAUNCHES = {"route": 1, "permute": 4, "gemm13": 1, "gemm2": 1, "shared": 2, "combine": 1}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(cfg):
+    s = f"{cfg.name}: N={cfg.N} H={cfg.H} I={cfg.I} E={cfg.E} top-{cfg.k}"
+    if cfg.Is:
+        s += f" shared Is={cfg.Is}"
+    if cfg.skew:
+        s += f" skew bias x{cfg.bias_scale}"
+    return s + ", bf16, SwiGLU experts"
+
+
+def layer_flops(cfg):
+    """Algorithmic FLOPs: router 2NHE + routed experts 6RHI + shared 6NHIs."""
+    return 2 * cfg.N * cfg.H * cfg.E + 6 * cfg.R * cfg.H * cfg.I + 6 * cfg.N * cfg.H * cfg.Is
+
+
+def gemm13_bytes(cfg, touched):
+    """W1+W3 tiles of the touched experts, x_perm read, h written."""
+    return touched * 2 * cfg.I * cfg.H * 2 + cfg.R * cfg.H * 2 + cfg.R * cfg.I * 2
+
+
+def gemm2_bytes(cfg, touched):
+    return touched * cfg.H * cfg.I * 2 + cfg.R * cfg.I * 2 + cfg.R * cfg.H * 2
+
+
+def layer_bytes(cfg, touched):
+    """Touched expert weights + shared weights + router weights + x in + out."""
+    return (touched * 3 * cfg.H * cfg.I * 2 + 3 * cfg.H * cfg.Is * 2 + cfg.H * cfg.E * 4
+            + 2 * cfg.N * cfg.H * 2)
+
+
+def kernel_traffic(kernel, workload):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.txt,
+    valid only while the kernel source is unchanged (its sha256 prefix matches)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    src = os.path.join(ROOT, "expert_ffn_layer_moe_b200", "csrc", "grouped_gemm.cu")
+    if not os.path.exists(path):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
+    for line in open(path):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload and f[3] == digest:
+            return float(f[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = [l.split(",") for l in open(self.path).read().splitlines() if l.strip()]
+        os.unlink(self.path)
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def oracle_sample_rate(cfg, t_host, tokens, seed=0):
+    """Tokens/s of the CPU oracle on `tokens` seeded tokens of the workload (whole
+    layer from x: logits, top-k, dispatch, experts, combine)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    sel = np.sort(rng.choice(cfg.N, tokens, replace=False))
+    x = t_host["x"][sel]
+    t0 = time.perf_counter()
+    oracle.layer(x, t_host["W_gate"], t_host["W1"], t_host["W3"], t_host["W2"], cfg.k, bias=t_host["bias"],
+                 Ws1=t_host["Ws1"], Ws3=t_host["Ws3"], Ws2=t_host["Ws2"])
+    dt = time.perf_counter() - t0
+    return tokens / dt, dt
+
+
+def host_inputs(cfg):
+    """Oracle-side copies (numpy, bf16 as uint16) of the seeded inputs."""
+    gen = "cuda" if torch.cuda.is_available() else "cpu"
+    t = make_inputs(cfg, seed=0, device=gen)
+    out = {}
+    for n, v in t.items():
+        if v is None:
+            out[n] = None
+        elif v.dtype == torch.bfloat16:
+            out[n] = v.cpu().view(torch.int16).numpy().view(np.uint16)
+        else:
+            out[n] = v.cpu().numpy()
+    del t
+    if torch.cuda.is_available():
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    th = host_inputs(cfg)
+    per_step = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_sample_rate(cfg, th, per_step)
+    total_tok, total_t = 0, 0.0
+    for i in range(args.steps):
+        r, dt = oracle_sample_rate(cfg, th, per_step, seed=i + 1)
+        total_tok += per_step
+        total_t += dt
+    value = total_tok / total_t
+    sample = f"{per_step} seeded tokens of the {cfg.N}-token batch per step, whole layer from x"
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * cfg.N / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": workload_desc(cfg), "global_batch": cfg.N, "parallelism": "rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, cfg, world, rank, local):
+    from expert_ffn_layer_moe_b200 import moe
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    t = make_inputs(cfg, seed=0, device=dev)
+    if world > 1:  # every rank its own token batch
+        t["x"] = make_inputs(cfg, seed=rank, device=dev, weights=False)["x"]
+    N, H, I, E, k = cfg.N, cfg.H, cfg.I, cfg.E, cfg.k
+    ws = torch.empty(moe.moe_workspace_bytes(N, H, I, E, k, cfg.Is), dtype=torch.uint8, device=dev)
+    out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+
+    def step(events=None):
+        moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], k, bias=t["bias"],
+                                 Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=out, stream=stream,
+                                 phase_events=events)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if moe.moe_get_device_error(stream) != 0:
+        raise RuntimeError("device error reported during warm-up")
+    counts = moe.moe_permute(t["x"], moe.moe_route(t["x"], t["W_gate"], k, bias=t["bias"])[0], E)["counts"]
+    touched = int((counts > 0).sum().item())
+    max_load = int(counts.max().item())
+    torch.cuda.synchronize()
+
+    phase_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(PHASES) + 1)] for _ in range(args.steps)]
+    for evs in phase_ev:  # materialise the events before handing their handles to C
+        for e in evs:
+            e.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(phase_ev[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = start.elapsed_time(end)
+    phase_ms = {p: statistics.mean(evs[j].elapsed_time(evs[j + 1]) for evs in phase_ev)
+                for j, p in enumerate(PHASES)}
+    if moe.moe_get_device_error(stream) != 0:
+        raise RuntimeError("device error reported during the timed steps")
+
+    # end to end through the public short form: host x in, host out back, every step
+    e2e = None
+    if cfg.Is == 0 and cfg.bias_scale == 1.0 and not cfg.skew:
+        x_host = t["x"].cpu().pin_memory()
+        out_host = torch.empty((N, H), dtype=torch.bfloat16).pin_memory()
+        for _ in range(args.warmup):
+            moe.moe_layer_forward(x_host, t["W_gate"], t["W1"], t["W3"], t["W2"], k, out=out_host)
+        barrier(world)
+        torch.cuda.synchronize()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        legacy = torch.cuda.default_stream(dev)
+        s0.record(legacy)
+        for _ in range(args.steps):
+            moe.moe_layer_forward(x_host, t["W_gate"], t["W1"], t["W3"], t["W2"], k, out=out_host)
+        s1.record(legacy)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+        e2e = {"value": world * N * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": N * H * 2, "d2h_bytes_per_step": N * H * 2}
+
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    step_s = elapsed_ms / 1e3 / args.steps
+    value = world * N / step_s
+    g13_s = phase_ms["gemm13"] / 1e3
+    g2_s = phase_ms["gemm2"] / 1e3
+    g13_b = gemm13_bytes(cfg, touched)
+    hbm = pk["hbm_gbs"]
+    achieved = g13_b / g13_s / 1e9
+    flops = layer_flops(cfg)
+    gemm_flops = 6 * cfg.R * H * I
+    lbytes = layer_bytes(cfg, touched)
+    floor_s = max(flops / (pk["bf16_tflops"] * 1e12), lbytes / (hbm * 1e9))
+    workload = cfg.name
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "global_batch": world * N, "tokens_per_gpu": N,
+                   "parallelism": f"dp{world} (token batches, replicated weights, no exchange)",
+                   "l2": f"inputs larger than L2: {touched} touched experts' weights "
+                         f"({touched * 3 * H * I * 2 / 1e9:.2f} GB) streamed from HBM every step",
+                   "touched_experts": touched, "max_expert_rows": max_load},
+        "roofline": {"bound": "hbm", "kernel": "grouped_gemm SwiGLU W1/W3 (gemm13)", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "peak_kind": pk_kind,
+                     "traffic": kernel_traffic("gemm13", workload), "alg_bytes_per_launch": g13_b,
+                     "avg_launch_ms": phase_ms["gemm13"]},
+        "layer": {"tflops": flops / step_s / 1e12, "alg_bytes": lbytes, "gb_s": lbytes / step_s / 1e9,
+                  "roofline_floor_us": floor_s * 1e6, "roofline_frac": floor_s / step_s,
+                  "useful_flop_fraction_k_over_E": k / E},
+        "grouped_gemm": {"tflops": gemm_flops / (g13_s + g2_s) / 1e12,
+                         "gb_s": (g13_b + gemm2_bytes(cfg, touched)) / (g13_s + g2_s) / 1e9,
+                         "gemm2_frac_hbm": gemm2_bytes(cfg, touched) / g2_s / 1e9 / hbm},
+        "phase_ms": phase_ms,
+        "gpu_launches": args.steps * sum(LAUNCHES[p] for p in PHASES if p != "shared" or cfg.Is > 0),
+        "e2e": e2e,
+    }
+    clk_sum = clk.summary()
+    if clk_sum:
+        line["clocks"] = clk_sum
+    if world == 1 and not args.no_cpu_baseline:
+        del t, ws
+        torch.cuda.empty_cache()
+        import oracle
+        oracle.build()
+        th = host_inputs(cfg)
+        rate, dt = oracle_sample_rate(cfg, th, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{args.cpu_tokens} seeded tokens of the {N}-token batch, whole "
+                                          f"layer from x, single thread, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    tt = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="mixtral_8x22b_decode", choices=sorted(CONFIGS))
+    ap.add_argument("--tokens", type=int, default=0, help="override N")
+    ap.add_argument("--cpu-tokens", type=int, default=12)
+    ap.add_argument("--ref-tokens", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    cfg = CONFIGS[args.config]
+    if args.tokens:
+        cfg = cfg.with_tokens(args.tokens)
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, world, rank)
+        else:
+            run_ours(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,363 @@
+// api.cu -- the C ABI (include/moe.h): argument checks, workspace layout, launch order.
+//
+// Every entry point validates its arguments on the host and launches nothing when a
+// check fails.  Kernels report device-side faults through one error word per device
+// (read and cleared by moe_get_device_error), never by trapping.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace {
+
+__device__ int g_moe_device_error;  // per device: first MOE_DEVERR_* code since the last read
+
+thread_local char g_last_cuda_error[256] = "no error";
+
+moe_status_t cuda_fail(cudaError_t e)
+{
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
+
+#define MOE_CUDA(call)                                   \
+    do {                                                 \
+        cudaError_t e_ = (call);                         \
+        if (e_ != cudaSuccess) return cuda_fail(e_);     \
+    } while (0)
+
+// Device address of the error word on the current device (host code must not use
+// the symbol itself as a pointer).
+int *device_error_word()
+{
+    static std::mutex mu;
+    static int *addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_moe_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_hidden(int v) { return v >= 64 && v <= 65536 && v % 64 == 0; }
+
+bool valid_ek(int E, int k) { return E >= 1 && E <= 256 && k >= 1 && k <= 8 && k <= E; }
+
+bool valid_rows(int64_t N, int k) { return N >= 0 && N * (int64_t)k < (int64_t(1) << 31); }
+
+size_t round_up(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct WsLayout {
+    size_t logits, idx, w, counts, offsets, r2t, t2r, perm, x_perm, h, hs, y_perm, s, total;
+};
+
+// Carve the layer's workspace; every buffer starts on a 256-byte boundary.
+void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
+{
+    const int64_t R = N * k;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t at = off; off += round_up(bytes ? bytes : 1); return at; };
+    L->logits = take((size_t)N * E * 4);
+    L->idx = take((size_t)R * 4);
+    L->w = take((size_t)R * 4);
+    L->counts = take((size_t)E * 4);
+    L->offsets = take((size_t)(E + 1) * 4);
+    L->r2t = take((size_t)R * 4);
+    L->t2r = take((size_t)R * 4);
+    L->perm = take((size_t)moe::permute_scratch_ints(R, E) * 4);
+    L->x_perm = take((size_t)R * H * 2);
+    L->h = take((size_t)R * I * 2);
+    L->hs = take((size_t)N * (Is > 0 ? Is : 0) * 2);
+    L->y_perm = take((size_t)R * H * 2);
+    L->s = take((size_t)N * (Is > 0 ? H : 0) * 2);
+    L->total = off;
+}
+
+moe_status_t expert_ffn_impl(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
+                             const uint16_t *W3, const uint16_t *W2, int64_t R, int H, int I, int E,
+                             uint16_t *h, uint16_t *y_perm, int *err, cudaStream_t s)
+{
+    if (R == 0) return MOE_OK;
+    moe::GroupedGemmArgs a{};
+    a.act = x_perm; a.w_a = W1; a.w_b = W3; a.offsets = offsets; a.groups = E; a.R = R;
+    a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
+    MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
+    moe::GroupedGemmArgs b{};
+    b.act = h; b.w_a = W2; b.w_b = nullptr; b.offsets = offsets; b.groups = E; b.R = R;
+    b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
+    MOE_CUDA(moe::launch_gemm2(b, s));
+    return MOE_OK;
+}
+
+// Shared experts: one dense SwiGLU FFN over all N rows = the grouped kernels with a
+// single group whose rows are x itself.
+moe_status_t shared_ffn_impl(const uint16_t *x, const uint16_t *Ws1, const uint16_t *Ws3,
+                             const uint16_t *Ws2, int64_t N, int H, int Is, uint16_t *hs, uint16_t *s_out,
+                             int *err, cudaStream_t s)
+{
+    if (N == 0) return MOE_OK;
+    moe::GroupedGemmArgs a{};
+    a.act = x; a.w_a = Ws1; a.w_b = Ws3; a.offsets = nullptr; a.groups = 1; a.R = N;
+    a.rows_single = (int)N; a.K = H; a.Nout = Is; a.out = hs; a.dev_err = err;
+    MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
+    moe::GroupedGemmArgs b{};
+    b.act = hs; b.w_a = Ws2; b.offsets = nullptr; b.groups = 1; b.R = N; b.rows_single = (int)N;
+    b.K = Is; b.Nout = H; b.out = s_out; b.dev_err = err;
+    MOE_CUDA(moe::launch_gemm2(b, s));
+    return MOE_OK;
+}
+
+moe_status_t record(void *const *ev, int i, cudaStream_t s)
+{
+    if (ev && ev[i]) MOE_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s));
+    return MOE_OK;
+}
+
+#define MOE_TRY(call)                            \
+    do {                                         \
+        moe_status_t st_ = (call);               \
+        if (st_ != MOE_OK) return st_;           \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(moe_status_t status)
+{
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape, alignment or device";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_DEVICE: return "device-side fault reported by a kernel";
+    }
+    return "unknown status";
+}
+
+const char *moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+int moe_device_sm_count(void) { return moe::device_sm_count(); }
+
+size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return 0;
+    if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return 0;
+    WsLayout L;
+    ws_layout(N, H, I, E, k, Is, &L);
+    return L.total;
+}
+
+moe_status_t moe_route(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
+                       int k, float *logits, int32_t *topk_idx, float *topk_w, void *stream)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
+    if (N == 0) return MOE_OK;
+    if (!x || !W_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x)) return MOE_ERR_UNSUPPORTED;
+    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w,
+                                static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+moe_status_t moe_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E, int k,
+                         int32_t *counts, int32_t *offsets, int32_t *row_to_token, int32_t *token_to_row,
+                         uint16_t *x_perm, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        // empty batch: the group table is still well defined (all zero)
+        MOE_CUDA(cudaMemsetAsync(counts, 0, (size_t)E * 4, s));
+        MOE_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * 4, s));
+        return MOE_OK;
+    }
+    if (!x || !topk_idx || !row_to_token || !token_to_row || !x_perm) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_UNSUPPORTED;
+    const size_t need = (size_t)moe::permute_scratch_ints(N * k, E) * 4;
+    if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
+    int *err = device_error_word();
+    if (!err) return cuda_fail(cudaGetLastError());
+    MOE_CUDA(moe::launch_permute(x, topk_idx, N, H, E, k, counts, offsets, row_to_token, token_to_row, x_perm,
+                                 static_cast<int32_t *>(ws), err, s));
+    return MOE_OK;
+}
+
+moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
+                            const uint16_t *W3, const uint16_t *W2, int64_t R, int H, int I, int E,
+                            uint16_t *y_perm, void *ws, size_t ws_bytes, void *stream)
+{
+    if (R < 0 || R >= (int64_t(1) << 31) || !valid_hidden(H) || !valid_hidden(I) || E < 1 || E > 256)
+        return MOE_ERR_INVALID_ARG;
+    if (R == 0) return MOE_OK;
+    if (!x_perm || !offsets || !W1 || !W3 || !W2 || !y_perm) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_perm) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(y_perm))
+        return MOE_ERR_UNSUPPORTED;
+    const size_t need = (size_t)R * I * 2;
+    if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    int *err = device_error_word();
+    if (!err) return cuda_fail(cudaGetLastError());
+    return expert_ffn_impl(x_perm, offsets, W1, W3, W2, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, err,
+                           static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const uint16_t *y_perm, const int32_t *token_to_row, const float *topk_w,
+                         const uint16_t *shared_out, int64_t N, int H, int k, uint16_t *out, void *stream)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || k < 1 || k > 8) return MOE_ERR_INVALID_ARG;
+    if (N == 0) return MOE_OK;
+    if (!y_perm || !token_to_row || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_perm) || !aligned16(out) || (shared_out && !aligned16(shared_out)))
+        return MOE_ERR_UNSUPPORTED;
+    MOE_CUDA(moe::launch_combine(y_perm, token_to_row, topk_w, shared_out, N, H, k, out,
+                                 static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const float *bias,
+                                  const uint16_t *W1, const uint16_t *W3, const uint16_t *W2,
+                                  const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2, int64_t N,
+                                  int H, int I, int E, int k, int Is, uint16_t *out, float *logits, void *ws,
+                                  size_t ws_bytes, void *stream, void *const *phase_events)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
+    if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (N == 0) return MOE_OK;
+    if (!x || !W_gate || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
+    if (Is > 0 && (!Ws1 || !Ws3 || !Ws2)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(out))
+        return MOE_ERR_UNSUPPORTED;
+    if (Is > 0 && (!aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2))) return MOE_ERR_UNSUPPORTED;
+    WsLayout L;
+    ws_layout(N, H, I, E, k, Is, &L);
+    if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    int *err = device_error_word();
+    if (!err) return cuda_fail(cudaGetLastError());
+
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *lg = logits ? logits : reinterpret_cast<float *>(base + L.logits);
+    int32_t *idx = reinterpret_cast<int32_t *>(base + L.idx);
+    float *w = reinterpret_cast<float *>(base + L.w);
+    int32_t *counts = reinterpret_cast<int32_t *>(base + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(base + L.offsets);
+    int32_t *r2t = reinterpret_cast<int32_t *>(base + L.r2t);
+    int32_t *t2r = reinterpret_cast<int32_t *>(base + L.t2r);
+    int32_t *perm = reinterpret_cast<int32_t *>(base + L.perm);
+    uint16_t *x_perm = reinterpret_cast<uint16_t *>(base + L.x_perm);
+    uint16_t *h = reinterpret_cast<uint16_t *>(base + L.h);
+    uint16_t *hs = reinterpret_cast<uint16_t *>(base + L.hs);
+    uint16_t *y_perm = reinterpret_cast<uint16_t *>(base + L.y_perm);
+    uint16_t *sh = Is > 0 ? reinterpret_cast<uint16_t *>(base + L.s) : nullptr;
+    const int64_t R = N * k;
+
+    MOE_TRY(record(phase_events, 0, s));
+    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
+    MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
+    {
+        moe::GroupedGemmArgs a{};
+        a.act = x_perm; a.w_a = W1; a.w_b = W3; a.offsets = offsets; a.groups = E; a.R = R;
+        a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
+        MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
+    }
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
+    {
+        moe::GroupedGemmArgs b{};
+        b.act = h; b.w_a = W2; b.offsets = offsets; b.groups = E; b.R = R;
+        b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
+        MOE_CUDA(moe::launch_gemm2(b, s));
+    }
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM2, s));
+    if (Is > 0) MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
+    MOE_CUDA(moe::launch_combine(y_perm, t2r, w, sh, N, H, k, out, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_COMBINE, s));
+    return MOE_OK;
+}
+
+moe_status_t moe_layer_forward(const uint16_t *x, const float *W_gate, const uint16_t *W1, const uint16_t *W3,
+                               const uint16_t *W2, int64_t N, int H, int I, int E, int k, uint16_t *out)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
+    if (N == 0) return MOE_OK;
+    if (!x || !W_gate || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
+
+    // Library-owned buffers, one set per device, grown on demand.
+    struct Cache { void *ws = nullptr; size_t ws_bytes = 0; void *io = nullptr; size_t io_bytes = 0; };
+    static Cache cache[64];
+    static std::mutex mu;
+    int dev = 0;
+    MOE_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    Cache &c = cache[dev];
+
+    auto is_device = [](const void *p) {
+        cudaPointerAttributes at{};
+        if (cudaPointerGetAttributes(&at, p) != cudaSuccess) { cudaGetLastError(); return false; }
+        return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+    };
+    const bool x_dev = is_device(x), out_dev = is_device(out);
+    const size_t act_bytes = round_up((size_t)N * H * 2);
+    const size_t io_need = (x_dev ? 0 : act_bytes) + (out_dev ? 0 : act_bytes);
+    const size_t ws_need = moe_workspace_bytes(N, H, I, E, k, 0);
+    if (c.ws_bytes < ws_need) {
+        if (c.ws) MOE_CUDA(cudaFree(c.ws));
+        c.ws = nullptr; c.ws_bytes = 0;
+        MOE_CUDA(cudaMalloc(&c.ws, ws_need));
+        c.ws_bytes = ws_need;
+    }
+    if (c.io_bytes < io_need) {
+        if (c.io) MOE_CUDA(cudaFree(c.io));
+        c.io = nullptr; c.io_bytes = 0;
+        MOE_CUDA(cudaMalloc(&c.io, io_need));
+        c.io_bytes = io_need;
+    }
+    const cudaStream_t s = 0;
+    uint8_t *io = static_cast<uint8_t *>(c.io);
+    const uint16_t *xd = x;
+    uint16_t *outd = out;
+    if (!x_dev) {
+        MOE_CUDA(cudaMemcpyAsync(io, x, (size_t)N * H * 2, cudaMemcpyHostToDevice, s));
+        xd = reinterpret_cast<const uint16_t *>(io);
+        io += act_bytes;
+    }
+    if (!out_dev) outd = reinterpret_cast<uint16_t *>(io);
+    MOE_TRY(moe_layer_forward_ex(xd, W_gate, nullptr, W1, W3, W2, nullptr, nullptr, nullptr, N, H, I, E, k, 0,
+                                 outd, nullptr, c.ws, c.ws_bytes, s, nullptr));
+    if (!out_dev) {
+        MOE_CUDA(cudaMemcpyAsync(out, outd, (size_t)N * H * 2, cudaMemcpyDeviceToHost, s));
+        MOE_CUDA(cudaStreamSynchronize(s));
+    }
+    return MOE_OK;
+}
+
+moe_status_t moe_get_device_error(void *stream, int32_t *code)
+{
+    if (!code) return MOE_ERR_INVALID_ARG;
+    MOE_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int v = 0;
+    MOE_CUDA(cudaMemcpyFromSymbol(&v, g_moe_device_error, sizeof v));
+    const int zero = 0;
+    MOE_CUDA(cudaMemcpyToSymbol(g_moe_device_error, &zero, sizeof zero));
+    *code = v;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+// combine.cu -- combine / unpermutation (sm_100a).
+//
+// MoE-latency article, section "router 之后还有一串动作": the inverse mapping brings
+// expert outputs back to token order, each is multiplied by its routing weight and
+// the k results are added.  Deterministic gather-reduce (no atomics):
+//
+//   acc = 0;  for j in pick order: acc = fmaf(w[t,j], y_perm[token_to_row[t,j]], acc)
+//   acc += shared_out[t]            (optional always-on shared experts, weight 1)
+//   out[t] = bf16_rn(acc)
+//
+// One block per token row, each thread 8 consecutive features (16-byte loads/stores);
+// HBM-bound: k rows read, one row written per token.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kMaxK = 8;
+
+__global__ void __launch_bounds__(kThreads)
+    combine_kernel(const uint16_t *__restrict__ y_perm, const int32_t *__restrict__ token_to_row,
+                   const float *__restrict__ topk_w, const uint16_t *__restrict__ shared_out, int64_t N,
+                   int H, int k, uint16_t *__restrict__ out)
+{
+    const int64_t t = blockIdx.x;
+    int rows[kMaxK];
+    float w[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        rows[j] = j < k ? token_to_row[t * k + j] : -1;
+        w[j] = j < k ? topk_w[t * k + j] : 0.f;
+    }
+    const int nvec = H / 8;
+    for (int v = threadIdx.x; v < nvec; v += kThreads) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+            if (j < k && rows[j] >= 0) {
+                const uint4 yv = __ldg(reinterpret_cast<const uint4 *>(y_perm + (int64_t)rows[j] * H) + v);
+                const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 f = unpack_bf16x2(yw[p]);
+                    acc[2 * p] = fmaf(w[j], f.x, acc[2 * p]);
+                    acc[2 * p + 1] = fmaf(w[j], f.y, acc[2 * p + 1]);
+                }
+            }
+        }
+        if (shared_out) {
+            const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(shared_out + t * H) + v);
+            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float2 f = unpack_bf16x2(sw[p]);
+                acc[2 * p] += f.x;
+                acc[2 * p + 1] += f.y;
+            }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        reinterpret_cast<uint4 *>(out + t * H)[v] = o;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *token_to_row, const float *topk_w,
+                           const uint16_t *shared_out, int64_t N, int H, int k, uint16_t *out, cudaStream_t s)
+{
+    if (N <= 0) return cudaSuccess;
+    combine_kernel<<<(unsigned)N, kThreads, 0, s>>>(y_perm, token_to_row, topk_w, shared_out, N, H, k, out);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

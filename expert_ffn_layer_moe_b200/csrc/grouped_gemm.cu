@@ -1,0 +1,523 @@
+// grouped_gemm.cu -- ragged grouped GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One persistent kernel per GEMM of the expert FFN.  Each expert's rows form a
+// group (MoE-latency article, section "router 之后还有一串动作": every expert runs
+// its own matrix, and a grouped GEMM merges them into one launch; FinDEP review,
+// section "核心公式": an expert is three GEMMs).  Two instantiations:
+//   * SWIGLU = true : h[r] = bf16( silu(x W1[e]^T) * (x W3[e]^T) ), the W1 and W3
+//                     products accumulate side by side in TMEM and the epilogue fuses
+//                     the SwiGLU;
+//   * SWIGLU = false: y[r] = bf16( h W2[e]^T ).
+//
+// Tile shape ("swap-AB"): the MMA's M side (128) walks the weight's output
+// features, its N side (BN = 32..256) walks the group's token rows.  Decode-sized
+// groups (a few dozen rows per expert) then fill the tensor core's N side instead
+// of padding M to 128, and every weight byte is read once per token tile.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over work items):
+//   warp 0 lane 0 : TMA producer  -- weight tile(s) [128 x 64] and activation tile
+//                   [BN x 64] per stage, 128-byte swizzle, mbarrier transaction counts;
+//   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (bf16 in, fp32 accumulate)
+//                   and tcgen05.commit to release stages and hand accumulators over;
+//   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
+//                   per warp), SwiGLU / rounding, bf16 stores of the tile's valid rows.
+// Work items are (group, feature tile, token tile), enumerated from the device-side
+// row offsets with no host synchronisation; empty groups produce no items (no
+// padding to a fixed capacity).  Every wait is bounded (globaltimer): on expiry the
+// kernel records MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain, frees
+// TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;     // weight rows (output features) per tile = MMA M
+constexpr int kBK = 64;      // K per pipeline stage: 64 bf16 = one 128-byte swizzle row
+constexpr int kUmmaK = 16;   // K of one tcgen05.mma kind::f16
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, far above any legal wait
+
+constexpr int pow2_at_least(int v, int p = 32) { return p >= v ? p : pow2_at_least(v, p * 2); }
+
+template <int BN, bool SWIGLU>
+struct Cfg {
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "token tile must be 32..256, step 32");
+    static constexpr int kNA = SWIGLU ? 2 : 1;          // weight tiles per stage
+    static constexpr int kABytes = kBM * kBK * 2;       // 16 KB
+    static constexpr int kBBytes = BN * kBK * 2;
+    static constexpr int kStageBytes = kNA * kABytes + kBBytes;
+    static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    static constexpr int kAccCols = kNA * BN;           // fp32 TMEM columns per accumulator set
+    static constexpr int kAccBufs = (2 * kAccCols <= 512) ? 2 : 1;
+    static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols);
+    static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs);
+    static constexpr int kSmemBytes =
+        1024 + kStages * kStageBytes + kBarBytes + 16 + 4 * 2 * (kMaxGroups + 1);
+    // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
+    // both operands K-major, N>>3 at bit 17, M>>4 at bit 24.
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+    static_assert(kStages >= 2, "pipeline needs at least two stages");
+    static_assert(kTmemCols <= 512, "TMEM has 512 columns");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+// ------------------------------------------------------------ PTX wrappers --
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity; false on timeout or abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *m)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, int c0, int c1, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, int c0, int c1, int c2,
+                                            uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA with
+// 128-byte swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart (SBO),
+// descriptor version 1 (bits 46..48), swizzle mode 2 = 128B (bits 61..63).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;              // leading byte offset: unused for swizzled K-major
+    d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane; the wait is inside the
+// same asm statement so no use of the registers can be scheduled before it.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+
+// ------------------------------------------------------------------ kernel --
+template <int BN, bool SWIGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
+                        const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
+                        int groups, int rows_single, int64_t R, int K, int Nout,
+                        uint16_t *__restrict__ out, int *dev_err)
+{
+    using C = Cfg<BN, SWIGLU>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);  // 1024-aligned for SW128
+
+    uint8_t *stages = smem;
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStageBytes);
+    uint64_t *empty_bar = full_bar + C::kStages;
+    uint64_t *tfull_bar = empty_bar + C::kStages;
+    uint64_t *tempty_bar = tfull_bar + C::kAccBufs;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty_bar + C::kAccBufs);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
+    int *g_tile = g_off + (kMaxGroups + 1);               // [groups+1] work-item prefix
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_feat = (Nout + kBM - 1) / kBM;
+    const int KB = (K + kBK - 1) / kBK;
+
+    // ---- work list: row offsets and the prefix of (token tiles x feature tiles) per group
+    if (offsets == nullptr) {
+        if (tid == 0) { g_off[0] = 0; g_off[1] = rows_single; }
+    } else {
+        for (int i = tid; i <= groups; i += kThreads) g_off[i] = offsets[i];
+    }
+    if (tid == 0) *abort_flag = 0;
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        bool bad = false;
+        for (int base = 0; base < groups; base += 32) {
+            const int gi = base + lane;
+            int items = 0;
+            if (gi < groups) {
+                const int lo = g_off[gi], hi = g_off[gi + 1];
+                if (lo < 0 || hi < lo || (int64_t)hi > R) bad = true;
+                else items = ((hi - lo + BN - 1) / BN) * n_feat;
+            }
+            int v = items;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (gi < groups) g_tile[gi + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) g_tile[0] = 0;
+        if (__any_sync(0xffffffffu, bad) && lane == 0) set_device_error(dev_err, MOE_DEVERR_BAD_OFFSETS);
+    }
+    __syncthreads();
+    const int total = g_tile[groups];
+    if ((int)blockIdx.x >= total) return;  // uniform: nothing allocated yet
+
+    // ---- barriers and TMEM
+    if (tid == 0) {
+        for (int s = 0; s < C::kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        for (int b = 0; b < C::kAccBufs; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // item -> (group, feature tile, first row, end row of the group)
+    auto decode = [&](int item, int &g, int &feat, int &row0, int &row_end) {
+        int lo = 0, hi = groups - 1;
+        while (lo < hi) {  // largest g with g_tile[g] <= item (skips empty groups)
+            const int mid = (lo + hi + 1) >> 1;
+            if (g_tile[mid] <= item) lo = mid; else hi = mid - 1;
+        }
+        g = lo;
+        const int local = item - g_tile[g];
+        const int ntok = (g_tile[g + 1] - g_tile[g]) / n_feat;
+        feat = local / ntok;
+        row0 = g_off[g] + (local % ntok) * BN;
+        row_end = g_off[g + 1];
+    };
+
+    bool failed = false;
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------ TMA producer
+        tma_prefetch_map(&tm_wa);
+        if (SWIGLU) tma_prefetch_map(&tm_wb);
+        tma_prefetch_map(&tm_act);
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
+            int g, feat, row0, row_end;
+            decode(item, g, feat, row0, row_end);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
+                uint8_t *st = stages + stage * C::kStageBytes;
+                mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
+                tma_load_3d(st, &tm_wa, kb * kBK, feat * kBM, g, &full_bar[stage]);
+                if (SWIGLU) tma_load_3d(st + C::kABytes, &tm_wb, kb * kBK, feat * kBM, g, &full_bar[stage]);
+                tma_load_2d(st + C::kNA * C::kABytes, &tm_act, kb * kBK, row0, &full_bar[stage]);
+                if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------------ MMA issuer
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, aphase = 0;
+        for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
+            if (!mbar_wait(&tempty_bar[acc], aphase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
+            tc_fence_after();
+            const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { failed = true; *abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(stages + stage * C::kStageBytes);
+                const uint64_t da = sdesc_sw128(sa);
+                const uint64_t da3 = sdesc_sw128(sa + C::kABytes);
+                const uint64_t db = sdesc_sw128(sa + C::kNA * C::kABytes);
+#pragma unroll
+                for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                    const uint32_t accumulate = (kb | kk) != 0;
+                    // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
+                    umma_bf16(d0, da + 2 * kk, db + 2 * kk, C::kIdesc, accumulate);
+                    if (SWIGLU) umma_bf16(d0 + BN, da3 + 2 * kk, db + 2 * kk, C::kIdesc, accumulate);
+                }
+                umma_commit(&empty_bar[stage]);  // stage free once these MMAs have read it
+                if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            }
+            if (failed) break;
+            umma_commit(&tfull_bar[acc]);        // accumulator complete
+            if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quadrant this warp may read
+        int acc = 0;
+        uint32_t aphase = 0;
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            int g, feat, row0, row_end;
+            decode(item, g, feat, row0, row_end);
+            // warp-uniform outcome: tcgen05.ld below is a warp-collective instruction
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], aphase, abort_flag));
+            if (!ok) { failed = true; *abort_flag = 1; break; }
+            tc_fence_after();
+            const int f = feat * kBM + q * 32 + lane;
+            const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
+            const int nrows = min(BN, row_end - row0);
+            for (int c0 = 0; c0 < nrows; c0 += 32) {
+                float a[32];
+                float b[32];
+                tmem_ld32(t0 + c0, a);
+                if (SWIGLU) tmem_ld32(t0 + BN + c0, b);
+                if (f < Nout) {
+                    uint16_t *dst = out + (size_t)(row0 + c0) * Nout + f;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        if (c0 + c < nrows) {
+                            const float v = SWIGLU ? silu(a[c]) * b[c] : a[c];
+                            dst[(size_t)c * Nout] = float_to_bf16_bits(v);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
+        }
+    }
+
+    if (failed) set_device_error(dev_err, MOE_DEVERR_PIPELINE_TIMEOUT);
+    __syncwarp();
+    __syncthreads();
+    if (*abort_flag) {
+        // let copies and MMAs already in flight land before the CTA's memory is released
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) { }
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// -------------------------------------------------------------------- host --
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// Weights [groups, Nout, K] bf16 as a 3-D map; box = 64 (K) x 128 (rows) x 1 (group).
+// Rows past Nout read as zero and never bleed into the next group.
+bool encode_weight_map(CUtensorMap *m, const void *ptr, int groups, int Nout, int K)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)Nout, (cuuint64_t)groups};
+    cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)Nout * (cuuint64_t)K * 2};
+    cuuint32_t box[3] = {(cuuint32_t)kBK, (cuuint32_t)kBM, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Activations [R, K] bf16 as a 2-D map; box = 64 (K) x BN (rows); rows >= R read as zero.
+bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int BN)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)R};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWIGLU>
+cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
+{
+    using C = Cfg<BN, SWIGLU>;
+    CUtensorMap ma, mb, mact;
+    if (!encode_weight_map(&ma, a.w_a, a.groups, a.Nout, a.K)) return cudaErrorInvalidValue;
+    if (SWIGLU) {
+        if (!encode_weight_map(&mb, a.w_b, a.groups, a.Nout, a.K)) return cudaErrorInvalidValue;
+    } else {
+        mb = ma;
+    }
+    if (!encode_act_map(&mact, a.act, a.R, a.K, BN)) return cudaErrorInvalidValue;
+    auto kern = grouped_gemm_kernel<BN, SWIGLU>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    kern<<<device_sm_count(), kThreads, C::kSmemBytes, s>>>(ma, mb, mact, a.offsets, a.groups, a.rows_single,
+                                                            a.R, a.K, a.Nout, a.out, a.dev_err);
+    return cudaGetLastError();
+}
+
+template <bool SWIGLU>
+cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
+{
+    if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
+    const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups);
+    switch (bn) {
+        case 32: return launch_impl<32, SWIGLU>(a, s);
+        case 64: return launch_impl<64, SWIGLU>(a, s);
+        case 128: return launch_impl<128, SWIGLU>(a, s);
+        case 256: return SWIGLU ? launch_impl<128, SWIGLU>(a, s) : launch_impl<256, SWIGLU>(a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+int device_sm_count()
+{
+    static int counts[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && counts[dev] > 0) return counts[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) counts[dev] = n;
+    return n;
+}
+
+// Token tile from the mean rows per group: decode-sized groups take narrow tiles
+// (less wasted MMA work, weights still read once per tile), large groups wide ones.
+int gemm_choose_token_tile(int64_t R, int groups)
+{
+    const int64_t mean = (R + groups - 1) / (groups > 0 ? groups : 1);
+    if (mean <= 24) return 32;
+    if (mean <= 48) return 64;
+    if (mean <= 160) return 128;
+    return 256;
+}
+
+cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s) { return launch_dispatch<true>(a, s); }
+cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s) { return launch_dispatch<false>(a, s); }
+
+}  // namespace moe

@@ -1,0 +1,51 @@
+// internal.h -- host-side launch interfaces between the kernel files and the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+// Router: logits (fp32), top-k indices and renormalised weights.
+cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *bias, int64_t N,
+                          int H, int E, int k, float *logits, int32_t *topk_idx, float *topk_w,
+                          cudaStream_t s);
+
+// Dispatch / permutation.  `scratch` holds permute_scratch_ints(R, E) ints.
+constexpr int kPermuteChunk = 1024;  // assignments per block in the count/rank passes
+inline int64_t permute_blocks(int64_t R) { return (R + kPermuteChunk - 1) / kPermuteChunk; }
+inline int64_t permute_scratch_ints(int64_t R, int E) { return permute_blocks(R) * E; }
+cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E,
+                           int k, int32_t *counts, int32_t *offsets, int32_t *row_to_token,
+                           int32_t *token_to_row, uint16_t *x_perm, int32_t *scratch,
+                           int *dev_err, cudaStream_t s);
+
+// Grouped GEMMs on tcgen05.  Weights are [groups, Nout, K]; activations [R, K];
+// rows of group g are offsets[g] .. offsets[g+1]-1 (offsets == nullptr: one group
+// of `rows_single` rows starting at row 0).
+struct GroupedGemmArgs {
+    const uint16_t *act;     // [R, K] bf16
+    const uint16_t *w_a;     // [groups, Nout, K] bf16 (W1, or W2)
+    const uint16_t *w_b;     // [groups, Nout, K] bf16 (W3) -- SwiGLU only
+    const int32_t *offsets;  // [groups + 1] device, or nullptr
+    int groups;
+    int64_t R;               // rows of `act` (and of `out`)
+    int rows_single;         // rows when offsets == nullptr
+    int K;
+    int Nout;
+    uint16_t *out;           // [R, Nout] bf16
+    int *dev_err;
+    int token_tile;          // 0 = choose from the shape
+};
+cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s);
+cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s);
+int gemm_choose_token_tile(int64_t R, int groups);
+int device_sm_count();
+
+// Combine / unpermutation.
+cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *token_to_row,
+                           const float *topk_w, const uint16_t *shared_out, int64_t N, int H,
+                           int k, uint16_t *out, cudaStream_t s);
+
+}  // namespace moe

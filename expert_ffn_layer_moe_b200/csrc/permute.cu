@@ -1,0 +1,158 @@
+// permute.cu -- dispatch and permutation of token rows into expert-contiguous order.
+//
+// MoE-latency article, section "router 之后还有一串动作": N tokens at top-k give N*k
+// assignments; grouping them by expert is dispatch, sorting the token rows by expert
+// is the permutation.  The result is deterministic and stable: assignment
+// a = t*k + j of expert e lands at row offsets[e] + #{a' < a : e(a') = e}.
+//
+// Four launches, no atomics on the row order:
+//   1. count  : per block of kPermuteChunk assignments, a per-expert histogram;
+//   2. scan   : one block -- counts[e], offsets = exclusive scan, and every block's
+//               starting row per expert (in place over the histograms);
+//   3. rank   : per block again, the stable rank of each assignment inside its
+//               block (warp match + per-warp counts, warps in order) -> row maps;
+//   4. gather : x_perm[r] = x[row_to_token[r]], one warp per row, 16-byte vectors.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxE = 256;
+static_assert(kPermuteChunk % kThreads == 0, "chunk is whole rounds of the block");
+
+__global__ void __launch_bounds__(kThreads)
+    count_kernel(const int32_t *__restrict__ idx, int64_t R, int E, int32_t *__restrict__ blk_cnt, int *err)
+{
+    __shared__ int hist[kMaxE];
+    for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
+    __syncthreads();
+    const int64_t a0 = (int64_t)blockIdx.x * kPermuteChunk;
+    for (int i = threadIdx.x; i < kPermuteChunk; i += kThreads) {
+        const int64_t a = a0 + i;
+        if (a >= R) break;
+        const int e = idx[a];
+        if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+        else set_device_error(err, MOE_DEVERR_BAD_EXPERT_INDEX);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kThreads) blk_cnt[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+// One block: totals per expert, exclusive scan, and per-block starting rows.
+__global__ void __launch_bounds__(kThreads)
+    scan_kernel(int32_t *__restrict__ blk_cnt, int64_t nblk, int E, int32_t *__restrict__ counts,
+                int32_t *__restrict__ offsets)
+{
+    __shared__ int s[kMaxE];
+    const int e = threadIdx.x;
+    int total = 0;
+    if (e < E)
+        for (int64_t b = 0; b < nblk; ++b) total += blk_cnt[b * E + e];
+    s[e] = e < E ? total : 0;
+    __syncthreads();
+    // inclusive Hillis-Steele scan over kThreads (>= E) entries
+    for (int o = 1; o < kThreads; o <<= 1) {
+        const int v = e >= o ? s[e - o] : 0;
+        __syncthreads();
+        s[e] += v;
+        __syncthreads();
+    }
+    if (e < E) {
+        const int start = s[e] - total;
+        counts[e] = total;
+        offsets[e] = start;
+        if (e == E - 1) offsets[E] = s[e];
+        int run = start;
+        for (int64_t b = 0; b < nblk; ++b) {
+            const int c = blk_cnt[b * E + e];
+            blk_cnt[b * E + e] = run;
+            run += c;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    rank_kernel(const int32_t *__restrict__ idx, int64_t R, int k, int E,
+                const int32_t *__restrict__ blk_base, int32_t *__restrict__ row_to_token,
+                int32_t *__restrict__ token_to_row)
+{
+    __shared__ int base[kMaxE];
+    __shared__ int wcnt[kWarps][kMaxE];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < E; e += kThreads) base[e] = blk_base[(int64_t)blockIdx.x * E + e];
+    const int64_t a0 = (int64_t)blockIdx.x * kPermuteChunk;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int round = 0; round < kPermuteChunk / kThreads; ++round) {
+        for (int i = threadIdx.x; i < kWarps * E; i += kThreads) (&wcnt[0][0])[(i / E) * kMaxE + i % E] = 0;
+        __syncthreads();
+        const int64_t a = a0 + (int64_t)round * kThreads + threadIdx.x;
+        int e = -1;
+        if (a < R) e = idx[a];
+        const bool valid = a < R && e >= 0 && e < E;
+        // lanes with equal keys form one group; invalid lanes get a key of their own
+        const int key = valid ? e : (kMaxE + lane);
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        const int rank_in_warp = __popc(peers & lt_mask);
+        if (valid && rank_in_warp == 0) wcnt[warp][e] = __popc(peers);
+        __syncthreads();
+        if (a < R) {
+            if (valid) {
+                int before = 0;
+                for (int w = 0; w < warp; ++w) before += wcnt[w][e];
+                const int row = base[e] + before + rank_in_warp;
+                row_to_token[row] = (int32_t)(a / k);
+                token_to_row[a] = row;
+            } else {
+                token_to_row[a] = -1;
+            }
+        }
+        __syncthreads();
+        for (int ee = threadIdx.x; ee < E; ee += kThreads) {
+            int add = 0;
+            for (int w = 0; w < kWarps; ++w) add += wcnt[w][ee];
+            base[ee] += add;
+        }
+        __syncthreads();
+        if (a0 + (int64_t)(round + 1) * kThreads >= R) break;  // uniform across the block
+    }
+}
+
+// x_perm[r] = x[row_to_token[r]] for r < offsets[E]; one warp per row.
+__global__ void __launch_bounds__(kThreads)
+    gather_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ row_to_token,
+                       const int32_t *__restrict__ offsets, int E, int H, uint16_t *__restrict__ x_perm)
+{
+    const int64_t rows = offsets[E];
+    const int nvec = H / 8;
+    const int64_t warp_global = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const int lane = threadIdx.x & 31;
+    for (int64_t r = warp_global; r < rows; r += nwarps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)row_to_token[r] * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * H);
+        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E, int k,
+                           int32_t *counts, int32_t *offsets, int32_t *row_to_token, int32_t *token_to_row,
+                           uint16_t *x_perm, int32_t *scratch, int *dev_err, cudaStream_t s)
+{
+    const int64_t R = N * k;
+    if (R <= 0) return cudaSuccess;
+    const int64_t nblk = permute_blocks(R);
+    count_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, E, scratch, dev_err);
+    scan_kernel<<<1, kThreads, 0, s>>>(scratch, nblk, E, counts, offsets);
+    rank_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, k, E, scratch, row_to_token, token_to_row);
+    const int64_t want = (R + kWarps - 1) / kWarps;
+    const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
+    gather_rows_kernel<<<gblocks, kThreads, 0, s>>>(x, row_to_token, offsets, E, H, x_perm);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

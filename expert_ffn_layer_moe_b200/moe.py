@@ -1,0 +1,184 @@
+"""Python binding of the C ABI in include/moe.h (argument marshalling only).
+
+Every function has the name of the C entry point it calls.  Tensors are torch
+tensors on the current CUDA device (bf16 as torch.bfloat16); outputs are
+allocated with torch when not given.  Each call runs on the current torch CUDA
+stream unless ``stream`` is given.  A non-OK status raises ``MoEError``.  There
+is no fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+_lib = None
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
+DEVERR = {0: "MOE_DEVERR_NONE", 1: "MOE_DEVERR_BAD_EXPERT_INDEX", 2: "MOE_DEVERR_PIPELINE_TIMEOUT",
+          3: "MOE_DEVERR_BAD_OFFSETS"}
+PHASES = ("route", "permute", "gemm13", "gemm2", "shared", "combine")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        detail = ""
+        if status == 4:
+            detail = ": " + lib().moe_last_cuda_error().decode()
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}{detail}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {_LIB_PATH} is missing "
+                               "(run __graft_entry__.build() or python expert_ffn_layer_moe_b200/build.py)")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i64, c_int, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.moe_status_string.argtypes = [c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_last_cuda_error.argtypes = []
+        L.moe_last_cuda_error.restype = ctypes.c_char_p
+        L.moe_workspace_bytes.argtypes = [i64, c_int, c_int, c_int, c_int, c_int]
+        L.moe_workspace_bytes.restype = sz
+        L.moe_route.argtypes = [vp, vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp]
+        L.moe_permute.argtypes = [vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_expert_ffn.argtypes = [vp, vp, vp, vp, vp, i64, c_int, c_int, c_int, vp, vp, sz, vp]
+        L.moe_combine.argtypes = [vp, vp, vp, vp, i64, c_int, c_int, vp, vp]
+        L.moe_layer_forward.argtypes = [vp, vp, vp, vp, vp, i64, c_int, c_int, c_int, c_int, vp]
+        L.moe_layer_forward_ex.argtypes = ([vp] * 9 + [i64] + [c_int] * 5 + [vp, vp, vp, sz, vp, vp])
+        L.moe_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+        L.moe_device_sm_count.argtypes = []
+        L.moe_device_sm_count.restype = c_int
+        for fn in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+                   "moe_layer_forward_ex", "moe_get_device_error"):
+            getattr(L, fn).restype = c_int
+        _lib = L
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    assert t.is_contiguous(), "tensors passed to the MoE library must be contiguous"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise MoEError(fn, status)
+
+
+def _empty(shape, dtype, like):
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+def moe_workspace_bytes(N: int, H: int, I: int, E: int, k: int, Is: int = 0) -> int:
+    return int(lib().moe_workspace_bytes(N, H, I, E, k, Is))
+
+
+def moe_device_sm_count() -> int:
+    return int(lib().moe_device_sm_count())
+
+
+def moe_route(x, W_gate, k, bias=None, logits=None, topk_idx=None, topk_w=None, stream=None):
+    """-> (topk_idx [N,k] int32, topk_w [N,k] fp32, logits [N,E] fp32 or None)."""
+    N, H = x.shape
+    E = W_gate.shape[1]
+    topk_idx = _empty((N, k), torch.int32, x) if topk_idx is None else topk_idx
+    topk_w = _empty((N, k), torch.float32, x) if topk_w is None else topk_w
+    _check("moe_route", lib().moe_route(_p(x), _p(W_gate), _p(bias), N, H, E, k, _p(logits),
+                                        _p(topk_idx), _p(topk_w), _s(stream)))
+    return topk_idx, topk_w, logits
+
+
+def moe_permute(x, topk_idx, E, ws=None, stream=None, out=None):
+    """-> dict(counts, offsets, row_to_token, token_to_row, x_perm)."""
+    N, H = x.shape
+    k = topk_idx.shape[1]
+    R = N * k
+    o = out or {}
+    counts = o.get("counts", _empty((E,), torch.int32, x))
+    offsets = o.get("offsets", _empty((E + 1,), torch.int32, x))
+    r2t = o.get("row_to_token", _empty((R,), torch.int32, x))
+    t2r = o.get("token_to_row", _empty((N, k), torch.int32, x))
+    x_perm = o.get("x_perm", _empty((R, H), torch.bfloat16, x))
+    if ws is None:
+        ws = _empty((max(1, moe_workspace_bytes(N, H, 64, E, k, 0)),), torch.uint8, x)
+    _check("moe_permute", lib().moe_permute(_p(x), _p(topk_idx), N, H, E, k, _p(counts), _p(offsets),
+                                            _p(r2t), _p(t2r), _p(x_perm), _p(ws), ws.numel(), _s(stream)))
+    return dict(counts=counts, offsets=offsets, row_to_token=r2t, token_to_row=t2r, x_perm=x_perm)
+
+
+def moe_expert_ffn(x_perm, offsets, W1, W3, W2, ws=None, y_perm=None, stream=None):
+    """-> y_perm [R,H] bf16 (rows past offsets[E] are left as allocated)."""
+    R, H = x_perm.shape
+    E, I, _ = W1.shape
+    y_perm = _empty((R, H), torch.bfloat16, x_perm) if y_perm is None else y_perm
+    if ws is None:
+        ws = _empty((max(16, R * I * 2),), torch.uint8, x_perm)
+    _check("moe_expert_ffn", lib().moe_expert_ffn(_p(x_perm), _p(offsets), _p(W1), _p(W3), _p(W2), R, H,
+                                                  I, E, _p(y_perm), _p(ws), ws.numel(), _s(stream)))
+    return y_perm
+
+
+def moe_combine(y_perm, token_to_row, topk_w, shared_out=None, out=None, stream=None):
+    """-> out [N,H] bf16."""
+    N, k = token_to_row.shape
+    H = y_perm.shape[1]
+    out = _empty((N, H), torch.bfloat16, y_perm) if out is None else out
+    _check("moe_combine", lib().moe_combine(_p(y_perm), _p(token_to_row), _p(topk_w), _p(shared_out), N,
+                                            H, k, _p(out), _s(stream)))
+    return out
+
+
+def moe_layer_forward(x, W_gate, W1, W3, W2, k, out=None):
+    """Short form: legacy default stream, library workspace; x and out may be
+    CPU tensors (host buffers, copied by the call) or CUDA tensors."""
+    N, H = x.shape
+    E, I, _ = W1.shape
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=x.device,
+                          pin_memory=(x.device.type == "cpu"))
+    _check("moe_layer_forward", lib().moe_layer_forward(_p(x), _p(W_gate), _p(W1), _p(W3), _p(W2), N, H,
+                                                        I, E, k, _p(out)))
+    return out
+
+
+def moe_layer_forward_ex(x, W_gate, W1, W3, W2, k, bias=None, Ws1=None, Ws3=None, Ws2=None, ws=None,
+                         out=None, logits=None, stream=None, phase_events: Optional[Sequence] = None):
+    """Explicit form: everything on `stream` (default: current), caller's workspace."""
+    N, H = x.shape
+    E, I, _ = W1.shape
+    Is = 0 if Ws1 is None else Ws1.shape[0]
+    out = _empty((N, H), torch.bfloat16, x) if out is None else out
+    if ws is None:
+        ws = _empty((max(16, moe_workspace_bytes(N, H, I, E, k, Is)),), torch.uint8, x)
+    ev = None
+    if phase_events is not None:
+        assert len(phase_events) == len(PHASES) + 1
+        ev = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
+    _check("moe_layer_forward_ex", lib().moe_layer_forward_ex(
+        _p(x), _p(W_gate), _p(bias), _p(W1), _p(W3), _p(W2), _p(Ws1), _p(Ws3), _p(Ws2), N, H, I, E, k, Is,
+        _p(out), _p(logits), _p(ws), ws.numel(), _s(stream), ev))
+    return out
+
+
+def moe_get_device_error(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device error word."""
+    code = ctypes.c_int32(0)
+    _check("moe_get_device_error", lib().moe_get_device_error(_s(stream), ctypes.byref(code)))
+    return int(code.value)

@@ -1,0 +1,198 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE expert layer library, libmoe_b200.so.
+ *
+ * One MoE layer: router top-k, dispatch/permutation of token rows into
+ * expert-contiguous groups, a SwiGLU FFN per expert as two grouped GEMMs
+ * (W1/W3 with a fused SwiGLU epilogue, then W2) on the tcgen05 tensor cores,
+ * optional always-on shared experts, and a deterministic weighted combine.
+ *
+ * Sources (web pages on the subject; cited by title and section):
+ *  [MoE-latency] "MoE 少算 FLOPs,延迟反而涨了:慢在搬 token 的路上",
+ *     sections "dense 和 MoE 的差别" (router, top-k, routing weights) and
+ *     "router 之后还有一串动作" (assignments, dispatch, permutation, grouped
+ *     GEMM, inverse mapping, weighting and summing = combine/unpermutation).
+ *  [FinDEP] "FinDEP: Efficient MoE Inference with Fine-Grained Scheduling of
+ *     Disaggregated Expert Parallelism", section "核心公式" (three GEMMs per
+ *     expert) and section "问题定义" (shared experts).
+ *
+ * Conventions for every call:
+ *  - bf16 tensors are passed as uint16_t storage (IEEE binary32's top half).
+ *  - Row-major layouts.  Weights are [out, in] (nn.Linear layout), so both
+ *    operands of every GEMM are K-contiguous.
+ *  - Pointers are DEVICE pointers owned by the caller unless a call says
+ *    otherwise; the library never frees them.  Every pointer a kernel reads
+ *    with TMA (x, x_perm, weights, outputs of the GEMMs) must be 16-byte
+ *    aligned; otherwise the call returns MOE_ERR_UNSUPPORTED.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls are asynchronous on it and launch nothing when argument
+ *    checks fail.
+ *  - Sizes: 1 <= E <= 256; 1 <= k <= min(E, 8); H and I multiples of 64
+ *    (H, I <= 65536); N*k < 2^31.  N == 0 returns MOE_OK with no launch.
+ *  - Device-side faults (an expert index outside [0,E) handed to
+ *    moe_permute, a pipeline wait that timed out) never trap: the kernel
+ *    skips the offending work and records a code in a per-device error word
+ *    that moe_get_device_error() reads and clears.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* a size or pointer is out of the documented range */
+    MOE_ERR_UNSUPPORTED = 2, /* a valid request this build does not handle (alignment, device) */
+    MOE_ERR_WORKSPACE = 3,   /* workspace pointer NULL or smaller than moe_workspace_bytes() */
+    MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed; see moe_last_cuda_error() */
+    MOE_ERR_DEVICE = 5       /* a kernel reported a device-side fault (moe_get_device_error) */
+} moe_status_t;
+
+/* Device error codes (moe_get_device_error). */
+#define MOE_DEVERR_NONE 0
+#define MOE_DEVERR_BAD_EXPERT_INDEX 1 /* moe_permute saw topk_idx outside [0,E) */
+#define MOE_DEVERR_PIPELINE_TIMEOUT 2 /* a grouped-GEMM pipeline wait exceeded its limit */
+#define MOE_DEVERR_BAD_OFFSETS 3      /* offsets not monotone or beyond R */
+
+/* Text of a status code (static storage). */
+MOE_API const char *moe_status_string(moe_status_t status);
+
+/* Text of the last CUDA error seen by this thread's calls (static storage). */
+MOE_API const char *moe_last_cuda_error(void);
+
+/*
+ * Bytes of device workspace moe_layer_forward_ex needs for this shape
+ * (Is = total width of the shared experts, 0 for none).  Returns 0 on
+ * invalid sizes.  The same number covers moe_permute and moe_expert_ffn.
+ */
+MOE_API size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is);
+
+/*
+ * Router ([MoE-latency] "dense 和 MoE 的差别"): score every expert, pick the
+ * top k, give k routing weights.
+ *   x         [N,H] bf16           token hidden states
+ *   W_gate    [H,E] fp32           router weights
+ *   bias      [E] fp32 or NULL     added to every logit (e.g. a load bias)
+ *   logits    [N,E] fp32 or NULL   output: logit[t,e] = sum_h x[t,h] W_gate[h,e] (+ bias[e]),
+ *                                  fp32 accumulation
+ *   topk_idx  [N,k] int32          output: experts in pick order -- larger logit
+ *                                  first, equal logits by lower expert index
+ *   topk_w    [N,k] fp32           output: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)
+ *                                  over the k picks (softmax renormalised over the picks)
+ * NaN logits are unsupported input (the pick among them is unspecified).
+ */
+MOE_API moe_status_t moe_route(const uint16_t *x, const float *W_gate, const float *bias, int64_t N,
+                       int H, int E, int k, float *logits, int32_t *topk_idx, float *topk_w,
+                       void *stream);
+
+/*
+ * Dispatch and permutation ([MoE-latency] "router 之后还有一串动作"): group
+ * the N*k assignments by expert and copy token rows into expert-contiguous
+ * order.  Deterministic and stable: within expert e, rows follow the
+ * assignment id a = t*k + j.
+ *   topk_idx      [N,k] int32      input
+ *   counts        [E] int32        output: rows per expert
+ *   offsets       [E+1] int32      output: exclusive scan of counts, offsets[E] = rows placed
+ *   row_to_token  [N*k] int32      output: token of each permuted row
+ *   token_to_row  [N,k] int32      output: permuted row of each assignment (-1 if the
+ *                                  assignment's expert index was invalid)
+ *   x_perm        [N*k,H] bf16     output: x_perm[r] = x[row_to_token[r]]
+ *   ws, ws_bytes                   device scratch, >= moe_workspace_bytes(N,H,64,E,k,0)
+ * An index outside [0,E) is skipped and sets MOE_DEVERR_BAD_EXPERT_INDEX.
+ */
+MOE_API moe_status_t moe_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E,
+                         int k, int32_t *counts, int32_t *offsets, int32_t *row_to_token,
+                         int32_t *token_to_row, uint16_t *x_perm, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/*
+ * Expert FFN as two grouped GEMMs ([MoE-latency] "router 之后还有一串动作":
+ * each expert runs its own matrix, merged into one launch; [FinDEP] "核心公式":
+ * three GEMMs per expert).  For rows r in [offsets[e], offsets[e+1]):
+ *   h[r]      = bf16( silu(x_perm[r] W1[e]^T) * (x_perm[r] W3[e]^T) )   fp32 accumulation,
+ *               silu(z) = z / (1 + exp(-z))
+ *   y_perm[r] = bf16( h[r] W2[e]^T )                                   fp32 accumulation
+ *   x_perm  [R,H] bf16; offsets [E+1] int32 (device; monotone, offsets[E] <= R)
+ *   W1, W3  [E,I,H] bf16; W2 [E,H,I] bf16; y_perm [R,H] bf16 (rows beyond offsets[E] untouched)
+ *   ws, ws_bytes: device scratch for h, >= moe_workspace_bytes(R,H,I,E,1,0)
+ */
+MOE_API moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
+                            const uint16_t *W3, const uint16_t *W2, int64_t R, int H, int I,
+                            int E, uint16_t *y_perm, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Combine / unpermutation ([MoE-latency] "router 之后还有一串动作": inverse
+ * mapping to token order, multiply by routing weight, add):
+ *   out[t] = bf16( fma-chain over j = 0..k-1 of topk_w[t,j] * y_perm[token_to_row[t,j]]
+ *                  (+ shared_out[t]) )   fp32, picks in order; rows < 0 are skipped
+ *   y_perm [R,H] bf16; token_to_row [N,k] int32; topk_w [N,k] fp32;
+ *   shared_out [N,H] bf16 or NULL; out [N,H] bf16.
+ */
+MOE_API moe_status_t moe_combine(const uint16_t *y_perm, const int32_t *token_to_row,
+                         const float *topk_w, const uint16_t *shared_out, int64_t N, int H, int k,
+                         uint16_t *out, void *stream);
+
+/*
+ * The whole layer, short form: route -> permute -> expert FFN -> combine,
+ * no bias, no shared experts, on the legacy default stream, with a
+ * library-owned workspace that grows on demand (not thread-safe).
+ *   x [N,H] bf16 and out [N,H] bf16 may be HOST or DEVICE pointers: host
+ *   buffers are copied in and out by the call (which then returns only after
+ *   out is written).  W_gate [H,E] fp32, W1, W3 [E,I,H] and W2 [E,H,I] bf16
+ *   must be device pointers (weights stay resident).
+ */
+MOE_API moe_status_t moe_layer_forward(const uint16_t *x, const float *W_gate, const uint16_t *W1,
+                               const uint16_t *W3, const uint16_t *W2, int64_t N, int H, int I,
+                               int E, int k, uint16_t *out);
+
+/*
+ * The whole layer, explicit form: everything on `stream`, caller's workspace,
+ * no allocation.  All pointers are device pointers.
+ *   bias [E] fp32 or NULL; Ws1, Ws3 [Is,H], Ws2 [H,Is] bf16 = shared experts
+ *   ([FinDEP] "问题定义"), their widths concatenated into Is (0 = none, then the
+ *   three pointers are ignored); their output is added with weight 1 after
+ *   the routed sum.  logits [N,E] fp32 is an optional output (NULL = keep it
+ *   in the workspace).
+ *   phase_events: NULL, or an array of MOE_NUM_PHASES + 1 cudaEvent_t (as
+ *   void*) recorded on `stream` before the first and after each phase, for
+ *   per-kernel timing.
+ */
+#define MOE_PHASE_ROUTE 0
+#define MOE_PHASE_PERMUTE 1
+#define MOE_PHASE_GEMM13 2
+#define MOE_PHASE_GEMM2 3
+#define MOE_PHASE_SHARED 4
+#define MOE_PHASE_COMBINE 5
+#define MOE_NUM_PHASES 6
+MOE_API moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const float *bias,
+                                  const uint16_t *W1, const uint16_t *W3, const uint16_t *W2,
+                                  const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2,
+                                  int64_t N, int H, int I, int E, int k, int Is, uint16_t *out,
+                                  float *logits, void *ws, size_t ws_bytes, void *stream,
+                                  void *const *phase_events);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  *code receives a MOE_DEVERR_* value.  Returns MOE_OK, or
+ * MOE_ERR_CUDA if the synchronisation itself failed.
+ */
+MOE_API moe_status_t moe_get_device_error(void *stream, int32_t *code);
+
+/* Number of streaming multiprocessors the grouped GEMM sizes its persistent grid to. */
+MOE_API int moe_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

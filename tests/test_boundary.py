@@ -1,0 +1,88 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/*.h declares, sizes workspaces, and rejects bad arguments before any
+CUDA call."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from expert_ffn_layer_moe_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names.update(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert {"moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"} <= names
+    L = moe.lib()
+    missing = [n for n in sorted(names) if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_workspace_bytes():
+    f = moe.moe_workspace_bytes
+    assert f(156, 6144, 16384, 8, 2) > 156 * 2 * (6144 * 2 * 2 + 16384 * 2)
+    assert f(156, 6144, 16384, 8, 2, 3072) > f(156, 6144, 16384, 8, 2, 0)
+    assert f(2000, 256, 512, 8, 2) > f(1000, 256, 512, 8, 2)
+    # invalid sizes -> 0
+    assert f(10, 100, 512, 8, 2) == 0        # H not a multiple of 64
+    assert f(10, 256, 512, 0, 1) == 0        # no experts
+    assert f(10, 256, 512, 4, 5) == 0        # k > E
+    assert f(10, 256, 512, 300, 2) == 0      # E > 256
+    assert f(10, 256, 512, 16, 9) == 0       # k > 8
+    assert f(-1, 256, 512, 8, 2) == 0
+    assert f(10, 256, 512, 8, 2, 100) == 0   # shared width not a multiple of 64
+
+
+def test_invalid_arguments_are_rejected_before_any_launch():
+    L = moe.lib()
+    nullp = None
+    s = ctypes.c_void_p(0)
+    # bad sizes: every call returns MOE_ERR_INVALID_ARG (1) without touching CUDA
+    assert L.moe_route(nullp, nullp, nullp, 4, 256, 0, 1, nullp, nullp, nullp, s) == 1
+    assert L.moe_route(nullp, nullp, nullp, 4, 256, 8, 9, nullp, nullp, nullp, s) == 1
+    assert L.moe_route(nullp, nullp, nullp, 4, 100, 8, 2, nullp, nullp, nullp, s) == 1
+    assert L.moe_route(nullp, nullp, nullp, 4, 256, 8, 2, nullp, nullp, nullp, s) == 1  # null pointers
+    assert L.moe_permute(nullp, nullp, 4, 256, 8, 2, nullp, nullp, nullp, nullp, nullp, nullp, 0, s) == 1
+    assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, -1, 256, 512, 8, nullp, nullp, 0, s) == 1
+    assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, 8, 256, 500, 8, nullp, nullp, 0, s) == 1
+    assert L.moe_combine(nullp, nullp, nullp, nullp, 4, 256, 0, nullp, s) == 1
+    assert L.moe_layer_forward(nullp, nullp, nullp, nullp, nullp, 4, 256, 512, 8, 2, nullp) == 1
+    assert L.moe_layer_forward_ex(*([nullp] * 9), 4, 256, 512, 8, 2, 64, nullp, nullp, nullp, 0, s,
+                                  nullp) == 1
+    # N == 0 is a no-op where no output needs defining
+    assert L.moe_route(nullp, nullp, nullp, 0, 256, 8, 2, nullp, nullp, nullp, s) == 0
+    assert L.moe_combine(nullp, nullp, nullp, nullp, 0, 256, 2, nullp, s) == 0
+    assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, 0, 256, 512, 8, nullp, nullp, 0, s) == 0
+
+
+def test_misaligned_pointers_are_unsupported():
+    L = moe.lib()
+    fake = ctypes.c_void_p(0x1000 + 8)   # never dereferenced: the check comes first
+    ok = ctypes.c_void_p(0x2000)
+    s = ctypes.c_void_p(0)
+    assert L.moe_route(fake, ok, None, 4, 256, 8, 2, None, ok, ok, s) == 2
+    assert L.moe_combine(fake, ok, ok, None, 4, 256, 2, ok, s) == 2
+
+
+def test_status_strings():
+    L = moe.lib()
+    assert L.moe_status_string(0) == b"ok"
+    assert L.moe_status_string(3).startswith(b"workspace")
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "_LIB_PATH", "/nonexistent/libmoe_b200.so")
+    with pytest.raises(RuntimeError, match="not built"):
+        moe.lib()

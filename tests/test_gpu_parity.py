@@ -1,0 +1,251 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bars: routing indices, counts, offsets, row maps and permuted rows bit-exact
+(the oracle picks experts from the GPU's fp32 logits, so both sides take that
+integer decision in the same precision); logits within a float64-derived bound;
+routing weights within a few fp32 ulp; h, y and out within
+|d| <= 2e-2*|ref| + 2e-3 with bf16 rounding at the same points.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from expert_ffn_layer_moe_b200 import moe
+from expert_ffn_layer_moe_b200.inputs import CONFIGS, MoEConfig, make_inputs
+from tests._bf16 import dec, to_u16
+
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL = 2e-2, 2e-3
+
+
+def assert_close_bf16(got_u16, want_u16, what):
+    g, w = dec(got_u16), dec(want_u16)
+    bad = np.abs(g - w) > RTOL * np.abs(w) + ATOL
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; first at "
+                           f"{np.argwhere(bad)[0].tolist()}: got {g[bad][0]} want {w[bad][0]}")
+
+
+def cuda_inputs(cfg, seed=0, gen_device="cpu"):
+    t = make_inputs(cfg, seed=seed, device=gen_device)
+    return {n: (v.cuda() if v is not None else None) for n, v in t.items()}
+
+
+def host(t):
+    if t is None:
+        return None
+    t = t.detach().cpu()
+    return to_u16(t) if t.dtype == torch.bfloat16 else t.numpy()
+
+
+def run_layer(cfg, t, **kw):
+    logits = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device="cuda")
+    out = moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k, bias=t["bias"],
+                                   Ws1=t.get("Ws1"), Ws3=t.get("Ws3"), Ws2=t.get("Ws2"), logits=logits, **kw)
+    assert moe.moe_get_device_error() == 0
+    return out, logits
+
+
+def check_layer_against_oracle(cfg, t, out, logits, tokens=None):
+    """Compare out (and routing) for `tokens` (default: all) with the oracle fed
+    the same inputs and the GPU's fp32 logits."""
+    sel = slice(None) if tokens is None else tokens
+    x = host(t["x"])[sel]
+    l32 = host(logits)[sel]
+    ref = oracle.layer_given_logits(x, l32, host(t["W1"]), host(t["W3"]), host(t["W2"]), cfg.k,
+                                    Ws1=host(t.get("Ws1")), Ws3=host(t.get("Ws3")), Ws2=host(t.get("Ws2")))
+    assert_close_bf16(host(out)[sel], ref, f"{cfg.name} out")
+
+
+def check_logits(cfg, t, logits):
+    l64 = oracle.router_logits(host(t["x"]), host(t["W_gate"]), host(t["bias"]))
+    xd = dec(host(t["x"]))
+    scale = np.abs(xd) @ np.abs(host(t["W_gate"]).astype(np.float64))
+    bound = 2.0 ** -20 * scale + 1e-6
+    assert np.all(np.abs(host(logits) - l64) <= bound)
+
+
+# --------------------------------------------------------------- the steps ---
+
+def test_route_matches_oracle():
+    cfg = CONFIGS["tiny"]
+    t = cuda_inputs(cfg)
+    logits = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device="cuda")
+    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k, logits=logits)
+    torch.cuda.synchronize()
+    check_logits(cfg, t, logits)
+    ref_idx, ref_w = oracle.topk(host(logits), cfg.k)
+    assert np.array_equal(host(idx), ref_idx)
+    assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (160, 6), (128, 8), (37, 3), (1, 1), (256, 8)])
+def test_route_shapes_and_bias(E, k):
+    cfg = MoEConfig("route", N=203, H=512, I=64, E=E, k=k)
+    t = cuda_inputs(cfg, seed=4)
+    bias = torch.linspace(-0.5, 0.5, E, device="cuda")
+    logits = torch.empty((cfg.N, E), dtype=torch.float32, device="cuda")
+    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], k, bias=bias, logits=logits)
+    torch.cuda.synchronize()
+    t["bias"] = bias
+    check_logits(cfg, t, logits)
+    ref_idx, ref_w = oracle.topk(host(logits), k)
+    assert np.array_equal(host(idx), ref_idx)
+    assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
+
+
+def test_route_ties_lower_index_first():
+    # all-zero hidden states: every logit equals the bias, with exact ties
+    N, H, E, k = 5, 256, 16, 4
+    x = torch.zeros((N, H), dtype=torch.bfloat16, device="cuda")
+    Wg = torch.randn((H, E), device="cuda")
+    bias = torch.tensor([0, 1, 1, 0, 2, 2, 2, 0, -1, 1, 0, 0, 2, 0, 0, 1], dtype=torch.float32, device="cuda")
+    idx, w, _ = moe.moe_route(x, Wg, k, bias=bias)
+    torch.cuda.synchronize()
+    assert host(idx).tolist() == [[4, 5, 6, 12]] * N
+    assert np.allclose(host(w), 0.25, rtol=0, atol=1e-7)
+
+
+@pytest.mark.parametrize("N,E,k", [(64, 8, 2), (1000, 160, 6), (3000, 128, 8), (7, 4, 4), (1, 1, 1)])
+def test_permute_bit_exact(N, E, k):
+    H = 128
+    g = torch.Generator().manual_seed(N + E)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(N)]).to(torch.int32)
+    idx[: N // 3, 0] = 0                           # a hot expert
+    x = (torch.randn((N, H), generator=g) * 3).to(torch.bfloat16)
+    res = moe.moe_permute(x.cuda(), idx.cuda(), E)
+    torch.cuda.synchronize()
+    counts, offsets, r2t, t2r = oracle.dispatch(idx.numpy(), E)
+    assert np.array_equal(host(res["counts"]), counts)
+    assert np.array_equal(host(res["offsets"]), offsets)
+    assert np.array_equal(host(res["row_to_token"]), r2t)
+    assert np.array_equal(host(res["token_to_row"]), t2r)
+    assert np.array_equal(host(res["x_perm"]), oracle.permute_rows(to_u16(x), r2t))
+    assert moe.moe_get_device_error() == 0
+
+
+def test_permute_bad_index_reports_without_trap():
+    N, H, E, k = 40, 64, 4, 2
+    idx = torch.randint(0, E, (N, k), dtype=torch.int32)
+    idx[:, 1] = (idx[:, 0] + 1) % E
+    idx[7, 1] = 9                                  # outside [0, E)
+    idx[12, 0] = -3
+    x = torch.randn((N, H)).to(torch.bfloat16).cuda()
+    res = moe.moe_permute(x, idx.cuda(), E)
+    assert moe.moe_get_device_error() == 1         # MOE_DEVERR_BAD_EXPERT_INDEX
+    assert moe.moe_get_device_error() == 0         # read clears it
+    t2r = host(res["token_to_row"])
+    assert t2r[7, 1] == -1 and t2r[12, 0] == -1
+    assert host(res["offsets"])[-1] == N * k - 2
+
+
+def test_expert_ffn_matches_oracle_tiny():
+    cfg = CONFIGS["tiny"]
+    t = cuda_inputs(cfg)
+    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k)
+    p = moe.moe_permute(t["x"], idx, cfg.E)
+    y = moe.moe_expert_ffn(p["x_perm"], p["offsets"], t["W1"], t["W3"], t["W2"])
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error() == 0
+    ref = oracle.expert_ffn(host(p["x_perm"]), host(p["offsets"]), host(t["W1"]), host(t["W3"]), host(t["W2"]))
+    assert_close_bf16(host(y), ref, "y_perm")
+
+
+def test_combine_matches_oracle():
+    N, H, k, R = 50, 192, 3, 150
+    g = torch.Generator().manual_seed(2)
+    y = torch.randn((R, H), generator=g).to(torch.bfloat16)
+    t2r = torch.randperm(R, generator=g).to(torch.int32).reshape(N, k)
+    w = torch.softmax(torch.randn((N, k), generator=g), 1).to(torch.float32)
+    s = torch.randn((N, H), generator=g).to(torch.bfloat16)
+    for shared in (None, s):
+        out = moe.moe_combine(y.cuda(), t2r.cuda(), w.cuda(), None if shared is None else shared.cuda())
+        ref = oracle.combine(to_u16(y), t2r.numpy(), w.numpy().astype(np.float64),
+                             None if shared is None else to_u16(shared))
+        assert_close_bf16(host(out), ref, "combine")
+
+
+# -------------------------------------------------------------- full layer ---
+
+def test_layer_tiny_matches_oracle():
+    cfg = CONFIGS["tiny"]
+    t = cuda_inputs(cfg)
+    out, logits = run_layer(cfg, t)
+    check_logits(cfg, t, logits)
+    check_layer_against_oracle(cfg, t, out, logits)
+
+
+@pytest.mark.parametrize("cfg", [
+    # several token tiles per expert with a ragged tail, K loop of 5, feature tiles 2.5 and 1.5
+    MoEConfig("ragged", N=300, H=320, I=192, E=5, k=2),
+    # mean 12 rows per expert -> 32-row token tiles
+    MoEConfig("narrow", N=48, H=256, I=256, E=16, k=4),
+    # mean ~100 rows -> 128-row tiles
+    MoEConfig("wide", N=400, H=256, I=384, E=8, k=2),
+    # mean ~400 rows -> 256-row tiles for W2
+    MoEConfig("wider", N=800, H=192, I=128, E=4, k=2),
+    # one expert, top-1: a dense SwiGLU FFN
+    MoEConfig("dense", N=77, H=128, I=256, E=1, k=1),
+    # shared experts on top of routed ones
+    MoEConfig("shared", N=90, H=256, I=128, E=6, k=2, Is=192),
+])
+def test_layer_shapes_match_oracle(cfg):
+    t = cuda_inputs(cfg, seed=1)
+    out, logits = run_layer(cfg, t)
+    check_layer_against_oracle(cfg, t, out, logits)
+
+
+def test_layer_skewed_routing_with_empty_experts():
+    cfg = MoEConfig("skew", N=256, H=256, I=256, E=12, k=2)
+    t = cuda_inputs(cfg, seed=5)
+    # experts 0 and 1 take every token; the others stay empty
+    t["bias"] = torch.tensor([50.0, 40.0] + [-50.0] * 10, device="cuda")
+    out, logits = run_layer(cfg, t)
+    check_layer_against_oracle(cfg, t, out, logits)
+
+
+def test_layer_empty_batch_is_a_no_op():
+    cfg = CONFIGS["tiny"]
+    t = cuda_inputs(cfg)
+    out = torch.full((0, cfg.H), 7, dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_forward_ex(t["x"][:0], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k, out=out)
+    assert moe.moe_get_device_error() == 0
+
+
+def test_layer_is_deterministic():
+    cfg = MoEConfig("det", N=500, H=256, I=256, E=8, k=2)
+    t = cuda_inputs(cfg, seed=9)
+    a, _ = run_layer(cfg, t)
+    b, _ = run_layer(cfg, t)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_short_form_with_host_buffers_matches_explicit_form():
+    cfg = CONFIGS["tiny"]
+    t = cuda_inputs(cfg)
+    ref = moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k)
+    x_host = t["x"].cpu().pin_memory()
+    out_host = moe.moe_layer_forward(x_host, t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k)
+    assert out_host.device.type == "cpu"
+    assert torch.equal(out_host.view(torch.int16), ref.cpu().view(torch.int16))
+    out_dev = moe.moe_layer_forward(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k)
+    assert torch.equal(out_dev.view(torch.int16), ref.view(torch.int16))
+
+
+def test_mixtral_decode_full_size_sampled():
+    """The benchmark's workload and launch path: full-size routing maps bit-exact,
+    outputs of a seeded sample of tokens against the oracle."""
+    cfg = CONFIGS["mixtral_8x22b_decode"]
+    t = cuda_inputs(cfg, gen_device="cuda")
+    out, logits = run_layer(cfg, t)
+    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k)
+    p = moe.moe_permute(t["x"], idx, cfg.E)
+    ref_idx, _ = oracle.topk(host(logits), cfg.k)
+    assert np.array_equal(host(idx), ref_idx)
+    counts, offsets, r2t, t2r = oracle.dispatch(ref_idx, cfg.E)
+    assert np.array_equal(host(p["offsets"]), offsets)
+    assert np.array_equal(host(p["row_to_token"]), r2t)
+    assert counts.sum() / cfg.E == 39
+    sample = np.random.default_rng(0).choice(cfg.N, 6, replace=False)
+    check_layer_against_oracle(cfg, t, out, logits, tokens=np.sort(sample))
