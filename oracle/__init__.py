@@ -63,16 +63,16 @@ def lib():
         L.oracle_dispatch.restype = c_int
         L.oracle_permute_rows.argtypes = [_P(u16), _P(i32), i64, c_int, _P(u16)]
         L.oracle_permute_rows.restype = None
-        L.oracle_swiglu_ffn.argtypes = [_P(u16), _P(u16), _P(u16), _P(u16), c_int, c_int, _P(u16)]
+        L.oracle_swiglu_ffn.argtypes = [_P(u16), _P(u16), _P(u16), _P(u16), c_int, c_int, _P(f64)]
         L.oracle_swiglu_ffn.restype = None
         L.oracle_expert_ffn.argtypes = [_P(u16), _P(i32), _P(u16), _P(u16), _P(u16), c_int, c_int,
-                                        c_int, _P(u16)]
+                                        c_int, _P(f64)]
         L.oracle_expert_ffn.restype = None
-        L.oracle_combine.argtypes = [_P(u16), _P(i32), _P(f64), _P(u16), i64, c_int, c_int, _P(u16)]
+        L.oracle_combine.argtypes = [_P(f64), _P(i32), _P(f64), _P(f64), i64, c_int, c_int, _P(u16)]
         L.oracle_combine.restype = None
         L.oracle_layer_given_logits.argtypes = (
             [_P(u16), _P(f32), _P(u16), _P(u16), _P(u16), _P(u16), _P(u16), _P(u16), i64] +
-            [c_int] * 5 + [_P(u16), _P(i32), _P(f64), _P(i32), _P(i32), _P(i32), _P(i32), _P(u16)])
+            [c_int] * 5 + [_P(u16), _P(i32), _P(f64), _P(i32), _P(i32), _P(i32), _P(i32), _P(f64)])
         L.oracle_layer_given_logits.restype = c_int
         L.oracle_layer.argtypes = ([_P(u16), _P(f32), _P(f32), _P(u16), _P(u16), _P(u16), _P(u16),
                                     _P(u16), _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f32)])
@@ -164,12 +164,12 @@ def permute_rows(x, row_to_token):
 
 
 def swiglu_ffn(xrow, W1e, W3e, W2e):
-    """One token row through one SwiGLU expert -> bf16 row (uint16)."""
+    """One token row through one SwiGLU expert -> float64 row (h rounded to bf16 inside)."""
     xrow = _u16(xrow); W1e = _u16(W1e); W3e = _u16(W3e); W2e = _u16(W2e)
     I, H = W1e.shape
-    y = np.zeros(H, np.uint16)
+    y = np.zeros(H, np.float64)
     lib().oracle_swiglu_ffn(_ptr(xrow, U16), _ptr(W1e, U16), _ptr(W3e, U16), _ptr(W2e, U16),
-                            H, I, _ptr(y, U16))
+                            H, I, _ptr(y, F64))
     return y
 
 
@@ -177,19 +177,21 @@ def expert_ffn(x_perm, offsets, W1, W3, W2):
     x_perm = _u16(x_perm); offsets = _i32(offsets)
     W1 = _u16(W1); W3 = _u16(W3); W2 = _u16(W2)
     E, I, H = W1.shape
-    y = np.zeros(x_perm.shape, np.uint16)
+    y = np.zeros(x_perm.shape, np.float64)
     lib().oracle_expert_ffn(_ptr(x_perm, U16), _ptr(offsets, I32), _ptr(W1, U16), _ptr(W3, U16),
-                            _ptr(W2, U16), E, H, I, _ptr(y, U16))
+                            _ptr(W2, U16), E, H, I, _ptr(y, F64))
     return y
 
 
 def combine(y_perm, token_to_row, w, s=None):
-    y_perm = _u16(y_perm); t2r = _i32(token_to_row)
-    w = np.ascontiguousarray(w, dtype=np.float64); s = _u16(s)
+    """y_perm [R,H] and s [N,H] as float64 (unrounded expert outputs)."""
+    y_perm = np.ascontiguousarray(y_perm, dtype=np.float64); t2r = _i32(token_to_row)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    s = None if s is None else np.ascontiguousarray(s, dtype=np.float64)
     N, k = t2r.shape
     H = y_perm.shape[1]
     out = np.zeros((N, H), np.uint16)
-    lib().oracle_combine(_ptr(y_perm, U16), _ptr(t2r, I32), _ptr(w, F64), _ptr(s, U16), N, H, k,
+    lib().oracle_combine(_ptr(y_perm, F64), _ptr(t2r, I32), _ptr(w, F64), _ptr(s, F64), N, H, k,
                          _ptr(out, U16))
     return out
 
@@ -207,12 +209,12 @@ def layer_given_logits(x, logits32, W1, W3, W2, k, Ws1=None, Ws3=None, Ws2=None,
     idx = np.zeros((N, k), np.int32); w = np.zeros((N, k), np.float64)
     counts = np.zeros(E, np.int32); offsets = np.zeros(E + 1, np.int32)
     r2t = np.zeros(R, np.int32); t2r = np.zeros((N, k), np.int32)
-    yp = np.zeros((R, H), np.uint16)
+    yp = np.zeros((R, H), np.float64)
     rc = lib().oracle_layer_given_logits(
         _ptr(x, U16), _ptr(l, F32), _ptr(W1, U16), _ptr(W3, U16), _ptr(W2, U16),
         _ptr(Ws1, U16), _ptr(Ws3, U16), _ptr(Ws2, U16), N, H, I, E, k, Is, _ptr(out, U16),
         _ptr(idx, I32), _ptr(w, F64), _ptr(counts, I32), _ptr(offsets, I32), _ptr(r2t, I32),
-        _ptr(t2r, I32), _ptr(yp, U16))
+        _ptr(t2r, I32), _ptr(yp, F64))
     if rc:
         raise ValueError("oracle_layer_given_logits failed")
     if not extras:

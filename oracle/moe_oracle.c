@@ -38,7 +38,10 @@
  *    a = t*k + j;
  *  - expert FFN is SwiGLU: h = silu(x W1^T) * (x W3^T), y = h W2^T,
  *    silu(z) = z / (1 + e^-z); all sums in fp64; bf16 rounding (to nearest,
- *    ties to even) at h, at y, at the shared-expert output s and at out;
+ *    ties to even) at h (the operand of the second GEMM) and at out only: the
+ *    expert outputs y and the shared-expert output s stay unrounded through
+ *    the combine, so the k-term weighted sum does not amplify a one-ulp
+ *    rounding of a term where the terms cancel;
  *  - combine: out[t] = bf16( sum_j w_j * y[row(t,j)] + s[t] ), j in pick order;
  *  - shared experts (optional, Is > 0): one SwiGLU FFN of width Is over every
  *    token, weight 1, added after the routed sum.
@@ -179,9 +182,9 @@ static double silu(double z) { return z / (1.0 + exp(-z)); }
 
 /* [FinDEP] "核心公式": an expert is three GEMMs; here the SwiGLU expert
  * y = W2 (silu(W1 x) * (W3 x)).  One row, one expert: W1, W3 [I,H], W2 [H,I].
- * fp64 sums; h and y rounded to bf16. */
+ * fp64 sums; h rounded to bf16, y left in fp64. */
 void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t *W3,
-                       const uint16_t *W2, int H, int I, uint16_t *yrow)
+                       const uint16_t *W2, int H, int I, double *yrow)
 {
     double *xd = (double *)malloc((size_t)H * sizeof(double));
     double *hd = (double *)malloc((size_t)I * sizeof(double));
@@ -197,7 +200,7 @@ void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t 
     for (int o = 0; o < H; ++o) {
         double y = 0.0;
         for (int i = 0; i < I; ++i) y += hd[i] * oracle_bf16_to_double(W2[(int64_t)o * I + i]);
-        yrow[o] = oracle_round_to_bf16(y);
+        yrow[o] = y;
     }
     free(xd);
     free(hd);
@@ -207,7 +210,7 @@ void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t 
  * Rows offsets[e] .. offsets[e+1]-1 of x_perm go through expert e. */
 void oracle_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
                        const uint16_t *W3, const uint16_t *W2, int E, int H, int I,
-                       uint16_t *y_perm)
+                       double *y_perm)
 {
     int64_t we = (int64_t)I * H;
     for (int e = 0; e < E; ++e)
@@ -221,16 +224,15 @@ void oracle_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uin
 /* [MoE-latency] "router 之后还有一串动作": inverse mapping back to token
  * order, multiply by the routing weight, add.  out[t] = bf16(sum_j w[t,j] *
  * y_perm[token_to_row[t,j]] + s[t]) in fp64, j in pick order; s may be NULL. */
-void oracle_combine(const uint16_t *y_perm, const int32_t *token_to_row, const double *w,
-                    const uint16_t *s, int64_t N, int H, int k, uint16_t *out)
+void oracle_combine(const double *y_perm, const int32_t *token_to_row, const double *w,
+                    const double *s, int64_t N, int H, int k, uint16_t *out)
 {
     for (int64_t t = 0; t < N; ++t)
         for (int o = 0; o < H; ++o) {
             double acc = 0.0;
             for (int j = 0; j < k; ++j)
-                acc += w[t * k + j] *
-                       oracle_bf16_to_double(y_perm[(int64_t)token_to_row[t * k + j] * H + o]);
-            if (s) acc += oracle_bf16_to_double(s[t * H + o]);
+                acc += w[t * k + j] * y_perm[(int64_t)token_to_row[t * k + j] * H + o];
+            if (s) acc += s[t * H + o];
             out[t * H + o] = oracle_round_to_bf16(acc);
         }
 }
@@ -240,14 +242,14 @@ void oracle_combine(const uint16_t *y_perm, const int32_t *token_to_row, const d
 /* The whole sparse path from given fp32 logits: top-k, dispatch, permuted
  * rows, per-expert SwiGLU, optional shared experts ([FinDEP] "问题定义"),
  * combine.  Optional outputs (may be NULL): idx [N,k], w [N,k], counts [E],
- * offsets [E+1], row_to_token [N*k], token_to_row [N*k], y_perm [N*k,H].
+ * offsets [E+1], row_to_token [N*k], token_to_row [N*k], y_perm [N*k,H] (fp64).
  * Returns 0, or -1 on bad arguments / allocation failure. */
 int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint16_t *W1,
                               const uint16_t *W3, const uint16_t *W2, const uint16_t *Ws1,
                               const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
                               int E, int k, int Is, uint16_t *out, int32_t *idx_out,
                               double *w_out, int32_t *counts_out, int32_t *offsets_out,
-                              int32_t *r2t_out, int32_t *t2r_out, uint16_t *y_perm_out)
+                              int32_t *r2t_out, int32_t *t2r_out, double *y_perm_out)
 {
     if (N < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E || Is < 0) return -1;
     int64_t R = N * k;
@@ -259,15 +261,15 @@ int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint
     int32_t *r2t = (int32_t *)malloc((size_t)(R ? R : 1) * sizeof(int32_t));
     int32_t *t2r = (int32_t *)malloc((size_t)(R ? R : 1) * sizeof(int32_t));
     uint16_t *xp = (uint16_t *)malloc((size_t)(R ? R : 1) * H * sizeof(uint16_t));
-    uint16_t *yp = (uint16_t *)malloc((size_t)(R ? R : 1) * H * sizeof(uint16_t));
-    uint16_t *s = NULL;
+    double *yp = (double *)malloc((size_t)(R ? R : 1) * H * sizeof(double));
+    double *s = NULL;
     if (!idx || !w || !counts || !offsets || !r2t || !t2r || !xp || !yp) goto done;
     if (oracle_topk(logits, N, E, k, idx, w)) goto done;
     if (oracle_dispatch(idx, N, E, k, counts, offsets, r2t, t2r)) goto done;
     oracle_permute_rows(x, r2t, R, H, xp);
     oracle_expert_ffn(xp, offsets, W1, W3, W2, E, H, I, yp);
     if (Is > 0) {
-        s = (uint16_t *)malloc((size_t)(N ? N : 1) * H * sizeof(uint16_t));
+        s = (double *)malloc((size_t)(N ? N : 1) * H * sizeof(double));
         if (!s) goto done;
         for (int64_t t = 0; t < N; ++t) oracle_swiglu_ffn(x + t * H, Ws1, Ws3, Ws2, H, Is, s + t * H);
     }
@@ -278,7 +280,7 @@ int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint
     if (offsets_out) memcpy(offsets_out, offsets, (size_t)(E + 1) * sizeof(int32_t));
     if (r2t_out) memcpy(r2t_out, r2t, (size_t)R * sizeof(int32_t));
     if (t2r_out) memcpy(t2r_out, t2r, (size_t)R * sizeof(int32_t));
-    if (y_perm_out) memcpy(y_perm_out, yp, (size_t)R * H * sizeof(uint16_t));
+    if (y_perm_out) memcpy(y_perm_out, yp, (size_t)R * H * sizeof(double));
     rc = 0;
 done:
     free(idx); free(w); free(counts); free(offsets); free(r2t); free(t2r); free(xp); free(yp);
