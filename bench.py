@@ -15,6 +15,7 @@ on rank 0 on a bounded sample of tokens of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -358,7 +359,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="mixtral_8x22b_decode", choices=sorted(CONFIGS))
-    ap.add_argument("--tokens", type=int, default=0, help="override N")
+    ap.add_argument("--tokens", type=int, default=0, help="override N (a smaller case for profiling)")
+    ap.add_argument("--experts", type=int, default=0, help="override E (a smaller case for profiling)")
     ap.add_argument("--cpu-tokens", type=int, default=12)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -368,6 +370,9 @@ def main():
     cfg = CONFIGS[args.config]
     if args.tokens:
         cfg = cfg.with_tokens(args.tokens)
+    if args.experts:
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}@E={args.experts}", E=args.experts,
+                                  k=min(cfg.k, args.experts))
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -80,14 +80,14 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
     L->x_perm = take((size_t)R * H * 2);
     L->h = take((size_t)R * I * 2);
     L->hs = take((size_t)N * (Is > 0 ? Is : 0) * 2);
-    L->y_perm = take((size_t)R * H * 2);
-    L->s = take((size_t)N * (Is > 0 ? H : 0) * 2);
+    L->y_perm = take((size_t)R * H * 4);
+    L->s = take((size_t)N * (Is > 0 ? H : 0) * 4);
     L->total = off;
 }
 
 moe_status_t expert_ffn_impl(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
                              const uint16_t *W3, const uint16_t *W2, int64_t R, int H, int I, int E,
-                             uint16_t *h, uint16_t *y_perm, int *err, cudaStream_t s)
+                             uint16_t *h, float *y_perm, int *err, cudaStream_t s)
 {
     if (R == 0) return MOE_OK;
     moe::GroupedGemmArgs a{};
@@ -104,7 +104,7 @@ moe_status_t expert_ffn_impl(const uint16_t *x_perm, const int32_t *offsets, con
 // Shared experts: one dense SwiGLU FFN over all N rows = the grouped kernels with a
 // single group whose rows are x itself.
 moe_status_t shared_ffn_impl(const uint16_t *x, const uint16_t *Ws1, const uint16_t *Ws3,
-                             const uint16_t *Ws2, int64_t N, int H, int Is, uint16_t *hs, uint16_t *s_out,
+                             const uint16_t *Ws2, int64_t N, int H, int Is, uint16_t *hs, float *s_out,
                              int *err, cudaStream_t s)
 {
     if (N == 0) return MOE_OK;
@@ -199,7 +199,7 @@ moe_status_t moe_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, 
 
 moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
                             const uint16_t *W3, const uint16_t *W2, int64_t R, int H, int I, int E,
-                            uint16_t *y_perm, void *ws, size_t ws_bytes, void *stream)
+                            float *y_perm, void *ws, size_t ws_bytes, void *stream)
 {
     if (R < 0 || R >= (int64_t(1) << 31) || !valid_hidden(H) || !valid_hidden(I) || E < 1 || E > 256)
         return MOE_ERR_INVALID_ARG;
@@ -215,8 +215,8 @@ moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, cons
                            static_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_combine(const uint16_t *y_perm, const int32_t *token_to_row, const float *topk_w,
-                         const uint16_t *shared_out, int64_t N, int H, int k, uint16_t *out, void *stream)
+moe_status_t moe_combine(const float *y_perm, const int32_t *token_to_row, const float *topk_w,
+                         const float *shared_out, int64_t N, int H, int k, uint16_t *out, void *stream)
 {
     if (!valid_rows(N, k) || !valid_hidden(H) || k < 1 || k > 8) return MOE_ERR_INVALID_ARG;
     if (N == 0) return MOE_OK;
@@ -261,8 +261,8 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
     uint16_t *x_perm = reinterpret_cast<uint16_t *>(base + L.x_perm);
     uint16_t *h = reinterpret_cast<uint16_t *>(base + L.h);
     uint16_t *hs = reinterpret_cast<uint16_t *>(base + L.hs);
-    uint16_t *y_perm = reinterpret_cast<uint16_t *>(base + L.y_perm);
-    uint16_t *sh = Is > 0 ? reinterpret_cast<uint16_t *>(base + L.s) : nullptr;
+    float *y_perm = reinterpret_cast<float *>(base + L.y_perm);
+    float *sh = Is > 0 ? reinterpret_cast<float *>(base + L.s) : nullptr;
     const int64_t R = N * k;
 
     MOE_TRY(record(phase_events, 0, s));

@@ -7,9 +7,11 @@
 //   acc = 0;  for j in pick order: acc = fmaf(w[t,j], y_perm[token_to_row[t,j]], acc)
 //   acc += shared_out[t]            (optional always-on shared experts, weight 1)
 //   out[t] = bf16_rn(acc)
+// The expert rows y_perm and the shared output arrive in fp32, so out is the only
+// rounding after the expert GEMMs.
 //
-// One block per token row, each thread 8 consecutive features (16-byte loads/stores);
-// HBM-bound: k rows read, one row written per token.
+// One block per token row, each thread 8 consecutive features (two 16-byte fp32
+// loads per row, one 16-byte bf16 store); HBM-bound: k rows read, one written.
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,8 +22,8 @@ constexpr int kThreads = 128;
 constexpr int kMaxK = 8;
 
 __global__ void __launch_bounds__(kThreads)
-    combine_kernel(const uint16_t *__restrict__ y_perm, const int32_t *__restrict__ token_to_row,
-                   const float *__restrict__ topk_w, const uint16_t *__restrict__ shared_out, int64_t N,
+    combine_kernel(const float *__restrict__ y_perm, const int32_t *__restrict__ token_to_row,
+                   const float *__restrict__ topk_w, const float *__restrict__ shared_out, int64_t N,
                    int H, int k, uint16_t *__restrict__ out)
 {
     const int64_t t = blockIdx.x;
@@ -40,25 +42,19 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int j = 0; j < kMaxK; ++j) {
             if (j < k && rows[j] >= 0) {
-                const uint4 yv = __ldg(reinterpret_cast<const uint4 *>(y_perm + (int64_t)rows[j] * H) + v);
-                const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+                const float4 *src = reinterpret_cast<const float4 *>(y_perm + (int64_t)rows[j] * H) + 2 * v;
+                const float4 lo = __ldg(src), hi = __ldg(src + 1);
+                const float yv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 f = unpack_bf16x2(yw[p]);
-                    acc[2 * p] = fmaf(w[j], f.x, acc[2 * p]);
-                    acc[2 * p + 1] = fmaf(w[j], f.y, acc[2 * p + 1]);
-                }
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], yv[i], acc[i]);
             }
         }
         if (shared_out) {
-            const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(shared_out + t * H) + v);
-            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+            const float4 *src = reinterpret_cast<const float4 *>(shared_out + t * H) + 2 * v;
+            const float4 lo = __ldg(src), hi = __ldg(src + 1);
+            const float sv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 f = unpack_bf16x2(sw[p]);
-                acc[2 * p] += f.x;
-                acc[2 * p + 1] += f.y;
-            }
+            for (int i = 0; i < 8; ++i) acc[i] += sv[i];
         }
         uint4 o;
         o.x = pack_bf16x2(acc[0], acc[1]);
@@ -71,8 +67,8 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *token_to_row, const float *topk_w,
-                           const uint16_t *shared_out, int64_t N, int H, int k, uint16_t *out, cudaStream_t s)
+cudaError_t launch_combine(const float *y_perm, const int32_t *token_to_row, const float *topk_w,
+                           const float *shared_out, int64_t N, int H, int k, uint16_t *out, cudaStream_t s)
 {
     if (N <= 0) return cudaSuccess;
     combine_kernel<<<(unsigned)N, kThreads, 0, s>>>(y_perm, token_to_row, topk_w, shared_out, N, H, k, out);

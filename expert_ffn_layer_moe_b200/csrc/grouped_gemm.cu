@@ -7,7 +7,8 @@
 //   * SWIGLU = true : h[r] = bf16( silu(x W1[e]^T) * (x W3[e]^T) ), the W1 and W3
 //                     products accumulate side by side in TMEM and the epilogue fuses
 //                     the SwiGLU;
-//   * SWIGLU = false: y[r] = bf16( h W2[e]^T ).
+//   * SWIGLU = false: y[r] = h W2[e]^T, stored in fp32 (the combine sums k of these
+//                     rows before the one rounding of the layer output).
 //
 // Tile shape ("swap-AB"): the MMA's M side (128) walks the weight's output
 // features, its N side (BN = 32..256) walks the group's token rows.  Decode-sized
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
-                        uint16_t *__restrict__ out, int *dev_err)
+                        void *__restrict__ out, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU>;
     extern __shared__ uint8_t smem_raw[];
@@ -382,13 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(t0 + c0, a);
                 if (SWIGLU) tmem_ld32(t0 + BN + c0, b);
                 if (f < Nout) {
-                    uint16_t *dst = out + (size_t)(row0 + c0) * Nout + f;
+                    const size_t o = (size_t)(row0 + c0) * Nout + f;
+                    if (SWIGLU) {
+                        uint16_t *dst = static_cast<uint16_t *>(out) + o;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        if (c0 + c < nrows) {
-                            const float v = SWIGLU ? silu(a[c]) * b[c] : a[c];
-                            dst[(size_t)c * Nout] = float_to_bf16_bits(v);
-                        }
+                        for (int c = 0; c < 32; ++c)
+                            if (c0 + c < nrows) dst[(size_t)c * Nout] = float_to_bf16_bits(silu(a[c]) * b[c]);
+                    } else {
+                        float *dst = static_cast<float *>(out) + o;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (c0 + c < nrows) dst[(size_t)c * Nout] = a[c];
                     }
                 }
             }

@@ -34,7 +34,7 @@ struct GroupedGemmArgs {
     int rows_single;         // rows when offsets == nullptr
     int K;
     int Nout;
-    uint16_t *out;           // [R, Nout] bf16
+    void *out;               // [R, Nout]: bf16 (SwiGLU GEMM) or fp32 (W2 GEMM)
     int *dev_err;
     int token_tile;          // 0 = choose from the shape
 };
@@ -44,8 +44,8 @@ int gemm_choose_token_tile(int64_t R, int groups);
 int device_sm_count();
 
 // Combine / unpermutation.
-cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *token_to_row,
-                           const float *topk_w, const uint16_t *shared_out, int64_t N, int H,
+cudaError_t launch_combine(const float *y_perm, const int32_t *token_to_row,
+                           const float *topk_w, const float *shared_out, int64_t N, int H,
                            int k, uint16_t *out, cudaStream_t s);
 
 }  // namespace moe

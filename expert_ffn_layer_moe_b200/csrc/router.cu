@@ -8,137 +8,182 @@
 //   w_j        = exp(l_j - l_0) / sum_i exp(l_i - l_0)          (softmax over all E
 //                renormalised over the picks equals the softmax of the picked logits)
 //
-// One warp per token.  The logits are a skinny fp32 product (E <= 256 columns),
-// too small and too precision-sensitive to be worth the tensor cores here; lanes
-// split H, each lane accumulates kEC experts at a time, and a butterfly reduction
-// gives every lane the sums.  The top-k then runs on the warp with one expert
-// slice per lane and a shuffle arg-max per pick.
+// One block per tile of TT tokens, 8 warps splitting H: warp w takes the 64-wide
+// column chunks w, w+8, ... and each lane two adjacent columns, so a warp reads
+// 128 contiguous bytes of x per token and 64 consecutive W_gate rows per step.  A
+// lane accumulates TT tokens x 8 experts at a time; lanes then reduce with a
+// butterfly and warps in a fixed order through shared memory (deterministic bits).
+// TT shrinks for small batches so the grid still covers the SMs.  The top-k runs
+// on one warp per token with an expert slice per lane and a shuffle arg-max per pick.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int kWarps = 8;     // tokens per block
-constexpr int kEC = 8;        // experts accumulated per pass
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kEC = 8;      // experts accumulated per pass
+constexpr int kChunk = 64;  // columns of H per warp step (2 per lane)
 constexpr int kMaxE = 256;
+constexpr int kMaxK = 8;
 
-__global__ void __launch_bounds__(kWarps * 32)
+template <int TT>
+__global__ void __launch_bounds__(kThreads)
     router_kernel(const uint16_t *__restrict__ x, const float *__restrict__ W_gate,
                   const float *__restrict__ bias, int64_t N, int H, int E, int k,
                   float *__restrict__ logits, int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
 {
-    __shared__ float s_logit[kWarps][kMaxE];
+    extern __shared__ float smem[];
+    float *partial = smem;                        // [kWarps][TT][E]
+    float *s_logit = smem + kWarps * TT * E;      // [TT][E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * kWarps + warp;
-    if (t >= N) return;  // whole warp leaves together; no block-wide barrier below
-    const uint16_t *xr = x + t * H;
+    const int64_t t0 = (int64_t)blockIdx.x * TT;
+    const int nt = (N - t0) < TT ? (int)(N - t0) : TT;
 
-    // ---- logits: lanes stride H by 8 elements (one 16-byte load of x per step)
     for (int e0 = 0; e0 < E; e0 += kEC) {
         const int ne = min(kEC, E - e0);
-        float acc[kEC];
+        float acc[TT][kEC];
 #pragma unroll
-        for (int j = 0; j < kEC; ++j) acc[j] = 0.f;
-        for (int h0 = lane * 8; h0 < H; h0 += 32 * 8) {
-            const uint4 xv = *reinterpret_cast<const uint4 *>(xr + h0);
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        for (int t = 0; t < TT; ++t)
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 xf = unpack_bf16x2(xw[p]);
-                const float *w0 = W_gate + (int64_t)(h0 + 2 * p) * E + e0;
-                const float *w1 = w0 + E;
+            for (int j = 0; j < kEC; ++j) acc[t][j] = 0.f;
+        for (int c = warp * kChunk; c < H; c += kWarps * kChunk) {
+            const int h = c + 2 * lane;
+            float2 xv[TT];
 #pragma unroll
-                for (int j = 0; j < kEC; ++j) {
-                    if (j < ne) {
-                        acc[j] = fmaf(xf.x, __ldg(w0 + j), acc[j]);
-                        acc[j] = fmaf(xf.y, __ldg(w1 + j), acc[j]);
-                    }
+            for (int t = 0; t < TT; ++t) {
+                const uint32_t v = t < nt ? __ldg(reinterpret_cast<const uint32_t *>(x + (t0 + t) * H + h)) : 0u;
+                xv[t] = unpack_bf16x2(v);
+            }
+            const float *w0 = W_gate + (int64_t)h * E + e0;
+            const float *w1 = w0 + E;
+#pragma unroll
+            for (int j = 0; j < kEC; ++j) {
+                if (j < ne) {
+                    const float a = __ldg(w0 + j), b = __ldg(w1 + j);
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) acc[t][j] = fmaf(xv[t].y, b, fmaf(xv[t].x, a, acc[t][j]));
                 }
             }
         }
 #pragma unroll
-        for (int j = 0; j < kEC; ++j) {
+        for (int t = 0; t < TT; ++t)
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-        }
-        if (lane < ne) {
-            float v = acc[0];
+            for (int j = 0; j < kEC; ++j)
 #pragma unroll
-            for (int j = 1; j < kEC; ++j)
-                if (lane == j) v = acc[j];
-            if (bias) v += bias[e0 + lane];
-            s_logit[warp][e0 + lane] = v;
-            if (logits) logits[t * E + e0 + lane] = v;
+                for (int o = 16; o > 0; o >>= 1) acc[t][j] += __shfl_xor_sync(0xffffffffu, acc[t][j], o);
+        if (lane == 0) {
+#pragma unroll
+            for (int t = 0; t < TT; ++t)
+#pragma unroll
+                for (int j = 0; j < kEC; ++j)
+                    if (j < ne) partial[(warp * TT + t) * E + e0 + j] = acc[t][j];
         }
     }
-    __syncwarp();
+    __syncthreads();
 
-    // ---- top-k: lane holds experts lane, lane+32, ...
-    constexpr int kPer = kMaxE / 32;
-    float v[kPer];
-    bool taken[kPer];
+    // fixed-order sum over warps, bias, write logits
+    for (int i = threadIdx.x; i < nt * E; i += kThreads) {
+        const int t = i / E, e = i % E;
+        float v = 0.f;
 #pragma unroll
-    for (int m = 0; m < kPer; ++m) {
-        const int e = lane + 32 * m;
-        v[m] = e < E ? s_logit[warp][e] : 0.f;
-        taken[m] = e >= E;
+        for (int w = 0; w < kWarps; ++w) v += partial[(w * TT + t) * E + e];
+        if (bias) v += bias[e];
+        s_logit[t * E + e] = v;
+        if (logits) logits[(t0 + t) * E + e] = v;
     }
-    float picked[8];
-    int picked_idx[8];
-    for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
+    __syncthreads();
+
+    // top-k: warp t handles token t; lane holds experts lane, lane+32, ...
+    for (int t = warp; t < nt; t += kWarps) {
+        constexpr int kPer = kMaxE / 32;
+        float v[kPer];
+        bool taken[kPer];
 #pragma unroll
         for (int m = 0; m < kPer; ++m) {
             const int e = lane + 32 * m;
-            if (!taken[m] && (v[m] > bv || (v[m] == bv && e < bi))) { bv = v[m]; bi = e; }
+            v[m] = e < E ? s_logit[t * E + e] : 0.f;
+            taken[m] = e >= E;
         }
+        float pv[kMaxK];
+        int pi[kMaxK];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        // a NaN-only remainder leaves bi unset: fall back to the lowest free index
-        if (bi == 0x7fffffff) {
-            int lo = 0x7fffffff;
+        for (int j = 0; j < kMaxK; ++j) {
+            if (j >= k) break;
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int m = 0; m < kPer; ++m) {
+                const int e = lane + 32 * m;
+                if (!taken[m] && (v[m] > bv || (v[m] == bv && e < bi))) { bv = v[m]; bi = e; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (bi == 0x7fffffff) {  // only NaN left: take the lowest free index
+                int lo = 0x7fffffff;
+#pragma unroll
+                for (int m = 0; m < kPer; ++m)
+                    if (!taken[m]) lo = min(lo, lane + 32 * m);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                bi = lo;
+                bv = s_logit[t * E + bi];
+            }
 #pragma unroll
             for (int m = 0; m < kPer; ++m)
-                if (!taken[m]) lo = min(lo, lane + 32 * m);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            bi = lo;
-            bv = s_logit[warp][bi];
+                if (lane + 32 * m == bi) taken[m] = true;
+            pv[j] = bv;
+            pi[j] = bi;
         }
+        if (lane == 0) {
+            const float l0 = pv[0];
+            float ex[kMaxK];
+            float den = 0.f;
 #pragma unroll
-        for (int m = 0; m < kPer; ++m)
-            if (lane + 32 * m == bi) taken[m] = true;
-        picked[j] = bv;
-        picked_idx[j] = bi;
-    }
-    if (lane == 0) {
-        const float l0 = picked[0];
-        float ex[8];
-        float den = 0.f;
-        for (int j = 0; j < k; ++j) { ex[j] = expf(picked[j] - l0); den += ex[j]; }
-        for (int j = 0; j < k; ++j) {
-            topk_idx[t * k + j] = picked_idx[j];
-            topk_w[t * k + j] = ex[j] / den;
+            for (int j = 0; j < kMaxK; ++j)
+                if (j < k) { ex[j] = expf(pv[j] - l0); den += ex[j]; }
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j)
+                if (j < k) {
+                    topk_idx[(t0 + t) * k + j] = pi[j];
+                    topk_w[(t0 + t) * k + j] = ex[j] / den;
+                }
         }
     }
 }
 
+template <int TT>
+cudaError_t launch_tt(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E, int k,
+                      float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
+{
+    const size_t smem = sizeof(float) * (size_t)(kWarps * TT * E + TT * E);
+    auto kern = router_kernel<TT>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t blocks = (N + TT - 1) / TT;
+    kern<<<(unsigned)blocks, kThreads, smem, s>>>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
-cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H,
-                          int E, int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
+cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
+                          int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
 {
     if (N <= 0) return cudaSuccess;
-    const int64_t blocks = (N + kWarps - 1) / kWarps;
-    router_kernel<<<(unsigned)blocks, kWarps * 32, 0, s>>>(x, W_gate, bias, N, H, E, k, logits, topk_idx,
-                                                           topk_w);
-    return cudaGetLastError();
+    // tokens per block: keep at least ~2 blocks per SM before sharing W_gate reads
+    const int64_t sms = device_sm_count();
+    if (N >= 8 * 2 * sms) return launch_tt<8>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+    if (N >= 4 * 2 * sms) return launch_tt<4>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+    if (N >= 2 * 2 * sms) return launch_tt<2>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+    return launch_tt<1>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
 }
 
 }  // namespace moe

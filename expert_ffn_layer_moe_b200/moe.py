@@ -124,10 +124,10 @@ def moe_permute(x, topk_idx, E, ws=None, stream=None, out=None):
 
 
 def moe_expert_ffn(x_perm, offsets, W1, W3, W2, ws=None, y_perm=None, stream=None):
-    """-> y_perm [R,H] bf16 (rows past offsets[E] are left as allocated)."""
+    """-> y_perm [R,H] fp32 (rows past offsets[E] are left as allocated)."""
     R, H = x_perm.shape
     E, I, _ = W1.shape
-    y_perm = _empty((R, H), torch.bfloat16, x_perm) if y_perm is None else y_perm
+    y_perm = _empty((R, H), torch.float32, x_perm) if y_perm is None else y_perm
     if ws is None:
         ws = _empty((max(16, R * I * 2),), torch.uint8, x_perm)
     _check("moe_expert_ffn", lib().moe_expert_ffn(_p(x_perm), _p(offsets), _p(W1), _p(W3), _p(W2), R, H,
@@ -136,7 +136,7 @@ def moe_expert_ffn(x_perm, offsets, W1, W3, W2, ws=None, y_perm=None, stream=Non
 
 
 def moe_combine(y_perm, token_to_row, topk_w, shared_out=None, out=None, stream=None):
-    """-> out [N,H] bf16."""
+    """y_perm [R,H] fp32, shared_out [N,H] fp32 or None -> out [N,H] bf16."""
     N, k = token_to_row.shape
     H = y_perm.shape[1]
     out = _empty((N, H), torch.bfloat16, y_perm) if out is None else out

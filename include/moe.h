@@ -121,25 +121,27 @@ MOE_API moe_status_t moe_permute(const uint16_t *x, const int32_t *topk_idx, int
  * three GEMMs per expert).  For rows r in [offsets[e], offsets[e+1]):
  *   h[r]      = bf16( silu(x_perm[r] W1[e]^T) * (x_perm[r] W3[e]^T) )   fp32 accumulation,
  *               silu(z) = z / (1 + exp(-z))
- *   y_perm[r] = bf16( h[r] W2[e]^T )                                   fp32 accumulation
+ *   y_perm[r] = h[r] W2[e]^T                                           fp32 accumulation, fp32 out
  *   x_perm  [R,H] bf16; offsets [E+1] int32 (device; monotone, offsets[E] <= R)
- *   W1, W3  [E,I,H] bf16; W2 [E,H,I] bf16; y_perm [R,H] bf16 (rows beyond offsets[E] untouched)
+ *   W1, W3  [E,I,H] bf16; W2 [E,H,I] bf16; y_perm [R,H] fp32 (rows beyond offsets[E] untouched)
+ * h is the only rounding inside the FFN (bf16, the second GEMM's operand); y stays
+ * fp32 so the combine rounds once.
  *   ws, ws_bytes: device scratch for h, >= moe_workspace_bytes(R,H,I,E,1,0)
  */
 MOE_API moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
                             const uint16_t *W3, const uint16_t *W2, int64_t R, int H, int I,
-                            int E, uint16_t *y_perm, void *ws, size_t ws_bytes, void *stream);
+                            int E, float *y_perm, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Combine / unpermutation ([MoE-latency] "router 之后还有一串动作": inverse
  * mapping to token order, multiply by routing weight, add):
  *   out[t] = bf16( fma-chain over j = 0..k-1 of topk_w[t,j] * y_perm[token_to_row[t,j]]
  *                  (+ shared_out[t]) )   fp32, picks in order; rows < 0 are skipped
- *   y_perm [R,H] bf16; token_to_row [N,k] int32; topk_w [N,k] fp32;
- *   shared_out [N,H] bf16 or NULL; out [N,H] bf16.
+ *   y_perm [R,H] fp32; token_to_row [N,k] int32; topk_w [N,k] fp32;
+ *   shared_out [N,H] fp32 or NULL; out [N,H] bf16 (the only rounding of the sum).
  */
-MOE_API moe_status_t moe_combine(const uint16_t *y_perm, const int32_t *token_to_row,
-                         const float *topk_w, const uint16_t *shared_out, int64_t N, int H, int k,
+MOE_API moe_status_t moe_combine(const float *y_perm, const int32_t *token_to_row,
+                         const float *topk_w, const float *shared_out, int64_t N, int H, int k,
                          uint16_t *out, void *stream);
 
 /*
