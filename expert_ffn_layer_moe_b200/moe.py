@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_bytes.restype = sz
         L.moe_route.argtypes = [vp, vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp]
         L.moe_permute.argtypes = [vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_permute_noalloc.argtypes = [vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp]
         L.moe_expert_ffn.argtypes = [vp, vp, vp, vp, vp, i64, c_int, c_int, c_int, vp, vp, sz, vp]
         L.moe_combine.argtypes = [vp, vp, vp, vp, i64, c_int, c_int, vp, vp]
         L.moe_layer_forward.argtypes = [vp, vp, vp, vp, vp, i64, c_int, c_int, c_int, c_int, vp]
@@ -57,7 +58,7 @@ def lib() -> ctypes.CDLL:
         L.moe_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         L.moe_device_sm_count.argtypes = []
         L.moe_device_sm_count.restype = c_int
-        for fn in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+        for fn in ("moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
                    "moe_layer_forward_ex", "moe_get_device_error"):
             getattr(L, fn).restype = c_int
         _lib = L
@@ -121,6 +122,18 @@ def moe_permute(x, topk_idx, E, ws=None, stream=None, out=None):
     _check("moe_permute", lib().moe_permute(_p(x), _p(topk_idx), N, H, E, k, _p(counts), _p(offsets),
                                             _p(r2t), _p(t2r), _p(x_perm), _p(ws), ws.numel(), _s(stream)))
     return dict(counts=counts, offsets=offsets, row_to_token=r2t, token_to_row=t2r, x_perm=x_perm)
+
+
+def moe_permute_noalloc(x, topk_idx, E, out, stream=None):
+    """moe_permute without a workspace, for callers that cannot allocate device
+    memory: the caller passes every output in `out` (keys counts, offsets,
+    row_to_token, token_to_row, x_perm); the library's fixed scratch array is used."""
+    N, H = x.shape
+    k = topk_idx.shape[1]
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(
+        _p(x), _p(topk_idx), N, H, E, k, _p(out["counts"]), _p(out["offsets"]), _p(out["row_to_token"]),
+        _p(out["token_to_row"]), _p(out["x_perm"]), _s(stream)))
+    return out
 
 
 def moe_expert_ffn(x_perm, offsets, W1, W3, W2, ws=None, y_perm=None, stream=None):

@@ -116,6 +116,36 @@ MOE_API moe_status_t moe_permute(const uint16_t *x, const int32_t *topk_idx, int
                          void *stream);
 
 /*
+ * moe_permute for callers that cannot allocate device memory.  The pages
+ * describe no such call; it exists for library users, not for the method.
+ *
+ * Some callers cannot call cudaMalloc at all or cannot hand out a workspace:
+ * a serving process whose own pool has already claimed the device memory, a
+ * plugin whose host framework owns every allocation, or code with a strict
+ * latency budget (cudaMalloc may synchronise the device and has no time
+ * bound).  This call takes the same inputs and outputs as moe_permute but no
+ * workspace: its scratch (the per-block expert histograms of the dispatch)
+ * lives in a fixed 1 MiB array inside the library, which every GPU that loads
+ * the library holds until the process exits.  Nothing is allocated by the call.
+ *
+ * Limit: ceil(N*k / 1024) * E <= MOE_PERMUTE_NOALLOC_MAX_SCRATCH_INTS, i.e.
+ * up to 1,048,576 assignments at E = 256 (more at smaller E).  Larger requests
+ * return MOE_ERR_UNSUPPORTED before any launch.
+ *
+ * The first call on each device looks up the array's device address on that
+ * device (the device must be current); make that first call before any stream
+ * capture.  All calls share the one array: two calls whose kernels overlap on
+ * the GPU (different streams, or host threads) race on it and must be ordered
+ * by the caller.  The array keeps the previous call's contents; the dispatch
+ * writes every entry it later reads, so no clearing is needed.
+ */
+#define MOE_PERMUTE_NOALLOC_MAX_SCRATCH_INTS 262144
+MOE_API moe_status_t moe_permute_noalloc(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H,
+                                 int E, int k, int32_t *counts, int32_t *offsets,
+                                 int32_t *row_to_token, int32_t *token_to_row, uint16_t *x_perm,
+                                 void *stream);
+
+/*
  * Expert FFN as two grouped GEMMs ([MoE-latency] "router 之后还有一串动作":
  * each expert runs its own matrix, merged into one launch; [FinDEP] "核心公式":
  * three GEMMs per expert).  For rows r in [offsets[e], offsets[e+1]):
