@@ -37,7 +37,14 @@ from expert_ffn_layer_moe_b200.inputs import CONFIGS, make_inputs  # noqa: E402
 METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PHASES = ("route", "permute", "gemm13", "gemm2", "shared", "combine")
-LAUNCHES = {"route": 1, "permute": 4, "gemm13": 1, "gemm2": 1, "shared": 2, "combine": 1}
+SMALL_DISPATCH_R = 8192  # assignments up to which the dispatch is one single-block launch
+
+
+def launches_per_step(cfg):
+    """Kernels of this library launched by one layer forward."""
+    permute = 2 if cfg.R <= SMALL_DISPATCH_R else 4
+    shared = 2 if cfg.Is > 0 else 0
+    return 1 + permute + 2 + shared + 1  # router, dispatch, W1/W3 and W2 GEMMs, shared, combine
 
 
 def peaks():
@@ -318,7 +325,7 @@ def run_ours(args, cfg, world, rank, local):
                          "gb_s": (g13_b + gemm2_bytes(cfg, touched)) / (g13_s + g2_s) / 1e9,
                          "gemm2_frac_hbm": gemm2_bytes(cfg, touched) / g2_s / 1e9 / hbm},
         "phase_ms": phase_ms,
-        "gpu_launches": args.steps * sum(LAUNCHES[p] for p in PHASES if p != "shared" or cfg.Is > 0),
+        "gpu_launches": args.steps * launches_per_step(cfg),
         "e2e": e2e,
     }
     clk_sum = clk.summary()

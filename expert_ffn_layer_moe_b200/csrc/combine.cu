@@ -10,8 +10,10 @@
 // The expert rows y_perm and the shared output arrive in fp32, so out is the only
 // rounding after the expert GEMMs.
 //
-// One block per token row, each thread 8 consecutive features (two 16-byte fp32
-// loads per row, one 16-byte bf16 store); HBM-bound: k rows read, one written.
+// Grid = tokens x feature slices of kThreads*8 features: each thread owns 8
+// consecutive features of one token (two 16-byte fp32 loads per picked row, one
+// 16-byte bf16 store), so every load of a small decode batch is in flight at once.
+// HBM-bound: k rows read, one row written per token.
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,7 +28,7 @@ __global__ void __launch_bounds__(kThreads)
                    const float *__restrict__ topk_w, const float *__restrict__ shared_out, int64_t N,
                    int H, int k, uint16_t *__restrict__ out)
 {
-    const int64_t t = blockIdx.x;
+    const int64_t t = blockIdx.y;
     int rows[kMaxK];
     float w[kMaxK];
 #pragma unroll
@@ -35,7 +37,7 @@ __global__ void __launch_bounds__(kThreads)
         w[j] = j < k ? topk_w[t * k + j] : 0.f;
     }
     const int nvec = H / 8;
-    for (int v = threadIdx.x; v < nvec; v += kThreads) {
+    for (int v = blockIdx.x * kThreads + threadIdx.x; v < nvec; v += gridDim.x * kThreads) {
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -71,7 +73,17 @@ cudaError_t launch_combine(const float *y_perm, const int32_t *token_to_row, con
                            const float *shared_out, int64_t N, int H, int k, uint16_t *out, cudaStream_t s)
 {
     if (N <= 0) return cudaSuccess;
-    combine_kernel<<<(unsigned)N, kThreads, 0, s>>>(y_perm, token_to_row, topk_w, shared_out, N, H, k, out);
+    if (N > 65535) {  // grid.y limit: process in slabs of 65535 tokens
+        for (int64_t t0 = 0; t0 < N; t0 += 65535) {
+            const int64_t n = N - t0 < 65535 ? N - t0 : 65535;
+            cudaError_t e = launch_combine(y_perm, token_to_row + t0 * k, topk_w + t0 * k,
+                                           shared_out ? shared_out + t0 * H : nullptr, n, H, k, out + t0 * H, s);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
+    const dim3 grid((unsigned)((H / 8 + kThreads - 1) / kThreads), (unsigned)N);
+    combine_kernel<<<grid, kThreads, 0, s>>>(y_perm, token_to_row, topk_w, shared_out, N, H, k, out);
     return cudaGetLastError();
 }
 

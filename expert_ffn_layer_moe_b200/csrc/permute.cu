@@ -5,13 +5,15 @@
 // is the permutation.  The result is deterministic and stable: assignment
 // a = t*k + j of expert e lands at row offsets[e] + #{a' < a : e(a') = e}.
 //
-// Four launches, no atomics on the row order:
+// No atomics decide the row order.  Large batches take four launches:
 //   1. count  : per block of kPermuteChunk assignments, a per-expert histogram;
 //   2. scan   : one block -- counts[e], offsets = exclusive scan, and every block's
 //               starting row per expert (in place over the histograms);
 //   3. rank   : per block again, the stable rank of each assignment inside its
 //               block (warp match + per-warp counts, warps in order) -> row maps;
 //   4. gather : x_perm[r] = x[row_to_token[r]], one warp per row, 16-byte vectors.
+// Batches of at most kSmallR assignments (decode) do 1-3 in one single-block
+// launch, then the gather: two launches instead of four.
 #include "common.cuh"
 #include "internal.h"
 
@@ -21,6 +23,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxE = 256;
+constexpr int64_t kSmallR = 8192;  // one-block dispatch up to this many assignments
 static_assert(kPermuteChunk % kThreads == 0, "chunk is whole rounds of the block");
 
 __global__ void __launch_bounds__(kThreads)
@@ -74,6 +77,84 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// One round of the stable rank: kThreads consecutive assignments starting at a0,
+// placed after base[e] rows of their expert; advances base.  Block-wide.
+__device__ __forceinline__ void rank_round(const int32_t *__restrict__ idx, int64_t R, int k, int E, int64_t a0,
+                                           int *base, int (*wcnt)[kMaxE], int32_t *__restrict__ row_to_token,
+                                           int32_t *__restrict__ token_to_row)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int i = threadIdx.x; i < kWarps * E; i += kThreads) wcnt[i / E][i % E] = 0;
+    __syncthreads();
+    const int64_t a = a0 + threadIdx.x;
+    int e = -1;
+    if (a < R) e = idx[a];
+    const bool valid = a < R && e >= 0 && e < E;
+    // lanes with equal keys form one group; invalid lanes get a key of their own
+    const int key = valid ? e : (kMaxE + lane);
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    const int rank_in_warp = __popc(peers & lt_mask);
+    if (valid && rank_in_warp == 0) wcnt[warp][e] = __popc(peers);
+    __syncthreads();
+    if (a < R) {
+        if (valid) {
+            int before = 0;
+            for (int w = 0; w < warp; ++w) before += wcnt[w][e];
+            const int row = base[e] + before + rank_in_warp;
+            row_to_token[row] = (int32_t)(a / k);
+            token_to_row[a] = row;
+        } else {
+            token_to_row[a] = -1;
+        }
+    }
+    __syncthreads();
+    for (int ee = threadIdx.x; ee < E; ee += kThreads) {
+        int add = 0;
+        for (int w = 0; w < kWarps; ++w) add += wcnt[w][ee];
+        base[ee] += add;
+    }
+    __syncthreads();
+}
+
+// Small batches: histogram, exclusive scan and stable ranks in one block.
+__global__ void __launch_bounds__(kThreads)
+    dispatch_small_kernel(const int32_t *__restrict__ idx, int64_t R, int k, int E, int32_t *__restrict__ counts,
+                          int32_t *__restrict__ offsets, int32_t *__restrict__ row_to_token,
+                          int32_t *__restrict__ token_to_row, int *err)
+{
+    __shared__ int base[kMaxE];
+    __shared__ int scan[kThreads];
+    __shared__ int wcnt[kWarps][kMaxE];
+    const int tid = threadIdx.x;
+    if (tid < E) base[tid] = 0;
+    __syncthreads();
+    for (int64_t a = tid; a < R; a += kThreads) {
+        const int e = idx[a];
+        if (e >= 0 && e < E) atomicAdd(&base[e], 1);
+        else set_device_error(err, MOE_DEVERR_BAD_EXPERT_INDEX);
+    }
+    __syncthreads();
+    const int c = tid < E ? base[tid] : 0;
+    scan[tid] = c;
+    __syncthreads();
+    for (int o = 1; o < kThreads; o <<= 1) {  // inclusive scan
+        const int v = tid >= o ? scan[tid - o] : 0;
+        __syncthreads();
+        scan[tid] += v;
+        __syncthreads();
+    }
+    if (tid < E) {
+        counts[tid] = c;
+        offsets[tid] = scan[tid] - c;
+        if (tid == E - 1) offsets[E] = scan[tid];
+        base[tid] = scan[tid] - c;
+    }
+    __syncthreads();
+    for (int64_t a0 = 0; a0 < R; a0 += kThreads)
+        rank_round(idx, R, k, E, a0, base, wcnt, row_to_token, token_to_row);
+}
+
 __global__ void __launch_bounds__(kThreads)
     rank_kernel(const int32_t *__restrict__ idx, int64_t R, int k, int E,
                 const int32_t *__restrict__ blk_base, int32_t *__restrict__ row_to_token,
@@ -81,42 +162,12 @@ __global__ void __launch_bounds__(kThreads)
 {
     __shared__ int base[kMaxE];
     __shared__ int wcnt[kWarps][kMaxE];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < E; e += kThreads) base[e] = blk_base[(int64_t)blockIdx.x * E + e];
     const int64_t a0 = (int64_t)blockIdx.x * kPermuteChunk;
-    const unsigned lt_mask = (1u << lane) - 1u;
     for (int round = 0; round < kPermuteChunk / kThreads; ++round) {
-        for (int i = threadIdx.x; i < kWarps * E; i += kThreads) (&wcnt[0][0])[(i / E) * kMaxE + i % E] = 0;
-        __syncthreads();
-        const int64_t a = a0 + (int64_t)round * kThreads + threadIdx.x;
-        int e = -1;
-        if (a < R) e = idx[a];
-        const bool valid = a < R && e >= 0 && e < E;
-        // lanes with equal keys form one group; invalid lanes get a key of their own
-        const int key = valid ? e : (kMaxE + lane);
-        const unsigned peers = __match_any_sync(0xffffffffu, key);
-        const int rank_in_warp = __popc(peers & lt_mask);
-        if (valid && rank_in_warp == 0) wcnt[warp][e] = __popc(peers);
-        __syncthreads();
-        if (a < R) {
-            if (valid) {
-                int before = 0;
-                for (int w = 0; w < warp; ++w) before += wcnt[w][e];
-                const int row = base[e] + before + rank_in_warp;
-                row_to_token[row] = (int32_t)(a / k);
-                token_to_row[a] = row;
-            } else {
-                token_to_row[a] = -1;
-            }
-        }
-        __syncthreads();
-        for (int ee = threadIdx.x; ee < E; ee += kThreads) {
-            int add = 0;
-            for (int w = 0; w < kWarps; ++w) add += wcnt[w][ee];
-            base[ee] += add;
-        }
-        __syncthreads();
-        if (a0 + (int64_t)(round + 1) * kThreads >= R) break;  // uniform across the block
+        const int64_t ar = a0 + (int64_t)round * kThreads;
+        if (ar >= R) break;  // uniform across the block
+        rank_round(idx, R, k, E, ar, base, wcnt, row_to_token, token_to_row);
     }
 }
 
@@ -145,10 +196,15 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
 {
     const int64_t R = N * k;
     if (R <= 0) return cudaSuccess;
-    const int64_t nblk = permute_blocks(R);
-    count_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, E, scratch, dev_err);
-    scan_kernel<<<1, kThreads, 0, s>>>(scratch, nblk, E, counts, offsets);
-    rank_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, k, E, scratch, row_to_token, token_to_row);
+    if (R <= kSmallR) {
+        dispatch_small_kernel<<<1, kThreads, 0, s>>>(topk_idx, R, k, E, counts, offsets, row_to_token, token_to_row,
+                                                     dev_err);
+    } else {
+        const int64_t nblk = permute_blocks(R);
+        count_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, E, scratch, dev_err);
+        scan_kernel<<<1, kThreads, 0, s>>>(scratch, nblk, E, counts, offsets);
+        rank_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, k, E, scratch, row_to_token, token_to_row);
+    }
     const int64_t want = (R + kWarps - 1) / kWarps;
     const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
     gather_rows_kernel<<<gblocks, kThreads, 0, s>>>(x, row_to_token, offsets, E, H, x_perm);

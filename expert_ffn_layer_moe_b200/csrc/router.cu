@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(kThreads)
         for (int t = 0; t < TT; ++t)
 #pragma unroll
             for (int j = 0; j < kEC; ++j) acc[t][j] = 0.f;
+        // full 8-expert slices of rows whose start is 16-byte aligned load as float4
+        const bool vec = ne == kEC && (E & 3) == 0;
+#pragma unroll 4
         for (int c = warp * kChunk; c < H; c += kWarps * kChunk) {
             const int h = c + 2 * lane;
             float2 xv[TT];
@@ -58,14 +61,25 @@ __global__ void __launch_bounds__(kThreads)
             }
             const float *w0 = W_gate + (int64_t)h * E + e0;
             const float *w1 = w0 + E;
+            float a[kEC], b[kEC];
+            if (vec) {
+                const float4 a0 = __ldg(reinterpret_cast<const float4 *>(w0));
+                const float4 a1 = __ldg(reinterpret_cast<const float4 *>(w0) + 1);
+                const float4 b0 = __ldg(reinterpret_cast<const float4 *>(w1));
+                const float4 b1 = __ldg(reinterpret_cast<const float4 *>(w1) + 1);
+                a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w; a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+                b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w; b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+            } else {
 #pragma unroll
-            for (int j = 0; j < kEC; ++j) {
-                if (j < ne) {
-                    const float a = __ldg(w0 + j), b = __ldg(w1 + j);
-#pragma unroll
-                    for (int t = 0; t < TT; ++t) acc[t][j] = fmaf(xv[t].y, b, fmaf(xv[t].x, a, acc[t][j]));
+                for (int j = 0; j < kEC; ++j) {
+                    a[j] = j < ne ? __ldg(w0 + j) : 0.f;
+                    b[j] = j < ne ? __ldg(w1 + j) : 0.f;
                 }
             }
+#pragma unroll
+            for (int j = 0; j < kEC; ++j)
+#pragma unroll
+                for (int t = 0; t < TT; ++t) acc[t][j] = fmaf(xv[t].y, b[j], fmaf(xv[t].x, a[j], acc[t][j]));
         }
 #pragma unroll
         for (int t = 0; t < TT; ++t)
