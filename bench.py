@@ -354,7 +354,8 @@ def max_over_ranks(v, world):
     if world == 1:
         return v
     import torch.distributed as dist
-    tt = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    tt = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(tt, op=dist.ReduceOp.MAX)
     return float(tt.item())
 
