@@ -60,7 +60,7 @@ bool valid_rows(int64_t N, int k) { return N >= 0 && N * (int64_t)k < (int64_t(1
 size_t round_up(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t logits, idx, w, counts, offsets, r2t, t2r, perm, x_perm, h, hs, y_perm, s, total;
+    size_t logits, idx, w, counts, offsets, r2t, t2r, perm, x_perm, h, hs, y_perm, s, router, router_bytes, total;
 };
 
 // Carve the layer's workspace; every buffer starts on a 256-byte boundary.
@@ -82,6 +82,8 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
     L->hs = take((size_t)N * (Is > 0 ? Is : 0) * 2);
     L->y_perm = take((size_t)R * H * 4);
     L->s = take((size_t)N * (Is > 0 ? H : 0) * 4);
+    L->router_bytes = moe::router_ws_bytes(N, H, E);
+    L->router = take(L->router_bytes);
     L->total = off;
 }
 
@@ -162,14 +164,17 @@ size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is)
 }
 
 moe_status_t moe_route(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
-                       int k, float *logits, int32_t *topk_idx, float *topk_w, void *stream)
+                       int k, float *logits, int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes,
+                       void *stream)
 {
     if (!valid_rows(N, k) || !valid_hidden(H) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
     if (N == 0) return MOE_OK;
     if (!x || !W_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(x)) return MOE_ERR_UNSUPPORTED;
-    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w,
-                                static_cast<cudaStream_t>(stream)));
+    if (!aligned16(x) || (ws && !aligned16(ws))) return MOE_ERR_UNSUPPORTED;
+    int *err = device_error_word();
+    if (!err) return cuda_fail(cudaGetLastError());
+    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, ws, ws ? ws_bytes : 0,
+                                err, static_cast<cudaStream_t>(stream)));
     return MOE_OK;
 }
 
@@ -266,7 +271,7 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
     const int64_t R = N * k;
 
     MOE_TRY(record(phase_events, 0, s));
-    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, s));
+    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
     MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));

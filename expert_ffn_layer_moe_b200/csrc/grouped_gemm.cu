@@ -11,9 +11,12 @@
 //                     rows before the one rounding of the layer output).
 //
 // Tile shape ("swap-AB"): the MMA's M side (128) walks the weight's output
-// features, its N side (BN = 32..256) walks the group's token rows.  Decode-sized
+// features, its N side (up to BN = 32..256) walks the group's token rows.  Decode-sized
 // groups (a few dozen rows per expert) then fill the tensor core's N side instead
-// of padding M to 128, and every weight byte is read once per token tile.
+// of padding M to 128, and every weight byte is read once per token tile.  The MMA
+// width is set per tile (the instruction descriptor is a runtime operand): a tile
+// holding r rows multiplies round_up(r, 16) of them, so a ragged group pays for at
+// most 15 padding rows instead of BN - r.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over work items):
 //   warp 0 lane 0 : TMA producer  -- weight tile(s) [128 x 64] and activation tile
@@ -63,9 +66,8 @@ struct Cfg {
     static constexpr int kSmemBytes =
         1024 + kStages * kStageBytes + kBarBytes + 16 + 4 * 2 * (kMaxGroups + 1);
     // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
-    // both operands K-major, N>>3 at bit 17, M>>4 at bit 24.
-    static constexpr uint32_t kIdesc =
-        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+    // both operands K-major, M>>4 at bit 24; N>>3 (bit 17) is added per tile.
+    static constexpr uint32_t kIdescNoN = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBM >> 4) << 24);
     static_assert(kStages >= 2, "pipeline needs at least two stages");
     static_assert(kTmemCols <= 512, "TMEM has 512 columns");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -338,6 +340,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, acc = 0;
         uint32_t phase = 0, aphase = 0;
         for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
+            int g, feat, row0, row_end;
+            decode(item, g, feat, row0, row_end);
+            // MMA width for this tile: its rows rounded up to the instruction's step of 16
+            const int n_mma = min(BN, (min(BN, row_end - row0) + 15) & ~15);
+            const uint32_t idesc = C::kIdescNoN | ((uint32_t)(n_mma >> 3) << 17);
             if (!mbar_wait(&tempty_bar[acc], aphase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
@@ -352,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                     const uint32_t accumulate = (kb | kk) != 0;
                     // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
-                    umma_bf16(d0, da + 2 * kk, db + 2 * kk, C::kIdesc, accumulate);
-                    if (SWIGLU) umma_bf16(d0 + BN, da3 + 2 * kk, db + 2 * kk, C::kIdesc, accumulate);
+                    umma_bf16(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
+                    if (SWIGLU) umma_bf16(d0 + BN, da3 + 2 * kk, db + 2 * kk, idesc, accumulate);
                 }
                 umma_commit(&empty_bar[stage]);  // stage free once these MMAs have read it
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -492,7 +499,7 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
         case 32: return launch_impl<32, SWIGLU>(a, s);
         case 64: return launch_impl<64, SWIGLU>(a, s);
         case 128: return launch_impl<128, SWIGLU>(a, s);
-        case 256: return SWIGLU ? launch_impl<128, SWIGLU>(a, s) : launch_impl<256, SWIGLU>(a, s);
+        case 256: return launch_impl<256, SWIGLU>(a, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -511,14 +518,17 @@ int device_sm_count()
     return n;
 }
 
-// Token tile from the mean rows per group: decode-sized groups take narrow tiles
-// (less wasted MMA work, weights still read once per tile), large groups wide ones.
+// Token tile from the mean rows per group.  The MMA width follows each tile's rows,
+// so a wide tile wastes no tensor work on a short group; what a wide tile costs is
+// shared memory (fewer pipeline stages) and, for the SwiGLU GEMM at 256, the second
+// TMEM accumulator buffer.  Groups then fit in one tile where possible, so each
+// weight tile streams through shared memory once.
 int gemm_choose_token_tile(int64_t R, int groups)
 {
     const int64_t mean = (R + groups - 1) / (groups > 0 ? groups : 1);
     if (mean <= 24) return 32;
     if (mean <= 48) return 64;
-    if (mean <= 160) return 128;
+    if (mean <= 112) return 128;
     return 256;
 }
 

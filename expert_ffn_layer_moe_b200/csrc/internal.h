@@ -7,10 +7,15 @@
 
 namespace moe {
 
-// Router: logits (fp32), top-k indices and renormalised weights.
+// Router: logits (fp32), top-k indices and renormalised weights.  `ws` (nullable)
+// of at least router_ws_bytes(N, H, E) bytes enables the tensor-core and
+// expert-split paths.
+enum class RouterPath { kFused, kSplitE, kTensor };
+RouterPath router_path(int64_t N, int E, bool have_logits_buffer, bool have_ws);
+size_t router_ws_bytes(int64_t N, int H, int E);
 cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *bias, int64_t N,
                           int H, int E, int k, float *logits, int32_t *topk_idx, float *topk_w,
-                          cudaStream_t s);
+                          void *ws, size_t ws_bytes, int *dev_err, cudaStream_t s);
 
 // Dispatch / permutation.  `scratch` holds permute_scratch_ints(R, E) ints.
 constexpr int kPermuteChunk = 1024;  // assignments per block in the count/rank passes

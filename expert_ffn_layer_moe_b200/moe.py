@@ -48,7 +48,7 @@ def lib() -> ctypes.CDLL:
         L.moe_last_cuda_error.restype = ctypes.c_char_p
         L.moe_workspace_bytes.argtypes = [i64, c_int, c_int, c_int, c_int, c_int]
         L.moe_workspace_bytes.restype = sz
-        L.moe_route.argtypes = [vp, vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp]
+        L.moe_route.argtypes = [vp, vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp, sz, vp]
         L.moe_permute.argtypes = [vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_permute_noalloc.argtypes = [vp, vp, i64, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp]
         L.moe_expert_ffn.argtypes = [vp, vp, vp, vp, vp, i64, c_int, c_int, c_int, vp, vp, sz, vp]
@@ -95,14 +95,21 @@ def moe_device_sm_count() -> int:
     return int(lib().moe_device_sm_count())
 
 
-def moe_route(x, W_gate, k, bias=None, logits=None, topk_idx=None, topk_w=None, stream=None):
-    """-> (topk_idx [N,k] int32, topk_w [N,k] fp32, logits [N,E] fp32 or None)."""
+def moe_route(x, W_gate, k, bias=None, logits=None, topk_idx=None, topk_w=None, ws=None, stream=None,
+              use_workspace=True):
+    """-> (topk_idx [N,k] int32, topk_w [N,k] fp32, logits [N,E] fp32 or None).
+    With use_workspace (default) a scratch buffer is passed, which lets large
+    batches take the tensor-core path; use_workspace=False runs the one-kernel
+    CUDA-core path."""
     N, H = x.shape
     E = W_gate.shape[1]
     topk_idx = _empty((N, k), torch.int32, x) if topk_idx is None else topk_idx
     topk_w = _empty((N, k), torch.float32, x) if topk_w is None else topk_w
+    if ws is None and use_workspace:
+        ws = _empty((max(16, moe_workspace_bytes(N, H, 64, E, k, 0)),), torch.uint8, x)
     _check("moe_route", lib().moe_route(_p(x), _p(W_gate), _p(bias), N, H, E, k, _p(logits),
-                                        _p(topk_idx), _p(topk_w), _s(stream)))
+                                        _p(topk_idx), _p(topk_w), _p(ws), 0 if ws is None else ws.numel(),
+                                        _s(stream)))
     return topk_idx, topk_w, logits
 
 

@@ -89,11 +89,20 @@ MOE_API size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is
  *                                  first, equal logits by lower expert index
  *   topk_w    [N,k] fp32           output: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)
  *                                  over the k picks (softmax renormalised over the picks)
+ *   ws, ws_bytes                   device scratch or NULL/0.  With at least
+ *                                  moe_workspace_bytes(N,H,64,E,k,0) bytes, large batches
+ *                                  compute the logits on the tensor cores (W_gate split
+ *                                  into three bf16 terms, exact products, fp32
+ *                                  accumulation) and small batches with many experts
+ *                                  spread the experts over more blocks; with NULL a
+ *                                  single fp32 CUDA-core kernel runs.
+ * The logits are fp32-grade on every path; which path ran can change their last bits,
+ * and the expert choice is taken on the logits this call produced.
  * NaN logits are unsupported input (the pick among them is unspecified).
  */
 MOE_API moe_status_t moe_route(const uint16_t *x, const float *W_gate, const float *bias, int64_t N,
                        int H, int E, int k, float *logits, int32_t *topk_idx, float *topk_w,
-                       void *stream);
+                       void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Dispatch and permutation ([MoE-latency] "router 之后还有一串动作"): group

@@ -49,10 +49,10 @@ def test_invalid_arguments_are_rejected_before_any_launch():
     nullp = None
     s = ctypes.c_void_p(0)
     # bad sizes: every call returns MOE_ERR_INVALID_ARG (1) without touching CUDA
-    assert L.moe_route(nullp, nullp, nullp, 4, 256, 0, 1, nullp, nullp, nullp, s) == 1
-    assert L.moe_route(nullp, nullp, nullp, 4, 256, 8, 9, nullp, nullp, nullp, s) == 1
-    assert L.moe_route(nullp, nullp, nullp, 4, 100, 8, 2, nullp, nullp, nullp, s) == 1
-    assert L.moe_route(nullp, nullp, nullp, 4, 256, 8, 2, nullp, nullp, nullp, s) == 1  # null pointers
+    assert L.moe_route(nullp, nullp, nullp, 4, 256, 0, 1, nullp, nullp, nullp, nullp, 0, s) == 1
+    assert L.moe_route(nullp, nullp, nullp, 4, 256, 8, 9, nullp, nullp, nullp, nullp, 0, s) == 1
+    assert L.moe_route(nullp, nullp, nullp, 4, 100, 8, 2, nullp, nullp, nullp, nullp, 0, s) == 1
+    assert L.moe_route(nullp, nullp, nullp, 4, 256, 8, 2, nullp, nullp, nullp, nullp, 0, s) == 1  # null ptrs
     assert L.moe_permute(nullp, nullp, 4, 256, 8, 2, nullp, nullp, nullp, nullp, nullp, nullp, 0, s) == 1
     assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, -1, 256, 512, 8, nullp, nullp, 0, s) == 1
     assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, 8, 256, 500, 8, nullp, nullp, 0, s) == 1
@@ -61,7 +61,7 @@ def test_invalid_arguments_are_rejected_before_any_launch():
     assert L.moe_layer_forward_ex(*([nullp] * 9), 4, 256, 512, 8, 2, 64, nullp, nullp, nullp, 0, s,
                                   nullp) == 1
     # N == 0 is a no-op where no output needs defining
-    assert L.moe_route(nullp, nullp, nullp, 0, 256, 8, 2, nullp, nullp, nullp, s) == 0
+    assert L.moe_route(nullp, nullp, nullp, 0, 256, 8, 2, nullp, nullp, nullp, nullp, 0, s) == 0
     assert L.moe_combine(nullp, nullp, nullp, nullp, 0, 256, 2, nullp, s) == 0
     assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, 0, 256, 512, 8, nullp, nullp, 0, s) == 0
 
@@ -71,7 +71,7 @@ def test_misaligned_pointers_are_unsupported():
     fake = ctypes.c_void_p(0x1000 + 8)   # never dereferenced: the check comes first
     ok = ctypes.c_void_p(0x2000)
     s = ctypes.c_void_p(0)
-    assert L.moe_route(fake, ok, None, 4, 256, 8, 2, None, ok, ok, s) == 2
+    assert L.moe_route(fake, ok, None, 4, 256, 8, 2, None, ok, ok, None, 0, s) == 2
     assert L.moe_combine(fake, ok, ok, None, 4, 256, 2, ok, s) == 2
 
 

@@ -40,10 +40,12 @@ def test_full_size_layer_sampled(cfg):
                                    Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], logits=logits)
     assert moe.moe_get_device_error() == 0
 
-    # routing and dispatch of every token, bit-exact
-    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k, bias=t["bias"])
+    # routing and dispatch of every token, bit-exact, on the logits the router produced
+    rlogits = torch.empty_like(logits)
+    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k, bias=t["bias"], logits=rlogits)
     p = moe.moe_permute(t["x"], idx, cfg.E)
     torch.cuda.synchronize()
+    assert torch.equal(rlogits, logits)        # the layer's router runs the same path
     l32 = _host(logits)
     ref_idx, ref_w = oracle.topk(l32, cfg.k)
     assert np.array_equal(_host(idx), ref_idx)

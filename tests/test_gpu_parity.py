@@ -82,19 +82,43 @@ def test_route_matches_oracle():
     assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
 
 
-@pytest.mark.parametrize("E,k", [(8, 2), (160, 6), (128, 8), (37, 3), (1, 1), (256, 8)])
-def test_route_shapes_and_bias(E, k):
-    cfg = MoEConfig("route", N=203, H=512, I=64, E=E, k=k)
+# (N, E, k, workspace): the one-kernel path (no workspace, or E <= 16), the
+# expert-split path (E > 16, small N) and the tensor-core path (N >= 256, N*E >= 32768)
+ROUTE_CASES = [(203, 8, 2, True), (203, 160, 6, False), (203, 160, 6, True), (203, 128, 8, True),
+               (203, 37, 3, True), (203, 1, 1, True), (203, 256, 8, True), (1, 128, 8, True),
+               (1000, 128, 8, True), (512, 160, 6, True), (4096, 8, 2, True), (300, 256, 8, True),
+               (777, 37, 3, True)]
+
+
+@pytest.mark.parametrize("N,E,k,use_ws", ROUTE_CASES)
+def test_route_shapes_and_bias(N, E, k, use_ws):
+    cfg = MoEConfig("route", N=N, H=512, I=64, E=E, k=k)
     t = cuda_inputs(cfg, seed=4)
     bias = torch.linspace(-0.5, 0.5, E, device="cuda")
     logits = torch.empty((cfg.N, E), dtype=torch.float32, device="cuda")
-    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], k, bias=bias, logits=logits)
+    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], k, bias=bias, logits=logits, use_workspace=use_ws)
     torch.cuda.synchronize()
     t["bias"] = bias
     check_logits(cfg, t, logits)
     ref_idx, ref_w = oracle.topk(host(logits), k)
     assert np.array_equal(host(idx), ref_idx)
     assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
+
+
+def test_route_paths_agree_on_logits():
+    """The tensor-core logits (three-term bf16 split of W_gate) and the CUDA-core fp32
+    logits agree to fp32 accuracy; most expert choices coincide."""
+    cfg = MoEConfig("paths", N=2048, H=1024, I=64, E=128, k=8)
+    t = cuda_inputs(cfg, seed=6)
+    la = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device="cuda")
+    lb = torch.empty_like(la)
+    ia, _, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k, logits=la, use_workspace=True)
+    ib, _, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k, logits=lb, use_workspace=False)
+    torch.cuda.synchronize()
+    scale = torch.from_numpy(np.abs(dec(host(t["x"]))) @ np.abs(host(t["W_gate"]).astype(np.float64)))
+    d = (la - lb).abs().double().cpu()
+    assert bool((d <= 2.0 ** -19 * scale + 1e-6).all())
+    assert (ia == ib).float().mean().item() > 0.99
 
 
 def test_route_ties_lower_index_first():
