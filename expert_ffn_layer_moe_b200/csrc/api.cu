@@ -80,7 +80,7 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
     L->x_perm = take((size_t)R * H * 2);
     L->h = take((size_t)R * I * 2);
     L->hs = take((size_t)N * (Is > 0 ? Is : 0) * 2);
-    L->y_perm = take((size_t)R * H * 4);
+    L->y_perm = take((size_t)moe::gemm2_ksplit(R, E, I, H) * R * H * 4);  // one buffer per K slice
     L->s = take((size_t)N * (Is > 0 ? H : 0) * 4);
     L->router_bytes = moe::router_ws_bytes(N, H, E);
     L->router = take(L->router_bytes);
@@ -228,7 +228,7 @@ moe_status_t moe_combine(const float *y_perm, const int32_t *token_to_row, const
     if (!y_perm || !token_to_row || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(y_perm) || !aligned16(out) || (shared_out && !aligned16(shared_out)))
         return MOE_ERR_UNSUPPORTED;
-    MOE_CUDA(moe::launch_combine(y_perm, token_to_row, topk_w, shared_out, N, H, k, out,
+    MOE_CUDA(moe::launch_combine(y_perm, 1, 0, token_to_row, topk_w, shared_out, N, H, k, out,
                                  static_cast<cudaStream_t>(stream)));
     return MOE_OK;
 }
@@ -282,16 +282,18 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
         MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
+    const int ksplit = moe::gemm2_ksplit(R, E, I, H);
     {
         moe::GroupedGemmArgs b{};
         b.act = h; b.w_a = W2; b.offsets = offsets; b.groups = E; b.R = R;
         b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
+        b.ksplit = ksplit; b.split_stride = R * (int64_t)H;
         MOE_CUDA(moe::launch_gemm2(b, s));
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM2, s));
     if (Is > 0) MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
-    MOE_CUDA(moe::launch_combine(y_perm, t2r, w, sh, N, H, k, out, s));
+    MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r, w, sh, N, H, k, out, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_COMBINE, s));
     return MOE_OK;
 }

@@ -25,9 +25,12 @@
 //                   and tcgen05.commit to release stages and hand accumulators over;
 //   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
 //                   per warp), SwiGLU / rounding, bf16 stores of the tile's valid rows.
-// Work items are (group, feature tile, token tile), enumerated from the device-side
-// row offsets with no host synchronisation; empty groups produce no items (no
-// padding to a fixed capacity).  Every wait is bounded (globaltimer): on expiry the
+// Work items are (group, feature tile, K slice, token tile), enumerated from the
+// device-side row offsets with no host synchronisation; empty groups produce no items
+// (no padding to a fixed capacity).  The plain (fp32-out) GEMM can split K into
+// `ksplit` slices whose partial sums land in separate buffers `split_stride` apart,
+// for shapes with too few tiles to cover the SMs; the consumer adds them in a fixed
+// order, so results stay deterministic.  Every wait is bounded (globaltimer): on expiry the
 // kernel records MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain, frees
 // TMEM and returns.
 #include <cuda.h>
@@ -63,8 +66,9 @@ struct Cfg {
     static constexpr int kAccBufs = (2 * kAccCols <= 512) ? 2 : 1;
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols);
     static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs);
-    static constexpr int kSmemBytes =
-        1024 + kStages * kStageBytes + kBarBytes + 16 + 4 * 2 * (kMaxGroups + 1);
+    static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
+    static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // per epilogue warp: 32 x 33 fp32 staging
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16 + kTableBytes + kEpiBytes;
     // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
     // both operands K-major, M>>4 at bit 24; N>>3 (bit 17) is added per tile.
     static constexpr uint32_t kIdescNoN = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBM >> 4) << 24);
@@ -227,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
-                        void *__restrict__ out, int *dev_err)
+                        void *__restrict__ out, int ksplit, int64_t split_stride, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU>;
     extern __shared__ uint8_t smem_raw[];
@@ -243,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
     int *g_tile = g_off + (kMaxGroups + 1);               // [groups+1] work-item prefix
+    float *epi_stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(g_off) + C::kTableBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_feat = (Nout + kBM - 1) / kBM;
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (gi < groups) {
                 const int lo = g_off[gi], hi = g_off[gi + 1];
                 if (lo < 0 || hi < lo || (int64_t)hi > R) bad = true;
-                else items = ((hi - lo + BN - 1) / BN) * n_feat;
+                else items = ((hi - lo + BN - 1) / BN) * n_feat * ksplit;
             }
             int v = items;
 #pragma unroll
@@ -299,8 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // item -> (group, feature tile, first row, end row of the group)
-    auto decode = [&](int item, int &g, int &feat, int &row0, int &row_end) {
+    // item -> (group, feature tile, K slice, first row, end row of the group); the
+    // token tile runs fastest so CTAs sharing a weight slice run side by side.
+    auto decode = [&](int item, int &g, int &feat, int &ks, int &row0, int &row_end) {
         int lo = 0, hi = groups - 1;
         while (lo < hi) {  // largest g with g_tile[g] <= item (skips empty groups)
             const int mid = (lo + hi + 1) >> 1;
@@ -308,10 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         g = lo;
         const int local = item - g_tile[g];
-        const int ntok = (g_tile[g + 1] - g_tile[g]) / n_feat;
-        feat = local / ntok;
+        const int ntok = (g_tile[g + 1] - g_tile[g]) / (n_feat * ksplit);
+        const int fk = local / ntok;
+        feat = fk / ksplit;
+        ks = fk % ksplit;
         row0 = g_off[g] + (local % ntok) * BN;
         row_end = g_off[g + 1];
+    };
+    auto kslice = [&](int ks, int &kb0, int &kb1) {
+        kb0 = (int)((int64_t)ks * KB / ksplit);
+        kb1 = (int)((int64_t)(ks + 1) * KB / ksplit);
     };
 
     bool failed = false;
@@ -323,9 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
-            int g, feat, row0, row_end;
-            decode(item, g, feat, row0, row_end);
-            for (int kb = 0; kb < KB; ++kb) {
+            int g, feat, ks, row0, row_end, kb0, kb1;
+            decode(item, g, feat, ks, row0, row_end);
+            kslice(ks, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
                 uint8_t *st = stages + stage * C::kStageBytes;
                 mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
@@ -340,15 +353,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, acc = 0;
         uint32_t phase = 0, aphase = 0;
         for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
-            int g, feat, row0, row_end;
-            decode(item, g, feat, row0, row_end);
+            int g, feat, ks, row0, row_end, kb0, kb1;
+            decode(item, g, feat, ks, row0, row_end);
+            kslice(ks, kb0, kb1);
             // MMA width for this tile: its rows rounded up to the instruction's step of 16
             const int n_mma = min(BN, (min(BN, row_end - row0) + 15) & ~15);
             const uint32_t idesc = C::kIdescNoN | ((uint32_t)(n_mma >> 3) << 17);
             if (!mbar_wait(&tempty_bar[acc], aphase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { failed = true; *abort_flag = 1; break; }
                 tc_fence_after();
                 const uint32_t sa = smem_u32(stages + stage * C::kStageBytes);
@@ -357,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t db = sdesc_sw128(sa + C::kNA * C::kABytes);
 #pragma unroll
                 for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                    const uint32_t accumulate = (kb | kk) != 0;
+                    const uint32_t accumulate = (kb != kb0 || kk != 0) ? 1u : 0u;
                     // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
                     umma_bf16(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
                     if (SWIGLU) umma_bf16(d0 + BN, da3 + 2 * kk, db + 2 * kk, idesc, accumulate);
@@ -371,12 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 2) {
         // ------------------------------------------------------ epilogue
+        // Each 32-row chunk: tcgen05.ld gives a lane one feature across 32 rows; the
+        // values go through a padded 32x33 shared tile (conflict-free both ways) so the
+        // global stores are 16-byte vectors of consecutive features of one row.
         const int q = warp & 3;  // TMEM lane quadrant this warp may read
+        float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + (warp - 2) * 32 * 33);
+        const bool vec_ok = (Nout & 7) == 0;  // then no 16-byte vector straddles the row end
         int acc = 0;
         uint32_t aphase = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            int g, feat, row0, row_end;
-            decode(item, g, feat, row0, row_end);
+            int g, feat, ks, row0, row_end;
+            decode(item, g, feat, ks, row0, row_end);
+            float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;  // plain GEMM only
             // warp-uniform outcome: tcgen05.ld below is a warp-collective instruction
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], aphase, abort_flag));
             if (!ok) { failed = true; *abort_flag = 1; break; }
@@ -384,12 +404,47 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = feat * kBM + q * 32 + lane;
             const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
             const int nrows = min(BN, row_end - row0);
+            const int fbase = feat * kBM + q * 32;
             for (int c0 = 0; c0 < nrows; c0 += 32) {
                 float a[32];
                 float b[32];
                 tmem_ld32(t0 + c0, a);
                 if (SWIGLU) tmem_ld32(t0 + BN + c0, b);
-                if (f < Nout) {
+                if (vec_ok) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) stage_t[lane][c] = SWIGLU ? silu(a[c]) * b[c] : a[c];
+                    __syncwarp();
+                    if (SWIGLU) {
+                        const int rr = lane >> 2, j = lane & 3;  // 8 rows x 4 feature octets per step
+                        const int fv = fbase + 8 * j;
+#pragma unroll
+                        for (int it = 0; it < 4; ++it) {
+                            const int r = it * 8 + rr;
+                            if (c0 + r < nrows && fv < Nout) {
+                                uint4 v;
+                                v.x = pack_bf16x2(stage_t[8 * j + 0][r], stage_t[8 * j + 1][r]);
+                                v.y = pack_bf16x2(stage_t[8 * j + 2][r], stage_t[8 * j + 3][r]);
+                                v.z = pack_bf16x2(stage_t[8 * j + 4][r], stage_t[8 * j + 5][r]);
+                                v.w = pack_bf16x2(stage_t[8 * j + 6][r], stage_t[8 * j + 7][r]);
+                                *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) +
+                                                           (size_t)(row0 + c0 + r) * Nout + fv) = v;
+                            }
+                        }
+                    } else {
+                        const int rr = lane >> 3, j = lane & 7;  // 4 rows x 8 feature quads per step
+                        const int fv = fbase + 4 * j;
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int r = it * 4 + rr;
+                            if (c0 + r < nrows && fv < Nout) {
+                                const float4 v = make_float4(stage_t[4 * j + 0][r], stage_t[4 * j + 1][r],
+                                                             stage_t[4 * j + 2][r], stage_t[4 * j + 3][r]);
+                                *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * Nout + fv) = v;
+                            }
+                        }
+                    }
+                    __syncwarp();
+                } else if (f < Nout) {
                     const size_t o = (size_t)(row0 + c0) * Nout + f;
                     if (SWIGLU) {
                         uint16_t *dst = static_cast<uint16_t *>(out) + o;
@@ -397,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int c = 0; c < 32; ++c)
                             if (c0 + c < nrows) dst[(size_t)c * Nout] = float_to_bf16_bits(silu(a[c]) * b[c]);
                     } else {
-                        float *dst = static_cast<float *>(out) + o;
+                        float *dst = outf + o;
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
                             if (c0 + c < nrows) dst[(size_t)c * Nout] = a[c];
@@ -485,8 +540,10 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     auto kern = grouped_gemm_kernel<BN, SWIGLU>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
+    const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
     kern<<<device_sm_count(), kThreads, C::kSmemBytes, s>>>(ma, mb, mact, a.offsets, a.groups, a.rows_single,
-                                                            a.R, a.K, a.Nout, a.out, a.dev_err);
+                                                            a.R, a.K, a.Nout, a.out, ksplit, a.split_stride,
+                                                            a.dev_err);
     return cudaGetLastError();
 }
 
@@ -494,7 +551,7 @@ template <bool SWIGLU>
 cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
-    const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups);
+    const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups, SWIGLU);
     switch (bn) {
         case 32: return launch_impl<32, SWIGLU>(a, s);
         case 64: return launch_impl<64, SWIGLU>(a, s);
@@ -523,13 +580,42 @@ int device_sm_count()
 // shared memory (fewer pipeline stages) and, for the SwiGLU GEMM at 256, the second
 // TMEM accumulator buffer.  Groups then fit in one tile where possible, so each
 // weight tile streams through shared memory once.
-int gemm_choose_token_tile(int64_t R, int groups)
+//
+// The SwiGLU GEMM keeps two accumulators per tile, so 256-row tiles fill TMEM and
+// lose the second buffer (the epilogue then cannot overlap the next tile).  That pays
+// when a group fits one 256-row tile (weights stream once, the HBM-bound middle
+// range); for groups of several hundred rows the tensor-bound regime prefers
+// double-buffered 128-row tiles.
+int gemm_choose_token_tile(int64_t R, int groups, bool swiglu)
 {
     const int64_t mean = (R + groups - 1) / (groups > 0 ? groups : 1);
     if (mean <= 24) return 32;
     if (mean <= 48) return 64;
     if (mean <= 112) return 128;
+    if (swiglu && mean > 256) return 128;
     return 256;
+}
+
+// K slices for the W2 GEMM of a decode-shaped layer: when the tiles (estimated from
+// the mean group size) cover the SMs in few waves with a ragged last one, split K so
+// the last wave is nearly full.  1 for everything with enough tiles.
+int gemm2_ksplit(int64_t R, int groups, int K, int Nout)
+{
+    const int sms = device_sm_count();
+    const int bn = gemm_choose_token_tile(R, groups, false);
+    const int64_t active = R < groups ? R : groups;
+    const int64_t mean = (R + active - 1) / (active > 0 ? active : 1);
+    const int64_t tiles = active * ((mean + bn - 1) / bn) * ((Nout + kBM - 1) / kBM);
+    if (tiles <= 0 || tiles >= 4 * (int64_t)sms) return 1;
+    int best = 1;
+    double best_eff = 0.0;
+    for (int ks = 1; ks <= 4; ++ks) {
+        if (K / kBK < 16 * ks) break;  // keep every slice at least 16 K-blocks long
+        const int64_t n = tiles * ks;
+        const double eff = (double)n / (double)(((n + sms - 1) / sms) * sms);
+        if (eff > best_eff + 0.02) { best_eff = eff; best = ks; }
+    }
+    return best;
 }
 
 cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s) { return launch_dispatch<true>(a, s); }

@@ -42,15 +42,19 @@ struct GroupedGemmArgs {
     void *out;               // [R, Nout]: bf16 (SwiGLU GEMM) or fp32 (W2 GEMM)
     int *dev_err;
     int token_tile;          // 0 = choose from the shape
+    int ksplit;              // plain GEMM: K slices (0/1 = none); partial sums at out + s*split_stride
+    int64_t split_stride;    // elements between the partial-sum buffers
 };
 cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s);
-int gemm_choose_token_tile(int64_t R, int groups);
+int gemm_choose_token_tile(int64_t R, int groups, bool swiglu);
+int gemm2_ksplit(int64_t R, int groups, int K, int Nout);
 int device_sm_count();
 
 // Combine / unpermutation.
-cudaError_t launch_combine(const float *y_perm, const int32_t *token_to_row,
-                           const float *topk_w, const float *shared_out, int64_t N, int H,
-                           int k, uint16_t *out, cudaStream_t s);
+// y_perm holds `nsplit` partial-sum buffers `split_stride` elements apart (1 = one).
+cudaError_t launch_combine(const float *y_perm, int nsplit, int64_t split_stride,
+                           const int32_t *token_to_row, const float *topk_w, const float *shared_out,
+                           int64_t N, int H, int k, uint16_t *out, cudaStream_t s);
 
 }  // namespace moe

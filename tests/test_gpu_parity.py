@@ -215,6 +215,8 @@ def test_layer_tiny_matches_oracle():
     MoEConfig("dense", N=77, H=128, I=256, E=1, k=1),
     # shared experts on top of routed ones
     MoEConfig("shared", N=90, H=256, I=128, E=6, k=2, Is=192),
+    # few tiles and a long K: the W2 GEMM splits K and the combine adds the slices
+    MoEConfig("splitk", N=64, H=256, I=2048, E=4, k=2),
 ])
 def test_layer_shapes_match_oracle(cfg):
     t = cuda_inputs(cfg, seed=1)
