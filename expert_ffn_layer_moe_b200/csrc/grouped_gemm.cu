@@ -4,11 +4,14 @@
 // group (MoE-latency article, section "router 之后还有一串动作": every expert runs
 // its own matrix, and a grouped GEMM merges them into one launch; FinDEP review,
 // section "核心公式": an expert is three GEMMs).  Two instantiations:
-//   * SWIGLU = true : h[r] = bf16( silu(x W1[e]^T) * (x W3[e]^T) ), the W1 and W3
-//                     products accumulate side by side in TMEM and the epilogue fuses
-//                     the SwiGLU;
-//   * SWIGLU = false: y[r] = h W2[e]^T, stored in fp32 (the combine sums k of these
-//                     rows before the one rounding of the layer output).
+//   * SWIGLU = true : h[r] = bf16( silu(x W1[e]^T) * (x W3[e]^T) ).  The MMA's 128
+//                     weight rows are 64 rows of W1 and the same 64 rows of W3, so one
+//                     accumulator holds g (TMEM lanes 0-63) and u (lanes 64-127) for 64
+//                     output features, the activation tile is read once per K step, and
+//                     the epilogue pairs the lanes through shared memory;
+//   * SWIGLU = false: y[r] = h W2[e]^T over 128 output features, stored in fp32 (the
+//                     combine sums k of these rows before the one rounding of the layer
+//                     output).
 //
 // Tile shape ("swap-AB"): the MMA's M side (128) walks the weight's output
 // features, its N side (up to BN = 32..256) walks the group's token rows.  Decode-sized
@@ -19,24 +22,24 @@
 // most 15 padding rows instead of BN - r.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over work items):
-//   warp 0 lane 0 : TMA producer  -- weight tile(s) [128 x 64] and activation tile
-//                   [BN x 64] per stage, 128-byte swizzle, mbarrier transaction counts;
+//   warp 0 lane 0 : TMA producer  -- the 128-row weight tile and the [BN x 64]
+//                   activation tile per stage, 128-byte swizzle, mbarrier transaction counts;
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (bf16 in, fp32 accumulate)
 //                   and tcgen05.commit to release stages and hand accumulators over;
 //   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
-//                   per warp), SwiGLU / rounding, bf16 stores of the tile's valid rows.
+//                   per warp), staged through shared memory into 16-byte row stores.
+// TMEM holds two accumulators of BN columns (BN <= 256), so the epilogue of one tile
+// overlaps the main loop of the next.
 // Work items are (group, feature tile, K slice, token tile), enumerated from the
 // device-side row offsets with no host synchronisation; empty groups produce no items
 // (no padding to a fixed capacity).  The plain (fp32-out) GEMM can split K into
 // `ksplit` slices whose partial sums land in separate buffers `split_stride` apart,
 // for shapes with too few tiles to cover the SMs; the consumer adds them in a fixed
-// order, so results stay deterministic.  Every wait is bounded (globaltimer): on expiry the
-// kernel records MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain, frees
-// TMEM and returns.
+// order, so results stay deterministic.  Every wait is bounded (globaltimer): on
+// expiry the kernel records MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain,
+// frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
-
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -44,7 +47,7 @@
 namespace moe {
 namespace {
 
-constexpr int kBM = 128;     // weight rows (output features) per tile = MMA M
+constexpr int kBM = 128;     // MMA M: weight rows per tile
 constexpr int kBK = 64;      // K per pipeline stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;   // K of one tcgen05.mma kind::f16
 constexpr int kThreads = 192;
@@ -56,18 +59,18 @@ constexpr int pow2_at_least(int v, int p = 32) { return p >= v ? p : pow2_at_lea
 template <int BN, bool SWIGLU>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "token tile must be 32..256, step 32");
-    static constexpr int kNA = SWIGLU ? 2 : 1;          // weight tiles per stage
-    static constexpr int kABytes = kBM * kBK * 2;       // 16 KB
+    static constexpr int kFeat = SWIGLU ? kBM / 2 : kBM;  // output features per tile
+    static constexpr int kABytes = kBM * kBK * 2;          // 16 KB weight tile per stage
     static constexpr int kBBytes = BN * kBK * 2;
-    static constexpr int kStageBytes = kNA * kABytes + kBBytes;
+    static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-    static constexpr int kAccCols = kNA * BN;           // fp32 TMEM columns per accumulator set
-    static constexpr int kAccBufs = (2 * kAccCols <= 512) ? 2 : 1;
+    static constexpr int kAccCols = BN;                   // fp32 TMEM columns per accumulator
+    static constexpr int kAccBufs = 2;
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols);
     static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs);
     static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
-    static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // per epilogue warp: 32 x 33 fp32 staging
+    static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // staging: 4 x [32][33] fp32 (= 2 x [64][33])
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16 + kTableBytes + kEpiBytes;
     // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
     // both operands K-major, M>>4 at bit 24; N>>3 (bit 17) is added per tile.
@@ -225,6 +228,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
+// Named barrier for the four epilogue warps (barrier 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 // ------------------------------------------------------------------ kernel --
 template <int BN, bool SWIGLU>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -245,15 +251,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *tempty_bar = tfull_bar + C::kAccBufs;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty_bar + C::kAccBufs);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
     int *g_tile = g_off + (kMaxGroups + 1);               // [groups+1] work-item prefix
     float *epi_stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(g_off) + C::kTableBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_feat = (Nout + kBM - 1) / kBM;
+    const int n_feat = (Nout + C::kFeat - 1) / C::kFeat;
     const int KB = (K + kBK - 1) / kBK;
 
-    // ---- work list: row offsets and the prefix of (token tiles x feature tiles) per group
+    // ---- work list: row offsets and the prefix of (token tiles x feature tiles x K slices) per group
     if (offsets == nullptr) {
         if (tid == 0) { g_off[0] = 0; g_off[1] = rows_single; }
     } else {
@@ -342,9 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
                 uint8_t *st = stages + stage * C::kStageBytes;
                 mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
-                tma_load_3d(st, &tm_wa, kb * kBK, feat * kBM, g, &full_bar[stage]);
-                if (SWIGLU) tma_load_3d(st + C::kABytes, &tm_wb, kb * kBK, feat * kBM, g, &full_bar[stage]);
-                tma_load_2d(st + C::kNA * C::kABytes, &tm_act, kb * kBK, row0, &full_bar[stage]);
+                if (SWIGLU) {
+                    // rows 0-63: W1 features [64 feat, +64); rows 64-127: the same features of W3
+                    tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
+                    tma_load_3d(st + C::kABytes / 2, &tm_wb, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
+                } else {
+                    tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
+                }
+                tma_load_2d(st + C::kABytes, &tm_act, kb * kBK, row0, &full_bar[stage]);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
         }
@@ -367,14 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t sa = smem_u32(stages + stage * C::kStageBytes);
                 const uint64_t da = sdesc_sw128(sa);
-                const uint64_t da3 = sdesc_sw128(sa + C::kABytes);
-                const uint64_t db = sdesc_sw128(sa + C::kNA * C::kABytes);
+                const uint64_t db = sdesc_sw128(sa + C::kABytes);
 #pragma unroll
                 for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                     const uint32_t accumulate = (kb != kb0 || kk != 0) ? 1u : 0u;
                     // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
                     umma_bf16(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
-                    if (SWIGLU) umma_bf16(d0 + BN, da3 + 2 * kk, db + 2 * kk, idesc, accumulate);
                 }
                 umma_commit(&empty_bar[stage]);  // stage free once these MMAs have read it
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -385,52 +395,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 2) {
         // ------------------------------------------------------ epilogue
-        // Each 32-row chunk: tcgen05.ld gives a lane one feature across 32 rows; the
-        // values go through a padded 32x33 shared tile (conflict-free both ways) so the
-        // global stores are 16-byte vectors of consecutive features of one row.
-        const int q = warp & 3;  // TMEM lane quadrant this warp may read
-        float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + (warp - 2) * 32 * 33);
+        // Per 32-row chunk every warp loads its TMEM lane quadrant (one feature, or one
+        // half of a SwiGLU pair, across 32 rows) into a padded shared tile; after the
+        // epilogue barrier the tile is read back so each lane stores 16 bytes of
+        // consecutive features of one row.
+        const int q = warp & 3;   // TMEM lane quadrant this warp may read
+        const int ew = warp - 2;  // 0..3
         const bool vec_ok = (Nout & 7) == 0;  // then no 16-byte vector straddles the row end
         int acc = 0;
         uint32_t aphase = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
             int g, feat, ks, row0, row_end;
             decode(item, g, feat, ks, row0, row_end);
-            float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;  // plain GEMM only
-            // warp-uniform outcome: tcgen05.ld below is a warp-collective instruction
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], aphase, abort_flag));
+            // one waiter decides for all four warps, so the named barriers below are
+            // always reached by all of them
+            if (ew == 0 && lane == 0) *epi_ok = mbar_wait(&tfull_bar[acc], aphase, abort_flag) ? 1 : 0;
+            epilogue_sync();
+            const bool ok = *epi_ok != 0;
+            epilogue_sync();  // everyone has read the flag before it can be rewritten
             if (!ok) { failed = true; *abort_flag = 1; break; }
             tc_fence_after();
-            const int f = feat * kBM + q * 32 + lane;
             const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
             const int nrows = min(BN, row_end - row0);
-            const int fbase = feat * kBM + q * 32;
-            for (int c0 = 0; c0 < nrows; c0 += 32) {
-                float a[32];
-                float b[32];
-                tmem_ld32(t0 + c0, a);
-                if (SWIGLU) tmem_ld32(t0 + BN + c0, b);
-                if (vec_ok) {
+            if (SWIGLU) {
+                float(*Gs)[33] = reinterpret_cast<float(*)[33]>(epi_stage);            // [64][33] g
+                float(*Us)[33] = reinterpret_cast<float(*)[33]>(epi_stage + 64 * 33);  // [64][33] u
+                float(*mine)[33] = q < 2 ? Gs : Us;
+                const int fl = (q & 1) * 32 + lane;  // feature within the 64-feature tile
+                const int rr = lane >> 3, j = lane & 7;
+                const int fv = feat * C::kFeat + 8 * j;
+                uint16_t *outh = static_cast<uint16_t *>(out);
+                for (int c0 = 0; c0 < nrows; c0 += 32) {
+                    float a[32];
+                    tmem_ld32(t0 + c0, a);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) stage_t[lane][c] = SWIGLU ? silu(a[c]) * b[c] : a[c];
-                    __syncwarp();
-                    if (SWIGLU) {
-                        const int rr = lane >> 2, j = lane & 3;  // 8 rows x 4 feature octets per step
-                        const int fv = fbase + 8 * j;
+                    for (int c = 0; c < 32; ++c) mine[fl][c] = a[c];
+                    epilogue_sync();
+                    // warp ew stores rows 8*ew .. 8*ew+7 of the chunk: 4 rows x 8 feature octets per step
 #pragma unroll
-                        for (int it = 0; it < 4; ++it) {
-                            const int r = it * 8 + rr;
-                            if (c0 + r < nrows && fv < Nout) {
-                                uint4 v;
-                                v.x = pack_bf16x2(stage_t[8 * j + 0][r], stage_t[8 * j + 1][r]);
-                                v.y = pack_bf16x2(stage_t[8 * j + 2][r], stage_t[8 * j + 3][r]);
-                                v.z = pack_bf16x2(stage_t[8 * j + 4][r], stage_t[8 * j + 5][r]);
-                                v.w = pack_bf16x2(stage_t[8 * j + 6][r], stage_t[8 * j + 7][r]);
-                                *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) +
-                                                           (size_t)(row0 + c0 + r) * Nout + fv) = v;
-                            }
+                    for (int it = 0; it < 2; ++it) {
+                        const int r = 8 * ew + 4 * it + rr;
+                        if (c0 + r < nrows && fv < Nout) {
+                            float h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) h[i] = silu(Gs[8 * j + i][r]) * Us[8 * j + i][r];
+                            uint4 v;
+                            v.x = pack_bf16x2(h[0], h[1]);
+                            v.y = pack_bf16x2(h[2], h[3]);
+                            v.z = pack_bf16x2(h[4], h[5]);
+                            v.w = pack_bf16x2(h[6], h[7]);
+                            *reinterpret_cast<uint4 *>(outh + (size_t)(row0 + c0 + r) * Nout + fv) = v;
                         }
-                    } else {
+                    }
+                    epilogue_sync();
+                }
+            } else {
+                float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + ew * 32 * 33);
+                float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
+                const int fbase = feat * C::kFeat + q * 32;
+                for (int c0 = 0; c0 < nrows; c0 += 32) {
+                    float a[32];
+                    tmem_ld32(t0 + c0, a);
+                    if (vec_ok) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) stage_t[lane][c] = a[c];
+                        __syncwarp();
                         const int rr = lane >> 3, j = lane & 7;  // 4 rows x 8 feature quads per step
                         const int fv = fbase + 4 * j;
 #pragma unroll
@@ -442,17 +471,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * Nout + fv) = v;
                             }
                         }
-                    }
-                    __syncwarp();
-                } else if (f < Nout) {
-                    const size_t o = (size_t)(row0 + c0) * Nout + f;
-                    if (SWIGLU) {
-                        uint16_t *dst = static_cast<uint16_t *>(out) + o;
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (c0 + c < nrows) dst[(size_t)c * Nout] = float_to_bf16_bits(silu(a[c]) * b[c]);
-                    } else {
-                        float *dst = outf + o;
+                        __syncwarp();
+                    } else if (fbase + lane < Nout) {
+                        float *dst = outf + (size_t)(row0 + c0) * Nout + fbase + lane;
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
                             if (c0 + c < nrows) dst[(size_t)c * Nout] = a[c];
@@ -496,15 +517,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// Weights [groups, Nout, K] bf16 as a 3-D map; box = 64 (K) x 128 (rows) x 1 (group).
+// Weights [groups, Nout, K] bf16 as a 3-D map; box = 64 (K) x box_rows x 1 (group).
 // Rows past Nout read as zero and never bleed into the next group.
-bool encode_weight_map(CUtensorMap *m, const void *ptr, int groups, int Nout, int K)
+bool encode_weight_map(CUtensorMap *m, const void *ptr, int groups, int Nout, int K, int box_rows)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)Nout, (cuuint64_t)groups};
     cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)Nout * (cuuint64_t)K * 2};
-    cuuint32_t box[3] = {(cuuint32_t)kBK, (cuuint32_t)kBM, 1};
+    cuuint32_t box[3] = {(cuuint32_t)kBK, (cuuint32_t)box_rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -530,9 +551,10 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
     using C = Cfg<BN, SWIGLU>;
     CUtensorMap ma, mb, mact;
-    if (!encode_weight_map(&ma, a.w_a, a.groups, a.Nout, a.K)) return cudaErrorInvalidValue;
+    const int box_rows = SWIGLU ? kBM / 2 : kBM;
+    if (!encode_weight_map(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     if (SWIGLU) {
-        if (!encode_weight_map(&mb, a.w_b, a.groups, a.Nout, a.K)) return cudaErrorInvalidValue;
+        if (!encode_weight_map(&mb, a.w_b, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     } else {
         mb = ma;
     }
@@ -551,6 +573,7 @@ template <bool SWIGLU>
 cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
+    if (SWIGLU && (a.Nout % (kBM / 2)) != 0) return cudaErrorInvalidValue;  // whole 64-feature tiles
     const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups, SWIGLU);
     switch (bn) {
         case 32: return launch_impl<32, SWIGLU>(a, s);
@@ -577,22 +600,15 @@ int device_sm_count()
 
 // Token tile from the mean rows per group.  The MMA width follows each tile's rows,
 // so a wide tile wastes no tensor work on a short group; what a wide tile costs is
-// shared memory (fewer pipeline stages) and, for the SwiGLU GEMM at 256, the second
-// TMEM accumulator buffer.  Groups then fit in one tile where possible, so each
-// weight tile streams through shared memory once.
-//
-// The SwiGLU GEMM keeps two accumulators per tile, so 256-row tiles fill TMEM and
-// lose the second buffer (the epilogue then cannot overlap the next tile).  That pays
-// when a group fits one 256-row tile (weights stream once, the HBM-bound middle
-// range); for groups of several hundred rows the tensor-bound regime prefers
-// double-buffered 128-row tiles.
+// shared memory (fewer pipeline stages).  Groups then fit in one tile where possible,
+// so each weight tile streams through shared memory once.
 int gemm_choose_token_tile(int64_t R, int groups, bool swiglu)
 {
+    (void)swiglu;
     const int64_t mean = (R + groups - 1) / (groups > 0 ? groups : 1);
     if (mean <= 24) return 32;
     if (mean <= 48) return 64;
     if (mean <= 112) return 128;
-    if (swiglu && mean > 256) return 128;
     return 256;
 }
 
