@@ -28,9 +28,9 @@
 //                   (row_map != nullptr) the activation rows are token rows of x picked
 //                   through row_map, so the permuted copy of x is never written to HBM:
 //                   the warp's lanes copy them with 16-byte cp.async (8 lanes per row,
-//                   the 128-byte swizzle applied by hand) and each lane's
-//                   cp.async.mbarrier.arrive completes the stage barrier when its rows
-//                   have landed (the MMA thread fences them over to the async proxy);
+//                   the 128-byte swizzle applied by hand), commit one group per stage
+//                   and, kStages-1 stages later, wait for it, fence the writes over to
+//                   the async proxy and arrive on the stage's barrier;
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (bf16 in, fp32 accumulate)
 //                   and tcgen05.commit to release stages and hand accumulators over;
 //   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
@@ -239,13 +239,12 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint3
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-// Arrive on `bar` once every cp.async this thread issued so far has completed (the
-// barrier's expected count includes this arrival: .noinc).
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
 {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
@@ -280,7 +279,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *s_tok = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(epi_stage) + C::kEpiBytes);  // [BN]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool gather_mode = row_map != nullptr;
     const int n_feat = (Nout + C::kFeat - 1) / C::kFeat;
     const int KB = (K + kBK - 1) / kBK;
 
@@ -322,9 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- barriers and TMEM
     if (tid == 0) {
         for (int s = 0; s < C::kStages; ++s) mbar_init(&empty_bar[s], 1);
-        // a gathered stage gets 33 arrivals: the TMA's expect_tx and one per producer
-        // lane when that lane's cp.async rows have landed
-        const uint32_t full_count = row_map != nullptr ? 33u : 1u;
+        // a gathered stage gets two arrivals: the TMA's expect_tx and the producer's
+        // declaration that its cp.async rows have landed
+        const uint32_t full_count = row_map != nullptr ? 2u : 1u;
         for (int s = 0; s < C::kStages; ++s) mbar_init(&full_bar[s], full_count);
         for (int b = 0; b < C::kAccBufs; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -364,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool failed = false;
     if (warp == 0) {
         // ------------------------------------------------------ producer
+        constexpr int kLag = C::kStages - 1;  // gather groups in flight before a stage is declared full
         const bool gather = row_map != nullptr;
         if (lane == 0) {
             tma_prefetch_map(&tm_wa);
@@ -371,8 +370,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!gather) tma_prefetch_map(&tm_act);
         }
         const uint16_t *xg = static_cast<const uint16_t *>(act_ptr);
-        int stage = 0;
+        int stage = 0, pend_stage = 0;  // pend_stage: oldest stage whose gather is not yet declared
         uint32_t phase = 0;
+        int issued = 0, declared = 0;
+        // declare the oldest gathered stage complete: its cp.async group has landed
+        auto declare_oldest = [&]() {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_bar[pend_stage]);
+            if (++pend_stage == C::kStages) pend_stage = 0;
+            ++declared;
+        };
         for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
@@ -410,12 +418,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t dst = bt + r * (kBK * 2) + ((c ^ (r & 7)) << 4);
                         cp_async_16(dst, src, r < nload ? 16u : 0u);  // rows past the group: zeros
                     }
-                    cp_async_arrive(&full_bar[stage]);  // fires when this lane's copies have landed
+                    cp_async_commit();
+                    if (++issued > kLag) {
+                        cp_async_wait_group<kLag>();
+                        declare_oldest();
+                    }
                 }
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
         }
-        if (gather) cp_async_wait_all();  // nothing of ours may land after the CTA exits
+        if (gather) {
+            cp_async_wait_group<0>();
+            while (declared < issued) declare_oldest();
+        }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------ MMA issuer
         int stage = 0, acc = 0;
@@ -432,8 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
             for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { failed = true; *abort_flag = 1; break; }
-                // rows gathered by cp.async were written through the generic proxy
-                if (gather_mode) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 tc_fence_after();
                 const uint32_t sa = smem_u32(stages + stage * C::kStageBytes);
                 const uint64_t da = sdesc_sw128(sa);
