@@ -22,15 +22,14 @@
 // most 15 padding rows instead of BN - r.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over work items):
-//   warp 0        : producer -- lane 0 loads the 128-row weight tile with TMA and, for
-//                   contiguous activations, the [BN x 64] activation tile (128-byte
-//                   swizzle, mbarrier transaction counts).  In gather mode
+//   warp 0        : TMA producer  -- lane 0 loads the 128-row weight tile and, for
+//                   contiguous activations, the [BN x 64] activation tile per stage
+//                   (128-byte swizzle, mbarrier transaction counts).  In gather mode
 //                   (row_map != nullptr) the activation rows are token rows of x picked
-//                   through row_map, so the permuted copy of x is never written to HBM:
-//                   the warp's lanes copy them with 16-byte cp.async (8 lanes per row,
-//                   the 128-byte swizzle applied by hand), commit one group per stage
-//                   and, kStages-1 stages later, wait for it, fence the writes over to
-//                   the async proxy and arrive on the stage's barrier;
+//                   through row_map: the 32 lanes each issue one-row TMA loads for their
+//                   rows, straight into the swizzled tile, so the permuted copy of x is
+//                   never written to HBM (the swizzle is a function of the shared-memory
+//                   address, so a row landing at tile + 128*r gets row r's pattern);
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (bf16 in, fp32 accumulate)
 //                   and tcgen05.commit to release stages and hand accumulators over;
 //   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
@@ -78,8 +77,7 @@ struct Cfg {
     static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs);
     static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
     static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // staging: 4 x [32][33] fp32 (= 2 x [64][33])
-    static constexpr int kSmemBytes =
-        1024 + kStages * kStageBytes + kBarBytes + 16 + kTableBytes + kEpiBytes + 4 * BN;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16 + kTableBytes + kEpiBytes;
     // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
     // both operands K-major, M>>4 at bit 24; N>>3 (bit 17) is added per tile.
     static constexpr uint32_t kIdescNoN = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBM >> 4) << 24);
@@ -234,18 +232,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// 16-byte global -> shared copy through L2 (cp.async.cg); src_bytes 0 writes zeros.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
 // Named barrier for the four epilogue warps (barrier 0 is __syncthreads).
@@ -258,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
                         void *__restrict__ out, int ksplit, int64_t split_stride,
-                        const int32_t *__restrict__ row_map, const void *__restrict__ act_ptr, int *dev_err)
+                        const int32_t *__restrict__ row_map, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU>;
     extern __shared__ uint8_t smem_raw[];
@@ -276,7 +262,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
     int *g_tile = g_off + (kMaxGroups + 1);               // [groups+1] work-item prefix
     float *epi_stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(g_off) + C::kTableBytes);
-    int *s_tok = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(epi_stage) + C::kEpiBytes);  // [BN]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_feat = (Nout + C::kFeat - 1) / C::kFeat;
@@ -319,11 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- barriers and TMEM
     if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) mbar_init(&empty_bar[s], 1);
-        // a gathered stage gets two arrivals: the TMA's expect_tx and the producer's
-        // declaration that its cp.async rows have landed
-        const uint32_t full_count = row_map != nullptr ? 2u : 1u;
-        for (int s = 0; s < C::kStages; ++s) mbar_init(&full_bar[s], full_count);
+        for (int s = 0; s < C::kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
         for (int b = 0; b < C::kAccBufs; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -361,36 +342,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     bool failed = false;
     if (warp == 0) {
-        // ------------------------------------------------------ producer
-        constexpr int kLag = C::kStages - 1;  // gather groups in flight before a stage is declared full
+        // ------------------------------------------------------ TMA producer
+        constexpr int kRowsPerLane = BN / 32;
         const bool gather = row_map != nullptr;
         if (lane == 0) {
             tma_prefetch_map(&tm_wa);
             if (SWIGLU) tma_prefetch_map(&tm_wb);
-            if (!gather) tma_prefetch_map(&tm_act);
+            tma_prefetch_map(&tm_act);
         }
-        const uint16_t *xg = static_cast<const uint16_t *>(act_ptr);
-        int stage = 0, pend_stage = 0;  // pend_stage: oldest stage whose gather is not yet declared
+        int stage = 0;
         uint32_t phase = 0;
-        int issued = 0, declared = 0;
-        // declare the oldest gathered stage complete: its cp.async group has landed
-        auto declare_oldest = [&]() {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_bar[pend_stage]);
-            if (++pend_stage == C::kStages) pend_stage = 0;
-            ++declared;
-        };
         for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
             kslice(ks, kb0, kb1);
             const int nload = min(BN, row_end - row0);  // rows of this tile that exist
-            if (gather) {
-                __syncwarp();  // every lane is done reading the previous item's table
-                for (int r = lane; r < BN; r += 32) s_tok[r] = r < nload ? row_map[row0 + r] : 0;
-                __syncwarp();
+            int tok[kRowsPerLane];                      // gather mode: x row of tile row lane + 32 i
+#pragma unroll
+            for (int i = 0; i < kRowsPerLane; ++i) {
+                const int r = lane + 32 * i;
+                tok[i] = (gather && r < nload) ? row_map[row0 + r] : -1;
             }
+            const uint32_t stage_tx = C::kABytes + (gather ? (uint32_t)nload * (kBK * 2) : (uint32_t)C::kBBytes);
             for (int kb = kb0; kb < kb1; ++kb) {
                 int ok = 1;
                 if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag) ? 1 : 0;
@@ -398,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) { failed = true; if (lane == 0) *abort_flag = 1; break; }
                 uint8_t *st = stages + stage * C::kStageBytes;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full_bar[stage], gather ? C::kABytes : C::kStageBytes);
+                    mbar_arrive_expect_tx(&full_bar[stage], stage_tx);
                     if (SWIGLU) {
                         // rows 0-63: W1 features [64 feat, +64); rows 64-127: the same features of W3
                         tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
@@ -409,27 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!gather) tma_load_2d(st + C::kABytes, &tm_act, kb * kBK, row0, &full_bar[stage]);
                 }
                 if (gather) {
-                    // row r, 16-byte chunk c = lane & 7 lands at chunk c ^ (r & 7) of the row's 128 bytes
-                    const int c = lane & 7;
-                    const uint32_t bt = smem_u32(st + C::kABytes);
-#pragma unroll 4
-                    for (int r = lane >> 3; r < BN; r += 4) {
-                        const uint16_t *src = xg + (int64_t)s_tok[r] * K + kb * kBK + c * 8;
-                        const uint32_t dst = bt + r * (kBK * 2) + ((c ^ (r & 7)) << 4);
-                        cp_async_16(dst, src, r < nload ? 16u : 0u);  // rows past the group: zeros
-                    }
-                    cp_async_commit();
-                    if (++issued > kLag) {
-                        cp_async_wait_group<kLag>();
-                        declare_oldest();
-                    }
+#pragma unroll
+                    for (int i = 0; i < kRowsPerLane; ++i)
+                        if (tok[i] >= 0)
+                            tma_load_2d(st + C::kABytes + (lane + 32 * i) * (kBK * 2), &tm_act, kb * kBK, tok[i],
+                                        &full_bar[stage]);
                 }
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
-        }
-        if (gather) {
-            cp_async_wait_group<0>();
-            while (declared < issued) declare_oldest();
         }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------ MMA issuer
@@ -604,6 +564,7 @@ bool encode_weight_map(CUtensorMap *m, const void *ptr, int groups, int Nout, in
 }
 
 // Activations [R, K] bf16 as a 2-D map; box = 64 (K) x BN (rows); rows >= R read as zero.
+// Gather mode uses BN = 1: one row per load.
 bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int BN)
 {
     auto enc = tensor_map_encoder();
@@ -629,15 +590,15 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     } else {
         mb = ma;
     }
-    const int64_t act_rows = a.row_map ? a.act_rows : a.R;  // gather mode: the map is unused
-    if (!encode_act_map(&mact, a.act, act_rows, a.K, BN)) return cudaErrorInvalidValue;
+    const int64_t act_rows = a.row_map ? a.act_rows : a.R;
+    if (!encode_act_map(&mact, a.act, act_rows, a.K, a.row_map ? 1 : BN)) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_kernel<BN, SWIGLU>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
     const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
     kern<<<device_sm_count(), kThreads, C::kSmemBytes, s>>>(ma, mb, mact, a.offsets, a.groups, a.rows_single,
                                                             a.R, a.K, a.Nout, a.out, ksplit, a.split_stride,
-                                                            a.row_map, a.act, a.dev_err);
+                                                            a.row_map, a.dev_err);
     return cudaGetLastError();
 }
 
