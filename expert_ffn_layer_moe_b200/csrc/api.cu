@@ -60,7 +60,7 @@ bool valid_rows(int64_t N, int k) { return N >= 0 && N * (int64_t)k < (int64_t(1
 size_t round_up(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t logits, idx, w, counts, offsets, r2t, t2r, perm, h, hs, y_perm, s, router, router_bytes, total;
+    size_t logits, idx, w, counts, offsets, r2t, t2r, perm, x_perm, h, hs, y_perm, s, router, router_bytes, total;
 };
 
 // Carve the layer's workspace; every buffer starts on a 256-byte boundary.
@@ -77,6 +77,7 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
     L->r2t = take((size_t)R * 4);
     L->t2r = take((size_t)R * 4);
     L->perm = take((size_t)moe::permute_scratch_ints(R, E) * 4);
+    L->x_perm = take((size_t)R * H * 2);
     L->h = take((size_t)R * I * 2);
     L->hs = take((size_t)N * (Is > 0 ? Is : 0) * 2);
     L->y_perm = take((size_t)moe::gemm2_ksplit(R, E, I, H) * R * H * 4);  // one buffer per K slice
@@ -262,6 +263,7 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
     int32_t *r2t = reinterpret_cast<int32_t *>(base + L.r2t);
     int32_t *t2r = reinterpret_cast<int32_t *>(base + L.t2r);
     int32_t *perm = reinterpret_cast<int32_t *>(base + L.perm);
+    uint16_t *x_perm = reinterpret_cast<uint16_t *>(base + L.x_perm);
     uint16_t *h = reinterpret_cast<uint16_t *>(base + L.h);
     uint16_t *hs = reinterpret_cast<uint16_t *>(base + L.hs);
     float *y_perm = reinterpret_cast<float *>(base + L.y_perm);
@@ -271,13 +273,12 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
     MOE_TRY(record(phase_events, 0, s));
     MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
-    // row maps only: the W1/W3 GEMM gathers its token rows from x through row_to_token
-    MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
+    MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
     {
         moe::GroupedGemmArgs a{};
-        a.act = x; a.row_map = r2t; a.act_rows = N; a.w_a = W1; a.w_b = W3; a.offsets = offsets; a.groups = E;
-        a.R = R; a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
+        a.act = x_perm; a.w_a = W1; a.w_b = W3; a.offsets = offsets; a.groups = E; a.R = R;
+        a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
         MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));

@@ -22,14 +22,8 @@
 // most 15 padding rows instead of BN - r.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over work items):
-//   warp 0        : TMA producer  -- lane 0 loads the 128-row weight tile and, for
-//                   contiguous activations, the [BN x 64] activation tile per stage
-//                   (128-byte swizzle, mbarrier transaction counts).  In gather mode
-//                   (row_map != nullptr) the activation rows are token rows of x picked
-//                   through row_map: the 32 lanes each issue one-row TMA loads for their
-//                   rows, straight into the swizzled tile, so the permuted copy of x is
-//                   never written to HBM (the swizzle is a function of the shared-memory
-//                   address, so a row landing at tile + 128*r gets row r's pattern);
+//   warp 0 lane 0 : TMA producer  -- the 128-row weight tile and the [BN x 64]
+//                   activation tile per stage, 128-byte swizzle, mbarrier transaction counts;
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (bf16 in, fp32 accumulate)
 //                   and tcgen05.commit to release stages and hand accumulators over;
 //   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
@@ -243,8 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
-                        void *__restrict__ out, int ksplit, int64_t split_stride,
-                        const int32_t *__restrict__ row_map, int *dev_err)
+                        void *__restrict__ out, int ksplit, int64_t split_stride, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU>;
     extern __shared__ uint8_t smem_raw[];
@@ -341,53 +334,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     bool failed = false;
-    if (warp == 0) {
+    if (warp == 0 && lane == 0) {
         // ------------------------------------------------------ TMA producer
-        constexpr int kRowsPerLane = BN / 32;
-        const bool gather = row_map != nullptr;
-        if (lane == 0) {
-            tma_prefetch_map(&tm_wa);
-            if (SWIGLU) tma_prefetch_map(&tm_wb);
-            tma_prefetch_map(&tm_act);
-        }
+        tma_prefetch_map(&tm_wa);
+        if (SWIGLU) tma_prefetch_map(&tm_wb);
+        tma_prefetch_map(&tm_act);
         int stage = 0;
         uint32_t phase = 0;
         for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
             kslice(ks, kb0, kb1);
-            const int nload = min(BN, row_end - row0);  // rows of this tile that exist
-            int tok[kRowsPerLane];                      // gather mode: x row of tile row lane + 32 i
-#pragma unroll
-            for (int i = 0; i < kRowsPerLane; ++i) {
-                const int r = lane + 32 * i;
-                tok[i] = (gather && r < nload) ? row_map[row0 + r] : -1;
-            }
-            const uint32_t stage_tx = C::kABytes + (gather ? (uint32_t)nload * (kBK * 2) : (uint32_t)C::kBBytes);
             for (int kb = kb0; kb < kb1; ++kb) {
-                int ok = 1;
-                if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) { failed = true; if (lane == 0) *abort_flag = 1; break; }
+                if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
                 uint8_t *st = stages + stage * C::kStageBytes;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full_bar[stage], stage_tx);
-                    if (SWIGLU) {
-                        // rows 0-63: W1 features [64 feat, +64); rows 64-127: the same features of W3
-                        tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
-                        tma_load_3d(st + C::kABytes / 2, &tm_wb, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
-                    } else {
-                        tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
-                    }
-                    if (!gather) tma_load_2d(st + C::kABytes, &tm_act, kb * kBK, row0, &full_bar[stage]);
+                mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
+                if (SWIGLU) {
+                    // rows 0-63: W1 features [64 feat, +64); rows 64-127: the same features of W3
+                    tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
+                    tma_load_3d(st + C::kABytes / 2, &tm_wb, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
+                } else {
+                    tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
                 }
-                if (gather) {
-#pragma unroll
-                    for (int i = 0; i < kRowsPerLane; ++i)
-                        if (tok[i] >= 0)
-                            tma_load_2d(st + C::kABytes + (lane + 32 * i) * (kBK * 2), &tm_act, kb * kBK, tok[i],
-                                        &full_bar[stage]);
-                }
+                tma_load_2d(st + C::kABytes, &tm_act, kb * kBK, row0, &full_bar[stage]);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
         }
@@ -564,7 +533,6 @@ bool encode_weight_map(CUtensorMap *m, const void *ptr, int groups, int Nout, in
 }
 
 // Activations [R, K] bf16 as a 2-D map; box = 64 (K) x BN (rows); rows >= R read as zero.
-// Gather mode uses BN = 1: one row per load.
 bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int BN)
 {
     auto enc = tensor_map_encoder();
@@ -590,15 +558,14 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     } else {
         mb = ma;
     }
-    const int64_t act_rows = a.row_map ? a.act_rows : a.R;
-    if (!encode_act_map(&mact, a.act, act_rows, a.K, a.row_map ? 1 : BN)) return cudaErrorInvalidValue;
+    if (!encode_act_map(&mact, a.act, a.R, a.K, BN)) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_kernel<BN, SWIGLU>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
     const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
     kern<<<device_sm_count(), kThreads, C::kSmemBytes, s>>>(ma, mb, mact, a.offsets, a.groups, a.rows_single,
                                                             a.R, a.K, a.Nout, a.out, ksplit, a.split_stride,
-                                                            a.row_map, a.dev_err);
+                                                            a.dev_err);
     return cudaGetLastError();
 }
 

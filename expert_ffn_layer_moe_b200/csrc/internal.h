@@ -21,7 +21,6 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
 constexpr int kPermuteChunk = 1024;  // assignments per block in the count/rank passes
 inline int64_t permute_blocks(int64_t R) { return (R + kPermuteChunk - 1) / kPermuteChunk; }
 inline int64_t permute_scratch_ints(int64_t R, int E) { return permute_blocks(R) * E; }
-// x_perm == nullptr: row maps only (the grouped GEMM gathers rows from x itself).
 cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E,
                            int k, int32_t *counts, int32_t *offsets, int32_t *row_to_token,
                            int32_t *token_to_row, uint16_t *x_perm, int32_t *scratch,
@@ -45,8 +44,6 @@ struct GroupedGemmArgs {
     int token_tile;          // 0 = choose from the shape
     int ksplit;              // plain GEMM: K slices (0/1 = none); partial sums at out + s*split_stride
     int64_t split_stride;    // elements between the partial-sum buffers
-    const int32_t *row_map;  // gather mode: tile row r reads act row row_map[r] (nullptr = contiguous)
-    int64_t act_rows;        // gather mode: rows of `act`
 };
 cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s);

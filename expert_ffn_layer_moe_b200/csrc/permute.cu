@@ -205,11 +205,9 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
         scan_kernel<<<1, kThreads, 0, s>>>(scratch, nblk, E, counts, offsets);
         rank_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, k, E, scratch, row_to_token, token_to_row);
     }
-    if (x_perm) {
-        const int64_t want = (R + kWarps - 1) / kWarps;
-        const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
-        gather_rows_kernel<<<gblocks, kThreads, 0, s>>>(x, row_to_token, offsets, E, H, x_perm);
-    }
+    const int64_t want = (R + kWarps - 1) / kWarps;
+    const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
+    gather_rows_kernel<<<gblocks, kThreads, 0, s>>>(x, row_to_token, offsets, E, H, x_perm);
     return cudaGetLastError();
 }
 
