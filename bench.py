@@ -41,10 +41,18 @@ SMALL_DISPATCH_R = 8192  # assignments up to which the dispatch is one single-bl
 
 
 def launches_per_step(cfg):
-    """Kernels of this library launched by one layer forward."""
-    permute = 2 if cfg.R <= SMALL_DISPATCH_R else 4
+    """Kernels of this library launched by one layer forward (the layer's router
+    takes its tensor-core path for N >= 256 with N*E >= 32768: split, GEMM, top-k;
+    its expert-split path for E > 16: logits, top-k; else one kernel)."""
+    if cfg.N >= 256 and cfg.N * cfg.E >= 32768:
+        router = 3
+    elif cfg.E > 16:
+        router = 2
+    else:
+        router = 1
+    permute = 2 if cfg.R <= SMALL_DISPATCH_R else 4  # dispatch (1 or 3 kernels) + row gather
     shared = 2 if cfg.Is > 0 else 0
-    return 1 + permute + 2 + shared + 1  # router, dispatch, W1/W3 and W2 GEMMs, shared, combine
+    return router + permute + 2 + shared + 1  # + W1/W3 and W2 GEMMs, shared, combine
 
 
 def peaks():
