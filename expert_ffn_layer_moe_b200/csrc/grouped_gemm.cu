@@ -56,25 +56,29 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, far above any
 
 constexpr int pow2_at_least(int v, int p = 32) { return p >= v ? p : pow2_at_least(v, p * 2); }
 
-template <int BN, bool SWIGLU>
+template <int BN, bool SWIGLU, bool PAIR>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "token tile must be 32..256, step 32");
-    static constexpr int kFeat = SWIGLU ? kBM / 2 : kBM;  // output features per tile
+    static constexpr int kCtas = PAIR ? 2 : 1;             // CTAs sharing one MMA (cta_group)
+    static constexpr int kFeat = SWIGLU ? kBM / 2 : kBM;   // output features per CTA per tile
+    static constexpr int kFeatTile = kCtas * kFeat;        // output features per work item
+    static constexpr int kBRows = BN / kCtas;              // token rows of B held by each CTA
     static constexpr int kABytes = kBM * kBK * 2;          // 16 KB weight tile per stage
-    static constexpr int kBBytes = BN * kBK * 2;
+    static constexpr int kBBytes = kBRows * kBK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-    static constexpr int kAccCols = BN;                   // fp32 TMEM columns per accumulator
-    static constexpr int kAccBufs = 2;
+    static constexpr int kAccCols = BN;                    // fp32 TMEM columns per accumulator
+    static constexpr int kAccBufs = (PAIR && BN > 128) ? 1 : 2;
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols);
     static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs);
     static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
     static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // staging: 4 x [32][33] fp32 (= 2 x [64][33])
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16 + kTableBytes + kEpiBytes;
     // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
-    // both operands K-major, M>>4 at bit 24; N>>3 (bit 17) is added per tile.
-    static constexpr uint32_t kIdescNoN = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBM >> 4) << 24);
+    // both operands K-major, M>>4 at bit 24 (M = 128 per CTA); N>>3 (bit 17) per tile.
+    static constexpr uint32_t kIdescNoN =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)((kBM * kCtas) >> 4) << 24);
     static_assert(kStages >= 2, "pipeline needs at least two stages");
     static_assert(kTmemCols <= 512, "TMEM has 512 columns");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -134,44 +138,8 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *m)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, int c0, int c1, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, int c0, int c1, int c2,
-                                            uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-        : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
-                 "r"(ncols)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish()
-{
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA with
 // 128-byte swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart (SBO),
@@ -226,20 +194,151 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ---------------------------------------------- CTA-pair (cta_group::2) forms --
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA loads into this CTA's shared memory that complete on `bar` (a shared::cluster
+// address; with PAIR it may be the leader CTA's barrier).  Never multicast.
+template <bool PAIR>
+__device__ __forceinline__ void tma_3d(void *dst, const CUtensorMap *m, int c0, int c1, int c2, uint32_t bar)
+{
+    if (PAIR)
+        asm volatile(
+            "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+            : "memory");
+    else
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+            : "memory");
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *m, int c0, int c1, uint32_t bar)
+{
+    if (PAIR)
+        asm volatile(
+            "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(bar)
+            : "memory");
+    else
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(bar)
+            : "memory");
+}
+
+// TMEM allocation: with PAIR one warp of each CTA of the pair takes part.
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc_g(uint32_t *slot, uint32_t ncols)
+{
+    if (PAIR)
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                     "r"(ncols)
+                     : "memory");
+    else
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                     "r"(ncols)
+                     : "memory");
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void tmem_relinquish_g()
+{
+    if (PAIR) asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    else asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void tmem_dealloc_g(uint32_t taddr, uint32_t ncols)
+{
+    if (PAIR)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+    else
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// One MMA: with PAIR, M = 256 across the pair (each CTA's 128 weight rows), N split
+// between the CTAs' halves of the token tile; issued by the leader CTA only.
+template <bool PAIR>
+__device__ __forceinline__ void umma_g(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate)
+{
+    if (PAIR)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        umma_bf16(d_tmem, adesc, bdesc, idesc, accumulate);
+}
+
+// Arrive on `bar` when the MMAs issued so far complete; with PAIR the arrival goes
+// to the barrier at the same offset in both CTAs of the pair.
+template <bool PAIR>
+__device__ __forceinline__ void umma_commit_g(uint64_t *bar)
+{
+    if (PAIR) {
+        const uint16_t both = 0x3;
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                smem_u32(bar)),
+            "h"(both)
+            : "memory");
+    } else {
+        umma_commit(bar);
+    }
+}
+
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
 // Named barrier for the four epilogue warps (barrier 0 is __syncthreads).
 __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // ------------------------------------------------------------------ kernel --
-template <int BN, bool SWIGLU>
+// PAIR = true runs as clusters of two CTAs on two SMs: CTA r of a pair holds weight
+// rows [128 r, 128 r + 128) of the work item's 256 and token rows
+// [n/2 r, n/2 r + n/2) of its n; the leader (r = 0) issues the M=256 MMAs, both CTAs'
+// TMA loads complete on the leader's stage barrier, its commits reach both CTAs'
+// barriers, and each CTA drains its own half of the accumulator.
+template <int BN, bool SWIGLU, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
                         void *__restrict__ out, int ksplit, int64_t split_stride, int *dev_err)
 {
-    using C = Cfg<BN, SWIGLU>;
+    using C = Cfg<BN, SWIGLU, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);  // 1024-aligned for SW128
@@ -257,7 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *epi_stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(g_off) + C::kTableBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_feat = (Nout + C::kFeat - 1) / C::kFeat;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // work-list walker: one per pair
+    const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const int n_feat = (Nout + C::kFeatTile - 1) / C::kFeatTile;
     const int KB = (K + kBK - 1) / kBK;
 
     // ---- work list: row offsets and the prefix of (token tiles x feature tiles x K slices) per group
@@ -289,30 +391,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             carry += __shfl_sync(0xffffffffu, v, 31);
         }
         if (lane == 0) g_tile[0] = 0;
-        if (__any_sync(0xffffffffu, bad) && lane == 0) set_device_error(dev_err, MOE_DEVERR_BAD_OFFSETS);
+        if (__any_sync(0xffffffffu, bad) && lane == 0 && rank == 0)
+            set_device_error(dev_err, MOE_DEVERR_BAD_OFFSETS);
     }
     __syncthreads();
     const int total = g_tile[groups];
-    if ((int)blockIdx.x >= total) return;  // uniform: nothing allocated yet
+    if (unit >= total) return;  // uniform over the pair: nothing allocated, no cluster barrier yet
 
     // ---- barriers and TMEM
     if (tid == 0) {
         for (int s = 0; s < C::kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-        for (int b = 0; b < C::kAccBufs; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
+        for (int b = 0; b < C::kAccBufs; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 4 * C::kCtas);  // every epilogue warp of the pair releases
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_g<PAIR>(tmem_slot, C::kTmemCols);
+        tmem_relinquish_g<PAIR>();
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // both CTAs' barriers exist before either signals the other
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     // item -> (group, feature tile, K slice, first row, end row of the group); the
-    // token tile runs fastest so CTAs sharing a weight slice run side by side.
+    // token tile runs fastest so units sharing a weight slice run side by side.
     auto decode = [&](int item, int &g, int &feat, int &ks, int &row0, int &row_end) {
         int lo = 0, hi = groups - 1;
         while (lo < hi) {  // largest g with g_tile[g] <= item (skips empty groups)
@@ -332,6 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         kb0 = (int)((int64_t)ks * KB / ksplit);
         kb1 = (int)((int64_t)(ks + 1) * KB / ksplit);
     };
+    // MMA width of a tile: its rows rounded up to the instruction's step of 16
+    auto mma_width = [&](int row0, int row_end) { return min(BN, (min(BN, row_end - row0) + 15) & ~15); };
 
     bool failed = false;
     if (warp == 0 && lane == 0) {
@@ -339,38 +448,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tm_wa);
         if (SWIGLU) tma_prefetch_map(&tm_wb);
         tma_prefetch_map(&tm_act);
+        // every load of the pair completes on the leader's stage barrier
+        const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&full_bar[0]), 0) : smem_u32(&full_bar[0]);
         int stage = 0;
         uint32_t phase = 0;
-        for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
+        for (int item = unit; item < total && !failed; item += nunits) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
             kslice(ks, kb0, kb1);
+            const int frow = feat * C::kFeatTile + (int)rank * C::kFeat;        // first weight row (W1 / W)
+            const int trow = row0 + (PAIR ? (int)rank * (mma_width(row0, row_end) >> 1) : 0);
             for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
                 uint8_t *st = stages + stage * C::kStageBytes;
-                mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
+                const uint32_t fb = full0 + 8u * stage;
+                if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kCtas * C::kStageBytes);
                 if (SWIGLU) {
-                    // rows 0-63: W1 features [64 feat, +64); rows 64-127: the same features of W3
-                    tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
-                    tma_load_3d(st + C::kABytes / 2, &tm_wb, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
+                    // rows 0-63: W1 features [frow, +64); rows 64-127: the same features of W3
+                    tma_3d<PAIR>(st, &tm_wa, kb * kBK, frow, g, fb);
+                    tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kb * kBK, frow, g, fb);
                 } else {
-                    tma_load_3d(st, &tm_wa, kb * kBK, feat * C::kFeat, g, &full_bar[stage]);
+                    tma_3d<PAIR>(st, &tm_wa, kb * kBK, frow, g, fb);
                 }
-                tma_load_2d(st + C::kABytes, &tm_act, kb * kBK, row0, &full_bar[stage]);
+                tma_2d<PAIR>(st + C::kABytes, &tm_act, kb * kBK, trow, fb);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
         }
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------------ MMA issuer
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ------------------------------------------------------ MMA issuer (leader CTA)
         int stage = 0, acc = 0;
         uint32_t phase = 0, aphase = 0;
-        for (int item = blockIdx.x; item < total && !failed; item += gridDim.x) {
+        for (int item = unit; item < total && !failed; item += nunits) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
             kslice(ks, kb0, kb1);
-            // MMA width for this tile: its rows rounded up to the instruction's step of 16
-            const int n_mma = min(BN, (min(BN, row_end - row0) + 15) & ~15);
-            const uint32_t idesc = C::kIdescNoN | ((uint32_t)(n_mma >> 3) << 17);
+            const uint32_t idesc = C::kIdescNoN | ((uint32_t)(mma_width(row0, row_end) >> 3) << 17);
             if (!mbar_wait(&tempty_bar[acc], aphase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
@@ -384,13 +496,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                     const uint32_t accumulate = (kb != kb0 || kk != 0) ? 1u : 0u;
                     // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
-                    umma_bf16(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
+                    umma_g<PAIR>(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
                 }
-                umma_commit(&empty_bar[stage]);  // stage free once these MMAs have read it
+                umma_commit_g<PAIR>(&empty_bar[stage]);  // stage free (in both CTAs) once read
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
             if (failed) break;
-            umma_commit(&tfull_bar[acc]);        // accumulator complete
+            umma_commit_g<PAIR>(&tfull_bar[acc]);        // accumulator complete (in both CTAs)
             if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
         }
     } else if (warp >= 2) {
@@ -402,9 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;   // TMEM lane quadrant this warp may read
         const int ew = warp - 2;  // 0..3
         const bool vec_ok = (Nout & 7) == 0;  // then no 16-byte vector straddles the row end
+        const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(&tempty_bar[0]), 0) : 0u;
         int acc = 0;
         uint32_t aphase = 0;
-        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        for (int item = unit; item < total; item += nunits) {
             int g, feat, ks, row0, row_end;
             decode(item, g, feat, ks, row0, row_end);
             // one waiter decides for all four warps, so the named barriers below are
@@ -421,9 +534,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float(*Gs)[33] = reinterpret_cast<float(*)[33]>(epi_stage);            // [64][33] g
                 float(*Us)[33] = reinterpret_cast<float(*)[33]>(epi_stage + 64 * 33);  // [64][33] u
                 float(*mine)[33] = q < 2 ? Gs : Us;
-                const int fl = (q & 1) * 32 + lane;  // feature within the 64-feature tile
+                const int fl = (q & 1) * 32 + lane;  // feature within this CTA's 64
                 const int rr = lane >> 3, j = lane & 7;
-                const int fv = feat * C::kFeat + 8 * j;
+                const int fv = feat * C::kFeatTile + (int)rank * C::kFeat + 8 * j;
                 uint16_t *outh = static_cast<uint16_t *>(out);
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
@@ -452,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + ew * 32 * 33);
                 float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
-                const int fbase = feat * C::kFeat + q * 32;
+                const int fbase = feat * C::kFeatTile + (int)rank * C::kFeat + q * 32;
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
@@ -482,7 +595,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * acc);  // the leader's barrier
+                else mbar_arrive(&tempty_bar[acc]);
+            }
             if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
         }
     }
@@ -490,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (failed) set_device_error(dev_err, MOE_DEVERR_PIPELINE_TIMEOUT);
     __syncwarp();
     __syncthreads();
+    if (PAIR) cluster_sync();  // no arrival from the peer can still be on its way
     if (*abort_flag) {
         // let copies and MMAs already in flight land before the CTA's memory is released
         const uint64_t t0 = global_timer_ns();
@@ -498,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        tmem_dealloc_g<PAIR>(tmem_base, C::kTmemCols);
     }
 }
 
@@ -532,24 +649,24 @@ bool encode_weight_map(CUtensorMap *m, const void *ptr, int groups, int Nout, in
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Activations [R, K] bf16 as a 2-D map; box = 64 (K) x BN (rows); rows >= R read as zero.
-bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int BN)
+// Activations [R, K] bf16 as a 2-D map; box = 64 (K) x box_rows; rows >= R read as zero.
+bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_rows)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)R};
     cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU>
+template <int BN, bool SWIGLU, bool PAIR>
 cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
-    using C = Cfg<BN, SWIGLU>;
+    using C = Cfg<BN, SWIGLU, PAIR>;
     CUtensorMap ma, mb, mact;
     const int box_rows = SWIGLU ? kBM / 2 : kBM;
     if (!encode_weight_map(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
@@ -558,14 +675,29 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     } else {
         mb = ma;
     }
-    if (!encode_act_map(&mact, a.act, a.R, a.K, BN)) return cudaErrorInvalidValue;
-    auto kern = grouped_gemm_kernel<BN, SWIGLU>;
+    if (!encode_act_map(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
+    auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
     const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
-    kern<<<device_sm_count(), kThreads, C::kSmemBytes, s>>>(ma, mb, mact, a.offsets, a.groups, a.rows_single,
-                                                            a.R, a.K, a.Nout, a.out, ksplit, a.split_stride,
-                                                            a.dev_err);
+    const int sms = device_sm_count();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)(PAIR ? (sms / 2) * 2 : sms));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
+                             ksplit, a.split_stride, a.dev_err);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
@@ -575,11 +707,14 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
     if (SWIGLU && (a.Nout % (kBM / 2)) != 0) return cudaErrorInvalidValue;  // whole 64-feature tiles
     const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups, SWIGLU);
+    // token tiles of 128 rows and more run as CTA pairs (M = 256 weight rows per MMA):
+    // each SM streams half the activation rows and the pair reads each activation tile
+    // once per 256 weight rows instead of once per 128
     switch (bn) {
-        case 32: return launch_impl<32, SWIGLU>(a, s);
-        case 64: return launch_impl<64, SWIGLU>(a, s);
-        case 128: return launch_impl<128, SWIGLU>(a, s);
-        case 256: return launch_impl<256, SWIGLU>(a, s);
+        case 32: return launch_impl<32, SWIGLU, false>(a, s);
+        case 64: return launch_impl<64, SWIGLU, false>(a, s);
+        case 128: return launch_impl<128, SWIGLU, true>(a, s);
+        case 256: return launch_impl<256, SWIGLU, true>(a, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -619,6 +754,7 @@ int gemm2_ksplit(int64_t R, int groups, int K, int Nout)
 {
     const int sms = device_sm_count();
     const int bn = gemm_choose_token_tile(R, groups, false);
+    if (bn >= 128) return 1;  // paired tiles: large groups, enough work per tile
     const int64_t active = R < groups ? R : groups;
     const int64_t mean = (R + active - 1) / (active > 0 ? active : 1);
     const int64_t tiles = active * ((mean + bn - 1) / bn) * ((Nout + kBM - 1) / kBM);
