@@ -69,7 +69,7 @@ struct Cfg {
     static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
     static constexpr int kAccCols = BN;                    // fp32 TMEM columns per accumulator
-    static constexpr int kAccBufs = (PAIR && BN > 128) ? 1 : 2;
+    static constexpr int kAccBufs = 2;
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols);
     static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs);
     static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
