@@ -37,7 +37,7 @@ from expert_ffn_layer_moe_b200.inputs import CONFIGS, make_inputs  # noqa: E402
 METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PHASES = ("route", "permute", "gemm13", "gemm2", "shared", "combine")
-SMALL_DISPATCH_R = 8192  # assignments up to which the dispatch is one single-block launch
+SMALL_DISPATCH_R = 2048  # assignments up to which the dispatch is one single-block launch
 
 
 def launches_per_step(cfg):

@@ -67,7 +67,7 @@ struct Cfg {
     static constexpr int kBBytes = kBRows * kBK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
-    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
     static constexpr int kAccCols = BN;                    // fp32 TMEM columns per accumulator
     static constexpr int kAccBufs = 2;
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols);
@@ -418,8 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // item -> (group, feature tile, K slice, first row, end row of the group); the
-    // token tile runs fastest so units sharing a weight slice run side by side.
+    // item -> (group, feature tile, K slice, first row, end row of the group).  The
+    // feature tile (and K slice) runs fastest: units running side by side share a token
+    // tile, so a large group streams its activation rows from HBM once while its weights
+    // (a few tens of MB per expert) stay in L2.
     auto decode = [&](int item, int &g, int &feat, int &ks, int &row0, int &row_end) {
         int lo = 0, hi = groups - 1;
         while (lo < hi) {  // largest g with g_tile[g] <= item (skips empty groups)
@@ -428,11 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         g = lo;
         const int local = item - g_tile[g];
-        const int ntok = (g_tile[g + 1] - g_tile[g]) / (n_feat * ksplit);
-        const int fk = local / ntok;
+        const int nfk = n_feat * ksplit;
+        const int fk = local % nfk;
         feat = fk / ksplit;
         ks = fk % ksplit;
-        row0 = g_off[g] + (local % ntok) * BN;
+        row0 = g_off[g] + (local / nfk) * BN;
         row_end = g_off[g + 1];
     };
     auto kslice = [&](int ks, int &kb0, int &kb1) {
@@ -513,7 +515,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // consecutive features of one row.
         const int q = warp & 3;   // TMEM lane quadrant this warp may read
         const int ew = warp - 2;  // 0..3
-        const bool vec_ok = (Nout & 7) == 0;  // then no 16-byte vector straddles the row end
         const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(&tempty_bar[0]), 0) : 0u;
         int acc = 0;
         uint32_t aphase = 0;
@@ -563,29 +564,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     epilogue_sync();
                 }
             } else {
-                float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + ew * 32 * 33);
                 float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
                 const int fbase = feat * C::kFeatTile + (int)rank * C::kFeat + q * 32;
+                // fp32 out: the warp's 32 lanes hold 32 consecutive features of one row per
+                // column, so each store instruction writes 128 contiguous bytes
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
-                    if (vec_ok) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) stage_t[lane][c] = a[c];
-                        __syncwarp();
-                        const int rr = lane >> 3, j = lane & 7;  // 4 rows x 8 feature quads per step
-                        const int fv = fbase + 4 * j;
-#pragma unroll
-                        for (int it = 0; it < 8; ++it) {
-                            const int r = it * 4 + rr;
-                            if (c0 + r < nrows && fv < Nout) {
-                                const float4 v = make_float4(stage_t[4 * j + 0][r], stage_t[4 * j + 1][r],
-                                                             stage_t[4 * j + 2][r], stage_t[4 * j + 3][r]);
-                                *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * Nout + fv) = v;
-                            }
-                        }
-                        __syncwarp();
-                    } else if (fbase + lane < Nout) {
+                    if (fbase + lane < Nout) {
                         float *dst = outf + (size_t)(row0 + c0) * Nout + fbase + lane;
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
@@ -707,12 +693,12 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
     if (SWIGLU && (a.Nout % (kBM / 2)) != 0) return cudaErrorInvalidValue;  // whole 64-feature tiles
     const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups, SWIGLU);
-    // token tiles of 128 rows and more run as CTA pairs (M = 256 weight rows per MMA):
-    // each SM streams half the activation rows and the pair reads each activation tile
-    // once per 256 weight rows instead of once per 128
+    // every tile runs on a CTA pair (M = 256 weight rows per MMA): each SM streams half
+    // the token tile, and the pair reads each activation tile once per 256 weight rows
+    // instead of once per 128
     switch (bn) {
-        case 32: return launch_impl<32, SWIGLU, false>(a, s);
-        case 64: return launch_impl<64, SWIGLU, false>(a, s);
+        case 32: return launch_impl<32, SWIGLU, true>(a, s);
+        case 64: return launch_impl<64, SWIGLU, true>(a, s);
         case 128: return launch_impl<128, SWIGLU, true>(a, s);
         case 256: return launch_impl<256, SWIGLU, true>(a, s);
         default: return cudaErrorInvalidValue;
@@ -752,19 +738,19 @@ int gemm_choose_token_tile(int64_t R, int groups, bool swiglu)
 // the last wave is nearly full.  1 for everything with enough tiles.
 int gemm2_ksplit(int64_t R, int groups, int K, int Nout)
 {
-    const int sms = device_sm_count();
+    const int units = device_sm_count() / 2;  // CTA pairs
     const int bn = gemm_choose_token_tile(R, groups, false);
-    if (bn >= 128) return 1;  // paired tiles: large groups, enough work per tile
+    if (bn >= 128) return 1;  // large groups: enough work per tile
     const int64_t active = R < groups ? R : groups;
     const int64_t mean = (R + active - 1) / (active > 0 ? active : 1);
-    const int64_t tiles = active * ((mean + bn - 1) / bn) * ((Nout + kBM - 1) / kBM);
-    if (tiles <= 0 || tiles >= 4 * (int64_t)sms) return 1;
+    const int64_t tiles = active * ((mean + bn - 1) / bn) * ((Nout + 2 * kBM - 1) / (2 * kBM));
+    if (tiles <= 0 || tiles >= 4 * (int64_t)units) return 1;
     int best = 1;
     double best_eff = 0.0;
     for (int ks = 1; ks <= 4; ++ks) {
         if (K / kBK < 16 * ks) break;  // keep every slice at least 16 K-blocks long
         const int64_t n = tiles * ks;
-        const double eff = (double)n / (double)(((n + sms - 1) / sms) * sms);
+        const double eff = (double)n / (double)(((n + units - 1) / units) * units);
         if (eff > best_eff + 0.02) { best_eff = eff; best = ks; }
     }
     return best;

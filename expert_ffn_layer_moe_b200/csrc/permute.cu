@@ -23,7 +23,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxE = 256;
-constexpr int64_t kSmallR = 8192;  // one-block dispatch up to this many assignments
+constexpr int64_t kSmallR = 2048;  // one-block dispatch up to this many assignments
 static_assert(kPermuteChunk % kThreads == 0, "chunk is whole rounds of the block");
 
 __global__ void __launch_bounds__(kThreads)
