@@ -515,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // consecutive features of one row.
         const int q = warp & 3;   // TMEM lane quadrant this warp may read
         const int ew = warp - 2;  // 0..3
+        const bool vec_ok = (Nout & 7) == 0;  // then no 16-byte vector straddles the row end
         const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(&tempty_bar[0]), 0) : 0u;
         int acc = 0;
         uint32_t aphase = 0;
@@ -566,12 +567,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
                 const int fbase = feat * C::kFeatTile + (int)rank * C::kFeat + q * 32;
-                // fp32 out: the warp's 32 lanes hold 32 consecutive features of one row per
-                // column, so each store instruction writes 128 contiguous bytes
+                // fp32 out through the padded tile: 8 16-byte stores per 32 rows instead of
+                // 32 4-byte ones (store instruction issue, not bytes, limits short-K tiles)
+                float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + ew * 32 * 33);
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
-                    if (fbase + lane < Nout) {
+                    if (vec_ok) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) stage_t[lane][c] = a[c];
+                        __syncwarp();
+                        const int rr = lane >> 3, j = lane & 7;  // 4 rows x 8 feature quads per step
+                        const int fv = fbase + 4 * j;
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int r = it * 4 + rr;
+                            if (c0 + r < nrows && fv < Nout) {
+                                const float4 v = make_float4(stage_t[4 * j + 0][r], stage_t[4 * j + 1][r],
+                                                             stage_t[4 * j + 2][r], stage_t[4 * j + 3][r]);
+                                *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * Nout + fv) = v;
+                            }
+                        }
+                        __syncwarp();
+                    } else if (fbase + lane < Nout) {
                         float *dst = outf + (size_t)(row0 + c0) * Nout + fbase + lane;
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
