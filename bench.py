@@ -51,7 +51,8 @@ def launches_per_step(cfg):
     else:
         router = 1
     permute = 2 if cfg.R <= SMALL_DISPATCH_R else 4  # dispatch (1 or 3 kernels) + row gather
-    return router + permute + 2 + 1  # + W1/W3 and W2 GEMMs (shared experts ride inside), combine
+    shared = 2 if cfg.Is > 0 else 0
+    return router + permute + 2 + shared + 1  # + W1/W3 and W2 GEMMs, shared, combine
 
 
 def peaks():

@@ -103,6 +103,24 @@ moe_status_t expert_ffn_impl(const uint16_t *x_perm, const int32_t *offsets, con
     return MOE_OK;
 }
 
+// Shared experts: one dense SwiGLU FFN over all N rows = the grouped kernels with a
+// single group whose rows are x itself.
+moe_status_t shared_ffn_impl(const uint16_t *x, const uint16_t *Ws1, const uint16_t *Ws3,
+                             const uint16_t *Ws2, int64_t N, int H, int Is, uint16_t *hs, float *s_out,
+                             int *err, cudaStream_t s)
+{
+    if (N == 0) return MOE_OK;
+    moe::GroupedGemmArgs a{};
+    a.act = x; a.w_a = Ws1; a.w_b = Ws3; a.offsets = nullptr; a.groups = 1; a.R = N;
+    a.rows_single = (int)N; a.K = H; a.Nout = Is; a.out = hs; a.dev_err = err;
+    MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
+    moe::GroupedGemmArgs b{};
+    b.act = hs; b.w_a = Ws2; b.offsets = nullptr; b.groups = 1; b.R = N; b.rows_single = (int)N;
+    b.K = Is; b.Nout = H; b.out = s_out; b.dev_err = err;
+    MOE_CUDA(moe::launch_gemm2(b, s));
+    return MOE_OK;
+}
+
 moe_status_t record(void *const *ev, int i, cudaStream_t s)
 {
     if (ev && ev[i]) MOE_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s));
@@ -257,15 +275,10 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
     MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
-    // the shared experts (FinDEP review, section "问题定义": always-on experts) ride in
-    // the routed GEMM launches as a second segment: one group over all N tokens
     {
         moe::GroupedGemmArgs a{};
         a.act = x_perm; a.w_a = W1; a.w_b = W3; a.offsets = offsets; a.groups = E; a.R = R;
         a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
-        if (Is > 0) {
-            a.act2 = x; a.w_a2 = Ws1; a.w_b2 = Ws3; a.out2 = hs; a.rows2 = (int)N; a.K2 = H; a.Nout2 = Is;
-        }
         MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
@@ -275,13 +288,11 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
         b.act = h; b.w_a = W2; b.offsets = offsets; b.groups = E; b.R = R;
         b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
         b.ksplit = ksplit; b.split_stride = R * (int64_t)H;
-        if (Is > 0) {
-            b.act2 = hs; b.w_a2 = Ws2; b.out2 = sh; b.rows2 = (int)N; b.K2 = Is; b.Nout2 = H;
-        }
         MOE_CUDA(moe::launch_gemm2(b, s));
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM2, s));
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));  // shared experts ran inside the two GEMMs
+    if (Is > 0) MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
     MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r, w, sh, N, H, k, out, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_COMBINE, s));
     return MOE_OK;

@@ -35,11 +35,7 @@
 // (no padding to a fixed capacity).  The plain (fp32-out) GEMM can split K into
 // `ksplit` slices whose partial sums land in separate buffers `split_stride` apart,
 // for shapes with too few tiles to cover the SMs; the consumer adds them in a fixed
-// order, so results stay deterministic.  An optional second segment (the layer's
-// always-on shared experts: one group over all tokens, with its own weights, input,
-// output and widths) rides in the same launch; its tiles are spread evenly through the
-// work list, so compute-heavy shared tiles run beside weight-streaming routed tiles
-// instead of in a phase of their own.  Every wait is bounded (globaltimer): on
+// order, so results stay deterministic.  Every wait is bounded (globaltimer): on
 // expiry the kernel records MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain,
 // frees TMEM and returns.
 #include <cuda.h>
@@ -338,11 +334,9 @@ __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;
 template <int BN, bool SWIGLU, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
-                        const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_wa2,
-                        const __grid_constant__ CUtensorMap tm_wb2, const __grid_constant__ CUtensorMap tm_act2,
-                        const int32_t *__restrict__ offsets, int groups, int rows_single, int64_t R, int K,
-                        int Nout, void *__restrict__ out, int ksplit, int64_t split_stride, int rows2, int K2,
-                        int Nout2, void *__restrict__ out2, int *dev_err)
+                        const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
+                        int groups, int rows_single, int64_t R, int K, int Nout,
+                        void *__restrict__ out, int ksplit, int64_t split_stride, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU, PAIR>;
     extern __shared__ uint8_t smem_raw[];
@@ -367,8 +361,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     const int n_feat = (Nout + C::kFeatTile - 1) / C::kFeatTile;
     const int KB = (K + kBK - 1) / kBK;
-    const int n_feat2 = rows2 > 0 ? (Nout2 + C::kFeatTile - 1) / C::kFeatTile : 0;
-    const int KB2 = (K2 + kBK - 1) / kBK;
 
     // ---- work list: row offsets and the prefix of (token tiles x feature tiles x K slices) per group
     if (offsets == nullptr) {
@@ -403,9 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             set_device_error(dev_err, MOE_DEVERR_BAD_OFFSETS);
     }
     __syncthreads();
-    const int total_routed = g_tile[groups];
-    const int total_second = rows2 > 0 ? ((rows2 + BN - 1) / BN) * n_feat2 : 0;
-    const int total = total_routed + total_second;
+    const int total = g_tile[groups];
     if (unit >= total) return;  // uniform over the pair: nothing allocated, no cluster barrier yet
 
     // ---- barriers and TMEM
@@ -432,22 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // feature tile (and K slice) runs fastest: units running side by side share a token
     // tile, so a large group streams its activation rows from HBM once while its weights
     // (a few tens of MB per expert) stay in L2.
-    // seg = 1: a tile of the second segment; its tiles take positions where
-    // floor(i * total_second / total) steps up, i.e. evenly spread.
-    auto decode = [&](int item, int &seg, int &g, int &feat, int &ks, int &row0, int &row_end) {
-        seg = 0;
-        if (total_second > 0) {
-            const int s_i = (int)((int64_t)item * total_second / total);
-            const int s_n = (int)((int64_t)(item + 1) * total_second / total);
-            if (s_n > s_i) {
-                seg = 1; g = 0; ks = 0;
-                feat = s_i % n_feat2;
-                row0 = (s_i / n_feat2) * BN;
-                row_end = rows2;
-                return;
-            }
-            item -= s_i;  // index among the routed tiles
-        }
+    auto decode = [&](int item, int &g, int &feat, int &ks, int &row0, int &row_end) {
         int lo = 0, hi = groups - 1;
         while (lo < hi) {  // largest g with g_tile[g] <= item (skips empty groups)
             const int mid = (lo + hi + 1) >> 1;
@@ -475,22 +450,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tm_wa);
         if (SWIGLU) tma_prefetch_map(&tm_wb);
         tma_prefetch_map(&tm_act);
-        if (total_second > 0) {
-            tma_prefetch_map(&tm_wa2);
-            if (SWIGLU) tma_prefetch_map(&tm_wb2);
-            tma_prefetch_map(&tm_act2);
-        }
         // every load of the pair completes on the leader's stage barrier
         const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&full_bar[0]), 0) : smem_u32(&full_bar[0]);
         int stage = 0;
         uint32_t phase = 0;
         for (int item = unit; item < total && !failed; item += nunits) {
-            int seg, g, feat, ks, row0, row_end, kb0, kb1;
-            decode(item, seg, g, feat, ks, row0, row_end);
-            if (seg) { kb0 = 0; kb1 = KB2; } else kslice(ks, kb0, kb1);
-            const CUtensorMap *mwa = seg ? &tm_wa2 : &tm_wa;
-            const CUtensorMap *mwb = seg ? &tm_wb2 : &tm_wb;
-            const CUtensorMap *mact = seg ? &tm_act2 : &tm_act;
+            int g, feat, ks, row0, row_end, kb0, kb1;
+            decode(item, g, feat, ks, row0, row_end);
+            kslice(ks, kb0, kb1);
             const int frow = feat * C::kFeatTile + (int)rank * C::kFeat;        // first weight row (W1 / W)
             const int trow = row0 + (PAIR ? (int)rank * (mma_width(row0, row_end) >> 1) : 0);
             for (int kb = kb0; kb < kb1; ++kb) {
@@ -500,12 +467,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kCtas * C::kStageBytes);
                 if (SWIGLU) {
                     // rows 0-63: W1 features [frow, +64); rows 64-127: the same features of W3
-                    tma_3d<PAIR>(st, mwa, kb * kBK, frow, g, fb);
-                    tma_3d<PAIR>(st + C::kABytes / 2, mwb, kb * kBK, frow, g, fb);
+                    tma_3d<PAIR>(st, &tm_wa, kb * kBK, frow, g, fb);
+                    tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kb * kBK, frow, g, fb);
                 } else {
-                    tma_3d<PAIR>(st, mwa, kb * kBK, frow, g, fb);
+                    tma_3d<PAIR>(st, &tm_wa, kb * kBK, frow, g, fb);
                 }
-                tma_2d<PAIR>(st + C::kABytes, mact, kb * kBK, trow, fb);
+                tma_2d<PAIR>(st + C::kABytes, &tm_act, kb * kBK, trow, fb);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
         }
@@ -514,9 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, acc = 0;
         uint32_t phase = 0, aphase = 0;
         for (int item = unit; item < total && !failed; item += nunits) {
-            int seg, g, feat, ks, row0, row_end, kb0, kb1;
-            decode(item, seg, g, feat, ks, row0, row_end);
-            if (seg) { kb0 = 0; kb1 = KB2; } else kslice(ks, kb0, kb1);
+            int g, feat, ks, row0, row_end, kb0, kb1;
+            decode(item, g, feat, ks, row0, row_end);
+            kslice(ks, kb0, kb1);
             const uint32_t idesc = C::kIdescNoN | ((uint32_t)(mma_width(row0, row_end) >> 3) << 17);
             if (!mbar_wait(&tempty_bar[acc], aphase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
             tc_fence_after();
@@ -548,15 +515,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // consecutive features of one row.
         const int q = warp & 3;   // TMEM lane quadrant this warp may read
         const int ew = warp - 2;  // 0..3
+        const bool vec_ok = (Nout & 7) == 0;  // then no 16-byte vector straddles the row end
         const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(&tempty_bar[0]), 0) : 0u;
         int acc = 0;
         uint32_t aphase = 0;
         for (int item = unit; item < total; item += nunits) {
-            int seg, g, feat, ks, row0, row_end;
-            decode(item, seg, g, feat, ks, row0, row_end);
-            const int nout = seg ? Nout2 : Nout;
-            void *outp = seg ? out2 : out;
-            const bool vec_ok = (nout & 7) == 0;  // then no 16-byte vector straddles the row end
+            int g, feat, ks, row0, row_end;
+            decode(item, g, feat, ks, row0, row_end);
             // one waiter decides for all four warps, so the named barriers below are
             // always reached by all of them
             if (ew == 0 && lane == 0) *epi_ok = mbar_wait(&tfull_bar[acc], aphase, abort_flag) ? 1 : 0;
@@ -574,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int fl = (q & 1) * 32 + lane;  // feature within this CTA's 64
                 const int rr = lane >> 3, j = lane & 7;
                 const int fv = feat * C::kFeatTile + (int)rank * C::kFeat + 8 * j;
-                uint16_t *outh = static_cast<uint16_t *>(outp);
+                uint16_t *outh = static_cast<uint16_t *>(out);
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
@@ -585,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int it = 0; it < 2; ++it) {
                         const int r = 8 * ew + 4 * it + rr;
-                        if (c0 + r < nrows && fv < nout) {
+                        if (c0 + r < nrows && fv < Nout) {
                             float h[8];
 #pragma unroll
                             for (int i = 0; i < 8; ++i) h[i] = silu(Gs[8 * j + i][r]) * Us[8 * j + i][r];
@@ -594,13 +559,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             v.y = pack_bf16x2(h[2], h[3]);
                             v.z = pack_bf16x2(h[4], h[5]);
                             v.w = pack_bf16x2(h[6], h[7]);
-                            *reinterpret_cast<uint4 *>(outh + (size_t)(row0 + c0 + r) * nout + fv) = v;
+                            *reinterpret_cast<uint4 *>(outh + (size_t)(row0 + c0 + r) * Nout + fv) = v;
                         }
                     }
                     epilogue_sync();
                 }
             } else {
-                float *outf = static_cast<float *>(outp) + (seg ? 0 : (int64_t)ks * split_stride);
+                float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
                 const int fbase = feat * C::kFeatTile + (int)rank * C::kFeat + q * 32;
                 // fp32 out through the padded tile: 8 16-byte stores per 32 rows instead of
                 // 32 4-byte ones (store instruction issue, not bytes, limits short-K tiles)
@@ -617,18 +582,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int it = 0; it < 8; ++it) {
                             const int r = it * 4 + rr;
-                            if (c0 + r < nrows && fv < nout) {
+                            if (c0 + r < nrows && fv < Nout) {
                                 const float4 v = make_float4(stage_t[4 * j + 0][r], stage_t[4 * j + 1][r],
                                                              stage_t[4 * j + 2][r], stage_t[4 * j + 3][r]);
-                                *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * nout + fv) = v;
+                                *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * Nout + fv) = v;
                             }
                         }
                         __syncwarp();
-                    } else if (fbase + lane < nout) {
-                        float *dst = outf + (size_t)(row0 + c0) * nout + fbase + lane;
+                    } else if (fbase + lane < Nout) {
+                        float *dst = outf + (size_t)(row0 + c0) * Nout + fbase + lane;
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
-                            if (c0 + c < nrows) dst[(size_t)c * nout] = a[c];
+                            if (c0 + c < nrows) dst[(size_t)c * Nout] = a[c];
                     }
                 }
             }
@@ -706,7 +671,7 @@ template <int BN, bool SWIGLU, bool PAIR>
 cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
     using C = Cfg<BN, SWIGLU, PAIR>;
-    CUtensorMap ma, mb, mact, ma2, mb2, mact2;
+    CUtensorMap ma, mb, mact;
     const int box_rows = SWIGLU ? kBM / 2 : kBM;
     if (!encode_weight_map(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     if (SWIGLU) {
@@ -715,17 +680,6 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
         mb = ma;
     }
     if (!encode_act_map(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
-    if (a.rows2 > 0) {
-        if (!encode_weight_map(&ma2, a.w_a2, 1, a.Nout2, a.K2, box_rows)) return cudaErrorInvalidValue;
-        if (SWIGLU) {
-            if (!encode_weight_map(&mb2, a.w_b2, 1, a.Nout2, a.K2, box_rows)) return cudaErrorInvalidValue;
-        } else {
-            mb2 = ma2;
-        }
-        if (!encode_act_map(&mact2, a.act2, a.rows2, a.K2, C::kBRows)) return cudaErrorInvalidValue;
-    } else {
-        ma2 = ma; mb2 = mb; mact2 = mact;  // never read
-    }
     auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
@@ -745,9 +699,8 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, ma2, mb2, mact2, a.offsets, a.groups, a.rows_single, a.R,
-                             a.K, a.Nout, a.out, ksplit, a.split_stride, a.rows2 > 0 ? a.rows2 : 0, a.K2, a.Nout2,
-                             a.out2, a.dev_err);
+    err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
+                             ksplit, a.split_stride, a.dev_err);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
@@ -757,7 +710,6 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
     if (SWIGLU && (a.Nout % (kBM / 2)) != 0) return cudaErrorInvalidValue;  // whole 64-feature tiles
-    if (SWIGLU && a.rows2 > 0 && (a.Nout2 % (kBM / 2)) != 0) return cudaErrorInvalidValue;
     const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups, SWIGLU);
     // every tile runs on a CTA pair (M = 256 weight rows per MMA): each SM streams half
     // the token tile, and the pair reads each activation tile once per 256 weight rows

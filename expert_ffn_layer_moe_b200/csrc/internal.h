@@ -44,14 +44,6 @@ struct GroupedGemmArgs {
     int token_tile;          // 0 = choose from the shape
     int ksplit;              // plain GEMM: K slices (0/1 = none); partial sums at out + s*split_stride
     int64_t split_stride;    // elements between the partial-sum buffers
-    // optional second segment in the same launch: one group of rows2 rows of act2
-    const uint16_t *act2;    // [rows2, K2] bf16
-    const uint16_t *w_a2;    // [Nout2, K2] bf16
-    const uint16_t *w_b2;    // [Nout2, K2] bf16 -- SwiGLU only
-    void *out2;              // [rows2, Nout2], same element type as out
-    int rows2;               // 0 = no second segment
-    int K2;
-    int Nout2;
 };
 cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s);

@@ -206,8 +206,7 @@ MOE_API moe_status_t moe_layer_forward(const uint16_t *x, const float *W_gate, c
  *   in the workspace).
  *   phase_events: NULL, or an array of MOE_NUM_PHASES + 1 cudaEvent_t (as
  *   void*) recorded on `stream` before the first and after each phase, for
- *   per-kernel timing.  The shared experts run inside the two GEMM phases (a
- *   second segment of the same launches), so the SHARED phase is empty.
+ *   per-kernel timing.
  */
 #define MOE_PHASE_ROUTE 0
 #define MOE_PHASE_PERMUTE 1
