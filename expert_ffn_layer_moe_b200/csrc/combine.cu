@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(kThreads)
                    const int32_t *__restrict__ token_to_row, const float *__restrict__ topk_w,
                    const float *__restrict__ shared_out, int64_t N, int H, int k, uint16_t *__restrict__ out)
 {
+    pdl_entry();
     const int64_t t = blockIdx.y;
     int rows[kMaxK];
     float w[kMaxK];
@@ -92,9 +93,8 @@ cudaError_t launch_combine(const float *y_perm, int nsplit, int64_t split_stride
         return cudaSuccess;
     }
     const dim3 grid((unsigned)((H / 8 + kThreads - 1) / kThreads), (unsigned)N);
-    combine_kernel<<<grid, kThreads, 0, s>>>(y_perm, nsplit, split_stride, token_to_row, topk_w, shared_out, N, H,
-                                             k, out);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, grid, dim3(kThreads), 0, s, y_perm, nsplit, split_stride, token_to_row, topk_w,
+                      shared_out, N, H, k, out);
 }
 
 }  // namespace moe

@@ -37,6 +37,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
            (static_cast<uint32_t>(float_to_bf16_bits(hi)) << 16);
 }
 
+// Programmatic dependent launch.  Every kernel of the layer lets the next kernel in the
+// stream begin launching at once, then waits until the kernels it depends on have
+// finished and their writes are visible -- before touching global memory, so no
+// read-after-write or write-after-read hazard can cross the overlap.  What overlaps is
+// launch latency and any prologue placed before the wait.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_entry()
+{
+    pdl_launch_dependents();
+    pdl_wait();
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns()
 {
     uint64_t t;

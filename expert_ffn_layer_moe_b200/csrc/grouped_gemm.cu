@@ -362,13 +362,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_feat = (Nout + C::kFeatTile - 1) / C::kFeatTile;
     const int KB = (K + kBK - 1) / kBK;
 
+    // ---- barriers and TMEM: nothing here reads global memory, so it overlaps the tail
+    // of the previous kernel in the stream (programmatic dependent launch)
+    pdl_launch_dependents();
+    if (tid == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < C::kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        for (int b = 0; b < C::kAccBufs; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 4 * C::kCtas);  // every epilogue warp of the pair releases
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc_g<PAIR>(tmem_slot, C::kTmemCols);
+        tmem_relinquish_g<PAIR>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (PAIR) cluster_sync();  // both CTAs' barriers exist before either signals the other
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // from here on the previous kernels' outputs are complete and visible
+
     // ---- work list: row offsets and the prefix of (token tiles x feature tiles x K slices) per group
     if (offsets == nullptr) {
         if (tid == 0) { g_off[0] = 0; g_off[1] = rows_single; }
     } else {
         for (int i = tid; i <= groups; i += kThreads) g_off[i] = offsets[i];
     }
-    if (tid == 0) *abort_flag = 0;
     __syncthreads();
     if (warp == 0) {
         int carry = 0;
@@ -395,28 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             set_device_error(dev_err, MOE_DEVERR_BAD_OFFSETS);
     }
     __syncthreads();
-    const int total = g_tile[groups];
-    if (unit >= total) return;  // uniform over the pair: nothing allocated, no cluster barrier yet
-
-    // ---- barriers and TMEM
-    if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-        for (int b = 0; b < C::kAccBufs; ++b) {
-            mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 4 * C::kCtas);  // every epilogue warp of the pair releases
-        }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    if (warp == 1) {
-        tmem_alloc_g<PAIR>(tmem_slot, C::kTmemCols);
-        tmem_relinquish_g<PAIR>();
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (PAIR) cluster_sync();  // both CTAs' barriers exist before either signals the other
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    const int total = g_tile[groups];  // units with no work skip every role loop below
 
     // item -> (group, feature tile, K slice, first row, end row of the group).  The
     // feature tile (and K slice) runs fastest: units running side by side share a token
@@ -686,19 +688,19 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
     const int sms = device_sm_count();
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cfg.gridDim = dim3((unsigned)(PAIR ? (sms / 2) * 2 : sms));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = s;
-    if (PAIR) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = PAIR ? 2 : 1;
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
                              ksplit, a.split_stride, a.dev_err);
     if (err != cudaSuccess) return err;

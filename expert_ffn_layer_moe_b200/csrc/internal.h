@@ -7,6 +7,24 @@
 
 namespace moe {
 
+// Launch with programmatic stream serialization (the kernel calls pdl_entry/pdl_wait
+// before its first global memory access).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Router: logits (fp32), top-k indices and renormalised weights.  `ws` (nullable)
 // of at least router_ws_bytes(N, H, E) bytes enables the tensor-core and
 // expert-split paths.

@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(kThreads)
     count_kernel(const int32_t *__restrict__ idx, int64_t R, int E, int32_t *__restrict__ blk_cnt, int *err)
 {
     __shared__ int hist[kMaxE];
+    pdl_entry();
     for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
     __syncthreads();
     const int64_t a0 = (int64_t)blockIdx.x * kPermuteChunk;
@@ -50,6 +51,7 @@ __global__ void __launch_bounds__(kThreads)
                 int32_t *__restrict__ offsets)
 {
     __shared__ int s[kMaxE];
+    pdl_entry();
     const int e = threadIdx.x;
     int total = 0;
     if (e < E)
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(kThreads)
     __shared__ int base[kMaxE];
     __shared__ int scan[kThreads];
     __shared__ int wcnt[kWarps][kMaxE];
+    pdl_entry();
     const int tid = threadIdx.x;
     if (tid < E) base[tid] = 0;
     __syncthreads();
@@ -162,6 +165,7 @@ __global__ void __launch_bounds__(kThreads)
 {
     __shared__ int base[kMaxE];
     __shared__ int wcnt[kWarps][kMaxE];
+    pdl_entry();
     for (int e = threadIdx.x; e < E; e += kThreads) base[e] = blk_base[(int64_t)blockIdx.x * E + e];
     const int64_t a0 = (int64_t)blockIdx.x * kPermuteChunk;
     for (int round = 0; round < kPermuteChunk / kThreads; ++round) {
@@ -176,6 +180,7 @@ __global__ void __launch_bounds__(kThreads)
     gather_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ row_to_token,
                        const int32_t *__restrict__ offsets, int E, int H, uint16_t *__restrict__ x_perm)
 {
+    pdl_entry();
     const int64_t rows = offsets[E];
     const int nvec = H / 8;
     const int64_t warp_global = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
@@ -197,18 +202,24 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
     const int64_t R = N * k;
     if (R <= 0) return cudaSuccess;
     if (R <= kSmallR) {
-        dispatch_small_kernel<<<1, kThreads, 0, s>>>(topk_idx, R, k, E, counts, offsets, row_to_token, token_to_row,
-                                                     dev_err);
+        cudaError_t e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(kThreads), 0, s, topk_idx, R, k, E, counts,
+                                   offsets, row_to_token, token_to_row, dev_err);
+        if (e != cudaSuccess) return e;
     } else {
         const int64_t nblk = permute_blocks(R);
-        count_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, E, scratch, dev_err);
-        scan_kernel<<<1, kThreads, 0, s>>>(scratch, nblk, E, counts, offsets);
-        rank_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, R, k, E, scratch, row_to_token, token_to_row);
+        cudaError_t e = launch_pdl(count_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s, topk_idx, R, E, scratch,
+                                   dev_err);
+        if (e == cudaSuccess)
+            e = launch_pdl(scan_kernel, dim3(1), dim3(kThreads), 0, s, scratch, nblk, E, counts, offsets);
+        if (e == cudaSuccess)
+            e = launch_pdl(rank_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s, (const int32_t *)topk_idx, R, k,
+                           E, (const int32_t *)scratch, row_to_token, token_to_row);
+        if (e != cudaSuccess) return e;
     }
     const int64_t want = (R + kWarps - 1) / kWarps;
     const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
-    gather_rows_kernel<<<gblocks, kThreads, 0, s>>>(x, row_to_token, offsets, E, H, x_perm);
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, dim3(gblocks), dim3(kThreads), 0, s, x, (const int32_t *)row_to_token,
+                      (const int32_t *)offsets, E, H, x_perm);
 }
 
 }  // namespace moe

@@ -157,6 +157,7 @@ __global__ void __launch_bounds__(kThreads)
     extern __shared__ float smem[];
     float *partial = smem;                        // [kWarps][TT][E]
     float *s_logit = smem + kWarps * TT * E;      // [TT][E]
+    pdl_entry();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * TT;
     const int nt = (N - t0) < TT ? (int)(N - t0) : TT;
@@ -194,6 +195,7 @@ __global__ void __launch_bounds__(kThreads)
                          const float *__restrict__ bias, int64_t N, int H, int E, float *__restrict__ logits)
 {
     __shared__ float partial[kWarps][TT][kEC];
+    pdl_entry();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * TT;
     const int nt = (N - t0) < TT ? (int)(N - t0) : TT;
@@ -229,6 +231,7 @@ __global__ void __launch_bounds__(kThreads)
                        float *__restrict__ topk_w)
 {
     __shared__ float row[kWarps][kMaxE];
+    pdl_entry();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * kWarps + warp;
     if (t >= N) return;  // the whole warp leaves; no block-wide barrier below
@@ -255,6 +258,7 @@ __global__ void __launch_bounds__(kThreads)
     router_split_kernel(const float *__restrict__ W_gate, int H, int E, uint16_t *__restrict__ wsplit)
 {
     __shared__ float tile[32][33];
+    pdl_entry();
     const int h0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
     for (int i = ty; i < 32; i += kWarps) {
@@ -288,9 +292,8 @@ cudaError_t launch_fused(const uint16_t *x, const float *W_gate, const float *bi
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    kern<<<(unsigned)((N + TT - 1) / TT), kThreads, smem, s>>>(x, W_gate, bias, N, H, E, k, logits, topk_idx,
-                                                               topk_w);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)((N + TT - 1) / TT)), dim3(kThreads), smem, s, x, W_gate, bias, N, H, E, k,
+                      logits, topk_idx, topk_w);
 }
 
 template <int TT>
@@ -298,10 +301,10 @@ cudaError_t launch_split_e(const uint16_t *x, const float *W_gate, const float *
                            int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
 {
     const dim3 grid((unsigned)((N + TT - 1) / TT), (unsigned)((E + kEC - 1) / kEC));
-    router_logits_kernel<TT><<<grid, kThreads, 0, s>>>(x, W_gate, bias, N, H, E, logits);
-    router_topk_kernel<<<(unsigned)((N + kWarps - 1) / kWarps), kThreads, 0, s>>>(logits, 1, nullptr, N, E, k,
-                                                                                  nullptr, topk_idx, topk_w);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(router_logits_kernel<TT>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H, E, logits);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(router_topk_kernel, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s,
+                      (const float *)logits, 1, (const float *)nullptr, N, E, k, (float *)nullptr, topk_idx, topk_w);
 }
 
 // Tokens per block for the CUDA-core paths: keep about two blocks per SM (times the
@@ -347,15 +350,15 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
         uint16_t *wsplit = reinterpret_cast<uint16_t *>(w8);
         float *parts = reinterpret_cast<float *>(w8 + split_bytes);
         const dim3 sgrid((unsigned)((H + 31) / 32), (unsigned)((E + 31) / 32));
-        router_split_kernel<<<sgrid, kThreads, 0, s>>>(W_gate, H, E, wsplit);
+        cudaError_t e = launch_pdl(router_split_kernel, sgrid, dim3(kThreads), 0, s, W_gate, H, E, wsplit);
+        if (e != cudaSuccess) return e;
         GroupedGemmArgs g{};
         g.act = x; g.w_a = wsplit; g.w_b = nullptr; g.offsets = nullptr; g.groups = 1; g.R = N;
         g.rows_single = (int)N; g.K = H; g.Nout = 3 * E; g.out = parts; g.dev_err = dev_err; g.token_tile = 128;
-        cudaError_t e = launch_gemm2(g, s);
+        e = launch_gemm2(g, s);
         if (e != cudaSuccess) return e;
-        router_topk_kernel<<<(unsigned)((N + kWarps - 1) / kWarps), kThreads, 0, s>>>(parts, 3, bias, N, E, k, lbuf,
-                                                                                      topk_idx, topk_w);
-        return cudaGetLastError();
+        return launch_pdl(router_topk_kernel, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s,
+                          (const float *)parts, 3, bias, N, E, k, lbuf, topk_idx, topk_w);
     }
     if (path == RouterPath::kSplitE) {
         switch (tokens_per_block(N, (E + kEC - 1) / kEC)) {
