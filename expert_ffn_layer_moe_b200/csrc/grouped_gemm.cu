@@ -707,15 +707,34 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// Expected work items on CTA pairs, from the mean group size (the true count is only
+// known on the device).
+int64_t gemm_pair_tiles(int64_t R, int groups, int Nout, bool swiglu, int ksplit)
+{
+    const int bn = gemm_choose_token_tile(R, groups, swiglu);
+    const int64_t active = R < groups ? R : groups;
+    if (active <= 0) return 0;
+    const int64_t mean = (R + active - 1) / active;
+    const int feat = swiglu ? kBM : 2 * kBM;  // output features per pair tile
+    return active * ((mean + bn - 1) / bn) * ((Nout + feat - 1) / feat) * (ksplit > 1 ? ksplit : 1);
+}
+
 template <bool SWIGLU>
 cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
     if (SWIGLU && (a.Nout % (kBM / 2)) != 0) return cudaErrorInvalidValue;  // whole 64-feature tiles
     const int bn = a.token_tile ? a.token_tile : gemm_choose_token_tile(a.R, a.groups, SWIGLU);
-    // every tile runs on a CTA pair (M = 256 weight rows per MMA): each SM streams half
-    // the token tile, and the pair reads each activation tile once per 256 weight rows
-    // instead of once per 128
+    // Tiles run on CTA pairs (M = 256 weight rows per MMA): each SM streams half the
+    // token tile, and the pair reads each activation tile once per 256 weight rows
+    // instead of once per 128.  A tiny batch whose pair tiles would not even cover the
+    // SM pairs once runs single-CTA tiles instead (twice the tiles, every SM streaming).
+    if (bn <= 64 && gemm_pair_tiles(a.R, a.groups, a.Nout, SWIGLU, a.ksplit) < device_sm_count() / 2) {
+        switch (bn) {
+            case 32: return launch_impl<32, SWIGLU, false>(a, s);
+            case 64: return launch_impl<64, SWIGLU, false>(a, s);
+        }
+    }
     switch (bn) {
         case 32: return launch_impl<32, SWIGLU, true>(a, s);
         case 64: return launch_impl<64, SWIGLU, true>(a, s);
@@ -761,14 +780,12 @@ int gemm2_ksplit(int64_t R, int groups, int K, int Nout)
     const int units = device_sm_count() / 2;  // CTA pairs
     const int bn = gemm_choose_token_tile(R, groups, false);
     if (bn >= 128) return 1;  // large groups: enough work per tile
-    const int64_t active = R < groups ? R : groups;
-    const int64_t mean = (R + active - 1) / (active > 0 ? active : 1);
-    const int64_t tiles = active * ((mean + bn - 1) / bn) * ((Nout + 2 * kBM - 1) / (2 * kBM));
+    const int64_t tiles = gemm_pair_tiles(R, groups, Nout, false, 1);
     if (tiles <= 0 || tiles >= 4 * (int64_t)units) return 1;
     int best = 1;
     double best_eff = 0.0;
     for (int ks = 1; ks <= 4; ++ks) {
-        if (K / kBK < 16 * ks) break;  // keep every slice at least 16 K-blocks long
+        if (K / kBK < 6 * ks) break;  // keep every slice at least 6 K-blocks long
         const int64_t n = tiles * ks;
         const double eff = (double)n / (double)(((n + units - 1) / units) * units);
         if (eff > best_eff + 0.02) { best_eff = eff; best = ks; }

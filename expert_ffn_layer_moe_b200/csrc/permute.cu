@@ -189,7 +189,13 @@ __global__ void __launch_bounds__(kThreads)
     for (int64_t r = warp_global; r < rows; r += nwarps) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)row_to_token[r] * H);
         uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * H);
-        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        int v = lane;
+        for (; v + 96 < nvec; v += 128) {  // four 16-byte loads in flight per lane
+            const uint4 a = __ldg(src + v), b = __ldg(src + v + 32), c = __ldg(src + v + 64),
+                        d = __ldg(src + v + 96);
+            dst[v] = a; dst[v + 32] = b; dst[v + 64] = c; dst[v + 96] = d;
+        }
+        for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
     }
 }
 
