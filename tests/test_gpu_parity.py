@@ -217,6 +217,12 @@ def test_layer_tiny_matches_oracle():
     MoEConfig("shared", N=90, H=256, I=128, E=6, k=2, Is=192),
     # few tiles and a long K: the W2 GEMM splits K and the combine adds the slices
     MoEConfig("splitk", N=64, H=256, I=2048, E=4, k=2),
+    # the largest expert count and top-k the library takes
+    MoEConfig("maxEk", N=512, H=256, I=128, E=256, k=8),
+    # k == E: every token visits every expert
+    MoEConfig("allexperts", N=96, H=192, I=192, E=4, k=4),
+    # the smallest widths (one 64-column K block, one feature half-tile)
+    MoEConfig("narrowest", N=40, H=64, I=64, E=3, k=2),
 ])
 def test_layer_shapes_match_oracle(cfg):
     t = cuda_inputs(cfg, seed=1)
