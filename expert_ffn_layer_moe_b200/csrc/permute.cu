@@ -11,7 +11,9 @@
 //               starting row per expert (in place over the histograms);
 //   3. rank   : per block again, the stable rank of each assignment inside its
 //               block (warp match + per-warp counts, warps in order) -> row maps;
-//   4. gather : x_perm[r] = x[row_to_token[r]], one warp per row, 16-byte vectors.
+//   4. copy   : x_perm[token_to_row[t,j]] = x[t] for j < k -- one warp per token reads
+//               its row once (16-byte vectors) and writes its k copies, so x is read
+//               from HBM once however many experts share a token.
 // Batches of at most kSmallR assignments (decode) do 1-3 in one single-block
 // launch, then the gather: two launches instead of four.
 #include "common.cuh"
@@ -175,27 +177,36 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// x_perm[r] = x[row_to_token[r]] for r < offsets[E]; one warp per row.
+// x_perm[token_to_row[t,j]] = x[t] for every assignment with a valid row; one warp
+// per token (grid-stride), each lane 16-byte vectors, four loads in flight.
 __global__ void __launch_bounds__(kThreads)
-    gather_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ row_to_token,
-                       const int32_t *__restrict__ offsets, int E, int H, uint16_t *__restrict__ x_perm)
+    scatter_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ token_to_row, int64_t N, int k,
+                        int H, uint16_t *__restrict__ x_perm)
 {
     pdl_entry();
-    const int64_t rows = offsets[E];
     const int nvec = H / 8;
     const int64_t warp_global = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
     const int lane = threadIdx.x & 31;
-    for (int64_t r = warp_global; r < rows; r += nwarps) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)row_to_token[r] * H);
-        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * H);
-        int v = lane;
-        for (; v + 96 < nvec; v += 128) {  // four 16-byte loads in flight per lane
-            const uint4 a = __ldg(src + v), b = __ldg(src + v + 32), c = __ldg(src + v + 64),
-                        d = __ldg(src + v + 96);
-            dst[v] = a; dst[v + 32] = b; dst[v + 64] = c; dst[v + 96] = d;
+    for (int64_t t = warp_global; t < N; t += nwarps) {
+        int rows[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rows[j] = j < k ? token_to_row[t * k + j] : -1;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
+        for (int v0 = lane; v0 < nvec; v0 += 128) {
+            uint4 buf[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (v0 + 32 * u < nvec) buf[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (rows[j] < 0) continue;
+                uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (int64_t)rows[j] * H);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = buf[u];
+            }
         }
-        for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
     }
 }
 
@@ -222,10 +233,10 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
                            E, (const int32_t *)scratch, row_to_token, token_to_row);
         if (e != cudaSuccess) return e;
     }
-    const int64_t want = (R + kWarps - 1) / kWarps;
+    const int64_t want = (N + kWarps - 1) / kWarps;
     const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
-    return launch_pdl(gather_rows_kernel, dim3(gblocks), dim3(kThreads), 0, s, x, (const int32_t *)row_to_token,
-                      (const int32_t *)offsets, E, H, x_perm);
+    return launch_pdl(scatter_rows_kernel, dim3(gblocks), dim3(kThreads), 0, s, x, (const int32_t *)token_to_row,
+                      N, k, H, x_perm);
 }
 
 }  // namespace moe

@@ -2,7 +2,7 @@
 import numpy as np
 import pytest
 
-from expert_ffn_layer_moe_b200.perfmodel import fit_linear
+from expert_ffn_layer_moe_b200.perfmodel import fit_linear, fit_multilinear, fit_roofline
 
 
 def test_exact_line():
@@ -29,3 +29,18 @@ def test_matches_polyfit_on_noisy_data():
 def test_needs_two_points():
     with pytest.raises(ValueError):
         fit_linear([1], [1])
+
+
+def test_roofline_fit_recovers_a_knee():
+    m = np.array([1, 2, 4, 8, 16, 32, 64, 128, 256])
+    t = np.maximum(5.0, 1.0 + 0.05 * m)       # flat at 5 until m = 80, then linear
+    c, a, b, r2 = fit_roofline(m, t)
+    assert np.isclose(c, 5.0) and np.isclose(a, 1.0) and np.isclose(b, 0.05) and np.isclose(r2, 1.0)
+
+
+def test_multilinear_recovers_two_coefficients():
+    touched = [8, 82, 128, 128, 128, 128]
+    rows = [0.06, 1, 4, 16, 64, 256]
+    t = [0.01 + 0.002 * a + 0.0005 * b for a, b in zip(touched, rows)]
+    coef, r2 = fit_multilinear([touched, rows], t)
+    assert np.allclose(coef, [0.01, 0.002, 0.0005]) and np.isclose(r2, 1.0)
