@@ -6,13 +6,14 @@ modelled as linear in the tokens each expert receives, t_e(m_e) = a_e + b_e * m_
 with coefficients collected offline by microbenchmarks and a fit quality (R^2)
 reported for its GEMM model.  This module measures the two grouped GEMMs of this
 library (W1/W3 with SwiGLU, then W2) over a sweep of batch sizes at one layer shape,
-takes m_e = N*k/E (mean rows per expert), and fits t = a + b*m by least squares, and
-also the roofline-shaped t = max(c, a + b*m) (flat while weights stream, linear once
-the rows' arithmetic dominates).
+takes m_e = N*k/E (mean rows per expert), and fits t = a + b*m by least squares -- over
+every point, and over the points where all experts receive rows (the model's premise).
+Because small batches leave experts untouched (their weights are then not streamed), it
+also fits t = c0 + c1*touched + c2*m_e.
 
     python -m expert_ffn_layer_moe_b200.perfmodel [--config qwen3_30b_a3b] [--tokens 1,16,...]
 
-prints one JSON object: the per-N measurements, (a, b) and R^2.
+prints one JSON object: the per-N measurements and the fits with their R^2.
 """
 from __future__ import annotations
 
@@ -49,33 +50,6 @@ def fit_multilinear(cols: Sequence[Sequence[float]], t: Sequence[float]) -> Tupl
     resid = y - A @ coef
     ss_tot = float(((y - y.mean()) ** 2).sum())
     return [float(v) for v in coef], (1.0 - float(resid @ resid) / ss_tot if ss_tot > 0 else 1.0)
-
-
-def fit_roofline(m: Sequence[float], t: Sequence[float]) -> Tuple[float, float, float, float]:
-    """Least-squares fit of the roofline-shaped model t ~ max(c, a + b*m).
-
-    Below the knee the time is flat (the expert weights stream from memory whatever the
-    row count); above it the rows' arithmetic grows it linearly.  Tries every split of
-    the points sorted by m into a flat part and a linear part, fits each by least
-    squares and keeps the split with the smallest squared error.  Returns
-    (c, a, b, R^2)."""
-    x = np.asarray(m, dtype=np.float64)
-    y = np.asarray(t, dtype=np.float64)
-    order = np.argsort(x)
-    x, y = x[order], y[order]
-    best = None
-    for split in range(1, x.size - 1):  # at least one flat point and two linear points
-        c = float(y[:split].mean())
-        a, b, _ = fit_linear(x[split:], y[split:])
-        pred = np.maximum(c, a + b * x)
-        sse = float(((y - pred) ** 2).sum())
-        if best is None or sse < best[0]:
-            best = (sse, c, a, b)
-    if best is None:
-        raise ValueError("need at least three points")
-    sse, c, a, b = best
-    ss_tot = float(((y - y.mean()) ** 2).sum())
-    return c, a, b, (1.0 - sse / ss_tot if ss_tot > 0 else 1.0)
 
 
 def measure(config: str, tokens: Sequence[int], steps: int = 10, warmup: int = 3) -> List[Dict]:
@@ -132,7 +106,6 @@ def main():
     rows = measure(args.config, tokens, steps=args.steps)
     a, b, r2 = fit_linear([r["m_e"] for r in rows], [r["gemm_ms"] for r in rows])
     la, lb, lr2 = fit_linear([r["m_e"] for r in rows], [r["layer_ms"] for r in rows])
-    c, ra, rb, rr2 = fit_roofline([r["m_e"] for r in rows], [r["gemm_ms"] for r in rows])
     full = [r for r in rows if r["touched"] == max(q["touched"] for q in rows)]
     fa, fb, fr2 = fit_linear([r["m_e"] for r in full], [r["gemm_ms"] for r in full]) if len(full) >= 2 else (0, 0, 0)
     coef, mr2 = fit_multilinear([[r["touched"] for r in rows], [r["m_e"] for r in rows]],
@@ -143,7 +116,6 @@ def main():
                                                             "points": len(full)},
                       "expert_ffn_fit_touched_and_rows": {"const_ms": coef[0], "ms_per_touched_expert": coef[1],
                                                           "ms_per_row_per_expert": coef[2], "r2": mr2},
-                      "expert_ffn_roofline_fit": {"flat_ms": c, "alpha_ms": ra, "beta_ms_per_row": rb, "r2": rr2},
                       "layer_fit": {"alpha_ms": la, "beta_ms_per_row": lb, "r2": lr2}}))
 
 

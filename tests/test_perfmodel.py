@@ -2,7 +2,7 @@
 import numpy as np
 import pytest
 
-from expert_ffn_layer_moe_b200.perfmodel import fit_linear, fit_multilinear, fit_roofline
+from expert_ffn_layer_moe_b200.perfmodel import fit_linear, fit_multilinear
 
 
 def test_exact_line():
@@ -29,13 +29,6 @@ def test_matches_polyfit_on_noisy_data():
 def test_needs_two_points():
     with pytest.raises(ValueError):
         fit_linear([1], [1])
-
-
-def test_roofline_fit_recovers_a_knee():
-    m = np.array([1, 2, 4, 8, 16, 32, 64, 128, 256])
-    t = np.maximum(5.0, 1.0 + 0.05 * m)       # flat at 5 until m = 80, then linear
-    c, a, b, r2 = fit_roofline(m, t)
-    assert np.isclose(c, 5.0) and np.isclose(a, 1.0) and np.isclose(b, 0.05) and np.isclose(r2, 1.0)
 
 
 def test_multilinear_recovers_two_coefficients():
