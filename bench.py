@@ -93,6 +93,17 @@ def layer_bytes(cfg, touched):
             + 2 * cfg.N * cfg.H * 2)
 
 
+def kernel_source_digest(path):
+    """sha256[:12] of a CUDA source with its comments and blank lines removed (a comment
+    edit leaves the compiled kernel, and so its measured traffic, unchanged)."""
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:12]
+
+
 def kernel_traffic(kernel, workload):
     """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.txt,
     valid only while the kernel source is unchanged (its sha256 prefix matches)."""
@@ -100,7 +111,7 @@ def kernel_traffic(kernel, workload):
     src = os.path.join(ROOT, "expert_ffn_layer_moe_b200", "csrc", "grouped_gemm.cu")
     if not os.path.exists(path):
         return None
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
+    digest = kernel_source_digest(src)
     for line in open(path):
         f = line.split()
         if len(f) >= 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload and f[3] == digest:

@@ -4,40 +4,47 @@
 // group (MoE-latency article, section "router 之后还有一串动作": every expert runs
 // its own matrix, and a grouped GEMM merges them into one launch; FinDEP review,
 // section "核心公式": an expert is three GEMMs).  Two instantiations:
-//   * SWIGLU = true : h[r] = bf16( silu(x W1[e]^T) * (x W3[e]^T) ).  The MMA's 128
-//                     weight rows are 64 rows of W1 and the same 64 rows of W3, so one
-//                     accumulator holds g (TMEM lanes 0-63) and u (lanes 64-127) for 64
-//                     output features, the activation tile is read once per K step, and
-//                     the epilogue pairs the lanes through shared memory;
-//   * SWIGLU = false: y[r] = h W2[e]^T over 128 output features, stored in fp32 (the
-//                     combine sums k of these rows before the one rounding of the layer
-//                     output).
+//   * SWIGLU = true : h[r] = bf16( silu(x W1[e]^T) * (x W3[e]^T) ).  A CTA's 128 weight
+//                     rows are 64 rows of W1 and the same 64 rows of W3, so one
+//                     accumulator holds g (TMEM lanes 0-63) and u (lanes 64-127), the
+//                     activation tile is read once per K step, and the epilogue pairs
+//                     the lanes through shared memory;
+//   * SWIGLU = false: y[r] = h W2[e]^T, stored in fp32 (the combine sums k of these rows
+//                     before the one rounding of the layer output).
 //
-// Tile shape ("swap-AB"): the MMA's M side (128) walks the weight's output
-// features, its N side (up to BN = 32..256) walks the group's token rows.  Decode-sized
-// groups (a few dozen rows per expert) then fill the tensor core's N side instead
-// of padding M to 128, and every weight byte is read once per token tile.  The MMA
-// width is set per tile (the instruction descriptor is a runtime operand): a tile
-// holding r rows multiplies round_up(r, 16) of them, so a ragged group pays for at
-// most 15 padding rows instead of BN - r.
+// Tile shape ("swap-AB"): the MMA's M side walks the weight's output features, its N
+// side (up to BN = 32..256 rows) walks the group's token rows.  Decode-sized groups (a
+// few dozen rows per expert) then fill the tensor core's N side instead of padding M,
+// and every weight byte is read once per token tile.  The MMA width is set per tile
+// (the instruction descriptor is a runtime operand): a tile holding r rows multiplies
+// round_up(r, 16) of them.
+//
+// CTA pairs (PAIR = true, the default): a cluster of two CTAs on two SMs shares one
+// tcgen05.mma.cta_group::2 of M = 256.  CTA r holds weight rows [128 r, 128 r + 128) and
+// half of the token tile; both CTAs' TMA loads complete on the leader's stage barrier,
+// the leader issues the MMAs and its commits arrive at both CTAs' barriers, and each CTA
+// drains its own TMEM.  An activation tile is then read once per 256 weight rows.  Tiny
+// batches whose tiles would not cover the SM pairs use single-CTA tiles (PAIR = false).
 //
 // Warp roles (192 threads, one CTA per SM, persistent over work items):
-//   warp 0 lane 0 : TMA producer  -- the 128-row weight tile and the [BN x 64]
-//                   activation tile per stage, 128-byte swizzle, mbarrier transaction counts;
-//   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (bf16 in, fp32 accumulate)
-//                   and tcgen05.commit to release stages and hand accumulators over;
+//   warp 0 lane 0 : TMA producer -- the 128-row weight tile and this CTA's part of the
+//                   token tile per stage, 128-byte swizzle, mbarrier transaction counts;
+//   warp 1        : TMEM allocator; lane 0 of the leader issues tcgen05.mma (bf16 in,
+//                   fp32 accumulate) and tcgen05.commit to free stages and hand
+//                   accumulators over;
 //   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
 //                   per warp), staged through shared memory into 16-byte row stores.
-// TMEM holds two accumulators of BN columns (BN <= 256), so the epilogue of one tile
-// overlaps the main loop of the next.
-// Work items are (group, feature tile, K slice, token tile), enumerated from the
-// device-side row offsets with no host synchronisation; empty groups produce no items
-// (no padding to a fixed capacity).  The plain (fp32-out) GEMM can split K into
-// `ksplit` slices whose partial sums land in separate buffers `split_stride` apart,
-// for shapes with too few tiles to cover the SMs; the consumer adds them in a fixed
-// order, so results stay deterministic.  Every wait is bounded (globaltimer): on
-// expiry the kernel records MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain,
-// frees TMEM and returns.
+// TMEM holds two accumulators of BN columns, so one tile's epilogue overlaps the next
+// tile's main loop.  Barrier set-up and TMEM allocation run before the kernel waits on
+// the previous kernel in the stream (programmatic dependent launch).
+//
+// Work items are (group, feature tile, K slice, token tile), enumerated on the device
+// from the row offsets with no host synchronisation; empty groups produce no items (no
+// padding to a fixed capacity).  The plain GEMM can split K into `ksplit` slices whose
+// partial sums land in separate buffers `split_stride` apart, for shapes with too few
+// tiles to cover the SMs; the consumer adds them in a fixed order, so results stay
+// deterministic.  Every wait is bounded (globaltimer): on expiry the kernel records
+// MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

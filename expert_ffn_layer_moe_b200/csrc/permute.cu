@@ -177,23 +177,28 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// x_perm[token_to_row[t,j]] = x[t] for every assignment with a valid row; one warp
-// per token (grid-stride), each lane 16-byte vectors, four loads in flight.
+// x_perm[token_to_row[t,j]] = x[t] for every assignment with a valid row.  A warp's
+// unit of work is 2 KB of one token's row (128 16-byte vectors, four per lane, all in
+// flight at once), read once and written to the token's k rows; units run grid-stride.
+constexpr int kScatterVec = 128;
 __global__ void __launch_bounds__(kThreads)
     scatter_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ token_to_row, int64_t N, int k,
                         int H, uint16_t *__restrict__ x_perm)
 {
     pdl_entry();
     const int nvec = H / 8;
+    const int chunks = (nvec + kScatterVec - 1) / kScatterVec;
     const int64_t warp_global = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
     const int lane = threadIdx.x & 31;
-    for (int64_t t = warp_global; t < N; t += nwarps) {
+    for (int64_t unit = warp_global; unit < N * chunks; unit += nwarps) {
+        const int64_t t = unit / chunks;
+        const int v0 = (int)(unit % chunks) * kScatterVec + lane;
         int rows[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) rows[j] = j < k ? token_to_row[t * k + j] : -1;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
-        for (int v0 = lane; v0 < nvec; v0 += 128) {
+        {
             uint4 buf[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
@@ -233,7 +238,8 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
                            E, (const int32_t *)scratch, row_to_token, token_to_row);
         if (e != cudaSuccess) return e;
     }
-    const int64_t want = (N + kWarps - 1) / kWarps;
+    const int64_t units = N * ((H / 8 + kScatterVec - 1) / kScatterVec);
+    const int64_t want = (units + kWarps - 1) / kWarps;
     const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
     return launch_pdl(scatter_rows_kernel, dim3(gblocks), dim3(kThreads), 0, s, x, (const int32_t *)token_to_row,
                       N, k, H, x_perm);
