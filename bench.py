@@ -37,22 +37,6 @@ from expert_ffn_layer_moe_b200.inputs import CONFIGS, make_inputs  # noqa: E402
 METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PHASES = ("route", "permute", "gemm13", "gemm2", "shared", "combine")
-SMALL_DISPATCH_R = 2048  # assignments up to which the dispatch is one single-block launch
-
-
-def launches_per_step(cfg):
-    """Kernels of this library launched by one layer forward (the layer's router
-    takes its tensor-core path for N >= 256 with N*E >= 32768: split, GEMM, top-k;
-    its expert-split path for E > 16: logits, top-k; else one kernel)."""
-    if cfg.N >= 256 and cfg.N * cfg.E >= 32768:
-        router = 3
-    elif cfg.E > 16:
-        router = 2
-    else:
-        router = 1
-    permute = 2 if cfg.R <= SMALL_DISPATCH_R else 4  # dispatch (1 or 3 kernels) + row gather
-    shared = 2 if cfg.Is > 0 else 0
-    return router + permute + 2 + shared + 1  # + W1/W3 and W2 GEMMs, shared, combine
 
 
 def peaks():
@@ -119,52 +103,94 @@ def kernel_traffic(kernel, workload):
     return None
 
 
-class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+CLOCK_SAMPLER = r"""
+import sys, time
+import pynvml as N
+bus, period = sys.argv[1], float(sys.argv[2])
+N.nvmlInit()
+try:
+    h = N.nvmlDeviceGetHandleByPciBusId(bus)
+except Exception:
+    h = N.nvmlDeviceGetHandleByIndex(int(sys.argv[3]))
+mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+get_reasons = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or N.nvmlDeviceGetCurrentClocksThrottleReasons
+print("ready", flush=True)
+while True:
+    t = time.time()
+    print(t, N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM), mx, N.nvmlDeviceGetPowerUsage(h), get_reasons(h), flush=True)
+    time.sleep(max(0.0, period - (time.time() - t)))
+"""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+class ClockSampler:
+    """SM clock, power and clock-event (throttle) reasons sampled through NVML every
+    2 ms by a helper process (no GIL shared with the launching thread), kept for the
+    samples whose host timestamps fall inside the timed region [enter, exit]."""
+
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+    PERIOD_S = 0.002
 
     def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
-        self.path = None
+        self.t0 = self.t1 = None
+        self.lines = []
 
-    def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+    def start(self):
+        """Start the helper before the region (it needs a moment to initialise NVML)."""
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except (OSError, FileNotFoundError):
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        except (AttributeError, RuntimeError):
+            bus = ""
+        try:
+            self.proc = subprocess.Popen([sys.executable, "-c", CLOCK_SAMPLER, bus, str(self.PERIOD_S),
+                                          str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            if self.proc.stdout.readline().strip() != "ready":
+                self.stop()
+        except OSError:
             self.proc = None
         return self
 
+    def __enter__(self):
+        self.t0 = time.time()
+        return self
+
     def __exit__(self, *a):
+        self.t1 = time.time()
+        self.stop()
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                out, _ = self.proc.communicate(timeout=5)
+                self.lines = out.splitlines()
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            self.proc = None
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
+        rows = []
+        for l in self.lines:
+            f = l.split()
+            if len(f) == 5:
+                try:
+                    rows.append((float(f[0]), float(f[1]), float(f[2]), float(f[3]) / 1e3, int(f[4])))
+                except ValueError:
+                    pass
+        if not rows or self.t0 is None:
             return None
-        rows = [l.split(",") for l in open(self.path).read().splitlines() if l.strip()]
-        os.unlink(self.path)
-        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        inside = [r for r in rows if self.t0 <= r[0] <= self.t1]
+        if not inside:  # region shorter than one period: the first sample after it began
+            later = [r for r in rows if r[0] >= self.t0]
+            inside = later[:1] or rows[-1:]
+        reasons = sorted(n for n, b in self.REASON_BITS.items() if any(r[4] & b for r in inside))
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "power_w_max": max(r[3] for r in inside), "reasons": reasons, "samples": len(inside),
+                "sampler": f"NVML every {self.PERIOD_S * 1e3:.0f} ms, samples inside the timed region"}
 
 
 def dist_setup(args):
@@ -270,11 +296,14 @@ def run_ours(args, cfg, world, rank, local):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    clk = ClockSampler(local).start()
+    with clk:
+        n0 = moe.moe_kernel_launches()
         start.record(stream)
         for i in range(args.steps):
             step()
         end.record(stream)
+        launches = moe.moe_kernel_launches() - n0
         torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = start.elapsed_time(end)
@@ -334,6 +363,20 @@ def run_ours(args, cfg, world, rank, local):
     lbytes = layer_bytes(cfg, touched)
     floor_s = max(flops / (pk["bf16_tflops"] * 1e12), lbytes / (hbm * 1e9))
     workload = cfg.name
+    # the W1/W3 kernel's bound: weight streaming (HBM) at decode sizes, the tensor cores
+    # once the token tiles are long enough (its FLOPs at the bf16 peak outlast its bytes)
+    g13_flops = 4 * cfg.R * H * I
+    if g13_flops / (pk["bf16_tflops"] * 1e12) > g13_b / (hbm * 1e9):
+        roofline = {"bound": "tensor", "achieved": g13_flops / g13_s / 1e12, "peak": pk["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": g13_flops / g13_s / 1e12 / pk["bf16_tflops"],
+                    "alg_flops_per_launch": g13_flops}
+        if "bf16_tflops_sustained" in pk:
+            roofline["frac_of_sustained_peak"] = g13_flops / g13_s / 1e12 / pk["bf16_tflops_sustained"]
+    else:
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                    "alg_bytes_per_launch": g13_b}
+    roofline.update({"kernel": "grouped_gemm SwiGLU W1/W3 (gemm13)", "peak_kind": pk_kind,
+                     "traffic": kernel_traffic("gemm13", workload), "avg_launch_ms": phase_ms["gemm13"]})
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
@@ -343,10 +386,7 @@ def run_ours(args, cfg, world, rank, local):
                    "l2": f"inputs larger than L2: {touched} touched experts' weights "
                          f"({touched * 3 * H * I * 2 / 1e9:.2f} GB) streamed from HBM every step",
                    "touched_experts": touched, "max_expert_rows": max_load},
-        "roofline": {"bound": "hbm", "kernel": "grouped_gemm SwiGLU W1/W3 (gemm13)", "achieved": achieved,
-                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "peak_kind": pk_kind,
-                     "traffic": kernel_traffic("gemm13", workload), "alg_bytes_per_launch": g13_b,
-                     "avg_launch_ms": phase_ms["gemm13"]},
+        "roofline": roofline,
         "layer": {"tflops": flops / step_s / 1e12, "alg_bytes": lbytes, "gb_s": lbytes / step_s / 1e9,
                   "roofline_floor_us": floor_s * 1e6, "roofline_frac": floor_s / step_s,
                   "useful_flop_fraction_k_over_E": k / E},
@@ -355,7 +395,8 @@ def run_ours(args, cfg, world, rank, local):
                          "gemm2_frac_hbm": gemm2_bytes(cfg, touched) / g2_s / 1e9 / hbm},
         "phase_ms": phase_ms,
         "phase_ms_note": "mean per-phase CUDA-event times from a second timed pass with events between phases",
-        "gpu_launches": args.steps * launches_per_step(cfg),
+        "gpu_launches": launches,
+        "gpu_launches_note": "the library's own host-side count of its kernel launches over the timed steps",
         "e2e": e2e,
     }
     clk_sum = clk.summary()

@@ -7,11 +7,20 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/moe.h"
 #include "internal.h"
+
+namespace moe {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+uint64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace moe
 
 namespace {
 
@@ -153,6 +162,8 @@ const char *moe_status_string(moe_status_t status)
 const char *moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 int moe_device_sm_count(void) { return moe::device_sm_count(); }
+
+uint64_t moe_kernel_launches(void) { return moe::launches_so_far(); }
 
 size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is)
 {

@@ -711,6 +711,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
                              ksplit, a.split_stride, a.dev_err);
     if (err != cudaSuccess) return err;
+    count_launch();
     return cudaGetLastError();
 }
 

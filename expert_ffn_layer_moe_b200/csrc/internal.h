@@ -7,6 +7,11 @@
 
 namespace moe {
 
+// Host-side count of kernels this library launched (every launch goes through
+// launch_pdl or the grouped GEMM's launcher, which call this on success).
+void count_launch();
+uint64_t launches_so_far();
+
 // Launch with programmatic stream serialization (the kernel calls pdl_entry/pdl_wait
 // before its first global memory access).
 template <typename... KArgs, typename... Args>
@@ -22,13 +27,15 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+    if (e == cudaSuccess) count_launch();
+    return e;
 }
 
 // Router: logits (fp32), top-k indices and renormalised weights.  `ws` (nullable)
-// of at least router_ws_bytes(N, H, E) bytes enables the tensor-core and
-// expert-split paths.
-enum class RouterPath { kFused, kSplitE, kTensor };
+// of at least router_ws_bytes(N, H, E) bytes enables the tensor-core path and
+// the split path's slices of H; a logits buffer alone enables the split path.
+enum class RouterPath { kFused, kSplit, kTensor };
 RouterPath router_path(int64_t N, int E, bool have_logits_buffer, bool have_ws);
 size_t router_ws_bytes(int64_t N, int H, int E);
 cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *bias, int64_t N,

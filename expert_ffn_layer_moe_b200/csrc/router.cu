@@ -9,12 +9,15 @@
 //                renormalised over the picks equals the softmax of the picked logits)
 //
 // Three paths, chosen by shape (router_path):
-//  * kFused (E <= 16, or no buffer for logits): one kernel -- a block per tile of TT
+//  * kFused (no buffer for logits at all): one kernel -- a block per tile of TT
 //    tokens, 8 warps splitting H (warp w takes 64-column chunks w, w+8, ...; a lane two
 //    adjacent columns), all experts in passes of 8, then the top-k in the same block;
-//  * kSplitE (E > 16, small N): the logits kernel's grid also splits the experts into
-//    slices of 8, so a batch of a few tokens still spreads W_gate over many SMs; a
-//    second kernel does the top-k;
+//  * kSplit (small N): the logits kernel's grid splits the tokens into tiles of up to
+//    8, the experts into slices of 8 and H into Z slices, so that a batch of a few
+//    tokens still spreads the W_gate read over every SM; the top-k kernel adds the Z
+//    partial sums in slice order.  Where one slice of H is all it would use and the
+//    experts fit two slices of 8, the fused kernel runs instead (same blocks, one
+//    launch);
 //  * kTensor (large N x E): the logits are a GEMM on the tcgen05 tensor cores.  W_gate
 //    is split into three bf16 terms hi + mid + lo (each the bf16 rounding of what the
 //    previous terms left; the remainder is below 2^-26 |w|), so x (bf16) times each
@@ -35,11 +38,11 @@ constexpr int kMaxE = 256;
 constexpr int kMaxK = 8;
 
 // Partial logits of TT tokens x one 8-expert slice [e0, e0+ne) over this warp's
-// share of H, reduced over the warp's lanes (every lane ends with the sums).
+// share of the columns [h_begin, h_end) of H, per lane (warp_sum_store adds the lanes).
 template <int TT>
 __device__ __forceinline__ void logits_slice(const uint16_t *__restrict__ x, const float *__restrict__ W_gate,
-                                             int64_t t0, int nt, int H, int E, int e0, int ne, int warp, int lane,
-                                             float (&acc)[TT][kEC])
+                                             int64_t t0, int nt, int H, int h_begin, int h_end, int E, int e0,
+                                             int ne, int warp, int lane, float (&acc)[TT][kEC])
 {
 #pragma unroll
     for (int t = 0; t < TT; ++t)
@@ -48,7 +51,7 @@ __device__ __forceinline__ void logits_slice(const uint16_t *__restrict__ x, con
     // full 8-expert slices of rows whose start is 16-byte aligned load as float4
     const bool vec = ne == kEC && (E & 3) == 0;
 #pragma unroll 4
-    for (int c = warp * kChunk; c < H; c += kWarps * kChunk) {
+    for (int c = h_begin + warp * kChunk; c < h_end; c += kWarps * kChunk) {
         const int h = c + 2 * lane;
         float2 xv[TT];
 #pragma unroll
@@ -78,12 +81,51 @@ __device__ __forceinline__ void logits_slice(const uint16_t *__restrict__ x, con
 #pragma unroll
             for (int t = 0; t < TT; ++t) acc[t][j] = fmaf(xv[t].y, b[j], fmaf(xv[t].x, a[j], acc[t][j]));
     }
+}
+
+// Sum each of the V = TT*8 per-lane values acc[t][j] over the warp's 32 lanes and
+// store the sums to out[t * tstride + j] (j < ne).  A reduce-scatter: at each step a
+// lane keeps one half of its values, sends the other half to the lane `o` apart and
+// adds what it receives, so the sums end up spread over the lanes after V - V/32
+// shuffles (instead of 5 V for a butterfly on every value); once a lane holds one
+// value the remaining steps are a butterfly.  The additions run in a fixed order.
+template <int TT>
+__device__ __forceinline__ void warp_sum_store(const float (&acc)[TT][kEC], int lane, float *out, int tstride,
+                                               int ne)
+{
+    constexpr int V = TT * kEC;
+    float v[V];
 #pragma unroll
-    for (int t = 0; t < TT; ++t)
+    for (int f = 0; f < V; ++f) v[f] = acc[f / kEC][f % kEC];
+    int base = 0;  // index of v[0] among the V values after the halving steps
 #pragma unroll
-        for (int j = 0; j < kEC; ++j)
+    for (int st = 0; st < 5; ++st) {
+        const int o = 16 >> st;
+        const int S = V >> st;  // values per lane before this step (a constant once unrolled)
+        if (S > 1) {
+            const int h = S >> 1;
+            const bool up = (lane & o) != 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc[t][j] += __shfl_xor_sync(0xffffffffu, acc[t][j], o);
+            for (int i = 0; i < h; ++i) {
+                const float send = up ? v[i] : v[i + h];
+                const float keep = up ? v[i + h] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+            if (up) base += h;
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+        }
+    }
+    constexpr int kLeft = V >= 32 ? V / 32 : 1;           // sums held per lane
+    constexpr int kSame = V >= 32 ? 0 : (32 / V) - 1;    // lanes holding copies of a sum
+    if ((lane & kSame) == 0) {
+#pragma unroll
+        for (int r = 0; r < kLeft; ++r) {
+            const int f = base + r;
+            const int t = f / kEC, j = f % kEC;
+            if (j < ne) out[t * tstride + j] = v[r];
+        }
+    }
 }
 
 // Top-k of one token's E logits (in `row`) on one warp; lane 0 writes the picks
@@ -164,14 +206,8 @@ __global__ void __launch_bounds__(kThreads)
     for (int e0 = 0; e0 < E; e0 += kEC) {
         const int ne = min(kEC, E - e0);
         float acc[TT][kEC];
-        logits_slice<TT>(x, W_gate, t0, nt, H, E, e0, ne, warp, lane, acc);
-        if (lane == 0) {
-#pragma unroll
-            for (int t = 0; t < TT; ++t)
-#pragma unroll
-                for (int j = 0; j < kEC; ++j)
-                    if (j < ne) partial[(warp * TT + t) * E + e0 + j] = acc[t][j];
-        }
+        logits_slice<TT>(x, W_gate, t0, nt, H, 0, H, E, e0, ne, warp, lane, acc);
+        warp_sum_store<TT>(acc, lane, partial + warp * TT * E + e0, E, ne);
     }
     __syncthreads();
     for (int i = threadIdx.x; i < nt * E; i += kThreads) {  // fixed-order sum over warps
@@ -188,11 +224,14 @@ __global__ void __launch_bounds__(kThreads)
         topk_warp(s_logit + t * E, E, k, lane, topk_idx + (t0 + t) * k, topk_w + (t0 + t) * k);
 }
 
-// kSplitE: logits of TT tokens x one 8-expert slice (blockIdx.y) per block.
+// kSplit: partial logits of TT tokens x one 8-expert slice (blockIdx.y) over one
+// slice of H (blockIdx.z, columns [z*hz, z*hz + hz)) per block, summed over the
+// block's warps in warp order, stored as part[z][t][e].  With one H slice the bias is
+// added here and `part` holds the logits.
 template <int TT>
 __global__ void __launch_bounds__(kThreads)
-    router_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ W_gate,
-                         const float *__restrict__ bias, int64_t N, int H, int E, float *__restrict__ logits)
+    router_partial_kernel(const uint16_t *__restrict__ x, const float *__restrict__ W_gate,
+                          const float *__restrict__ bias, int64_t N, int H, int E, int hz, float *__restrict__ part)
 {
     __shared__ float partial[kWarps][TT][kEC];
     pdl_entry();
@@ -201,14 +240,10 @@ __global__ void __launch_bounds__(kThreads)
     const int nt = (N - t0) < TT ? (int)(N - t0) : TT;
     const int e0 = blockIdx.y * kEC;
     const int ne = min(kEC, E - e0);
+    const int h0 = (int)blockIdx.z * hz;
     float acc[TT][kEC];
-    logits_slice<TT>(x, W_gate, t0, nt, H, E, e0, ne, warp, lane, acc);
-    if (lane == 0) {
-#pragma unroll
-        for (int t = 0; t < TT; ++t)
-#pragma unroll
-            for (int j = 0; j < kEC; ++j) partial[warp][t][j] = acc[t][j];
-    }
+    logits_slice<TT>(x, W_gate, t0, nt, H, h0, min(H, h0 + hz), E, e0, ne, warp, lane, acc);
+    warp_sum_store<TT>(acc, lane, &partial[warp][0][0], kEC, kEC);
     __syncthreads();
     if (threadIdx.x < nt * kEC) {
         const int t = threadIdx.x / kEC, j = threadIdx.x % kEC;
@@ -216,19 +251,23 @@ __global__ void __launch_bounds__(kThreads)
             float v = 0.f;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) v += partial[w][t][j];
-            if (bias) v += bias[e0 + j];
-            logits[(t0 + t) * E + e0 + j] = v;
+            if (bias && gridDim.z == 1) v += bias[e0 + j];
+            part[((int64_t)blockIdx.z * N + t0 + t) * E + e0 + j] = v;
         }
     }
 }
 
-// Top-k, one warp per token.  parts == 1: `lin` holds the logits [N,E].  parts == 3:
-// `lin` holds the three partial logits [N,3E] of the tensor path (hi, mid, lo terms
-// of W_gate); they are summed (+ bias), written to `logits`, then ranked.
+// Top-k, one warp per token.  `lin` holds P partial logits of each token: part p of
+// token t, expert e at lin[p * pstride + t * tstride + e] -- the P slices of H of the
+// split path ([P][N][E]) or the hi, mid, lo terms of the tensor path ([N][3E]).  They
+// are added in part order (+ bias), written to `logits` when it is given, then ranked.
+// With P == 1 and no bias `lin` already holds the logits.  P is a template argument so
+// that the loads of one expert's parts, and of consecutive experts, issue together.
+template <int P>
 __global__ void __launch_bounds__(kThreads)
-    router_topk_kernel(const float *__restrict__ lin, int parts, const float *__restrict__ bias, int64_t N, int E,
-                       int k, float *__restrict__ logits, int32_t *__restrict__ topk_idx,
-                       float *__restrict__ topk_w)
+    router_topk_kernel(const float *__restrict__ lin, int64_t pstride, int64_t tstride,
+                       const float *__restrict__ bias, int64_t N, int E, int k, float *__restrict__ logits,
+                       int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
 {
     __shared__ float row[kWarps][kMaxE];
     pdl_entry();
@@ -236,19 +275,27 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t t = (int64_t)blockIdx.x * kWarps + warp;
     if (t >= N) return;  // the whole warp leaves; no block-wide barrier below
     for (int e = lane; e < E; e += 32) {
-        float v;
-        if (parts == 3) {
-            const float *p = lin + t * 3 * E;
-            v = (p[e] + p[E + e]) + p[2 * E + e];
-            if (bias) v += bias[e];
-            if (logits) logits[t * E + e] = v;
-        } else {
-            v = lin[t * E + e];
-        }
+        const float *p = lin + t * tstride + e;
+        float part[P];
+#pragma unroll
+        for (int i = 0; i < P; ++i) part[i] = p[i * pstride];
+        float v = part[0];
+#pragma unroll
+        for (int i = 1; i < P; ++i) v += part[i];
+        if (bias) v += bias[e];
+        if (logits) logits[t * E + e] = v;
         row[warp][e] = v;
     }
     __syncwarp();
     topk_warp(row[warp], E, k, lane, topk_idx + t * k, topk_w + t * k);
+}
+
+template <int P>
+cudaError_t launch_topk(const float *lin, int64_t pstride, int64_t tstride, const float *bias, int64_t N, int E,
+                        int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
+{
+    return launch_pdl(router_topk_kernel<P>, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, lin,
+                      pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
 }
 
 // kTensor: W_gate [H,E] fp32 -> three bf16 terms, stacked K-major as [3E, H]:
@@ -297,25 +344,67 @@ cudaError_t launch_fused(const uint16_t *x, const float *W_gate, const float *bi
 }
 
 template <int TT>
-cudaError_t launch_split_e(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
-                           int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
+cudaError_t launch_split(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E, int k,
+                         int Z, float *part, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
 {
-    const dim3 grid((unsigned)((N + TT - 1) / TT), (unsigned)((E + kEC - 1) / kEC));
-    cudaError_t e = launch_pdl(router_logits_kernel<TT>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H, E, logits);
+    const int hz = (H / Z / kChunk) * kChunk;  // Z divides H / 64 (split_shape)
+    const dim3 grid((unsigned)((N + TT - 1) / TT), (unsigned)((E + kEC - 1) / kEC), (unsigned)Z);
+    cudaError_t e = launch_pdl(router_partial_kernel<TT>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H, E, hz,
+                               part);
     if (e != cudaSuccess) return e;
-    return launch_pdl(router_topk_kernel, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s,
-                      (const float *)logits, 1, (const float *)nullptr, N, E, k, (float *)nullptr, topk_idx, topk_w);
+    const int64_t ps = N * E;
+    switch (Z) {  // Z == 1: `part` holds the logits, bias included
+        case 1: return launch_topk<1>(part, ps, E, nullptr, N, E, k, nullptr, topk_idx, topk_w, s);
+        case 2: return launch_topk<2>(part, ps, E, bias, N, E, k, logits, topk_idx, topk_w, s);
+        case 4: return launch_topk<4>(part, ps, E, bias, N, E, k, logits, topk_idx, topk_w, s);
+        case 8: return launch_topk<8>(part, ps, E, bias, N, E, k, logits, topk_idx, topk_w, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
-// Tokens per block for the CUDA-core paths: keep about two blocks per SM (times the
-// expert slices) before sharing W_gate reads between tokens.
-int tokens_per_block(int64_t N, int64_t slices)
+// Tokens per block for the fused path: keep about two blocks per SM before sharing
+// W_gate reads between tokens.
+int tokens_per_block(int64_t N)
 {
     const int64_t want = 2 * (int64_t)device_sm_count();
-    if (N * slices >= 8 * want) return 8;
-    if (N * slices >= 4 * want) return 4;
-    if (N * slices >= 2 * want) return 2;
+    if (N >= 8 * want) return 8;
+    if (N >= 4 * want) return 4;
+    if (N >= 2 * want) return 2;
     return 1;
+}
+
+// Shape of the split path: the most tokens per block (up to 4, each W_gate load then
+// serves them all; 8 would take more than 128 registers a thread and halve the blocks
+// an SM holds) for which the blocks, times at most `zmax` slices of H, still come to
+// about two per SM; then the fewest H slices that get there.  The slice count is a
+// power of two up to 8 that divides H / 64 and leaves every warp at least one 64-column
+// chunk.
+void split_shape(int64_t N, int H, int E, int64_t zcap, int *tt, int *z)
+{
+    const int64_t want = 2 * (int64_t)device_sm_count();
+    const int64_t slices = (E + kEC - 1) / kEC;
+    const int nch = H / kChunk;
+    int zmax = 1;
+    for (int c = 2; c <= 8; c *= 2)
+        if (nch % c == 0 && nch / c >= kWarps && c <= zcap) zmax = c;
+    *tt = 1;
+    for (int c = 4; c > 1; c >>= 1)
+        if (N >= c && ((N + c - 1) / c) * slices * zmax >= want) { *tt = c; break; }
+    const int64_t blocks = ((N + *tt - 1) / *tt) * slices;
+    int zz = 1;
+    while (zz < zmax && blocks * zz < want) zz *= 2;
+    *z = zz;
+}
+
+cudaError_t launch_fused_for(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
+                             int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
+{
+    switch (tokens_per_block(N)) {
+        case 8: return launch_fused<8>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+        case 4: return launch_fused<4>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+        case 2: return launch_fused<2>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+        default: return launch_fused<1>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+    }
 }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -325,7 +414,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 RouterPath router_path(int64_t N, int E, bool have_logits_buffer, bool have_ws)
 {
     if (have_ws && N >= 256 && N * (int64_t)E >= 32768) return RouterPath::kTensor;
-    if (E > 16 && (have_logits_buffer || have_ws)) return RouterPath::kSplitE;
+    if (have_logits_buffer || have_ws) return RouterPath::kSplit;
     return RouterPath::kFused;
 }
 
@@ -357,23 +446,27 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
         g.rows_single = (int)N; g.K = H; g.Nout = 3 * E; g.out = parts; g.dev_err = dev_err; g.token_tile = 128;
         e = launch_gemm2(g, s);
         if (e != cudaSuccess) return e;
-        return launch_pdl(router_topk_kernel, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s,
-                          (const float *)parts, 3, bias, N, E, k, lbuf, topk_idx, topk_w);
+        return launch_topk<3>(parts, (int64_t)E, (int64_t)3 * E, bias, N, E, k, lbuf, topk_idx, topk_w, s);
     }
-    if (path == RouterPath::kSplitE) {
-        switch (tokens_per_block(N, (E + kEC - 1) / kEC)) {
-            case 8: return launch_split_e<8>(x, W_gate, bias, N, H, E, k, lbuf, topk_idx, topk_w, s);
-            case 4: return launch_split_e<4>(x, W_gate, bias, N, H, E, k, lbuf, topk_idx, topk_w, s);
-            case 2: return launch_split_e<2>(x, W_gate, bias, N, H, E, k, lbuf, topk_idx, topk_w, s);
-            default: return launch_split_e<1>(x, W_gate, bias, N, H, E, k, lbuf, topk_idx, topk_w, s);
+    if (path == RouterPath::kSplit) {
+        // the H-slice partials go to the scratch (its first two regions), else the
+        // caller's logits buffer holds the one slice
+        float *part = have_ws ? reinterpret_cast<float *>(w8) : lbuf;
+        const int64_t zcap = have_ws ? (int64_t)((split_bytes + parts_bytes) / ((size_t)N * E * 4)) : 1;
+        int tt, z;
+        split_shape(N, H, E, zcap, &tt, &z);
+        if (z == 1 && E <= 2 * kEC) {
+            // nothing to gain from slicing: the one-kernel path runs the same blocks
+            return launch_fused_for(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+        }
+        if (z == 1) part = lbuf;
+        switch (tt) {
+            case 4: return launch_split<4>(x, W_gate, bias, N, H, E, k, z, part, lbuf, topk_idx, topk_w, s);
+            case 2: return launch_split<2>(x, W_gate, bias, N, H, E, k, z, part, lbuf, topk_idx, topk_w, s);
+            default: return launch_split<1>(x, W_gate, bias, N, H, E, k, z, part, lbuf, topk_idx, topk_w, s);
         }
     }
-    switch (tokens_per_block(N, 1)) {
-        case 8: return launch_fused<8>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
-        case 4: return launch_fused<4>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
-        case 2: return launch_fused<2>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
-        default: return launch_fused<1>(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
-    }
+    return launch_fused_for(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
 }
 
 }  // namespace moe

@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
         L.moe_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         L.moe_device_sm_count.argtypes = []
         L.moe_device_sm_count.restype = c_int
+        L.moe_kernel_launches.argtypes = []
+        L.moe_kernel_launches.restype = ctypes.c_uint64
         for fn in ("moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
                    "moe_layer_forward_ex", "moe_get_device_error"):
             getattr(L, fn).restype = c_int
@@ -93,6 +95,11 @@ def moe_workspace_bytes(N: int, H: int, I: int, E: int, k: int, Is: int = 0) -> 
 
 def moe_device_sm_count() -> int:
     return int(lib().moe_device_sm_count())
+
+
+def moe_kernel_launches() -> int:
+    """Kernels the library has launched in this process (host-side count)."""
+    return int(lib().moe_kernel_launches())
 
 
 def moe_route(x, W_gate, k, bias=None, logits=None, topk_idx=None, topk_w=None, ws=None, stream=None,

@@ -93,9 +93,11 @@ MOE_API size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is
  *                                  moe_workspace_bytes(N,H,64,E,k,0) bytes, large batches
  *                                  compute the logits on the tensor cores (W_gate split
  *                                  into three bf16 terms, exact products, fp32
- *                                  accumulation) and small batches with many experts
- *                                  spread the experts over more blocks; with NULL a
- *                                  single fp32 CUDA-core kernel runs.
+ *                                  accumulation) and small batches split H, the
+ *                                  experts and the tokens over every SM (partial sums
+ *                                  added in a fixed order); with NULL ws and a logits
+ *                                  buffer the split runs without slices of H; with
+ *                                  neither, a single fp32 CUDA-core kernel runs.
  * The logits are fp32-grade on every path; which path ran can change their last bits,
  * and the expert choice is taken on the logits this call produced.
  * NaN logits are unsupported input (the pick among them is unspecified).
@@ -231,6 +233,13 @@ MOE_API moe_status_t moe_get_device_error(void *stream, int32_t *code);
 
 /* Number of streaming multiprocessors the grouped GEMM sizes its persistent grid to. */
 MOE_API int moe_device_sm_count(void);
+
+/*
+ * Kernels this library has launched in this process so far, counted on the host
+ * at each successful launch (all threads, all devices; never reset).  The
+ * difference across a region is the number of the library's kernels it ran.
+ */
+MOE_API uint64_t moe_kernel_launches(void);
 
 #ifdef __cplusplus
 }

@@ -82,27 +82,77 @@ def test_route_matches_oracle():
     assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
 
 
-# (N, E, k, workspace): the one-kernel path (no workspace, or E <= 16), the
-# expert-split path (E > 16, small N) and the tensor-core path (N >= 256, N*E >= 32768)
-ROUTE_CASES = [(203, 8, 2, True), (203, 160, 6, False), (203, 160, 6, True), (203, 128, 8, True),
-               (203, 37, 3, True), (203, 1, 1, True), (203, 256, 8, True), (1, 128, 8, True),
-               (1000, 128, 8, True), (512, 160, 6, True), (4096, 8, 2, True), (300, 256, 8, True),
-               (777, 37, 3, True)]
+# (N, H, E, k, workspace, logits buffer).  Paths: no workspace and no logits buffer ->
+# the fused one-kernel path; a logits buffer alone -> the split path with one slice of
+# H; a workspace -> the split path with up to H/512 slices of H (small N) or the
+# tensor-core path (N >= 256 and N*E >= 32768).  Where the split would use one slice
+# and E <= 16 the fused kernel runs instead (e.g. H=512, E=8).
+ROUTE_CASES = [
+    # fused
+    (203, 512, 8, 2, False, False), (203, 512, 160, 6, False, False), (1, 2048, 128, 8, False, False),
+    (37, 768, 37, 3, False, False),
+    # split, one slice of H (logits buffer, no workspace)
+    (203, 512, 160, 6, False, True), (1, 2048, 128, 8, False, True), (203, 512, 8, 2, False, True),
+    # split with slices of H
+    (203, 512, 8, 2, True, True), (203, 512, 128, 8, True, True), (203, 512, 37, 3, True, True),
+    (203, 512, 1, 1, True, True), (203, 512, 256, 8, True, True), (1, 2048, 128, 8, True, True),
+    (16, 2048, 128, 8, True, True), (156, 6144, 8, 2, True, True), (5, 4096, 160, 6, True, True),
+    (3, 1536, 256, 8, True, False), (128, 2048, 128, 8, True, False),
+    # tensor cores
+    (1000, 512, 128, 8, True, True), (512, 512, 160, 6, True, True), (4096, 512, 8, 2, True, True),
+    (300, 512, 256, 8, True, True), (777, 512, 37, 3, True, True), (1024, 2048, 128, 8, True, False),
+]
 
 
-@pytest.mark.parametrize("N,E,k,use_ws", ROUTE_CASES)
-def test_route_shapes_and_bias(N, E, k, use_ws):
-    cfg = MoEConfig("route", N=N, H=512, I=64, E=E, k=k)
+def check_picks_without_logits(cfg, t, idx, w):
+    """Routing returned without its logits: the picks must equal the top-k of the
+    float64 logits wherever that top-k is decided by more than the fp32 error bound
+    (the (k+1)-th logit and each consecutive pick apart by more than it); the weights
+    match the float64 softmax of the picks."""
+    l64 = oracle.router_logits(host(t["x"]), host(t["W_gate"]), host(t["bias"]))
+    scale = np.abs(dec(host(t["x"]))) @ np.abs(host(t["W_gate"]).astype(np.float64))
+    bound = 2.0 ** -20 * scale.max(axis=1) + 1e-6
+    order = np.lexsort((np.broadcast_to(np.arange(cfg.E), l64.shape), -l64), axis=1)
+    k = cfg.k
+    top = np.take_along_axis(l64, order[:, : min(k + 1, cfg.E)], axis=1)
+    gaps = -np.diff(top, axis=1)
+    clear = (gaps > 2 * bound[:, None]).all(axis=1)
+    got = host(idx)
+    assert clear.mean() > 0.5, "inputs too tied to check"
+    assert np.array_equal(got[clear], order[clear, :k])
+    picked = np.take_along_axis(l64, got.astype(np.int64), axis=1)
+    ref_w = np.exp(picked - picked[:, :1])
+    ref_w /= ref_w.sum(axis=1, keepdims=True)
+    assert np.allclose(host(w), ref_w, rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("N,H,E,k,use_ws,with_logits", ROUTE_CASES)
+def test_route_shapes_and_bias(N, H, E, k, use_ws, with_logits):
+    cfg = MoEConfig("route", N=N, H=H, I=64, E=E, k=k)
     t = cuda_inputs(cfg, seed=4)
     bias = torch.linspace(-0.5, 0.5, E, device="cuda")
-    logits = torch.empty((cfg.N, E), dtype=torch.float32, device="cuda")
+    logits = torch.empty((cfg.N, E), dtype=torch.float32, device="cuda") if with_logits else None
     idx, w, _ = moe.moe_route(t["x"], t["W_gate"], k, bias=bias, logits=logits, use_workspace=use_ws)
     torch.cuda.synchronize()
     t["bias"] = bias
-    check_logits(cfg, t, logits)
-    ref_idx, ref_w = oracle.topk(host(logits), k)
-    assert np.array_equal(host(idx), ref_idx)
-    assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
+    if with_logits:
+        check_logits(cfg, t, logits)
+        ref_idx, ref_w = oracle.topk(host(logits), k)
+        assert np.array_equal(host(idx), ref_idx)
+        assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
+    else:
+        check_picks_without_logits(cfg, t, idx, w)
+
+
+def test_kernel_launch_counter_counts_a_layer():
+    """The host-side launch count moves by the kernels one layer call runs: the
+    fused router, the single-block dispatch and the row scatter, the two grouped
+    GEMMs and the combine at the tiny shape."""
+    cfg = CONFIGS["tiny"]
+    t = cuda_inputs(cfg)
+    n0 = moe.moe_kernel_launches()
+    run_layer(cfg, t)
+    assert moe.moe_kernel_launches() - n0 == 6
 
 
 def test_route_paths_agree_on_logits():
