@@ -12,7 +12,11 @@ argsort and the pages' 156-token, 8-expert, top-2 worked example (mean 39 rows
 per expert); the expert FFN against a dense float64 matrix statement; combine
 against dense-masked evaluation (every expert on every token); the E=1, k=1
 reduction to a dense SwiGLU FFN; a hand-derived tiny layer; relabelling and
-scaling invariants.  No function is left unpinned.
+scaling invariants; e4m3 decoding against the format's own table of special
+values and every code, encoding against nearest-value search over all codes with
+ties to the even code, the quantizer's per-row scale and error bounds, and the
+fp8 layer against the bf16 layer on weights that the quantizer represents
+exactly.  No function is left unpinned.
 """
 from __future__ import annotations
 
@@ -77,6 +81,20 @@ def lib():
         L.oracle_layer.argtypes = ([_P(u16), _P(f32), _P(f32), _P(u16), _P(u16), _P(u16), _P(u16),
                                     _P(u16), _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f32)])
         L.oracle_layer.restype = c_int
+        u8 = ctypes.c_uint8
+        L.oracle_fp8_e4m3_to_double.argtypes = [u8]
+        L.oracle_fp8_e4m3_to_double.restype = f64
+        L.oracle_fp8_e4m3_from_float.argtypes = [f32]
+        L.oracle_fp8_e4m3_from_float.restype = u8
+        L.oracle_quantize_rows_fp8.argtypes = [_P(u16), i64, c_int, _P(u8), _P(f32)]
+        L.oracle_quantize_rows_fp8.restype = None
+        L.oracle_expert_ffn_fp8.argtypes = [_P(u16), _P(i32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8),
+                                            _P(f32), c_int, c_int, c_int, _P(f64)]
+        L.oracle_expert_ffn_fp8.restype = None
+        L.oracle_layer_given_logits_fp8.argtypes = (
+            [_P(u16), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u16), _P(u16),
+             _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f64)])
+        L.oracle_layer_given_logits_fp8.restype = c_int
         _lib = L
     return _lib
 
@@ -100,7 +118,11 @@ def _i32(a):
     return None if a is None else np.ascontiguousarray(a, dtype=np.int32)
 
 
-U16, I32, F32, F64 = ctypes.c_uint16, ctypes.c_int32, ctypes.c_float, ctypes.c_double
+U16, I32, F32, F64, U8 = ctypes.c_uint16, ctypes.c_int32, ctypes.c_float, ctypes.c_double, ctypes.c_uint8
+
+
+def _u8(a):
+    return None if a is None else np.ascontiguousarray(a).view(np.uint8)
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
@@ -239,3 +261,61 @@ def layer(x, W_gate, W1, W3, W2, k, bias=None, Ws1=None, Ws3=None, Ws2=None):
     if rc:
         raise ValueError("oracle_layer failed")
     return out, logits
+
+
+# ------------------------------------------------------------------ fp8 weights
+
+def fp8_to_f64(codes) -> np.ndarray:
+    """e4m3 codes (uint8) -> float64, element by element through the oracle."""
+    f = lib().oracle_fp8_e4m3_to_double
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([f(int(v)) for v in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def fp8_from_f32(values) -> np.ndarray:
+    """float32 -> e4m3 codes, element by element (nearest, ties to even, 448 at most)."""
+    f = lib().oracle_fp8_e4m3_from_float
+    v = np.asarray(values, dtype=np.float32)
+    return np.array([f(float(a)) for a in v.ravel()], dtype=np.uint8).reshape(v.shape)
+
+
+def quantize_rows_fp8(W):
+    """bf16 weights [..., K] (uint16) -> (e4m3 codes [..., K] uint8, fp32 scale per row [...])."""
+    W = _u16(W)
+    K = W.shape[-1]
+    rows = int(np.prod(W.shape[:-1]))
+    q = np.zeros(W.shape, np.uint8)
+    sc = np.zeros(W.shape[:-1], np.float32)
+    lib().oracle_quantize_rows_fp8(_ptr(W, U16), rows, K, _ptr(q, U8), _ptr(sc, F32))
+    return q, sc
+
+
+def expert_ffn_fp8(x_perm, offsets, q1, s1, q3, s3, q2, s2):
+    x_perm = _u16(x_perm); offsets = _i32(offsets)
+    q1, q3, q2 = _u8(q1), _u8(q3), _u8(q2)
+    s1, s3, s2 = _f32(s1), _f32(s3), _f32(s2)
+    E, I, H = q1.shape
+    y = np.zeros(x_perm.shape, np.float64)
+    lib().oracle_expert_ffn_fp8(_ptr(x_perm, U16), _ptr(offsets, I32), _ptr(q1, U8), _ptr(s1, F32),
+                                _ptr(q3, U8), _ptr(s3, F32), _ptr(q2, U8), _ptr(s2, F32), E, H, I,
+                                _ptr(y, F64))
+    return y
+
+
+def layer_given_logits_fp8(x, logits32, q1, s1, q3, s3, q2, s2, k, Ws1=None, Ws3=None, Ws2=None):
+    """The sparse layer from fp32 logits with e4m3 routed-expert weights; returns out (uint16 [N,H])."""
+    x = _u16(x); l = _f32(logits32)
+    q1, q3, q2 = _u8(q1), _u8(q3), _u8(q2)
+    s1, s3, s2 = _f32(s1), _f32(s3), _f32(s2)
+    Ws1 = _u16(Ws1); Ws3 = _u16(Ws3); Ws2 = _u16(Ws2)
+    N, H = x.shape
+    E, I, _ = q1.shape
+    Is = 0 if Ws1 is None else Ws1.shape[0]
+    out = np.zeros((N, H), np.uint16)
+    rc = lib().oracle_layer_given_logits_fp8(
+        _ptr(x, U16), _ptr(l, F32), _ptr(q1, U8), _ptr(s1, F32), _ptr(q3, U8), _ptr(s3, F32),
+        _ptr(q2, U8), _ptr(s2, F32), _ptr(Ws1, U16), _ptr(Ws3, U16), _ptr(Ws2, U16), N, H, I, E, k, Is,
+        _ptr(out, U16), None)
+    if rc:
+        raise ValueError("oracle_layer_given_logits_fp8 failed")
+    return out

@@ -20,6 +20,9 @@
  *                 "核心公式", MoE-layer formula: three GEMMs per expert
  *                 (here the SwiGLU form W1, W3, W2); section "问题定义":
  *                 shared experts are always-on experts.
+ *  [MoE-latency]  also section "优化从测量开始": quantizing weights (or
+ *                 activations) cuts memory bytes, and its numerical error has to
+ *                 be measured as an experiment of its own.
  *  [MegaScale]    "MegaScale-Infer: Serving Mixture-of-Experts at Scale with
  *                 Disaggregated Expert Parallelism", section "核心问题"
  *                 (Mixtral 8x22B: 156 tokens over 8 experts at top-2 gives
@@ -44,7 +47,12 @@
  *    rounding of a term where the terms cancel;
  *  - combine: out[t] = bf16( sum_j w_j * y[row(t,j)] + s[t] ), j in pick order;
  *  - shared experts (optional, Is > 0): one SwiGLU FFN of width Is over every
- *    token, weight 1, added after the routed sum.
+ *    token, weight 1, added after the routed sum;
+ *  - fp8 expert weights (the pages name no format): OCP e4m3 (no infinities,
+ *    largest finite 448) with one fp32 scale per output channel (weight row):
+ *    s = max|row| / 448 in fp32, q = e4m3(w / s) rounded to nearest even with
+ *    magnitudes past 448 kept at 448; the weight the FFN uses is e4m3(q) * s.
+ *    Activations, routing, combine and the shared experts are unchanged.
  *
  * Layouts: x [N,H] bf16 (uint16 storage); W_gate [H,E] fp32; bias [E] fp32 or
  * NULL; W1, W3 [E,I,H] bf16; W2 [E,H,I] bf16; Ws1, Ws3 [Is,H] bf16;
@@ -88,6 +96,65 @@ uint16_t oracle_round_to_bf16(double v)
     uint32_t u;
     memcpy(&u, &f, sizeof u);
     return (uint16_t)(sign | (u >> 16));
+}
+
+/* ----------------------------------------------------------------- fp8 ---- */
+
+/* OCP 8-bit float e4m3: sign bit, 4 exponent bits with bias 7, 3 mantissa bits.
+ * Exponent field 0 holds subnormals (m/8) * 2^-6; all-ones exponent with all-ones
+ * mantissa (0x7F, 0xFF) is NaN; there are no infinities; the largest finite
+ * magnitude is 1.75 * 2^8 = 448. */
+double oracle_fp8_e4m3_to_double(uint8_t q)
+{
+    int sign = (q >> 7) & 1, ex = (q >> 3) & 15, m = q & 7;
+    double v;
+    if (ex == 15 && m == 7) return NAN;
+    if (ex == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, ex - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest e4m3 value to v, ties to the even code (mantissa bit 0 clear);
+ * magnitudes at or past 448 give 448 (v must not be NaN). */
+uint8_t oracle_fp8_e4m3_from_float(float v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    int e2;
+    frexp(a, &e2);       /* a in [2^(e2-1), 2^e2) */
+    int E = e2 - 1;      /* unbiased exponent of a */
+    if (E < -6) E = -6;  /* subnormal range: spacing 2^-9 */
+    double step = ldexp(1.0, E - 3);
+    double n = nearbyint(a / step); /* a / step is exact; default rounding: ties to even */
+    double r = n * step;            /* at most 448 here */
+    if (r == 0.0) return sign;
+    if (r < ldexp(1.0, -6)) return (uint8_t)(sign | (int)(r / ldexp(1.0, -9)));
+    int er;
+    frexp(r, &er);
+    int Er = er - 1;
+    int m = (int)(r / ldexp(1.0, Er - 3)) - 8;
+    return (uint8_t)(sign | ((Er + 7) << 3) | m);
+}
+
+/* Per output channel quantization of a bf16 weight matrix [rows, K]:
+ * s[r] = max_c |W[r,c]| / 448 in fp32 (1 for an all-zero row), q[r,c] =
+ * e4m3(float(W[r,c]) / s[r]) with the division in fp32. */
+void oracle_quantize_rows_fp8(const uint16_t *W, int64_t rows, int K, uint8_t *q, float *s)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int c = 0; c < K; ++c) {
+            float a = fabsf((float)oracle_bf16_to_double(W[r * K + c]));
+            if (a > amax) amax = a;
+        }
+        float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        s[r] = sc;
+        for (int c = 0; c < K; ++c) {
+            volatile float t = (float)oracle_bf16_to_double(W[r * K + c]) / sc; /* fp32 quotient */
+            q[r * K + c] = oracle_fp8_e4m3_from_float(t);
+        }
+    }
 }
 
 /* -------------------------------------------------------------- router ---- */
@@ -180,11 +247,27 @@ void oracle_permute_rows(const uint16_t *x, const int32_t *row_to_token, int64_t
 
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
+/* One expert weight stack [E*rows, K] (row-major; expert e's rows start at
+ * e*rows): bf16 (w8 == NULL), or e4m3 codes with one fp32 scale per row, whose
+ * weight is e4m3(q) * s. */
+typedef struct {
+    const uint16_t *w16;
+    const uint8_t *w8;
+    const float *sc;
+} oracle_wmat;
+
+static double wval(const oracle_wmat *m, int64_t row, int K, int c)
+{
+    if (m->w8) return oracle_fp8_e4m3_to_double(m->w8[row * K + c]) * (double)m->sc[row];
+    return oracle_bf16_to_double(m->w16[row * K + c]);
+}
+
 /* [FinDEP] "核心公式": an expert is three GEMMs; here the SwiGLU expert
- * y = W2 (silu(W1 x) * (W3 x)).  One row, one expert: W1, W3 [I,H], W2 [H,I].
- * fp64 sums; h rounded to bf16, y left in fp64. */
-void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t *W3,
-                       const uint16_t *W2, int H, int I, double *yrow)
+ * y = W2 (silu(W1 x) * (W3 x)).  One row through the expert whose W1/W3 rows
+ * start at r13 and whose W2 rows start at r2.  fp64 sums; h rounded to bf16,
+ * y left in fp64. */
+static void swiglu_row(const uint16_t *xrow, const oracle_wmat *W1, const oracle_wmat *W3,
+                       const oracle_wmat *W2, int64_t r13, int64_t r2, int H, int I, double *yrow)
 {
     double *xd = (double *)malloc((size_t)H * sizeof(double));
     double *hd = (double *)malloc((size_t)I * sizeof(double));
@@ -192,31 +275,56 @@ void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t 
     for (int i = 0; i < I; ++i) {
         double g = 0.0, u = 0.0;
         for (int c = 0; c < H; ++c) {
-            g += xd[c] * oracle_bf16_to_double(W1[(int64_t)i * H + c]);
-            u += xd[c] * oracle_bf16_to_double(W3[(int64_t)i * H + c]);
+            g += xd[c] * wval(W1, r13 + i, H, c);
+            u += xd[c] * wval(W3, r13 + i, H, c);
         }
         hd[i] = oracle_bf16_to_double(oracle_round_to_bf16(silu(g) * u));
     }
     for (int o = 0; o < H; ++o) {
         double y = 0.0;
-        for (int i = 0; i < I; ++i) y += hd[i] * oracle_bf16_to_double(W2[(int64_t)o * I + i]);
+        for (int i = 0; i < I; ++i) y += hd[i] * wval(W2, r2 + o, I, i);
         yrow[o] = y;
     }
     free(xd);
     free(hd);
 }
 
+/* One row, one expert with bf16 weights: W1, W3 [I,H], W2 [H,I]. */
+void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t *W3,
+                       const uint16_t *W2, int H, int I, double *yrow)
+{
+    oracle_wmat a = {W1, NULL, NULL}, b = {W3, NULL, NULL}, c = {W2, NULL, NULL};
+    swiglu_row(xrow, &a, &b, &c, 0, 0, H, I, yrow);
+}
+
 /* [MoE-latency] "router 之后还有一串动作": each expert runs its own rows.
  * Rows offsets[e] .. offsets[e+1]-1 of x_perm go through expert e. */
+static void expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const oracle_wmat *W1,
+                       const oracle_wmat *W3, const oracle_wmat *W2, int E, int H, int I,
+                       double *y_perm)
+{
+    for (int e = 0; e < E; ++e)
+        for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r)
+            swiglu_row(x_perm + r * H, W1, W3, W2, (int64_t)e * I, (int64_t)e * H, H, I,
+                       y_perm + r * H);
+}
+
 void oracle_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
                        const uint16_t *W3, const uint16_t *W2, int E, int H, int I,
                        double *y_perm)
 {
-    int64_t we = (int64_t)I * H;
-    for (int e = 0; e < E; ++e)
-        for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r)
-            oracle_swiglu_ffn(x_perm + r * H, W1 + e * we, W3 + e * we, W2 + e * we, H, I,
-                              y_perm + r * H);
+    oracle_wmat a = {W1, NULL, NULL}, b = {W3, NULL, NULL}, c = {W2, NULL, NULL};
+    expert_ffn(x_perm, offsets, &a, &b, &c, E, H, I, y_perm);
+}
+
+/* [MoE-latency] "优化从测量开始": the same experts with e4m3 weights q1, q3
+ * [E,I,H], q2 [E,H,I] and per-row scales s1, s3 [E,I], s2 [E,H]. */
+void oracle_expert_ffn_fp8(const uint16_t *x_perm, const int32_t *offsets, const uint8_t *q1,
+                           const float *s1, const uint8_t *q3, const float *s3, const uint8_t *q2,
+                           const float *s2, int E, int H, int I, double *y_perm)
+{
+    oracle_wmat a = {NULL, q1, s1}, b = {NULL, q3, s3}, c = {NULL, q2, s2};
+    expert_ffn(x_perm, offsets, &a, &b, &c, E, H, I, y_perm);
 }
 
 /* ------------------------------------------------------------- combine ---- */
@@ -244,12 +352,11 @@ void oracle_combine(const double *y_perm, const int32_t *token_to_row, const dou
  * combine.  Optional outputs (may be NULL): idx [N,k], w [N,k], counts [E],
  * offsets [E+1], row_to_token [N*k], token_to_row [N*k], y_perm [N*k,H] (fp64).
  * Returns 0, or -1 on bad arguments / allocation failure. */
-int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint16_t *W1,
-                              const uint16_t *W3, const uint16_t *W2, const uint16_t *Ws1,
-                              const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
-                              int E, int k, int Is, uint16_t *out, int32_t *idx_out,
-                              double *w_out, int32_t *counts_out, int32_t *offsets_out,
-                              int32_t *r2t_out, int32_t *t2r_out, double *y_perm_out)
+static int layer_core(const uint16_t *x, const float *logits, const oracle_wmat *W1,
+                      const oracle_wmat *W3, const oracle_wmat *W2, const uint16_t *Ws1,
+                      const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I, int E, int k,
+                      int Is, uint16_t *out, int32_t *idx_out, double *w_out, int32_t *counts_out,
+                      int32_t *offsets_out, int32_t *r2t_out, int32_t *t2r_out, double *y_perm_out)
 {
     if (N < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E || Is < 0) return -1;
     int64_t R = N * k;
@@ -267,7 +374,7 @@ int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint
     if (oracle_topk(logits, N, E, k, idx, w)) goto done;
     if (oracle_dispatch(idx, N, E, k, counts, offsets, r2t, t2r)) goto done;
     oracle_permute_rows(x, r2t, R, H, xp);
-    oracle_expert_ffn(xp, offsets, W1, W3, W2, E, H, I, yp);
+    expert_ffn(xp, offsets, W1, W3, W2, E, H, I, yp);
     if (Is > 0) {
         s = (double *)malloc((size_t)(N ? N : 1) * H * sizeof(double));
         if (!s) goto done;
@@ -286,6 +393,31 @@ done:
     free(idx); free(w); free(counts); free(offsets); free(r2t); free(t2r); free(xp); free(yp);
     free(s);
     return rc;
+}
+
+int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint16_t *W1,
+                              const uint16_t *W3, const uint16_t *W2, const uint16_t *Ws1,
+                              const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
+                              int E, int k, int Is, uint16_t *out, int32_t *idx_out,
+                              double *w_out, int32_t *counts_out, int32_t *offsets_out,
+                              int32_t *r2t_out, int32_t *t2r_out, double *y_perm_out)
+{
+    oracle_wmat a = {W1, NULL, NULL}, b = {W3, NULL, NULL}, c = {W2, NULL, NULL};
+    return layer_core(x, logits, &a, &b, &c, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, idx_out, w_out,
+                      counts_out, offsets_out, r2t_out, t2r_out, y_perm_out);
+}
+
+/* The same path with e4m3 routed-expert weights (q1, q3 [E,I,H], q2 [E,H,I])
+ * and per-row scales (s1, s3 [E,I], s2 [E,H]); shared experts stay bf16. */
+int oracle_layer_given_logits_fp8(const uint16_t *x, const float *logits, const uint8_t *q1,
+                                  const float *s1, const uint8_t *q3, const float *s3,
+                                  const uint8_t *q2, const float *s2, const uint16_t *Ws1,
+                                  const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
+                                  int E, int k, int Is, uint16_t *out, double *y_perm_out)
+{
+    oracle_wmat a = {NULL, q1, s1}, b = {NULL, q3, s3}, c = {NULL, q2, s2};
+    return layer_core(x, logits, &a, &b, &c, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, NULL, NULL,
+                      NULL, NULL, NULL, NULL, y_perm_out);
 }
 
 /* The whole layer from x: fp64 logits rounded to fp32 (the precision the

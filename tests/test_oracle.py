@@ -293,3 +293,112 @@ def test_qwen3_30b_shape_matches_parameter_arithmetic():
     assert c.E == 128 and c.k == 8
     assert 0.9 * 30.5e9 < expert_params < 30.5e9
     assert abs(30.5e9 * 2 / 1e9 - 61) < 0.5
+
+
+# ------------------------------------------------------------- fp8 weights ----
+# [MoE-latency] "优化从测量开始": quantized weights are their own experiment.
+# The e4m3 format is pinned against torch's float8_e4m3fn (an independent
+# implementation of the same OCP format) and against nearest-value search.
+
+def test_e4m3_decode_every_code_matches_torch():
+    codes = torch.arange(256, dtype=torch.uint8)
+    want = codes.view(torch.float8_e4m3fn).double().numpy()
+    got = oracle.fp8_to_f64(codes.numpy())
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(want[ok]))
+    # the format's landmarks: smallest subnormal, smallest normal, one, largest; NaN only at 0x7F/0xFF
+    assert got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6 and got[0x38] == 1.0 and got[0x7E] == 448.0
+    assert set(np.flatnonzero(np.isnan(got)).tolist()) == {0x7F, 0xFF}
+
+
+def test_e4m3_encode_is_nearest_with_ties_to_even_code():
+    finite = [c for c in range(0x7F)]                       # 0x00 .. 0x7E, non-negative
+    vals = oracle.fp8_to_f64(np.array(finite, np.uint8))
+    assert np.all(np.diff(vals) > 0)                         # codes order the values
+    # every value encodes to its own code; every midpoint to the neighbour with an even code
+    assert np.array_equal(oracle.fp8_from_f32(vals.astype(np.float32)), np.array(finite, np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    assert np.all(mids.astype(np.float64) == (vals[:-1] + vals[1:]) / 2)   # midpoints exact in fp32
+    got = oracle.fp8_from_f32(mids)
+    lo = np.array(finite[:-1], np.uint8)
+    want = np.where(lo % 2 == 0, lo, lo + 1).astype(np.uint8)
+    assert np.array_equal(got, want)
+    # negative side mirrors; past 448 saturates at 448
+    assert np.array_equal(oracle.fp8_from_f32(-vals[1:].astype(np.float32)), np.array(finite[1:], np.uint8) | 0x80)
+    assert oracle.fp8_from_f32(np.array([464.0, 1e9, -1e9], np.float32)).tolist() == [0x7E, 0x7E, 0xFE]
+
+
+def test_e4m3_encode_matches_torch_in_range():
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-14, 6, 100000))).astype(np.float32)
+    x = x[np.abs(x) < 448]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.fp8_from_f32(x), want)
+
+
+def test_quantizer_scale_codes_and_error_bound():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((40, 192)) * np.exp(rng.uniform(-6, 3, (40, 1)))).astype(np.float32)
+    W[7] = 0.0                                                    # an all-zero row
+    Wb = enc(W)
+    q, sc = oracle.quantize_rows_fp8(Wb)
+    Wd = dec(Wb)
+    assert sc[7] == 1.0 and not q[7].any()
+    amax = np.abs(Wd).max(axis=1)
+    nz = amax > 0
+    assert np.array_equal(sc[nz], (amax[nz].astype(np.float32) / np.float32(448)).astype(np.float32))
+    # each nonzero row's largest magnitude lands on +-448
+    top = np.abs(Wd).argmax(axis=1)
+    assert all((q[r, top[r]] & 0x7F) == 0x7E for r in np.flatnonzero(nz))
+    # the rounding step is torch's e4m3 conversion of the fp32 quotient
+    quot = (Wd.astype(np.float32) / sc[:, None]).astype(np.float32)
+    assert np.array_equal(q, torch.from_numpy(quot).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+    # reconstruction: within half an e4m3 step (2^-4 relative, 2^-10 absolute in the subnormals) of the weight
+    rec = oracle.fp8_to_f64(q) * sc[:, None].astype(np.float64)
+    err = np.abs(rec - Wd)
+    bound = (2.0 ** -4 * np.abs(Wd) + 2.0 ** -10 * sc[:, None]) * (1 + 2.0 ** -20)
+    assert np.all(err <= bound)
+
+
+def _grid_weights(rng, shape):
+    """bf16 weights that are e4m3 values times a power of two per row, each row
+    holding +-448 times that power: the quantizer represents them exactly."""
+    pos = oracle.fp8_to_f64(np.arange(1, 0x7F, dtype=np.uint8))
+    v = rng.choice(pos, size=shape) * rng.choice([-1.0, 1.0], size=shape)
+    v[..., 0] = 448.0 * rng.choice([-1.0, 1.0], size=shape[:-1])
+    j = rng.integers(-14, -6, size=shape[:-1] + (1,))
+    return enc((v * np.exp2(j)).astype(np.float32))
+
+
+def test_fp8_layer_equals_bf16_layer_on_exactly_representable_weights():
+    cfg, t = small_layer(N=18, H=64, I=32, E=4, k=2)
+    rng = np.random.default_rng(9)
+    W1 = _grid_weights(rng, (cfg.E, cfg.I, cfg.H))
+    W3 = _grid_weights(rng, (cfg.E, cfg.I, cfg.H))
+    W2 = _grid_weights(rng, (cfg.E, cfg.H, cfg.I))
+    q1, s1 = oracle.quantize_rows_fp8(W1)
+    q3, s3 = oracle.quantize_rows_fp8(W3)
+    q2, s2 = oracle.quantize_rows_fp8(W2)
+    assert np.array_equal(enc((oracle.fp8_to_f64(q1) * s1[..., None]).astype(np.float32)), W1)
+    l32 = oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32)
+    want = oracle.layer_given_logits(t["x"], l32, W1, W3, W2, cfg.k)
+    got = oracle.layer_given_logits_fp8(t["x"], l32, q1, s1, q3, s3, q2, s2, cfg.k)
+    assert np.array_equal(got, want)
+    xp = t["x"][np.arange(cfg.N).repeat(1)]
+    off = np.array([0, 5, 9, 9, cfg.N], np.int32)
+    assert np.array_equal(oracle.expert_ffn_fp8(xp, off, q1, s1, q3, s3, q2, s2),
+                          oracle.expert_ffn(xp, off, W1, W3, W2))
+
+
+def test_fp8_layer_error_against_bf16_is_quantization_sized():
+    """Ordinary weights: the fp8 layer differs from the bf16 layer by about the
+    e4m3 step (2^-4 relative) averaged over the sums, far less than the outputs."""
+    cfg, t = small_layer(N=24, H=128, I=64, E=4, k=2)
+    l32 = oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32)
+    want = dec(oracle.layer_given_logits(t["x"], l32, t["W1"], t["W3"], t["W2"], cfg.k))
+    qs = [oracle.quantize_rows_fp8(t[n]) for n in ("W1", "W3", "W2")]
+    got = dec(oracle.layer_given_logits_fp8(t["x"], l32, *qs[0], *qs[1], *qs[2], cfg.k))
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    assert 1e-3 < rel < 5e-2
