@@ -62,18 +62,23 @@ def layer_flops(cfg):
     return 2 * cfg.N * cfg.H * cfg.E + 6 * cfg.R * cfg.H * cfg.I + 6 * cfg.N * cfg.H * cfg.Is
 
 
-def gemm13_bytes(cfg, touched):
-    """W1+W3 tiles of the touched experts, x_perm read, h written."""
-    return touched * 2 * cfg.I * cfg.H * 2 + cfg.R * cfg.H * 2 + cfg.R * cfg.I * 2
+def gemm13_bytes(cfg, touched, wbytes=2):
+    """W1+W3 tiles of the touched experts (wbytes per weight; fp8 adds a 4-byte scale
+    per row), x_perm read, h written."""
+    scales = touched * 2 * cfg.I * 4 if wbytes == 1 else 0
+    return touched * 2 * cfg.I * cfg.H * wbytes + scales + cfg.R * cfg.H * 2 + cfg.R * cfg.I * 2
 
 
-def gemm2_bytes(cfg, touched):
-    return touched * cfg.H * cfg.I * 2 + cfg.R * cfg.I * 2 + cfg.R * cfg.H * 2
+def gemm2_bytes(cfg, touched, wbytes=2):
+    scales = touched * cfg.H * 4 if wbytes == 1 else 0
+    return touched * cfg.H * cfg.I * wbytes + scales + cfg.R * cfg.I * 2 + cfg.R * cfg.H * 2
 
 
-def layer_bytes(cfg, touched):
-    """Touched expert weights + shared weights + router weights + x in + out."""
-    return (touched * 3 * cfg.H * cfg.I * 2 + 3 * cfg.H * cfg.Is * 2 + cfg.H * cfg.E * 4
+def layer_bytes(cfg, touched, wbytes=2):
+    """Touched expert weights (+ their scales for fp8) + shared weights + router weights
+    + x in + out."""
+    scales = touched * (2 * cfg.I + cfg.H) * 4 if wbytes == 1 else 0  # one per weight row
+    return (touched * 3 * cfg.H * cfg.I * wbytes + scales + 3 * cfg.H * cfg.Is * 2 + cfg.H * cfg.E * 4
             + 2 * cfg.N * cfg.H * 2)
 
 
@@ -277,17 +282,41 @@ def run_ours(args, cfg, world, rank, local):
     N, H, I, E, k = cfg.N, cfg.H, cfg.I, cfg.E, cfg.k
     ws = torch.empty(moe.moe_workspace_bytes(N, H, I, E, k, cfg.Is), dtype=torch.uint8, device=dev)
     out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    fp8 = args.weights == "fp8"
+    wbytes = 1 if fp8 else 2
+    if fp8:
+        # weight preparation, once, outside every timed region: e4m3 codes + row scales
+        q = {n: moe.moe_quantize_fp8(t[n], stream=stream) for n in ("W1", "W3", "W2")}
+        torch.cuda.synchronize()
 
-    def step(events=None):
-        moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], k, bias=t["bias"],
-                                 Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=out, stream=stream,
-                                 phase_events=events)
+    def step(events=None, x=None, o=None):
+        xx = t["x"] if x is None else x
+        oo = out if o is None else o
+        if fp8:
+            moe.moe_layer_forward_fp8_ex(xx, t["W_gate"], *q["W1"], *q["W3"], *q["W2"], k, bias=t["bias"],
+                                         Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=stream,
+                                         phase_events=events)
+        else:
+            moe.moe_layer_forward_ex(xx, t["W_gate"], t["W1"], t["W3"], t["W2"], k, bias=t["bias"],
+                                     Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=stream,
+                                     phase_events=events)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if moe.moe_get_device_error(stream) != 0:
         raise RuntimeError("device error reported during warm-up")
+    fp8_err = None
+    if fp8:
+        # the experiment's numerical cost: the fp8 layer against the bf16 layer, same inputs
+        ref = moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], k, bias=t["bias"],
+                                       Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, stream=stream)
+        step()
+        torch.cuda.synchronize()
+        d = (out.float() - ref.float()).norm() / ref.float().norm()
+        fp8_err = {"rel_l2_vs_bf16_layer": float(d),
+                   "max_abs_vs_bf16_layer": float((out.float() - ref.float()).abs().max())}
+        del ref
     counts = moe.moe_permute(t["x"], moe.moe_route(t["x"], t["W_gate"], k, bias=t["bias"])[0], E)["counts"]
     touched = int((counts > 0).sum().item())
     max_load = int(counts.max().item())
@@ -326,26 +355,42 @@ def run_ours(args, cfg, world, rank, local):
     if moe.moe_get_device_error(stream) != 0:
         raise RuntimeError("device error reported during the timed steps")
 
-    # end to end through the public short form: host x in, host out back, every step
-    e2e = None
-    if cfg.Is == 0 and cfg.bias_scale == 1.0 and not cfg.skew:
-        x_host = t["x"].cpu().pin_memory()
-        out_host = torch.empty((N, H), dtype=torch.bfloat16).pin_memory()
-        for _ in range(args.warmup):
+    # end to end through the public API, host x in and host out back every step: the
+    # short form (which takes host pointers and copies them itself) where it covers the
+    # workload, else the explicit call with the copies on its stream
+    x_host = t["x"].cpu().pin_memory()
+    out_host = torch.empty((N, H), dtype=torch.bfloat16).pin_memory()
+    short_form = not fp8 and cfg.Is == 0 and cfg.bias_scale == 1.0 and not cfg.skew
+    if short_form:
+        e2e_stream = torch.cuda.default_stream(dev)
+        e2e_how = "moe_layer_forward with host x and out (the call copies them)"
+
+        def e2e_step():
             moe.moe_layer_forward(x_host, t["W_gate"], t["W1"], t["W3"], t["W2"], k, out=out_host)
-        barrier(world)
-        torch.cuda.synchronize()
-        s0 = torch.cuda.Event(enable_timing=True)
-        s1 = torch.cuda.Event(enable_timing=True)
-        legacy = torch.cuda.default_stream(dev)
-        s0.record(legacy)
-        for _ in range(args.steps):
-            moe.moe_layer_forward(x_host, t["W_gate"], t["W1"], t["W3"], t["W2"], k, out=out_host)
-        s1.record(legacy)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
-        e2e = {"value": world * N * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": N * H * 2, "d2h_bytes_per_step": N * H * 2}
+    else:
+        e2e_stream = stream
+        e2e_how = (f"{'moe_layer_forward_fp8_ex' if fp8 else 'moe_layer_forward_ex'} with the copy of x in and "
+                   "of out back on its stream")
+        x_dev = torch.empty_like(t["x"])
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            step(x=x_dev)
+            out_host.copy_(out, non_blocking=True)
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(e2e_stream)
+    for _ in range(args.steps):
+        e2e_step()
+    s1.record(e2e_stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+    e2e = {"value": world * N * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": N * H * 2, "d2h_bytes_per_step": N * H * 2, "how": e2e_how}
 
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     if rank != 0:
@@ -355,12 +400,12 @@ def run_ours(args, cfg, world, rank, local):
     value = world * N / step_s
     g13_s = phase_ms["gemm13"] / 1e3
     g2_s = phase_ms["gemm2"] / 1e3
-    g13_b = gemm13_bytes(cfg, touched)
+    g13_b = gemm13_bytes(cfg, touched, wbytes)
     hbm = pk["hbm_gbs"]
     achieved = g13_b / g13_s / 1e9
     flops = layer_flops(cfg)
     gemm_flops = 6 * cfg.R * H * I
-    lbytes = layer_bytes(cfg, touched)
+    lbytes = layer_bytes(cfg, touched, wbytes)
     floor_s = max(flops / (pk["bf16_tflops"] * 1e12), lbytes / (hbm * 1e9))
     workload = cfg.name
     # the W1/W3 kernel's bound: weight streaming (HBM) at decode sizes, the tensor cores
@@ -375,8 +420,10 @@ def run_ours(args, cfg, world, rank, local):
     else:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "alg_bytes_per_launch": g13_b}
-    roofline.update({"kernel": "grouped_gemm SwiGLU W1/W3 (gemm13)", "peak_kind": pk_kind,
-                     "traffic": kernel_traffic("gemm13", workload), "avg_launch_ms": phase_ms["gemm13"]})
+    roofline.update({"kernel": "grouped_gemm SwiGLU W1/W3 (gemm13)" + (", e4m3 weights" if fp8 else ""),
+                     "peak_kind": pk_kind,
+                     "traffic": None if fp8 else kernel_traffic("gemm13", workload),
+                     "avg_launch_ms": phase_ms["gemm13"]})
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
@@ -384,21 +431,25 @@ def run_ours(args, cfg, world, rank, local):
         "config": {"workload": workload_desc(cfg), "global_batch": world * N, "tokens_per_gpu": N,
                    "parallelism": f"dp{world} (token batches, replicated weights, no exchange)",
                    "l2": f"inputs larger than L2: {touched} touched experts' weights "
-                         f"({touched * 3 * H * I * 2 / 1e9:.2f} GB) streamed from HBM every step",
-                   "touched_experts": touched, "max_expert_rows": max_load},
+                         f"({touched * 3 * H * I * wbytes / 1e9:.2f} GB) streamed from HBM every step",
+                   "touched_experts": touched, "max_expert_rows": max_load,
+                   "expert_weights": ("e4m3, one fp32 scale per output channel (quantized once before "
+                                      "timing; widened to bf16 on chip)") if fp8 else "bf16"},
         "roofline": roofline,
         "layer": {"tflops": flops / step_s / 1e12, "alg_bytes": lbytes, "gb_s": lbytes / step_s / 1e9,
                   "roofline_floor_us": floor_s * 1e6, "roofline_frac": floor_s / step_s,
                   "useful_flop_fraction_k_over_E": k / E},
         "grouped_gemm": {"tflops": gemm_flops / (g13_s + g2_s) / 1e12,
-                         "gb_s": (g13_b + gemm2_bytes(cfg, touched)) / (g13_s + g2_s) / 1e9,
-                         "gemm2_frac_hbm": gemm2_bytes(cfg, touched) / g2_s / 1e9 / hbm},
+                         "gb_s": (g13_b + gemm2_bytes(cfg, touched, wbytes)) / (g13_s + g2_s) / 1e9,
+                         "gemm2_frac_hbm": gemm2_bytes(cfg, touched, wbytes) / g2_s / 1e9 / hbm},
         "phase_ms": phase_ms,
         "phase_ms_note": "mean per-phase CUDA-event times from a second timed pass with events between phases",
         "gpu_launches": launches,
         "gpu_launches_note": "the library's own host-side count of its kernel launches over the timed steps",
         "e2e": e2e,
     }
+    if fp8_err is not None:
+        line["fp8_error"] = fp8_err
     clk_sum = clk.summary()
     if clk_sum:
         line["clocks"] = clk_sum
@@ -443,6 +494,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=12)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
+                    help="routed-expert weight format (fp8: e4m3 with per-channel scales, a separate experiment)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -96,18 +96,36 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
     L->total = off;
 }
 
-moe_status_t expert_ffn_impl(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
-                             const uint16_t *W3, const uint16_t *W2, int64_t R, int H, int I, int E,
-                             uint16_t *h, float *y_perm, int *err, cudaStream_t s)
+// The routed experts' weights: bf16, or e4m3 bytes with one fp32 scale per row.
+struct Experts {
+    const void *W1, *W3, *W2;
+    const float *s1, *s3, *s2;  // fp8 only
+    bool fp8;
+};
+
+void set_weights13(moe::GroupedGemmArgs *a, const Experts &X)
+{
+    a->w_a = X.W1; a->w_b = X.W3; a->w8 = X.fp8; a->scale_a = X.s1; a->scale_b = X.s3;
+}
+
+void set_weights2(moe::GroupedGemmArgs *b, const Experts &X)
+{
+    b->w_a = X.W2; b->w_b = nullptr; b->w8 = X.fp8; b->scale_a = X.s2; b->scale_b = nullptr;
+}
+
+moe_status_t expert_ffn_impl(const uint16_t *x_perm, const int32_t *offsets, const Experts &X, int64_t R, int H,
+                             int I, int E, uint16_t *h, float *y_perm, int *err, cudaStream_t s)
 {
     if (R == 0) return MOE_OK;
     moe::GroupedGemmArgs a{};
-    a.act = x_perm; a.w_a = W1; a.w_b = W3; a.offsets = offsets; a.groups = E; a.R = R;
+    a.act = x_perm; a.offsets = offsets; a.groups = E; a.R = R;
     a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
+    set_weights13(&a, X);
     MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     moe::GroupedGemmArgs b{};
-    b.act = h; b.w_a = W2; b.w_b = nullptr; b.offsets = offsets; b.groups = E; b.R = R;
+    b.act = h; b.offsets = offsets; b.groups = E; b.R = R;
     b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
+    set_weights2(&b, X);
     MOE_CUDA(moe::launch_gemm2(b, s));
     return MOE_OK;
 }
@@ -141,6 +159,72 @@ moe_status_t record(void *const *ev, int i, cudaStream_t s)
         moe_status_t st_ = (call);               \
         if (st_ != MOE_OK) return st_;           \
     } while (0)
+
+moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bias, const Experts &X,
+                        const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
+                        int E, int k, int Is, uint16_t *out, float *logits, void *ws, size_t ws_bytes,
+                        void *stream, void *const *phase_events)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
+    if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (N == 0) return MOE_OK;
+    if (!x || !W_gate || !X.W1 || !X.W3 || !X.W2 || !out) return MOE_ERR_INVALID_ARG;
+    if (Is > 0 && (!Ws1 || !Ws3 || !Ws2)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(X.W1) || !aligned16(X.W3) || !aligned16(X.W2) || !aligned16(out))
+        return MOE_ERR_UNSUPPORTED;
+    if (Is > 0 && (!aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2))) return MOE_ERR_UNSUPPORTED;
+    WsLayout L;
+    ws_layout(N, H, I, E, k, Is, &L);
+    if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    int *err = device_error_word();
+    if (!err) return cuda_fail(cudaGetLastError());
+
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *lg = logits ? logits : reinterpret_cast<float *>(base + L.logits);
+    int32_t *idx = reinterpret_cast<int32_t *>(base + L.idx);
+    float *w = reinterpret_cast<float *>(base + L.w);
+    int32_t *counts = reinterpret_cast<int32_t *>(base + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(base + L.offsets);
+    int32_t *r2t = reinterpret_cast<int32_t *>(base + L.r2t);
+    int32_t *t2r = reinterpret_cast<int32_t *>(base + L.t2r);
+    int32_t *perm = reinterpret_cast<int32_t *>(base + L.perm);
+    uint16_t *x_perm = reinterpret_cast<uint16_t *>(base + L.x_perm);
+    uint16_t *h = reinterpret_cast<uint16_t *>(base + L.h);
+    uint16_t *hs = reinterpret_cast<uint16_t *>(base + L.hs);
+    float *y_perm = reinterpret_cast<float *>(base + L.y_perm);
+    float *sh = Is > 0 ? reinterpret_cast<float *>(base + L.s) : nullptr;
+    const int64_t R = N * k;
+
+    MOE_TRY(record(phase_events, 0, s));
+    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
+    MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
+    {
+        moe::GroupedGemmArgs a{};
+        a.act = x_perm; a.offsets = offsets; a.groups = E; a.R = R;
+        a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
+        set_weights13(&a, X);
+        MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
+    }
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
+    const int ksplit = moe::gemm2_ksplit(R, E, I, H);
+    {
+        moe::GroupedGemmArgs b{};
+        b.act = h; b.offsets = offsets; b.groups = E; b.R = R;
+        b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
+        set_weights2(&b, X);
+        b.ksplit = ksplit; b.split_stride = R * (int64_t)H;
+        MOE_CUDA(moe::launch_gemm2(b, s));
+    }
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM2, s));
+    if (Is > 0) MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
+    MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r, w, sh, N, H, k, out, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_COMBINE, s));
+    return MOE_OK;
+}
 
 }  // namespace
 
@@ -227,7 +311,8 @@ moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, cons
     if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     int *err = device_error_word();
     if (!err) return cuda_fail(cudaGetLastError());
-    return expert_ffn_impl(x_perm, offsets, W1, W3, W2, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, err,
+    const Experts X{W1, W3, W2, nullptr, nullptr, nullptr, false};
+    return expert_ffn_impl(x_perm, offsets, X, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, err,
                            static_cast<cudaStream_t>(stream));
 }
 
@@ -250,63 +335,52 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
                                   int H, int I, int E, int k, int Is, uint16_t *out, float *logits, void *ws,
                                   size_t ws_bytes, void *stream, void *const *phase_events)
 {
-    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
-    if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return MOE_ERR_INVALID_ARG;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (N == 0) return MOE_OK;
-    if (!x || !W_gate || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
-    if (Is > 0 && (!Ws1 || !Ws3 || !Ws2)) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(out))
+    const Experts X{W1, W3, W2, nullptr, nullptr, nullptr, false};
+    return layer_impl(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, ws_bytes, stream,
+                      phase_events);
+}
+
+moe_status_t moe_layer_forward_fp8_ex(const uint16_t *x, const float *W_gate, const float *bias,
+                                      const uint8_t *W1q, const float *s1, const uint8_t *W3q, const float *s3,
+                                      const uint8_t *W2q, const float *s2, const uint16_t *Ws1,
+                                      const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I, int E,
+                                      int k, int Is, uint16_t *out, float *logits, void *ws, size_t ws_bytes,
+                                      void *stream, void *const *phase_events)
+{
+    if (N > 0 && (!s1 || !s3 || !s2)) return MOE_ERR_INVALID_ARG;
+    const Experts X{W1q, W3q, W2q, s1, s3, s2, true};
+    return layer_impl(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, ws_bytes, stream,
+                      phase_events);
+}
+
+moe_status_t moe_quantize_fp8(const uint16_t *W, int64_t rows, int K, uint8_t *q, float *scale, void *stream)
+{
+    if (rows < 0 || !valid_hidden(K)) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!W || !q || !scale) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(q) || !aligned16(scale)) return MOE_ERR_UNSUPPORTED;
+    MOE_CUDA(moe::launch_quantize_fp8(W, rows, K, q, scale, static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+moe_status_t moe_expert_ffn_fp8(const uint16_t *x_perm, const int32_t *offsets, const uint8_t *W1q,
+                                const float *s1, const uint8_t *W3q, const float *s3, const uint8_t *W2q,
+                                const float *s2, int64_t R, int H, int I, int E, float *y_perm, void *ws,
+                                size_t ws_bytes, void *stream)
+{
+    if (R < 0 || R >= (int64_t(1) << 31) || !valid_hidden(H) || !valid_hidden(I) || E < 1 || E > 256)
+        return MOE_ERR_INVALID_ARG;
+    if (R == 0) return MOE_OK;
+    if (!x_perm || !offsets || !W1q || !W3q || !W2q || !s1 || !s3 || !s2 || !y_perm) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_perm) || !aligned16(W1q) || !aligned16(W3q) || !aligned16(W2q) || !aligned16(y_perm))
         return MOE_ERR_UNSUPPORTED;
-    if (Is > 0 && (!aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2))) return MOE_ERR_UNSUPPORTED;
-    WsLayout L;
-    ws_layout(N, H, I, E, k, Is, &L);
-    if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    const size_t need = (size_t)R * I * 2;
+    if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     int *err = device_error_word();
     if (!err) return cuda_fail(cudaGetLastError());
-
-    uint8_t *base = static_cast<uint8_t *>(ws);
-    float *lg = logits ? logits : reinterpret_cast<float *>(base + L.logits);
-    int32_t *idx = reinterpret_cast<int32_t *>(base + L.idx);
-    float *w = reinterpret_cast<float *>(base + L.w);
-    int32_t *counts = reinterpret_cast<int32_t *>(base + L.counts);
-    int32_t *offsets = reinterpret_cast<int32_t *>(base + L.offsets);
-    int32_t *r2t = reinterpret_cast<int32_t *>(base + L.r2t);
-    int32_t *t2r = reinterpret_cast<int32_t *>(base + L.t2r);
-    int32_t *perm = reinterpret_cast<int32_t *>(base + L.perm);
-    uint16_t *x_perm = reinterpret_cast<uint16_t *>(base + L.x_perm);
-    uint16_t *h = reinterpret_cast<uint16_t *>(base + L.h);
-    uint16_t *hs = reinterpret_cast<uint16_t *>(base + L.hs);
-    float *y_perm = reinterpret_cast<float *>(base + L.y_perm);
-    float *sh = Is > 0 ? reinterpret_cast<float *>(base + L.s) : nullptr;
-    const int64_t R = N * k;
-
-    MOE_TRY(record(phase_events, 0, s));
-    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
-    MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
-    {
-        moe::GroupedGemmArgs a{};
-        a.act = x_perm; a.w_a = W1; a.w_b = W3; a.offsets = offsets; a.groups = E; a.R = R;
-        a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
-        MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
-    }
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
-    const int ksplit = moe::gemm2_ksplit(R, E, I, H);
-    {
-        moe::GroupedGemmArgs b{};
-        b.act = h; b.w_a = W2; b.offsets = offsets; b.groups = E; b.R = R;
-        b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
-        b.ksplit = ksplit; b.split_stride = R * (int64_t)H;
-        MOE_CUDA(moe::launch_gemm2(b, s));
-    }
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM2, s));
-    if (Is > 0) MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
-    MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r, w, sh, N, H, k, out, s));
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_COMBINE, s));
-    return MOE_OK;
+    const Experts X{W1q, W3q, W2q, s1, s3, s2, true};
+    return expert_ffn_impl(x_perm, offsets, X, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, err,
+                           static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_layer_forward(const uint16_t *x, const float *W_gate, const uint16_t *W1, const uint16_t *W3,

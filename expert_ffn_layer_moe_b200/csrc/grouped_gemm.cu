@@ -38,6 +38,20 @@
 // tile's main loop.  Barrier set-up and TMEM allocation run before the kernel waits on
 // the previous kernel in the stream (programmatic dependent launch).
 //
+// fp8 weights (W8 = true; MoE-latency article, section "优化从测量开始": quantized
+// weights as an experiment of their own): the weights are e4m3 bytes with one fp32 scale
+// per output row.  The tensor cores take bf16 here, so the bytes are widened on chip:
+//   warp 0        : TMA of 128 x 128-byte fp8 tiles (two 64-wide K blocks each);
+//   warp 14       : TMA of the activation tiles (their own ring, as deep in K);
+//   warps 6..13   : converters -- warp w widens the rows of TMEM lane quadrant w % 4,
+//                   half (w - 6) / 4 of each K block, with integer operations and one
+//                   exact bf16 multiplication, and stores them with tcgen05.st into one
+//                   of four operand slots in TMEM;
+//   warp 1        : MMA with A read from TMEM (tcgen05.mma [d], [a], b_desc);
+//   epilogue      : as above, multiplying each output row by its scale first.
+// W8 runs single-CTA tiles of up to 128 token rows (a pair's MMA would need the other
+// CTA to signal every K step across the cluster, which costs more than the pair saves).
+//
 // Work items are (group, feature tile, K slice, token tile), enumerated on the device
 // from the row offsets with no host synchronisation; empty groups produce no items (no
 // padding to a fixed capacity).  The plain GEMM can split K into `ksplit` slices whose
@@ -57,36 +71,53 @@ namespace {
 constexpr int kBM = 128;     // MMA M: weight rows per tile
 constexpr int kBK = 64;      // K per pipeline stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;   // K of one tcgen05.mma kind::f16
-constexpr int kThreads = 192;
 constexpr int kMaxGroups = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, far above any legal wait
 
 constexpr int pow2_at_least(int v, int p = 32) { return p >= v ? p : pow2_at_least(v, p * 2); }
 
-template <int BN, bool SWIGLU, bool PAIR>
+template <int BN, bool SWIGLU, bool PAIR, bool W8>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "token tile must be 32..256, step 32");
+    // warps: producer, MMA, 4 epilogue; with W8 also 8 converter warps (fp8 -> bf16)
+    // and an activation producer
+    static_assert(!(W8 && PAIR), "fp8 weights run single-CTA tiles");
+    static constexpr int kThreads = W8 ? 480 : 192;
     static constexpr int kCtas = PAIR ? 2 : 1;             // CTAs sharing one MMA (cta_group)
     static constexpr int kFeat = SWIGLU ? kBM / 2 : kBM;   // output features per CTA per tile
     static constexpr int kFeatTile = kCtas * kFeat;        // output features per work item
     static constexpr int kBRows = BN / kCtas;              // token rows of B held by each CTA
     static constexpr int kABytes = kBM * kBK * 2;          // 16 KB weight tile per stage
     static constexpr int kBBytes = kBRows * kBK * 2;
-    static constexpr int kStageBytes = kABytes + kBBytes;
+    // bf16: one TMA ring whose stages hold the weight and the activation tile.
+    // W8: three rings -- fp8 weight tiles (deep: those loads go to HBM), activation
+    // tiles (its stages are only kBBytes; the loads mostly hit L2) and the bf16 operand
+    // slots the converter warps write for the MMA.
+    static constexpr int kW8Bytes = W8 ? kBM * 2 * kBK : 0;  // one fp8 weight tile: K = 128 (16 KB)
+    static constexpr int kABufs = W8 ? 4 : 0;              // bf16 operand slots in TMEM (two per fp8 tile)
+    static constexpr int kACols = 32;                      // TMEM columns of one slot: 64 bf16 per lane
+    static constexpr int kStageBytes = W8 ? kBBytes : kABytes + kBBytes;
     static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
-    static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
+    // W8: the activation ring reaches as many K blocks ahead as the fp8 ring (two per
+    // fp8 tile): both kinds of load take microseconds under full HBM traffic
+    static constexpr int kFFit = W8 ? (200 * 1024) / (kW8Bytes + 2 * kBBytes) : 0;
+    static constexpr int kFStages = kFFit > 8 ? 8 : kFFit;     // fp8 ring (W8)
+    static constexpr int kStages = W8 ? 2 * kFStages : (kStagesFit > 10 ? 10 : kStagesFit);
     static constexpr int kAccCols = BN;                    // fp32 TMEM columns per accumulator
     static constexpr int kAccBufs = 2;
-    static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols);
-    static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs);
+    static constexpr int kASlot0 = kAccBufs * kAccCols;    // W8: first TMEM column of the operand slots
+    static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols + kABufs * kACols);
+    static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs + 2 * kFStages + 2 * kABufs);
     static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
     static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // staging: 4 x [32][33] fp32 (= 2 x [64][33])
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16 + kTableBytes + kEpiBytes;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kFStages * kW8Bytes + kBarBytes + 16 +
+                                      kTableBytes + kEpiBytes;
     // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
     // both operands K-major, M>>4 at bit 24 (M = 128 per CTA); N>>3 (bit 17) per tile.
     static constexpr uint32_t kIdescNoN =
         (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)((kBM * kCtas) >> 4) << 24);
     static_assert(kStages >= 2, "pipeline needs at least two stages");
+    static_assert(!W8 || kFStages >= 2, "fp8 ring needs at least two tiles");
     static_assert(kTmemCols <= 512, "TMEM has 512 columns");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -140,6 +171,59 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Two e4m3 bytes, placed in bits 0-7 and 16-23 of `t`, -> two bf16 (low half first).
+// t * 16 puts each byte's 7 exponent-and-mantissa bits at bits 4-10 of its half and
+// its sign at bit 11; adding 15 times the sign bit carries it to bit 15 (2^11 + 15 *
+// 2^11 = 2^15, no carry leaves the half).  The result is the bf16 whose value is the
+// e4m3 value times 2^-120 -- exactly, since the e4m3 subnormals (exponent field 0)
+// land on the bf16 subnormals with the same mantissa -- and one bf16 multiplication by
+// 2^120 (exact: a power of two, no overflow) gives the value itself.
+__device__ __forceinline__ uint32_t e4m3_pair_to_bf16x2(uint32_t t)
+{
+    const uint32_t a = t << 4;
+    const uint32_t w = a + (a & 0x08000800u) * 15u;
+    const __nv_bfloat162 two120 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)0x7B80),
+                                                     __ushort_as_bfloat16((unsigned short)0x7B80));
+    const __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&w), two120);
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// Four e4m3 bytes -> four bf16, as two words (bytes 0,1 and bytes 2,3).
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t v, uint32_t &lo, uint32_t &hi)
+{
+    lo = e4m3_pair_to_bf16x2(__byte_perm(v, 0u, 0x4140));  // byte 0 -> bits 0-7, byte 1 -> bits 16-23
+    hi = e4m3_pair_to_bf16x2(__byte_perm(v, 0u, 0x4342));
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane (the warp's lane quadrant).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+// 32 of the 128 fp8 values of row r of a 128 x 128 fp8 weight tile as TMA wrote it
+// (128-byte rows, 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)):
+// K block kh (0, 1), values [32 kq, 32 kq + 32) of its 64, as 16 bf16 pairs (low half =
+// lower K), the layout of one lane of an MMA A operand in TMEM.
+__device__ __forceinline__ void widen_e4m3_32(const uint8_t *src_tile, int r, int kh, int kq, uint32_t (&o)[16])
+{
+    const uint8_t *src = src_tile + r * 128;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = 4 * kh + 2 * kq + i;
+        const uint4 v = *reinterpret_cast<const uint4 *>(src + ((c ^ (r & 7)) << 4));
+        e4m3x4_to_bf16x4(v.x, o[8 * i + 0], o[8 * i + 1]);
+        e4m3x4_to_bf16x4(v.y, o[8 * i + 2], o[8 * i + 3]);
+        e4m3x4_to_bf16x4(v.z, o[8 * i + 4], o[8 * i + 5]);
+        e4m3x4_to_bf16x4(v.w, o[8 * i + 6], o[8 * i + 7]);
+    }
+}
+
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -170,6 +254,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// MMA with the A operand in TMEM (rows on lanes, K along the columns) and B in shared memory.
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -338,24 +434,31 @@ __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;
 // [n/2 r, n/2 r + n/2) of its n; the leader (r = 0) issues the M=256 MMAs, both CTAs'
 // TMA loads complete on the leader's stage barrier, its commits reach both CTAs'
 // barriers, and each CTA drains its own half of the accumulator.
-template <int BN, bool SWIGLU, bool PAIR>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, bool SWIGLU, bool PAIR, bool W8>
+__global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
-                        void *__restrict__ out, int ksplit, int64_t split_stride, int *dev_err)
+                        void *__restrict__ out, int ksplit, int64_t split_stride,
+                        const float *__restrict__ scale_a, const float *__restrict__ scale_b, int *dev_err)
 {
-    using C = Cfg<BN, SWIGLU, PAIR>;
+    using C = Cfg<BN, SWIGLU, PAIR, W8>;
+    constexpr int kThreads = C::kThreads;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);  // 1024-aligned for SW128
 
-    uint8_t *stages = smem;
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStageBytes);
+    uint8_t *stages = smem;                                     // TMA ring (W8: activations)
+    uint8_t *fring = smem + C::kStages * C::kStageBytes;        // W8: fp8 weight tiles
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(fring + C::kFStages * C::kW8Bytes);
     uint64_t *empty_bar = full_bar + C::kStages;
     uint64_t *tfull_bar = empty_bar + C::kStages;
     uint64_t *tempty_bar = tfull_bar + C::kAccBufs;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty_bar + C::kAccBufs);
+    uint64_t *ffull_bar = tempty_bar + C::kAccBufs;             // W8: fp8 tile landed
+    uint64_t *fempty_bar = ffull_bar + C::kFStages;             // W8: fp8 tile read by every converter warp
+    uint64_t *afull_bar = fempty_bar + C::kFStages;             // W8: operand slot written by every converter warp
+    uint64_t *aempty_bar = afull_bar + C::kABufs;               // W8: operand slot read by the MMA
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(aempty_bar + C::kABufs);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
@@ -378,6 +481,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < C::kAccBufs; ++b) {
             mbar_init(&tfull_bar[b], 1);
             mbar_init(&tempty_bar[b], 4 * C::kCtas);  // every epilogue warp of the pair releases
+        }
+        if (W8) {
+            for (int j = 0; j < C::kFStages; ++j) { mbar_init(&ffull_bar[j], 1); mbar_init(&fempty_bar[j], 8); }
+            for (int a = 0; a < C::kABufs; ++a) { mbar_init(&afull_bar[a], 8); mbar_init(&aempty_bar[a], 1); }
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -446,9 +553,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         row0 = g_off[g] + (local / nfk) * BN;
         row_end = g_off[g + 1];
     };
+    // W8: slices start and end on 128-wide K blocks (one fp8 load); a last half block
+    // past K reads zeros from both tensor maps and adds nothing
     auto kslice = [&](int ks, int &kb0, int &kb1) {
-        kb0 = (int)((int64_t)ks * KB / ksplit);
-        kb1 = (int)((int64_t)(ks + 1) * KB / ksplit);
+        if (W8) {
+            const int KB2 = (KB + 1) / 2;
+            kb0 = 2 * (int)((int64_t)ks * KB2 / ksplit);
+            kb1 = 2 * (int)((int64_t)(ks + 1) * KB2 / ksplit);
+        } else {
+            kb0 = (int)((int64_t)ks * KB / ksplit);
+            kb1 = (int)((int64_t)(ks + 1) * KB / ksplit);
+        }
     };
     // MMA width of a tile: its rows rounded up to the instruction's step of 16
     auto mma_width = [&](int row0, int row_end) { return min(BN, (min(BN, row_end - row0) + 15) & ~15); };
@@ -463,7 +578,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&full_bar[0]), 0) : smem_u32(&full_bar[0]);
         int stage = 0;
         uint32_t phase = 0;
-        for (int item = unit; item < total && !failed; item += nunits) {
+        for (int item = unit; W8 && item < total && !failed; item += nunits) {
+            // fp8 weight tiles, as far ahead as the fp8 ring reaches
+            int g, feat, ks, row0, row_end, kb0, kb1;
+            decode(item, g, feat, ks, row0, row_end);
+            kslice(ks, kb0, kb1);
+            const int frow = feat * C::kFeatTile;
+            for (int kb = kb0; kb < kb1; kb += 2) {
+                if (!mbar_wait(&fempty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
+                uint8_t *dst = fring + stage * C::kW8Bytes;
+                const uint32_t fb = smem_u32(&ffull_bar[stage]);
+                mbar_arrive_expect_tx(&ffull_bar[stage], C::kW8Bytes);
+                if (SWIGLU) {
+                    tma_3d<false>(dst, &tm_wa, kb * kBK, frow, g, fb);
+                    tma_3d<false>(dst + C::kW8Bytes / 2, &tm_wb, kb * kBK, frow, g, fb);
+                } else {
+                    tma_3d<false>(dst, &tm_wa, kb * kBK, frow, g, fb);
+                }
+                if (++stage == C::kFStages) { stage = 0; phase ^= 1u; }
+            }
+        }
+        for (int item = unit; !W8 && item < total && !failed; item += nunits) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
             kslice(ks, kb0, kb1);
@@ -487,8 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1 && lane == 0 && rank == 0) {
         // ------------------------------------------------------ MMA issuer (leader CTA)
-        int stage = 0, acc = 0;
-        uint32_t phase = 0, aphase = 0;
+        int stage = 0, acc = 0, ab = 0;
+        uint32_t phase = 0, aphase = 0, abphase = 0;
         for (int item = unit; item < total && !failed; item += nunits) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
@@ -499,24 +634,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
             for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { failed = true; *abort_flag = 1; break; }
+                if (W8 && !mbar_wait(&afull_bar[ab], abphase, abort_flag)) { failed = true; *abort_flag = 1; break; }
                 tc_fence_after();
-                const uint32_t sa = smem_u32(stages + stage * C::kStageBytes);
-                const uint64_t da = sdesc_sw128(sa);
-                const uint64_t db = sdesc_sw128(sa + C::kABytes);
+                const uint32_t sst = smem_u32(stages + stage * C::kStageBytes);
+                if (W8) {
+                    // A = the converters' bf16 slot in TMEM (8 columns per K step of 16),
+                    // B = the activation stage
+                    const uint32_t ta = tmem_base + (uint32_t)(C::kASlot0 + ab * C::kACols);
+                    const uint64_t db = sdesc_sw128(sst);
 #pragma unroll
-                for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                    const uint32_t accumulate = (kb != kb0 || kk != 0) ? 1u : 0u;
-                    // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
-                    umma_g<PAIR>(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                        const uint32_t accumulate = (kb != kb0 || kk != 0) ? 1u : 0u;
+                        umma_bf16_ta(d0, ta + 8 * kk, db + 2 * kk, idesc, accumulate);
+                    }
+                } else {
+                    const uint64_t da = sdesc_sw128(sst);
+                    const uint64_t db = sdesc_sw128(sst + C::kABytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                        const uint32_t accumulate = (kb != kb0 || kk != 0) ? 1u : 0u;
+                        // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
+                        umma_g<PAIR>(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
+                    }
                 }
                 umma_commit_g<PAIR>(&empty_bar[stage]);  // stage free (in both CTAs) once read
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                if (W8) {
+                    umma_commit_g<PAIR>(&aempty_bar[ab]);  // operand slot free (in both CTAs)
+                    if (++ab == C::kABufs) { ab = 0; abphase ^= 1u; }
+                }
             }
             if (failed) break;
             umma_commit_g<PAIR>(&tfull_bar[acc]);        // accumulator complete (in both CTAs)
             if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
         }
-    } else if (warp >= 2) {
+    } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------ epilogue
         // Per 32-row chunk every warp loads its TMEM lane quadrant (one feature, or one
         // half of a SwiGLU pair, across 32 rows) into a padded shared tile; after the
@@ -549,11 +701,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int rr = lane >> 3, j = lane & 7;
                 const int fv = feat * C::kFeatTile + (int)rank * C::kFeat + 8 * j;
                 uint16_t *outh = static_cast<uint16_t *>(out);
+                float sc = 1.0f;  // W8: the scale of this lane's weight row (W1 for g, W3 for u)
+                if (W8) {
+                    const int row = feat * C::kFeatTile + (int)rank * C::kFeat + fl;
+                    sc = row < Nout ? (q < 2 ? scale_a : scale_b)[(int64_t)g * Nout + row] : 0.0f;
+                }
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) mine[fl][c] = a[c];
+                    for (int c = 0; c < 32; ++c) mine[fl][c] = W8 ? a[c] * sc : a[c];
                     epilogue_sync();
                     // warp ew stores rows 8*ew .. 8*ew+7 of the chunk: 4 rows x 8 feature octets per step
 #pragma unroll
@@ -576,12 +733,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
                 const int fbase = feat * C::kFeatTile + (int)rank * C::kFeat + q * 32;
+                const float sc = W8 ? (fbase + lane < Nout ? scale_a[(int64_t)g * Nout + fbase + lane] : 0.0f) : 1.0f;
                 // fp32 out through the padded tile: 8 16-byte stores per 32 rows instead of
                 // 32 4-byte ones (store instruction issue, not bytes, limits short-K tiles)
                 float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + ew * 32 * 33);
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
+                    if (W8) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) a[c] *= sc;
+                    }
                     if (vec_ok) {
 #pragma unroll
                         for (int c = 0; c < 32; ++c) stage_t[lane][c] = a[c];
@@ -613,6 +775,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else mbar_arrive(&tempty_bar[acc]);
             }
             if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
+        }
+    }
+
+    if (W8 && warp >= 6 && warp < 14) {
+        // ------------------------------------------------------ converters (W8)
+        // A warp may only reach its own quadrant of TMEM lanes (warp % 4), so converter warp
+        // w takes rows [32 (w % 4), +32) -- one per lane -- and half kq = (w - 6) / 4 of
+        // every 64-wide K block: per fp8 tile (two K blocks) it widens 2 x 32 values a lane
+        // and stores them into the two K blocks' operand slots in TMEM.  The eight warps
+        // run on their own (no barrier between them): each waits, converts and arrives.
+        const int q = warp & 3, kq = (warp - 6) >> 2;
+        const int crow = 32 * q + lane;
+        const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(C::kASlot0 + 16 * kq);
+        int stage = 0, ab = 0;
+        uint32_t phase = 0, abphase = 0;
+        bool stop = false;
+        for (int item = unit; item < total && !stop; item += nunits) {
+            int g, feat, ks, row0, row_end, kb0, kb1;
+            decode(item, g, feat, ks, row0, row_end);
+            kslice(ks, kb0, kb1);
+            for (int kb = kb0; kb < kb1; kb += 2) {
+                // one fp8 tile -> the operand slots of its two K blocks (ab, ab + 1)
+                const bool ok = mbar_wait(&ffull_bar[stage], phase, abort_flag) &&
+                                mbar_wait(&aempty_bar[ab], abphase ^ 1u, abort_flag) &&
+                                mbar_wait(&aempty_bar[ab + 1], abphase ^ 1u, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) { stop = true; break; }
+                tc_fence_after();
+                uint32_t w0[16], w1[16];
+                widen_e4m3_32(fring + stage * C::kW8Bytes, crow, 0, kq, w0);
+                widen_e4m3_32(fring + stage * C::kW8Bytes, crow, 1, kq, w1);
+                tmem_st16(tq + (uint32_t)(ab * C::kACols), w0);
+                tmem_st16(tq + (uint32_t)((ab + 1) * C::kACols), w1);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&afull_bar[ab]);
+                    mbar_arrive(&afull_bar[ab + 1]);
+                    mbar_arrive(&fempty_bar[stage]);
+                }
+                ab += 2;
+                if (ab == C::kABufs) { ab = 0; abphase ^= 1u; }
+                if (++stage == C::kFStages) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (stop) { failed = true; *abort_flag = 1; }
+    } else if (W8 && warp == 14 && lane == 0) {
+        // ------------------------------------------------------ activation producer (W8)
+        tma_prefetch_map(&tm_act);
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int item = unit; item < total && !failed; item += nunits) {
+            int g, feat, ks, row0, row_end, kb0, kb1;
+            decode(item, g, feat, ks, row0, row_end);
+            kslice(ks, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&full_bar[stage], C::kBBytes);
+                tma_2d<false>(stages + stage * C::kStageBytes, &tm_act, kb * kBK, row0, smem_u32(&full_bar[stage]));
+                if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            }
         }
     }
 
@@ -662,6 +885,22 @@ bool encode_weight_map(CUtensorMap *m, const void *ptr, int groups, int Nout, in
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp8 (e4m3) weights [groups, Nout, K] as a 3-D byte map; box = 128 (K) x box_rows x 1:
+// 128-byte rows (two 64-wide K blocks per load, the same bytes per row request as the
+// bf16 tiles) with 128-byte swizzle.
+bool encode_weight_map_fp8(CUtensorMap *m, const void *ptr, int groups, int Nout, int K, int box_rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)Nout, (cuuint64_t)groups};
+    cuuint64_t strides[2] = {(cuuint64_t)K, (cuuint64_t)Nout * (cuuint64_t)K};
+    cuuint32_t box[3] = {(cuuint32_t)(2 * kBK), (cuuint32_t)box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Activations [R, K] bf16 as a 2-D map; box = 64 (K) x box_rows; rows >= R read as zero.
 bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_rows)
 {
@@ -676,20 +915,21 @@ bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_r
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU, bool PAIR>
+template <int BN, bool SWIGLU, bool PAIR, bool W8>
 cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
-    using C = Cfg<BN, SWIGLU, PAIR>;
+    using C = Cfg<BN, SWIGLU, PAIR, W8>;
     CUtensorMap ma, mb, mact;
     const int box_rows = SWIGLU ? kBM / 2 : kBM;
-    if (!encode_weight_map(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
+    auto enc_w = W8 ? encode_weight_map_fp8 : encode_weight_map;
+    if (!enc_w(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     if (SWIGLU) {
-        if (!encode_weight_map(&mb, a.w_b, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
+        if (!enc_w(&mb, a.w_b, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     } else {
         mb = ma;
     }
     if (!encode_act_map(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
-    auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR>;
+    auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR, W8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
     const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
@@ -697,7 +937,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     cfg.gridDim = dim3((unsigned)(PAIR ? (sms / 2) * 2 : sms));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = s;
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -709,7 +949,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = PAIR ? 2 : 1;
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
-                             ksplit, a.split_stride, a.dev_err);
+                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.dev_err);
     if (err != cudaSuccess) return err;
     count_launch();
     return cudaGetLastError();
@@ -727,7 +967,7 @@ int64_t gemm_pair_tiles(int64_t R, int groups, int Nout, bool swiglu, int ksplit
     return active * ((mean + bn - 1) / bn) * ((Nout + feat - 1) / feat) * (ksplit > 1 ? ksplit : 1);
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool W8>
 cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
@@ -737,18 +977,32 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
     // token tile, and the pair reads each activation tile once per 256 weight rows
     // instead of once per 128.  A tiny batch whose pair tiles would not even cover the
     // SM pairs once runs single-CTA tiles instead (twice the tiles, every SM streaming).
-    if (bn <= 64 && gemm_pair_tiles(a.R, a.groups, a.Nout, SWIGLU, a.ksplit) < device_sm_count() / 2) {
+    if (W8) {
+        // fp8 weights: single-CTA tiles.  A pair's MMA would read converted operands from
+        // the other CTA, which then has to signal every K step across the cluster.
+        // (token tiles up to 128 rows: two 256-column accumulators and the operand slots
+        // would not fit in TMEM's 512 columns)
         switch (bn) {
-            case 32: return launch_impl<32, SWIGLU, false>(a, s);
-            case 64: return launch_impl<64, SWIGLU, false>(a, s);
+            case 32: return launch_impl<32, SWIGLU, false, true>(a, s);
+            case 64: return launch_impl<64, SWIGLU, false, true>(a, s);
+            case 128:
+            case 256: return launch_impl<128, SWIGLU, false, true>(a, s);
+            default: return cudaErrorInvalidValue;
         }
-    }
-    switch (bn) {
-        case 32: return launch_impl<32, SWIGLU, true>(a, s);
-        case 64: return launch_impl<64, SWIGLU, true>(a, s);
-        case 128: return launch_impl<128, SWIGLU, true>(a, s);
-        case 256: return launch_impl<256, SWIGLU, true>(a, s);
-        default: return cudaErrorInvalidValue;
+    } else {
+        if (bn <= 64 && gemm_pair_tiles(a.R, a.groups, a.Nout, SWIGLU, a.ksplit) < device_sm_count() / 2) {
+            switch (bn) {
+                case 32: return launch_impl<32, SWIGLU, false, false>(a, s);
+                case 64: return launch_impl<64, SWIGLU, false, false>(a, s);
+            }
+        }
+        switch (bn) {
+            case 32: return launch_impl<32, SWIGLU, true, false>(a, s);
+            case 64: return launch_impl<64, SWIGLU, true, false>(a, s);
+            case 128: return launch_impl<128, SWIGLU, true, false>(a, s);
+            case 256: return launch_impl<256, SWIGLU, true, false>(a, s);
+            default: return cudaErrorInvalidValue;
+        }
     }
 }
 
@@ -801,7 +1055,16 @@ int gemm2_ksplit(int64_t R, int groups, int K, int Nout)
     return best;
 }
 
-cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s) { return launch_dispatch<true>(a, s); }
-cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s) { return launch_dispatch<false>(a, s); }
+cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s)
+{
+    if (a.w8 && (!a.scale_a || !a.scale_b)) return cudaErrorInvalidValue;
+    return a.w8 ? launch_dispatch<true, true>(a, s) : launch_dispatch<true, false>(a, s);
+}
+
+cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s)
+{
+    if (a.w8 && !a.scale_a) return cudaErrorInvalidValue;
+    return a.w8 ? launch_dispatch<false, true>(a, s) : launch_dispatch<false, false>(a, s);
+}
 
 }  // namespace moe

@@ -56,8 +56,11 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
 // of `rows_single` rows starting at row 0).
 struct GroupedGemmArgs {
     const uint16_t *act;     // [R, K] bf16
-    const uint16_t *w_a;     // [groups, Nout, K] bf16 (W1, or W2)
-    const uint16_t *w_b;     // [groups, Nout, K] bf16 (W3) -- SwiGLU only
+    const void *w_a;         // [groups, Nout, K] bf16, or e4m3 bytes when w8 (W1, or W2)
+    const void *w_b;         // [groups, Nout, K] likewise (W3) -- SwiGLU only
+    bool w8;                 // weights are e4m3 with one fp32 scale per row (scale_a, scale_b)
+    const float *scale_a;    // [groups, Nout] row scales of w_a (w8 only)
+    const float *scale_b;    // [groups, Nout] row scales of w_b (w8, SwiGLU only)
     const int32_t *offsets;  // [groups + 1] device, or nullptr
     int groups;
     int64_t R;               // rows of `act` (and of `out`)
@@ -75,6 +78,9 @@ cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s);
 int gemm_choose_token_tile(int64_t R, int groups, bool swiglu);
 int gemm2_ksplit(int64_t R, int groups, int K, int Nout);
 int device_sm_count();
+
+// e4m3 weights with one fp32 scale per row: q [rows, K] bytes, scale [rows].
+cudaError_t launch_quantize_fp8(const uint16_t *W, int64_t rows, int K, uint8_t *q, float *scale, cudaStream_t s);
 
 // Combine / unpermutation.
 // y_perm holds `nsplit` partial-sum buffers `split_stride` elements apart (1 = one).

@@ -225,6 +225,48 @@ MOE_API moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate
                                   void *const *phase_events);
 
 /*
+ * FP8 expert weights ([MoE-latency] "优化从测量开始": quantizing the weights cuts
+ * memory bytes; its numerical error is measured as an experiment of its own).
+ * The pages fix no format; this library uses OCP e4m3 bytes (largest finite 448)
+ * with one fp32 scale per output channel (weight row), and the weight a GEMM uses
+ * is e4m3(q) * scale.  Activations, routing, combine and shared experts stay as in
+ * the bf16 calls.
+ *
+ * moe_quantize_fp8: W [rows,K] bf16 -> q [rows,K] e4m3 bytes and scale [rows] fp32:
+ *   scale[r] = max_c |W[r,c]| / 448 (fp32, correctly rounded; 1 for an all-zero row),
+ *   q[r,c] = e4m3(W[r,c] / scale[r]) (fp32 quotient; nearest, ties to even; saturating).
+ *   Run once per weight set (W1 and W3 as [E*I, H], W2 as [E*H, I]).  K a multiple
+ *   of 64; W, q, scale 16-byte aligned device pointers.  Asynchronous on `stream`.
+ */
+MOE_API moe_status_t moe_quantize_fp8(const uint16_t *W, int64_t rows, int K, uint8_t *q, float *scale,
+                                      void *stream);
+
+/*
+ * moe_expert_ffn with e4m3 weights: W1q, W3q [E,I,H] and W2q [E,H,I] bytes, scales
+ * s1, s3 [E,I] and s2 [E,H] fp32 (from moe_quantize_fp8).  The grouped GEMMs stream
+ * the bytes and widen them to bf16 on chip; the products accumulate in fp32 and each
+ * output channel is multiplied by its scale before SwiGLU (W1/W3) or before the store
+ * (W2).  Other arguments, layouts and errors as moe_expert_ffn.
+ */
+MOE_API moe_status_t moe_expert_ffn_fp8(const uint16_t *x_perm, const int32_t *offsets, const uint8_t *W1q,
+                                        const float *s1, const uint8_t *W3q, const float *s3,
+                                        const uint8_t *W2q, const float *s2, int64_t R, int H, int I, int E,
+                                        float *y_perm, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * moe_layer_forward_ex with e4m3 routed-expert weights and their scales (as in
+ * moe_expert_ffn_fp8); the shared experts, when Is > 0, stay bf16.  Same workspace
+ * (moe_workspace_bytes), stream, phase events and errors as moe_layer_forward_ex.
+ */
+MOE_API moe_status_t moe_layer_forward_fp8_ex(const uint16_t *x, const float *W_gate, const float *bias,
+                                              const uint8_t *W1q, const float *s1, const uint8_t *W3q,
+                                              const float *s3, const uint8_t *W2q, const float *s2,
+                                              const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2,
+                                              int64_t N, int H, int I, int E, int k, int Is, uint16_t *out,
+                                              float *logits, void *ws, size_t ws_bytes, void *stream,
+                                              void *const *phase_events);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  *code receives a MOE_DEVERR_* value.  Returns MOE_OK, or
  * MOE_ERR_CUDA if the synchronisation itself failed.

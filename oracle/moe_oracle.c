@@ -256,9 +256,19 @@ typedef struct {
     const float *sc;
 } oracle_wmat;
 
+/* the 256 e4m3 values, filled from oracle_fp8_e4m3_to_double on first use */
+static double fp8_value[256];
+static int fp8_value_ready = 0;
+
 static double wval(const oracle_wmat *m, int64_t row, int K, int c)
 {
-    if (m->w8) return oracle_fp8_e4m3_to_double(m->w8[row * K + c]) * (double)m->sc[row];
+    if (m->w8) {
+        if (!fp8_value_ready) {
+            for (int i = 0; i < 256; ++i) fp8_value[i] = oracle_fp8_e4m3_to_double((uint8_t)i);
+            fp8_value_ready = 1;
+        }
+        return fp8_value[m->w8[row * K + c]] * (double)m->sc[row];
+    }
     return oracle_bf16_to_double(m->w16[row * K + c]);
 }
 

@@ -57,6 +57,15 @@ def test_invalid_arguments_are_rejected_before_any_launch():
     assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, -1, 256, 512, 8, nullp, nullp, 0, s) == 1
     assert L.moe_expert_ffn(nullp, nullp, nullp, nullp, nullp, 8, 256, 500, 8, nullp, nullp, 0, s) == 1
     assert L.moe_combine(nullp, nullp, nullp, nullp, 4, 256, 0, nullp, s) == 1
+    # fp8 weights: bad K, negative rows, null pointers, missing scales
+    assert L.moe_quantize_fp8(nullp, 4, 100, nullp, nullp, s) == 1
+    assert L.moe_quantize_fp8(nullp, -1, 256, nullp, nullp, s) == 1
+    assert L.moe_quantize_fp8(nullp, 4, 256, nullp, nullp, s) == 1
+    assert L.moe_quantize_fp8(nullp, 0, 256, nullp, nullp, s) == 0          # nothing to do
+    assert L.moe_expert_ffn_fp8(*([nullp] * 8), 8, 256, 500, 8, nullp, nullp, 0, s) == 1
+    assert L.moe_expert_ffn_fp8(*([nullp] * 8), 8, 256, 512, 8, nullp, nullp, 0, s) == 1
+    assert L.moe_layer_forward_fp8_ex(*([nullp] * 12), 4, 256, 512, 8, 2, 0, nullp, nullp, nullp, 0, s,
+                                      nullp) == 1
     assert L.moe_layer_forward(nullp, nullp, nullp, nullp, nullp, 4, 256, 512, 8, 2, nullp) == 1
     assert L.moe_layer_forward_ex(*([nullp] * 9), 4, 256, 512, 8, 2, 64, nullp, nullp, nullp, 0, s,
                                   nullp) == 1
@@ -73,6 +82,8 @@ def test_misaligned_pointers_are_unsupported():
     s = ctypes.c_void_p(0)
     assert L.moe_route(fake, ok, None, 4, 256, 8, 2, None, ok, ok, None, 0, s) == 2
     assert L.moe_combine(fake, ok, ok, None, 4, 256, 2, ok, s) == 2
+    assert L.moe_quantize_fp8(fake, 4, 256, ok, ok, s) == 2
+    assert L.moe_quantize_fp8(ok, 4, 256, fake, ok, s) == 2
 
 
 def test_status_strings():
