@@ -289,17 +289,33 @@ def run_ours(args, cfg, world, rank, local):
         q = {n: moe.moe_quantize_fp8(t[n], stream=stream) for n in ("W1", "W3", "W2")}
         torch.cuda.synchronize()
 
-    def step(events=None, x=None, o=None):
+    def step(events=None, x=None, o=None, st=None):
         xx = t["x"] if x is None else x
         oo = out if o is None else o
+        ss = stream if st is None else st
         if fp8:
             moe.moe_layer_forward_fp8_ex(xx, t["W_gate"], *q["W1"], *q["W3"], *q["W2"], k, bias=t["bias"],
-                                         Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=stream,
+                                         Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=ss,
                                          phase_events=events)
         else:
             moe.moe_layer_forward_ex(xx, t["W_gate"], t["W1"], t["W3"], t["W2"], k, bias=t["bias"],
-                                     Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=stream,
+                                     Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=ss,
                                      phase_events=events)
+
+    graph = None
+    graph_launches = 0
+    if args.graph:
+        # one layer step captured as a CUDA graph (the library only enqueues kernels on the
+        # stream it is given), replayed once per timed step
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        n0 = moe.moe_kernel_launches()
+        with torch.cuda.graph(graph):
+            step(st=torch.cuda.current_stream())
+        graph_launches = moe.moe_kernel_launches() - n0
+        torch.cuda.synchronize()
 
     for _ in range(args.warmup):
         step()
@@ -330,9 +346,12 @@ def run_ours(args, cfg, world, rank, local):
         n0 = moe.moe_kernel_launches()
         start.record(stream)
         for i in range(args.steps):
-            step()
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
         end.record(stream)
-        launches = moe.moe_kernel_launches() - n0
+        launches = moe.moe_kernel_launches() - n0 if graph is None else graph_launches * args.steps
         torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = start.elapsed_time(end)
@@ -445,7 +464,9 @@ def run_ours(args, cfg, world, rank, local):
         "phase_ms": phase_ms,
         "phase_ms_note": "mean per-phase CUDA-event times from a second timed pass with events between phases",
         "gpu_launches": launches,
-        "gpu_launches_note": "the library's own host-side count of its kernel launches over the timed steps",
+        "gpu_launches_note": ("the library's own host-side count of its kernel launches over the timed steps" +
+                              (" (counted once at graph capture, times the replays)" if graph is not None else "")),
+        "launch_mode": "cuda graph replay of one captured step" if graph is not None else "stream launches",
         "e2e": e2e,
     }
     if fp8_err is not None:
@@ -494,6 +515,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=12)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of one layer step captured as a CUDA graph (launch-bound decode sizes)")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
                     help="routed-expert weight format (fp8: e4m3 with per-channel scales, a separate experiment)")
     args = ap.parse_args()

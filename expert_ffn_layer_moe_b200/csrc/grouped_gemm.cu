@@ -107,7 +107,7 @@ struct Cfg {
     static constexpr int kAccBufs = 2;
     static constexpr int kASlot0 = kAccBufs * kAccCols;    // W8: first TMEM column of the operand slots
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols + kABufs * kACols);
-    static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs + 2 * kFStages + 2 * kABufs);
+    static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs + 2 * kFStages + kABufs);
     static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
     static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // staging: 4 x [32][33] fp32 (= 2 x [64][33])
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kFStages * kW8Bytes + kBarBytes + 16 +
@@ -457,8 +457,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
     uint64_t *ffull_bar = tempty_bar + C::kAccBufs;             // W8: fp8 tile landed
     uint64_t *fempty_bar = ffull_bar + C::kFStages;             // W8: fp8 tile read by every converter warp
     uint64_t *afull_bar = fempty_bar + C::kFStages;             // W8: operand slot written by every converter warp
-    uint64_t *aempty_bar = afull_bar + C::kABufs;               // W8: operand slot read by the MMA
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(aempty_bar + C::kABufs);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(afull_bar + C::kABufs);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
@@ -484,7 +483,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
         }
         if (W8) {
             for (int j = 0; j < C::kFStages; ++j) { mbar_init(&ffull_bar[j], 1); mbar_init(&fempty_bar[j], 8); }
-            for (int a = 0; a < C::kABufs; ++a) { mbar_init(&afull_bar[a], 8); mbar_init(&aempty_bar[a], 1); }
+            for (int a = 0; a < C::kABufs; ++a) mbar_init(&afull_bar[a], 8);  // every converter warp
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -660,7 +659,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
                 umma_commit_g<PAIR>(&empty_bar[stage]);  // stage free (in both CTAs) once read
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
                 if (W8) {
-                    umma_commit_g<PAIR>(&aempty_bar[ab]);  // operand slot free (in both CTAs)
+                    // the operand slot is free when this K block's MMAs complete, which the
+                    // commit above already signals on the activation stage's barrier
                     if (++ab == C::kABufs) { ab = 0; abphase ^= 1u; }
                 }
             }
@@ -788,18 +788,28 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
         const int q = warp & 3, kq = (warp - 6) >> 2;
         const int crow = 32 * q + lane;
         const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(C::kASlot0 + 16 * kq);
+        static_assert(!W8 || C::kStages > C::kABufs, "the activation ring must be deeper than the operand slots");
         int stage = 0, ab = 0;
-        uint32_t phase = 0, abphase = 0;
+        int64_t kbn = 0;  // K blocks of this CTA's sequence converted so far
+        uint32_t phase = 0;
         bool stop = false;
         for (int item = unit; item < total && !stop; item += nunits) {
             int g, feat, ks, row0, row_end, kb0, kb1;
             decode(item, g, feat, ks, row0, row_end);
             kslice(ks, kb0, kb1);
             for (int kb = kb0; kb < kb1; kb += 2) {
-                // one fp8 tile -> the operand slots of its two K blocks (ab, ab + 1)
-                const bool ok = mbar_wait(&ffull_bar[stage], phase, abort_flag) &&
-                                mbar_wait(&aempty_bar[ab], abphase ^ 1u, abort_flag) &&
-                                mbar_wait(&aempty_bar[ab + 1], abphase ^ 1u, abort_flag);
+                // one fp8 tile -> the operand slots of its two K blocks (ab, ab + 1).  Slot
+                // reuse: K block n takes the slot of K block n - kABufs, free once that K
+                // block's MMAs completed -- the commit on its activation stage's barrier
+                // (the activation ring is deeper than kABufs, so that barrier cannot have
+                // moved two phases past the one waited for)
+                bool ok = mbar_wait(&ffull_bar[stage], phase, abort_flag);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int64_t m = kbn + h - C::kABufs;  // the K block that last used the slot
+                    if (m >= 0)
+                        ok = ok && mbar_wait(&empty_bar[m % C::kStages], (uint32_t)((m / C::kStages) & 1), abort_flag);
+                }
                 if (!__all_sync(0xffffffffu, ok)) { stop = true; break; }
                 tc_fence_after();
                 uint32_t w0[16], w1[16];
@@ -816,7 +826,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
                     mbar_arrive(&fempty_bar[stage]);
                 }
                 ab += 2;
-                if (ab == C::kABufs) { ab = 0; abphase ^= 1u; }
+                kbn += 2;
+                if (ab == C::kABufs) ab = 0;
                 if (++stage == C::kFStages) { stage = 0; phase ^= 1u; }
             }
         }

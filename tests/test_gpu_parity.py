@@ -297,6 +297,34 @@ def test_layer_empty_batch_is_a_no_op():
     assert moe.moe_get_device_error() == 0
 
 
+@pytest.mark.parametrize("cfg", [CONFIGS["tiny"], MoEConfig("graph", N=300, H=256, I=384, E=16, k=4)])
+def test_layer_replays_from_a_cuda_graph(cfg):
+    """The explicit call only enqueues kernels on its stream (no allocation, no host
+    synchronisation), so one step captured as a CUDA graph replays to the same bits."""
+    t = cuda_inputs(cfg, seed=2)
+    ws = torch.empty(moe.moe_workspace_bytes(cfg.N, cfg.H, cfg.I, cfg.E, cfg.k, 0), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((cfg.N, cfg.H), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k, ws=ws, out=out,
+                                 stream=torch.cuda.current_stream())
+
+    step()
+    torch.cuda.synchronize()
+    eager = out.clone()
+    out.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error() == 0
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    del g
+
+
 def test_layer_is_deterministic():
     cfg = MoEConfig("det", N=500, H=256, I=256, E=8, k=2)
     t = cuda_inputs(cfg, seed=9)
