@@ -59,6 +59,7 @@
 // tiles to cover the SMs; the consumer adds them in a fixed order, so results stay
 // deterministic.  Every wait is bounded (globaltimer): on expiry the kernel records
 // MOE_DEVERR_PIPELINE_TIMEOUT, lets in-flight copies drain, frees TMEM and returns.
+#include <cmath>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -996,7 +997,9 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
         switch (bn) {
             case 32: return launch_impl<32, SWIGLU, false, true>(a, s);
             case 64: return launch_impl<64, SWIGLU, false, true>(a, s);
+            case 96:
             case 128:
+            case 192:
             case 256: return launch_impl<128, SWIGLU, false, true>(a, s);
             default: return cudaErrorInvalidValue;
         }
@@ -1010,7 +1013,9 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
         switch (bn) {
             case 32: return launch_impl<32, SWIGLU, true, false>(a, s);
             case 64: return launch_impl<64, SWIGLU, true, false>(a, s);
+            case 96: return launch_impl<96, SWIGLU, true, false>(a, s);
             case 128: return launch_impl<128, SWIGLU, true, false>(a, s);
+            case 192: return launch_impl<192, SWIGLU, true, false>(a, s);
             case 256: return launch_impl<256, SWIGLU, true, false>(a, s);
             default: return cudaErrorInvalidValue;
         }
@@ -1031,17 +1036,21 @@ int device_sm_count()
     return n;
 }
 
-// Token tile from the mean rows per group.  The MMA width follows each tile's rows,
+// Token tile from the expected largest group.  The MMA width follows each tile's rows,
 // so a wide tile wastes no tensor work on a short group; what a wide tile costs is
-// shared memory (fewer pipeline stages).  Groups then fit in one tile where possible,
-// so each weight tile streams through shared memory once.
+// shared memory (fewer pipeline stages, so fewer weight bytes in flight from HBM).
+// Groups should fit in one tile where possible, so each weight tile streams through
+// shared memory once: the tile covers the mean rows per group plus three standard
+// deviations of a balanced routing (mean + 3 sqrt(mean)), rounded up to the tiles
+// compiled (32, 64, 96, 128, 192, 256).
 int gemm_choose_token_tile(int64_t R, int groups, bool swiglu)
 {
     (void)swiglu;
-    const int64_t mean = (R + groups - 1) / (groups > 0 ? groups : 1);
-    if (mean <= 24) return 32;
-    if (mean <= 48) return 64;
-    if (mean <= 112) return 128;
+    const double mean = (double)R / (groups > 0 ? groups : 1);
+    const double want = mean + 3.0 * std::sqrt(mean);
+    static const int tiles[] = {32, 64, 96, 128, 192, 256};
+    for (int t : tiles)
+        if (want <= t) return t;
     return 256;
 }
 
