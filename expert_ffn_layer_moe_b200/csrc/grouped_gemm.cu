@@ -26,7 +26,7 @@
 // drains its own TMEM.  An activation tile is then read once per 256 weight rows.  Tiny
 // batches whose tiles would not cover the SM pairs use single-CTA tiles (PAIR = false).
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work items):
+// Warp roles (192 threads -- 480 with W8, below -- one CTA per SM, persistent over work items):
 //   warp 0 lane 0 : TMA producer -- the 128-row weight tile and this CTA's part of the
 //                   token tile per stage, 128-byte swizzle, mbarrier transaction counts;
 //   warp 1        : TMEM allocator; lane 0 of the leader issues tcgen05.mma (bf16 in,
@@ -34,8 +34,8 @@
 //                   accumulators over;
 //   warps 2..5    : epilogue -- tcgen05.ld of the accumulator (one TMEM lane quadrant
 //                   per warp), staged through shared memory into 16-byte row stores.
-// TMEM holds two accumulators of BN columns, so one tile's epilogue overlaps the next
-// tile's main loop.  Barrier set-up and TMEM allocation run before the kernel waits on
+// TMEM holds two accumulators of BN columns (W8: and four 32-column operand slots), so
+// one tile's epilogue overlaps the next tile's main loop.  Barrier set-up and TMEM allocation run before the kernel waits on
 // the previous kernel in the stream (programmatic dependent launch).
 //
 // fp8 weights (W8 = true; MoE-latency article, section "优化从测量开始": quantized
