@@ -16,7 +16,11 @@ scaling invariants; e4m3 decoding against the format's own table of special
 values and every code, encoding against nearest-value search over all codes with
 ties to the even code, the quantizer's per-row scale and error bounds, and the
 fp8 layer against the bf16 layer on weights that the quantizer represents
-exactly.  No function is left unpinned.
+exactly; with activations quantized too, the experts against the weight-only
+experts on rows the quantizer represents exactly, against a float64 BLAS
+statement fed the quantizer's dequantized rows, and against exact per-row
+power-of-two scaling, and the layer against its pinned steps.  No function is
+left unpinned.
 """
 from __future__ import annotations
 
@@ -95,6 +99,13 @@ def lib():
             [_P(u16), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u16), _P(u16),
              _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f64)])
         L.oracle_layer_given_logits_fp8.restype = c_int
+        L.oracle_expert_ffn_fp8_ex.argtypes = [_P(u16), _P(i32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8),
+                                               _P(f32), c_int, c_int, c_int, c_int, _P(u16), _P(f64), _P(u16)]
+        L.oracle_expert_ffn_fp8_ex.restype = None
+        L.oracle_layer_given_logits_fp8_ex.argtypes = (
+            [_P(u16), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u16), _P(u16),
+             _P(u16), i64] + [c_int] * 6 + [_P(u16), _P(u16), _P(f64)])
+        L.oracle_layer_given_logits_fp8_ex.restype = c_int
         _lib = L
     return _lib
 
@@ -319,3 +330,47 @@ def layer_given_logits_fp8(x, logits32, q1, s1, q3, s3, q2, s2, k, Ws1=None, Ws3
     if rc:
         raise ValueError("oracle_layer_given_logits_fp8 failed")
     return out
+
+
+# ------------------------------------------------ fp8 weights and fp8 activations
+
+def expert_ffn_fp8_ex(x_perm, offsets, q1, s1, q3, s3, q2, s2, quantize_acts, h_given=None):
+    """e4m3-weight experts; quantize_acts also quantizes each row of x_perm and of h
+    per row.  h_given [R,I] bf16 (uint16) replaces the computed h as the second GEMM's
+    input.  Returns (y_perm float64 [R,H], the computed h uint16 [R,I])."""
+    x_perm = _u16(x_perm); offsets = _i32(offsets)
+    q1, q3, q2 = _u8(q1), _u8(q3), _u8(q2)
+    s1, s3, s2 = _f32(s1), _f32(s3), _f32(s2)
+    h_given = _u16(h_given)
+    E, I, H = q1.shape
+    R = x_perm.shape[0]
+    y = np.zeros((R, H), np.float64)
+    h = np.zeros((R, I), np.uint16)
+    lib().oracle_expert_ffn_fp8_ex(_ptr(x_perm, U16), _ptr(offsets, I32), _ptr(q1, U8), _ptr(s1, F32),
+                                   _ptr(q3, U8), _ptr(s3, F32), _ptr(q2, U8), _ptr(s2, F32), E, H, I,
+                                   1 if quantize_acts else 0, _ptr(h_given, U16), _ptr(y, F64), _ptr(h, U16))
+    return y, h
+
+
+def layer_given_logits_fp8_ex(x, logits32, q1, s1, q3, s3, q2, s2, k, quantize_acts, h_given=None,
+                              Ws1=None, Ws3=None, Ws2=None, want_y=False):
+    """The e4m3-weight layer from fp32 logits with the activation options above;
+    h_given [N*k, I] bf16 is in assignment order (row t*k + j: token t's j-th pick).
+    Returns out (uint16 [N,H]), and y_perm (float64 [N*k,H]) with want_y."""
+    x = _u16(x); l = _f32(logits32)
+    q1, q3, q2 = _u8(q1), _u8(q3), _u8(q2)
+    s1, s3, s2 = _f32(s1), _f32(s3), _f32(s2)
+    Ws1 = _u16(Ws1); Ws3 = _u16(Ws3); Ws2 = _u16(Ws2)
+    h_given = _u16(h_given)
+    N, H = x.shape
+    E, I, _ = q1.shape
+    Is = 0 if Ws1 is None else Ws1.shape[0]
+    out = np.zeros((N, H), np.uint16)
+    y = np.zeros((N * k, H), np.float64) if want_y else None
+    rc = lib().oracle_layer_given_logits_fp8_ex(
+        _ptr(x, U16), _ptr(l, F32), _ptr(q1, U8), _ptr(s1, F32), _ptr(q3, U8), _ptr(s3, F32),
+        _ptr(q2, U8), _ptr(s2, F32), _ptr(Ws1, U16), _ptr(Ws3, U16), _ptr(Ws2, U16), N, H, I, E, k, Is,
+        1 if quantize_acts else 0, _ptr(h_given, U16), _ptr(out, U16), _ptr(y, F64))
+    if rc:
+        raise ValueError("oracle_layer_given_logits_fp8_ex failed")
+    return (out, y) if want_y else out

@@ -52,7 +52,12 @@
  *    largest finite 448) with one fp32 scale per output channel (weight row):
  *    s = max|row| / 448 in fp32, q = e4m3(w / s) rounded to nearest even with
  *    magnitudes past 448 kept at 448; the weight the FFN uses is e4m3(q) * s.
- *    Activations, routing, combine and the shared experts are unchanged.
+ *    Activations, routing, combine and the shared experts are unchanged;
+ *  - fp8 activations as well (the same section names activations beside
+ *    weights): each row the two routed GEMMs read -- a permuted token row x and
+ *    a row of h after its bf16 rounding -- goes through the same per-row
+ *    quantizer, and the GEMM uses e4m3(q) * s for it.  Routing, combine and the
+ *    shared experts are unchanged.
  *
  * Layouts: x [N,H] bf16 (uint16 storage); W_gate [H,E] fp32; bias [E] fp32 or
  * NULL; W1, W3 [E,I,H] bf16; W2 [E,H,I] bf16; Ws1, Ws3 [Is,H] bf16;
@@ -260,36 +265,60 @@ typedef struct {
 static double fp8_value[256];
 static int fp8_value_ready = 0;
 
+static double fp8_val(uint8_t q)
+{
+    if (!fp8_value_ready) {
+        for (int i = 0; i < 256; ++i) fp8_value[i] = oracle_fp8_e4m3_to_double((uint8_t)i);
+        fp8_value_ready = 1;
+    }
+    return fp8_value[q];
+}
+
 static double wval(const oracle_wmat *m, int64_t row, int K, int c)
 {
-    if (m->w8) {
-        if (!fp8_value_ready) {
-            for (int i = 0; i < 256; ++i) fp8_value[i] = oracle_fp8_e4m3_to_double((uint8_t)i);
-            fp8_value_ready = 1;
-        }
-        return fp8_value[m->w8[row * K + c]] * (double)m->sc[row];
-    }
+    if (m->w8) return fp8_val(m->w8[row * K + c]) * (double)m->sc[row];
     return oracle_bf16_to_double(m->w16[row * K + c]);
+}
+
+/* The values a GEMM reads for one bf16 activation row of K elements: the row
+ * itself, or (quantize != 0) e4m3(q) * s from the per-row quantizer above. */
+static void act_row(const uint16_t *row, int K, int quantize, double *d)
+{
+    if (quantize) {
+        uint8_t *q = (uint8_t *)malloc((size_t)K);
+        float s;
+        oracle_quantize_rows_fp8(row, 1, K, q, &s);
+        for (int c = 0; c < K; ++c) d[c] = fp8_val(q[c]) * (double)s;
+        free(q);
+    } else {
+        for (int c = 0; c < K; ++c) d[c] = oracle_bf16_to_double(row[c]);
+    }
 }
 
 /* [FinDEP] "核心公式": an expert is three GEMMs; here the SwiGLU expert
  * y = W2 (silu(W1 x) * (W3 x)).  One row through the expert whose W1/W3 rows
  * start at r13 and whose W2 rows start at r2.  fp64 sums; h rounded to bf16,
- * y left in fp64. */
+ * y left in fp64.  qa != 0 quantizes the activation rows (x, and h after its
+ * rounding) as described at the top.  h_out (may be NULL) receives the bf16 h;
+ * h_given (may be NULL) replaces it as the second GEMM's input. */
 static void swiglu_row(const uint16_t *xrow, const oracle_wmat *W1, const oracle_wmat *W3,
-                       const oracle_wmat *W2, int64_t r13, int64_t r2, int H, int I, double *yrow)
+                       const oracle_wmat *W2, int64_t r13, int64_t r2, int H, int I, int qa,
+                       const uint16_t *h_given, uint16_t *h_out, double *yrow)
 {
     double *xd = (double *)malloc((size_t)H * sizeof(double));
     double *hd = (double *)malloc((size_t)I * sizeof(double));
-    for (int c = 0; c < H; ++c) xd[c] = oracle_bf16_to_double(xrow[c]);
+    uint16_t *hb = (uint16_t *)malloc((size_t)I * sizeof(uint16_t));
+    act_row(xrow, H, qa, xd);
     for (int i = 0; i < I; ++i) {
         double g = 0.0, u = 0.0;
         for (int c = 0; c < H; ++c) {
             g += xd[c] * wval(W1, r13 + i, H, c);
             u += xd[c] * wval(W3, r13 + i, H, c);
         }
-        hd[i] = oracle_bf16_to_double(oracle_round_to_bf16(silu(g) * u));
+        hb[i] = oracle_round_to_bf16(silu(g) * u);
     }
+    if (h_out) memcpy(h_out, hb, (size_t)I * sizeof(uint16_t));
+    act_row(h_given ? h_given : hb, I, qa, hd);
     for (int o = 0; o < H; ++o) {
         double y = 0.0;
         for (int i = 0; i < I; ++i) y += hd[i] * wval(W2, r2 + o, I, i);
@@ -297,6 +326,7 @@ static void swiglu_row(const uint16_t *xrow, const oracle_wmat *W1, const oracle
     }
     free(xd);
     free(hd);
+    free(hb);
 }
 
 /* One row, one expert with bf16 weights: W1, W3 [I,H], W2 [H,I]. */
@@ -304,18 +334,20 @@ void oracle_swiglu_ffn(const uint16_t *xrow, const uint16_t *W1, const uint16_t 
                        const uint16_t *W2, int H, int I, double *yrow)
 {
     oracle_wmat a = {W1, NULL, NULL}, b = {W3, NULL, NULL}, c = {W2, NULL, NULL};
-    swiglu_row(xrow, &a, &b, &c, 0, 0, H, I, yrow);
+    swiglu_row(xrow, &a, &b, &c, 0, 0, H, I, 0, NULL, NULL, yrow);
 }
 
 /* [MoE-latency] "router 之后还有一串动作": each expert runs its own rows.
- * Rows offsets[e] .. offsets[e+1]-1 of x_perm go through expert e. */
+ * Rows offsets[e] .. offsets[e+1]-1 of x_perm go through expert e.  h_given
+ * and h_out (may be NULL) are [R,I] in the same (permuted) row order. */
 static void expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const oracle_wmat *W1,
-                       const oracle_wmat *W3, const oracle_wmat *W2, int E, int H, int I,
-                       double *y_perm)
+                       const oracle_wmat *W3, const oracle_wmat *W2, int E, int H, int I, int qa,
+                       const uint16_t *h_given, uint16_t *h_out, double *y_perm)
 {
     for (int e = 0; e < E; ++e)
         for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r)
-            swiglu_row(x_perm + r * H, W1, W3, W2, (int64_t)e * I, (int64_t)e * H, H, I,
+            swiglu_row(x_perm + r * H, W1, W3, W2, (int64_t)e * I, (int64_t)e * H, H, I, qa,
+                       h_given ? h_given + r * I : NULL, h_out ? h_out + r * I : NULL,
                        y_perm + r * H);
 }
 
@@ -324,7 +356,7 @@ void oracle_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uin
                        double *y_perm)
 {
     oracle_wmat a = {W1, NULL, NULL}, b = {W3, NULL, NULL}, c = {W2, NULL, NULL};
-    expert_ffn(x_perm, offsets, &a, &b, &c, E, H, I, y_perm);
+    expert_ffn(x_perm, offsets, &a, &b, &c, E, H, I, 0, NULL, NULL, y_perm);
 }
 
 /* [MoE-latency] "优化从测量开始": the same experts with e4m3 weights q1, q3
@@ -334,7 +366,23 @@ void oracle_expert_ffn_fp8(const uint16_t *x_perm, const int32_t *offsets, const
                            const float *s2, int E, int H, int I, double *y_perm)
 {
     oracle_wmat a = {NULL, q1, s1}, b = {NULL, q3, s3}, c = {NULL, q2, s2};
-    expert_ffn(x_perm, offsets, &a, &b, &c, E, H, I, y_perm);
+    expert_ffn(x_perm, offsets, &a, &b, &c, E, H, I, 0, NULL, NULL, y_perm);
+}
+
+/* The e4m3-weight experts with the two activation options: quantize_acts != 0
+ * quantizes every row of x_perm and of h per row as well (e4m3 with one fp32
+ * scale, as for the weights).  h_given [R,I] bf16 (may be NULL) replaces the
+ * computed h as the second GEMM's input -- so that a caller can hand in h as
+ * another implementation rounded it and take the quantization decision on the
+ * same values; h_out [R,I] (may be NULL) receives the computed bf16 h. */
+void oracle_expert_ffn_fp8_ex(const uint16_t *x_perm, const int32_t *offsets, const uint8_t *q1,
+                              const float *s1, const uint8_t *q3, const float *s3,
+                              const uint8_t *q2, const float *s2, int E, int H, int I,
+                              int quantize_acts, const uint16_t *h_given, double *y_perm,
+                              uint16_t *h_out)
+{
+    oracle_wmat a = {NULL, q1, s1}, b = {NULL, q3, s3}, c = {NULL, q2, s2};
+    expert_ffn(x_perm, offsets, &a, &b, &c, E, H, I, quantize_acts != 0, h_given, h_out, y_perm);
 }
 
 /* ------------------------------------------------------------- combine ---- */
@@ -365,8 +413,9 @@ void oracle_combine(const double *y_perm, const int32_t *token_to_row, const dou
 static int layer_core(const uint16_t *x, const float *logits, const oracle_wmat *W1,
                       const oracle_wmat *W3, const oracle_wmat *W2, const uint16_t *Ws1,
                       const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I, int E, int k,
-                      int Is, uint16_t *out, int32_t *idx_out, double *w_out, int32_t *counts_out,
-                      int32_t *offsets_out, int32_t *r2t_out, int32_t *t2r_out, double *y_perm_out)
+                      int Is, int qa, const uint16_t *h_given_tok, uint16_t *out, int32_t *idx_out,
+                      double *w_out, int32_t *counts_out, int32_t *offsets_out, int32_t *r2t_out,
+                      int32_t *t2r_out, double *y_perm_out)
 {
     if (N < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E || Is < 0) return -1;
     int64_t R = N * k;
@@ -380,11 +429,20 @@ static int layer_core(const uint16_t *x, const float *logits, const oracle_wmat 
     uint16_t *xp = (uint16_t *)malloc((size_t)(R ? R : 1) * H * sizeof(uint16_t));
     double *yp = (double *)malloc((size_t)(R ? R : 1) * H * sizeof(double));
     double *s = NULL;
+    uint16_t *hp = NULL;
     if (!idx || !w || !counts || !offsets || !r2t || !t2r || !xp || !yp) goto done;
     if (oracle_topk(logits, N, E, k, idx, w)) goto done;
     if (oracle_dispatch(idx, N, E, k, counts, offsets, r2t, t2r)) goto done;
     oracle_permute_rows(x, r2t, R, H, xp);
-    expert_ffn(xp, offsets, W1, W3, W2, E, H, I, yp);
+    if (h_given_tok) {
+        /* given h rows come in assignment order a = t*k + j; the experts read
+         * them in permuted order, at row token_to_row[a] */
+        hp = (uint16_t *)malloc((size_t)(R ? R : 1) * I * sizeof(uint16_t));
+        if (!hp) goto done;
+        for (int64_t a = 0; a < R; ++a)
+            memcpy(hp + (int64_t)t2r[a] * I, h_given_tok + a * I, (size_t)I * sizeof(uint16_t));
+    }
+    expert_ffn(xp, offsets, W1, W3, W2, E, H, I, qa, hp, NULL, yp);
     if (Is > 0) {
         s = (double *)malloc((size_t)(N ? N : 1) * H * sizeof(double));
         if (!s) goto done;
@@ -401,7 +459,7 @@ static int layer_core(const uint16_t *x, const float *logits, const oracle_wmat 
     rc = 0;
 done:
     free(idx); free(w); free(counts); free(offsets); free(r2t); free(t2r); free(xp); free(yp);
-    free(s);
+    free(s); free(hp);
     return rc;
 }
 
@@ -413,8 +471,8 @@ int oracle_layer_given_logits(const uint16_t *x, const float *logits, const uint
                               int32_t *r2t_out, int32_t *t2r_out, double *y_perm_out)
 {
     oracle_wmat a = {W1, NULL, NULL}, b = {W3, NULL, NULL}, c = {W2, NULL, NULL};
-    return layer_core(x, logits, &a, &b, &c, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, idx_out, w_out,
-                      counts_out, offsets_out, r2t_out, t2r_out, y_perm_out);
+    return layer_core(x, logits, &a, &b, &c, Ws1, Ws3, Ws2, N, H, I, E, k, Is, 0, NULL, out, idx_out,
+                      w_out, counts_out, offsets_out, r2t_out, t2r_out, y_perm_out);
 }
 
 /* The same path with e4m3 routed-expert weights (q1, q3 [E,I,H], q2 [E,H,I])
@@ -426,8 +484,24 @@ int oracle_layer_given_logits_fp8(const uint16_t *x, const float *logits, const 
                                   int E, int k, int Is, uint16_t *out, double *y_perm_out)
 {
     oracle_wmat a = {NULL, q1, s1}, b = {NULL, q3, s3}, c = {NULL, q2, s2};
-    return layer_core(x, logits, &a, &b, &c, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, NULL, NULL,
-                      NULL, NULL, NULL, NULL, y_perm_out);
+    return layer_core(x, logits, &a, &b, &c, Ws1, Ws3, Ws2, N, H, I, E, k, Is, 0, NULL, out, NULL,
+                      NULL, NULL, NULL, NULL, NULL, y_perm_out);
+}
+
+/* The e4m3-weight layer with the activation options of oracle_expert_ffn_fp8_ex:
+ * quantize_acts != 0 quantizes the routed experts' activation rows; h_given_tok
+ * (may be NULL) is [N*k, I] bf16 in assignment order (row a = t*k + j is the h
+ * of token t's j-th pick) and replaces the computed h. */
+int oracle_layer_given_logits_fp8_ex(const uint16_t *x, const float *logits, const uint8_t *q1,
+                                     const float *s1, const uint8_t *q3, const float *s3,
+                                     const uint8_t *q2, const float *s2, const uint16_t *Ws1,
+                                     const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H,
+                                     int I, int E, int k, int Is, int quantize_acts,
+                                     const uint16_t *h_given_tok, uint16_t *out, double *y_perm_out)
+{
+    oracle_wmat a = {NULL, q1, s1}, b = {NULL, q3, s3}, c = {NULL, q2, s2};
+    return layer_core(x, logits, &a, &b, &c, Ws1, Ws3, Ws2, N, H, I, E, k, Is, quantize_acts != 0,
+                      h_given_tok, out, NULL, NULL, NULL, NULL, NULL, NULL, y_perm_out);
 }
 
 /* The whole layer from x: fp64 logits rounded to fp32 (the precision the

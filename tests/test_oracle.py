@@ -362,13 +362,14 @@ def test_quantizer_scale_codes_and_error_bound():
     assert np.all(err <= bound)
 
 
-def _grid_weights(rng, shape):
-    """bf16 weights that are e4m3 values times a power of two per row, each row
-    holding +-448 times that power: the quantizer represents them exactly."""
+def _grid_weights(rng, shape, jlo=-14, jhi=-6):
+    """bf16 rows that are e4m3 values times a power of two 2^j per row (j in
+    [jlo, jhi)), each row holding +-448 times that power: the per-row quantizer
+    represents them exactly."""
     pos = oracle.fp8_to_f64(np.arange(1, 0x7F, dtype=np.uint8))
     v = rng.choice(pos, size=shape) * rng.choice([-1.0, 1.0], size=shape)
     v[..., 0] = 448.0 * rng.choice([-1.0, 1.0], size=shape[:-1])
-    j = rng.integers(-14, -6, size=shape[:-1] + (1,))
+    j = rng.integers(jlo, jhi, size=shape[:-1] + (1,))
     return enc((v * np.exp2(j)).astype(np.float32))
 
 
@@ -402,3 +403,136 @@ def test_fp8_layer_error_against_bf16_is_quantization_sized():
     got = dec(oracle.layer_given_logits_fp8(t["x"], l32, *qs[0], *qs[1], *qs[2], cfg.k))
     rel = np.linalg.norm(got - want) / np.linalg.norm(want)
     assert 1e-3 < rel < 5e-2
+
+
+# ---------------------------------------------- fp8 weights and fp8 activations
+# [MoE-latency] "优化从测量开始": activations quantized beside the weights, with the
+# error measured.  Each pin reduces the activation-quantized experts to something
+# pinned above (the weight-only fp8 experts, a float64 BLAS product) or to an exact
+# invariant of per-row scaling.
+
+def _fp8_experts(t):
+    return [a for n in ("W1", "W3", "W2") for a in oracle.quantize_rows_fp8(t[n])]
+
+
+def _ffn_case(R=20, H=128, I=64, E=4, seed=3):
+    cfg, t = small_layer(N=R, H=H, I=I, E=E, k=1, seed=seed)
+    off = np.array([0, 6, 6, 13, R], np.int32)             # one empty group, ragged others
+    return cfg, t, _fp8_experts(t), off
+
+
+def test_fp8_acts_exact_x_rows_give_the_weight_only_h():
+    """x rows the quantizer represents exactly (a power-of-two scale per row): the
+    quantized W1/W3 step gives the weight-only h bit for bit, and the weight-only
+    option of the extended function is the weight-only experts pinned above."""
+    cfg, t, q, off = _ffn_case()
+    xg = _grid_weights(np.random.default_rng(11), (cfg.N, cfg.H), -8, -4)
+    y0, h0 = oracle.expert_ffn_fp8_ex(xg, off, *q, quantize_acts=False)
+    _, h1 = oracle.expert_ffn_fp8_ex(xg, off, *q, quantize_acts=True)
+    assert np.array_equal(h1, h0)
+    assert np.array_equal(y0, oracle.expert_ffn_fp8(xg, off, *q))
+    # ordinary rows are not exact: h moves by about the e4m3 step averaged over the sums
+    x = t["x"]
+    _, hw = oracle.expert_ffn_fp8_ex(x, off, *q, quantize_acts=False)
+    _, ha = oracle.expert_ffn_fp8_ex(x, off, *q, quantize_acts=True)
+    d = np.linalg.norm(dec(ha) - dec(hw)) / np.linalg.norm(dec(hw))
+    assert 1e-3 < d < 5e-2, d
+
+
+def test_fp8_acts_exact_h_rows_give_the_blas_product():
+    """h rows given in the exactly representable form: the quantized W2 step equals
+    the weight-only one, and both equal a float64 BLAS product of the given h with
+    the dequantized W2 of each row's expert."""
+    cfg, t, q, off = _ffn_case()
+    rng = np.random.default_rng(12)
+    xg = _grid_weights(rng, (cfg.N, cfg.H), -8, -4)
+    hg = _grid_weights(rng, (cfg.N, cfg.I), -6, -2)
+    y0, _ = oracle.expert_ffn_fp8_ex(xg, off, *q, quantize_acts=False, h_given=hg)
+    y1, _ = oracle.expert_ffn_fp8_ex(xg, off, *q, quantize_acts=True, h_given=hg)
+    assert np.array_equal(y1, y0)
+    W2d = oracle.fp8_to_f64(q[4]) * q[5][..., None].astype(np.float64)
+    for e in range(cfg.E):
+        r = slice(off[e], off[e + 1])
+        assert np.allclose(y1[r], dec(hg[r]) @ W2d[e].T, rtol=1e-12, atol=1e-14)
+
+
+def _dequant_rows(a):
+    qa, sa = oracle.quantize_rows_fp8(a)
+    return oracle.fp8_to_f64(qa) * sa[:, None].astype(np.float64)
+
+
+def test_fp8_acts_steps_read_the_quantizer_output():
+    """Ordinary activations: the experts' output equals a float64 BLAS statement
+    that feeds each GEMM the pinned quantizer's dequantized rows -- x for W1/W3,
+    the experts' own bf16 h for W2 -- with the dequantized weights."""
+    cfg, t, q, off = _ffn_case()
+    y, h = oracle.expert_ffn_fp8_ex(t["x"], off, *q, quantize_acts=True)
+    W1d, W3d, W2d = (oracle.fp8_to_f64(q[i]) * q[i + 1][..., None].astype(np.float64) for i in (0, 2, 4))
+    xq, hq = _dequant_rows(t["x"]), _dequant_rows(h)
+    for e in range(cfg.E):
+        if off[e] == off[e + 1]:
+            continue
+        r = slice(off[e], off[e + 1])
+        g, u = xq[r] @ W1d[e].T, xq[r] @ W3d[e].T
+        assert ulp_diff(h[r], enc(g / (1 + np.exp(-g)) * u)).max() <= 1
+        assert np.allclose(y[r], hq[r] @ W2d[e].T, rtol=1e-12, atol=1e-14)
+    # and those are not the unquantized rows
+    assert not np.allclose(xq, dec(t["x"]), rtol=1e-3) and not np.allclose(hq, dec(h), rtol=1e-3)
+
+
+def test_fp8_acts_quantize_the_bf16_h_and_use_a_given_one():
+    """Handing back the experts' own bf16 h changes nothing (the quantizer reads h
+    after its bf16 rounding); a different given h changes the output."""
+    cfg, t, q, off = _ffn_case()
+    y, h = oracle.expert_ffn_fp8_ex(t["x"], off, *q, quantize_acts=True)
+    yg, _ = oracle.expert_ffn_fp8_ex(t["x"], off, *q, quantize_acts=True, h_given=h)
+    assert np.array_equal(yg, y)
+    h2 = h.copy()
+    h2[3] = enc(-dec(h[3]))
+    y2, _ = oracle.expert_ffn_fp8_ex(t["x"], off, *q, quantize_acts=True, h_given=h2)
+    assert np.array_equal(y2[3], -y[3]) and np.array_equal(np.delete(y2, 3, 0), np.delete(y, 3, 0))
+
+
+def test_fp8_acts_per_row_power_of_two_scaling_of_h_is_exact():
+    """Scaling each given h row by its own power of two scales that row's scale and
+    nothing else, so each output row scales by the same power exactly; a scale
+    along the wrong axis, or shared between rows, would change the codes."""
+    cfg, t, q, off = _ffn_case()
+    _, h = oracle.expert_ffn_fp8_ex(t["x"], off, *q, quantize_acts=True)
+    m = np.random.default_rng(13).integers(-3, 4, cfg.N).astype(np.float64)
+    hs = enc((dec(h) * np.exp2(m)[:, None]).astype(np.float32))
+    assert np.array_equal(dec(hs), dec(h) * np.exp2(m)[:, None])
+    y, _ = oracle.expert_ffn_fp8_ex(t["x"], off, *q, quantize_acts=True, h_given=h)
+    ys, _ = oracle.expert_ffn_fp8_ex(t["x"], off, *q, quantize_acts=True, h_given=hs)
+    assert np.array_equal(ys, y * np.exp2(m)[:, None])
+
+
+def test_fp8_acts_layer_is_its_steps_and_reads_h_in_assignment_order():
+    """The layer = pinned top-k, dispatch and combine around the quantized experts;
+    a given h in assignment order (row t*k + j) lands on the right permuted rows;
+    without activation quantization it is the weight-only fp8 layer."""
+    cfg, t = small_layer(N=24, H=128, I=64, E=4, k=2)
+    q = _fp8_experts(t)
+    l32 = oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32)
+    idx, w = oracle.topk(l32, cfg.k)
+    _, offsets, r2t, t2r = oracle.dispatch(idx, cfg.E)
+    assert not np.array_equal(t2r.ravel(), np.arange(cfg.N * cfg.k))
+    y, h = oracle.expert_ffn_fp8_ex(oracle.permute_rows(t["x"], r2t), offsets, *q, quantize_acts=True)
+    out = oracle.layer_given_logits_fp8_ex(t["x"], l32, *q, cfg.k, quantize_acts=True)
+    assert np.array_equal(out, oracle.combine(y, t2r, w))
+    h_tok = h[t2r.ravel()]
+    out_g = oracle.layer_given_logits_fp8_ex(t["x"], l32, *q, cfg.k, quantize_acts=True, h_given=h_tok)
+    assert np.array_equal(out_g, out)
+    assert np.array_equal(oracle.layer_given_logits_fp8_ex(t["x"], l32, *q, cfg.k, quantize_acts=False),
+                          oracle.layer_given_logits_fp8(t["x"], l32, *q, cfg.k))
+
+
+def test_fp8_acts_layer_error_against_bf16_is_quantization_sized():
+    cfg, t = small_layer(N=24, H=128, I=64, E=4, k=2)
+    l32 = oracle.router_logits(t["x"], t["W_gate"]).astype(np.float32)
+    want = dec(oracle.layer_given_logits(t["x"], l32, t["W1"], t["W3"], t["W2"], cfg.k))
+    got = dec(oracle.layer_given_logits_fp8_ex(t["x"], l32, *_fp8_experts(t), cfg.k, quantize_acts=True))
+    w8 = dec(oracle.layer_given_logits_fp8(t["x"], l32, *_fp8_experts(t), cfg.k))
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    rel_w8 = np.linalg.norm(w8 - want) / np.linalg.norm(want)
+    assert rel_w8 < rel < 8e-2, (rel, rel_w8)
