@@ -62,16 +62,19 @@ def layer_flops(cfg):
     return 2 * cfg.N * cfg.H * cfg.E + 6 * cfg.R * cfg.H * cfg.I + 6 * cfg.N * cfg.H * cfg.Is
 
 
-def gemm13_bytes(cfg, touched, wbytes=2):
+def gemm13_bytes(cfg, touched, wbytes=2, abytes=2):
     """W1+W3 tiles of the touched experts (wbytes per weight; fp8 adds a 4-byte scale
-    per row), x_perm read, h written."""
+    per row), x_perm read (abytes per value; fp8 adds a scale per row), h written."""
     scales = touched * 2 * cfg.I * 4 if wbytes == 1 else 0
-    return touched * 2 * cfg.I * cfg.H * wbytes + scales + cfg.R * cfg.H * 2 + cfg.R * cfg.I * 2
+    ascales = cfg.R * 4 if abytes == 1 else 0
+    return (touched * 2 * cfg.I * cfg.H * wbytes + scales + cfg.R * cfg.H * abytes + ascales
+            + cfg.R * cfg.I * 2)
 
 
-def gemm2_bytes(cfg, touched, wbytes=2):
+def gemm2_bytes(cfg, touched, wbytes=2, abytes=2):
     scales = touched * cfg.H * 4 if wbytes == 1 else 0
-    return touched * cfg.H * cfg.I * wbytes + scales + cfg.R * cfg.I * 2 + cfg.R * cfg.H * 2
+    ascales = cfg.R * 4 if abytes == 1 else 0
+    return touched * cfg.H * cfg.I * wbytes + scales + cfg.R * cfg.I * abytes + ascales + cfg.R * cfg.H * 2
 
 
 def layer_bytes(cfg, touched, wbytes=2):
@@ -165,14 +168,37 @@ class ClockSampler:
 
     def __exit__(self, *a):
         self.t1 = time.time()
+        self._read_until(self.t1, timeout_s=1.0)
         self.stop()
+
+    def _read_until(self, t, timeout_s):
+        """Keep the helper's lines until one is stamped at or after t (at most timeout_s),
+        so a region shorter than the helper's first query still has a sample."""
+        import select
+        if self.proc is None:
+            return
+        deadline = time.time() + timeout_s
+        while True:
+            left = deadline - time.time()
+            if left <= 0 or not select.select([self.proc.stdout], [], [], left)[0]:
+                return
+            line = self.proc.stdout.readline()
+            if not line:
+                return
+            self.lines.append(line)
+            f = line.split()
+            try:
+                if len(f) == 5 and float(f[0]) >= t:
+                    return
+            except ValueError:
+                pass
 
     def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
                 out, _ = self.proc.communicate(timeout=5)
-                self.lines = out.splitlines()
+                self.lines += out.splitlines()
             except subprocess.TimeoutExpired:
                 self.proc.kill()
             self.proc = None
@@ -280,10 +306,12 @@ def run_ours(args, cfg, world, rank, local):
     if world > 1:  # every rank its own token batch
         t["x"] = make_inputs(cfg, seed=rank, device=dev, weights=False)["x"]
     N, H, I, E, k = cfg.N, cfg.H, cfg.I, cfg.E, cfg.k
-    ws = torch.empty(moe.moe_workspace_bytes(N, H, I, E, k, cfg.Is), dtype=torch.uint8, device=dev)
-    out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
     fp8 = args.weights == "fp8"
-    wbytes = 1 if fp8 else 2
+    a8 = args.acts == "fp8"  # activations quantized too (fp8 weights only)
+    wbytes, abytes = (1 if fp8 else 2), (1 if a8 else 2)
+    ws_bytes = (moe.moe_workspace_bytes_w8a8 if a8 else moe.moe_workspace_bytes)(N, H, I, E, k, cfg.Is)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
     if fp8:
         # weight preparation, once, outside every timed region: e4m3 codes + row scales
         q = {n: moe.moe_quantize_fp8(t[n], stream=stream) for n in ("W1", "W3", "W2")}
@@ -294,9 +322,9 @@ def run_ours(args, cfg, world, rank, local):
         oo = out if o is None else o
         ss = stream if st is None else st
         if fp8:
-            moe.moe_layer_forward_fp8_ex(xx, t["W_gate"], *q["W1"], *q["W3"], *q["W2"], k, bias=t["bias"],
-                                         Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=ss,
-                                         phase_events=events)
+            fn = moe.moe_layer_forward_w8a8_ex if a8 else moe.moe_layer_forward_fp8_ex
+            fn(xx, t["W_gate"], *q["W1"], *q["W3"], *q["W2"], k, bias=t["bias"], Ws1=t["Ws1"], Ws3=t["Ws3"],
+               Ws2=t["Ws2"], ws=ws, out=oo, stream=ss, phase_events=events)
         else:
             moe.moe_layer_forward_ex(xx, t["W_gate"], t["W1"], t["W3"], t["W2"], k, bias=t["bias"],
                                      Ws1=t["Ws1"], Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=oo, stream=ss,
@@ -388,8 +416,8 @@ def run_ours(args, cfg, world, rank, local):
             moe.moe_layer_forward(x_host, t["W_gate"], t["W1"], t["W3"], t["W2"], k, out=out_host)
     else:
         e2e_stream = stream
-        e2e_how = (f"{'moe_layer_forward_fp8_ex' if fp8 else 'moe_layer_forward_ex'} with the copy of x in and "
-                   "of out back on its stream")
+        call = "moe_layer_forward_w8a8_ex" if a8 else ("moe_layer_forward_fp8_ex" if fp8 else "moe_layer_forward_ex")
+        e2e_how = f"{call} with the copy of x in and of out back on its stream"
         x_dev = torch.empty_like(t["x"])
 
         def e2e_step():
@@ -419,7 +447,7 @@ def run_ours(args, cfg, world, rank, local):
     value = world * N / step_s
     g13_s = phase_ms["gemm13"] / 1e3
     g2_s = phase_ms["gemm2"] / 1e3
-    g13_b = gemm13_bytes(cfg, touched, wbytes)
+    g13_b = gemm13_bytes(cfg, touched, wbytes, abytes)
     hbm = pk["hbm_gbs"]
     achieved = g13_b / g13_s / 1e9
     flops = layer_flops(cfg)
@@ -428,39 +456,50 @@ def run_ours(args, cfg, world, rank, local):
     floor_s = max(flops / (pk["bf16_tflops"] * 1e12), lbytes / (hbm * 1e9))
     workload = cfg.name
     # the W1/W3 kernel's bound: weight streaming (HBM) at decode sizes, the tensor cores
-    # once the token tiles are long enough (its FLOPs at the bf16 peak outlast its bytes)
+    # once the token tiles are long enough (its FLOPs at the tensor peak outlast its
+    # bytes).  An e4m3 x e4m3 contraction takes the measured bf16 peak times the nominal
+    # fp8 : bf16 ratio (4.5 : 2.25 PFLOP/s dense).
     g13_flops = 4 * cfg.R * H * I
-    if g13_flops / (pk["bf16_tflops"] * 1e12) > g13_b / (hbm * 1e9):
-        roofline = {"bound": "tensor", "achieved": g13_flops / g13_s / 1e12, "peak": pk["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": g13_flops / g13_s / 1e12 / pk["bf16_tflops"],
+    tratio = 2.0 if a8 else 1.0
+    tpeak = pk["bf16_tflops"] * tratio
+    if g13_flops / (tpeak * 1e12) > g13_b / (hbm * 1e9):
+        roofline = {"bound": "tensor", "achieved": g13_flops / g13_s / 1e12, "peak": tpeak,
+                    "unit": "TFLOP/s", "frac": g13_flops / g13_s / 1e12 / tpeak,
                     "alg_flops_per_launch": g13_flops}
+        if a8:
+            roofline["peak_note"] = "measured bf16 peak x 2 (nominal e4m3 : bf16 dense ratio)"
         if "bf16_tflops_sustained" in pk:
-            roofline["frac_of_sustained_peak"] = g13_flops / g13_s / 1e12 / pk["bf16_tflops_sustained"]
+            roofline["frac_of_sustained_peak"] = (g13_flops / g13_s / 1e12 /
+                                                  (pk["bf16_tflops_sustained"] * tratio))
     else:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "alg_bytes_per_launch": g13_b}
-    roofline.update({"kernel": "grouped_gemm SwiGLU W1/W3 (gemm13)" + (", e4m3 weights" if fp8 else ""),
+    kdesc = ", e4m3 weights and activations" if a8 else (", e4m3 weights" if fp8 else "")
+    roofline.update({"kernel": "grouped_gemm SwiGLU W1/W3 (gemm13)" + kdesc,
                      "peak_kind": pk_kind,
                      "traffic": None if fp8 else kernel_traffic("gemm13", workload),
                      "avg_launch_ms": phase_ms["gemm13"]})
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if a8 else "bf16", "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "global_batch": world * N, "tokens_per_gpu": N,
                    "parallelism": f"dp{world} (token batches, replicated weights, no exchange)",
                    "l2": f"inputs larger than L2: {touched} touched experts' weights "
                          f"({touched * 3 * H * I * wbytes / 1e9:.2f} GB) streamed from HBM every step",
                    "touched_experts": touched, "max_expert_rows": max_load,
-                   "expert_weights": ("e4m3, one fp32 scale per output channel (quantized once before "
-                                      "timing; widened to bf16 on chip)") if fp8 else "bf16"},
+                   "expert_weights": (("e4m3, one fp32 scale per output channel (quantized once before "
+                                       "timing; " + ("multiplied as e4m3" if a8 else "widened to bf16 on chip")
+                                       + ")") if fp8 else "bf16"),
+                   "expert_activations": ("e4m3, one fp32 scale per row (x_perm and h quantized on the device "
+                                          "every step)") if a8 else "bf16"},
         "roofline": roofline,
         "layer": {"tflops": flops / step_s / 1e12, "alg_bytes": lbytes, "gb_s": lbytes / step_s / 1e9,
                   "roofline_floor_us": floor_s * 1e6, "roofline_frac": floor_s / step_s,
                   "useful_flop_fraction_k_over_E": k / E},
         "grouped_gemm": {"tflops": gemm_flops / (g13_s + g2_s) / 1e12,
-                         "gb_s": (g13_b + gemm2_bytes(cfg, touched, wbytes)) / (g13_s + g2_s) / 1e9,
-                         "gemm2_frac_hbm": gemm2_bytes(cfg, touched, wbytes) / g2_s / 1e9 / hbm},
+                         "gb_s": (g13_b + gemm2_bytes(cfg, touched, wbytes, abytes)) / (g13_s + g2_s) / 1e9,
+                         "gemm2_frac_hbm": gemm2_bytes(cfg, touched, wbytes, abytes) / g2_s / 1e9 / hbm},
         "phase_ms": phase_ms,
         "phase_ms_note": "mean per-phase CUDA-event times from a second timed pass with events between phases",
         "gpu_launches": launches,
@@ -519,9 +558,13 @@ def main():
                     help="time replays of one layer step captured as a CUDA graph (launch-bound decode sizes)")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
                     help="routed-expert weight format (fp8: e4m3 with per-channel scales, a separate experiment)")
+    ap.add_argument("--acts", choices=["bf16", "fp8"], default="bf16",
+                    help="routed-expert activation format (fp8: e4m3 with per-row scales; needs --weights fp8)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.acts == "fp8" and args.weights != "fp8":
+        ap.error("--acts fp8 needs --weights fp8")
     cfg = CONFIGS[args.config]
     if args.tokens:
         cfg = cfg.with_tokens(args.tokens)

@@ -69,11 +69,14 @@ bool valid_rows(int64_t N, int k) { return N >= 0 && N * (int64_t)k < (int64_t(1
 size_t round_up(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t logits, idx, w, counts, offsets, r2t, t2r, perm, x_perm, h, hs, y_perm, s, router, router_bytes, total;
+    size_t logits, idx, w, counts, offsets, r2t, t2r, perm, x_perm, h, hs, y_perm, s, router, router_bytes;
+    size_t xqt, xst, xq, xsc, hq, hsc;  // fp8 activations only: quantized rows and their scales
+    size_t total;
 };
 
-// Carve the layer's workspace; every buffer starts on a 256-byte boundary.
-void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
+// Carve the layer's workspace; every buffer starts on a 256-byte boundary.  a8 adds
+// the quantized activation rows.
+void ws_layout(int64_t N, int H, int I, int E, int k, int Is, bool a8, WsLayout *L)
 {
     const int64_t R = N * k;
     size_t off = 0;
@@ -93,14 +96,28 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, WsLayout *L)
     L->s = take((size_t)N * (Is > 0 ? H : 0) * 4);
     L->router_bytes = moe::router_ws_bytes(N, H, E);
     L->router = take(L->router_bytes);
+    L->xqt = take(a8 ? (size_t)N * H : 0);  // token order
+    L->xst = take(a8 ? (size_t)N * 4 : 0);
+    L->xq = take(a8 ? (size_t)R * H : 0);
+    L->xsc = take(a8 ? (size_t)R * 4 : 0);
+    L->hq = take(a8 ? (size_t)R * I : 0);
+    L->hsc = take(a8 ? (size_t)R * 4 : 0);
     L->total = off;
 }
 
-// The routed experts' weights: bf16, or e4m3 bytes with one fp32 scale per row.
+// The routed experts' weights: bf16, or e4m3 bytes with one fp32 scale per row
+// (optionally with e4m3 activations as well).
 struct Experts {
     const void *W1, *W3, *W2;
     const float *s1, *s3, *s2;  // fp8 only
     bool fp8;
+    bool a8;                    // activations quantized too (fp8 weights only)
+};
+
+// Buffers of the quantized activation rows (a8 only): x_perm and h, with their scales
+// (the layer also quantizes x in token order first: xqt, xst).
+struct ActQ {
+    uint8_t *xq; float *xsc; uint8_t *hq; float *hsc; uint8_t *xqt; float *xst;
 };
 
 void set_weights13(moe::GroupedGemmArgs *a, const Experts &X)
@@ -113,19 +130,32 @@ void set_weights2(moe::GroupedGemmArgs *b, const Experts &X)
     b->w_a = X.W2; b->w_b = nullptr; b->w8 = X.fp8; b->scale_a = X.s2; b->scale_b = nullptr;
 }
 
+// The activation operand of a GEMM: the bf16 rows, or (a8) their quantized form,
+// produced here from the bf16 rows.
+moe_status_t set_act(moe::GroupedGemmArgs *g, const uint16_t *rows, int64_t R, int K, uint8_t *q, float *sc,
+                     bool a8, cudaStream_t s)
+{
+    if (!a8) { g->act = rows; return MOE_OK; }
+    MOE_CUDA(moe::launch_quantize_fp8(rows, R, K, q, sc, s));
+    g->act = q; g->a8 = true; g->scale_act = sc;
+    return MOE_OK;
+}
+
 moe_status_t expert_ffn_impl(const uint16_t *x_perm, const int32_t *offsets, const Experts &X, int64_t R, int H,
-                             int I, int E, uint16_t *h, float *y_perm, int *err, cudaStream_t s)
+                             int I, int E, uint16_t *h, float *y_perm, const ActQ &Q, int *err, cudaStream_t s)
 {
     if (R == 0) return MOE_OK;
     moe::GroupedGemmArgs a{};
-    a.act = x_perm; a.offsets = offsets; a.groups = E; a.R = R;
+    a.offsets = offsets; a.groups = E; a.R = R;
     a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
     set_weights13(&a, X);
+    if (moe_status_t st = set_act(&a, x_perm, R, H, Q.xq, Q.xsc, X.a8, s)) return st;
     MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     moe::GroupedGemmArgs b{};
-    b.act = h; b.offsets = offsets; b.groups = E; b.R = R;
+    b.offsets = offsets; b.groups = E; b.R = R;
     b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
     set_weights2(&b, X);
+    if (moe_status_t st = set_act(&b, h, R, I, Q.hq, Q.hsc, X.a8, s)) return st;
     MOE_CUDA(moe::launch_gemm2(b, s));
     return MOE_OK;
 }
@@ -175,12 +205,14 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
         return MOE_ERR_UNSUPPORTED;
     if (Is > 0 && (!aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2))) return MOE_ERR_UNSUPPORTED;
     WsLayout L;
-    ws_layout(N, H, I, E, k, Is, &L);
+    ws_layout(N, H, I, E, k, Is, X.a8, &L);
     if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     int *err = device_error_word();
     if (!err) return cuda_fail(cudaGetLastError());
 
     uint8_t *base = static_cast<uint8_t *>(ws);
+    const ActQ Q{base + L.xq, reinterpret_cast<float *>(base + L.xsc), base + L.hq,
+                 reinterpret_cast<float *>(base + L.hsc), base + L.xqt, reinterpret_cast<float *>(base + L.xst)};
     float *lg = logits ? logits : reinterpret_cast<float *>(base + L.logits);
     int32_t *idx = reinterpret_cast<int32_t *>(base + L.idx);
     float *w = reinterpret_cast<float *>(base + L.w);
@@ -199,25 +231,34 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
     MOE_TRY(record(phase_events, 0, s));
     MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
-    MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
+    moe::GroupedGemmArgs a{};
+    a.offsets = offsets; a.groups = E; a.R = R;
+    a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
+    set_weights13(&a, X);
+    if (X.a8) {
+        // each token row is quantized once (N rows, not N*k: a permuted row is a copy of
+        // its token's row, so its codes and scale are the same), then the codes and the
+        // scales move to the permuted rows
+        MOE_CUDA(moe::launch_quantize_fp8(x, N, H, Q.xqt, Q.xst, s));
+        MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
+        MOE_CUDA(moe::launch_scatter_rows(reinterpret_cast<const uint16_t *>(Q.xqt), Q.xst, t2r, N, k, H / 2,
+                                          reinterpret_cast<uint16_t *>(Q.xq), Q.xsc, s));
+        a.act = Q.xq; a.a8 = true; a.scale_act = Q.xsc;
+    } else {
+        MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
+        a.act = x_perm;
+    }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
-    {
-        moe::GroupedGemmArgs a{};
-        a.act = x_perm; a.offsets = offsets; a.groups = E; a.R = R;
-        a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
-        set_weights13(&a, X);
-        MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
-    }
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
+    MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     const int ksplit = moe::gemm2_ksplit(R, E, I, H);
-    {
-        moe::GroupedGemmArgs b{};
-        b.act = h; b.offsets = offsets; b.groups = E; b.R = R;
-        b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
-        set_weights2(&b, X);
-        b.ksplit = ksplit; b.split_stride = R * (int64_t)H;
-        MOE_CUDA(moe::launch_gemm2(b, s));
-    }
+    moe::GroupedGemmArgs b{};
+    b.offsets = offsets; b.groups = E; b.R = R;
+    b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
+    set_weights2(&b, X);
+    b.ksplit = ksplit; b.split_stride = R * (int64_t)H;
+    MOE_TRY(set_act(&b, h, R, I, Q.hq, Q.hsc, X.a8, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
+    MOE_CUDA(moe::launch_gemm2(b, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM2, s));
     if (Is > 0) MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
@@ -254,7 +295,16 @@ size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is)
     if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return 0;
     if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return 0;
     WsLayout L;
-    ws_layout(N, H, I, E, k, Is, &L);
+    ws_layout(N, H, I, E, k, Is, false, &L);
+    return L.total;
+}
+
+size_t moe_workspace_bytes_w8a8(int64_t N, int H, int I, int E, int k, int Is)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return 0;
+    if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return 0;
+    WsLayout L;
+    ws_layout(N, H, I, E, k, Is, true, &L);
     return L.total;
 }
 
@@ -311,8 +361,8 @@ moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, cons
     if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     int *err = device_error_word();
     if (!err) return cuda_fail(cudaGetLastError());
-    const Experts X{W1, W3, W2, nullptr, nullptr, nullptr, false};
-    return expert_ffn_impl(x_perm, offsets, X, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, err,
+    const Experts X{W1, W3, W2, nullptr, nullptr, nullptr, false, false};
+    return expert_ffn_impl(x_perm, offsets, X, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, ActQ{}, err,
                            static_cast<cudaStream_t>(stream));
 }
 
@@ -335,7 +385,7 @@ moe_status_t moe_layer_forward_ex(const uint16_t *x, const float *W_gate, const 
                                   int H, int I, int E, int k, int Is, uint16_t *out, float *logits, void *ws,
                                   size_t ws_bytes, void *stream, void *const *phase_events)
 {
-    const Experts X{W1, W3, W2, nullptr, nullptr, nullptr, false};
+    const Experts X{W1, W3, W2, nullptr, nullptr, nullptr, false, false};
     return layer_impl(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, ws_bytes, stream,
                       phase_events);
 }
@@ -348,7 +398,20 @@ moe_status_t moe_layer_forward_fp8_ex(const uint16_t *x, const float *W_gate, co
                                       void *stream, void *const *phase_events)
 {
     if (N > 0 && (!s1 || !s3 || !s2)) return MOE_ERR_INVALID_ARG;
-    const Experts X{W1q, W3q, W2q, s1, s3, s2, true};
+    const Experts X{W1q, W3q, W2q, s1, s3, s2, true, false};
+    return layer_impl(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, ws_bytes, stream,
+                      phase_events);
+}
+
+moe_status_t moe_layer_forward_w8a8_ex(const uint16_t *x, const float *W_gate, const float *bias,
+                                       const uint8_t *W1q, const float *s1, const uint8_t *W3q, const float *s3,
+                                       const uint8_t *W2q, const float *s2, const uint16_t *Ws1,
+                                       const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I, int E,
+                                       int k, int Is, uint16_t *out, float *logits, void *ws, size_t ws_bytes,
+                                       void *stream, void *const *phase_events)
+{
+    if (N > 0 && (!s1 || !s3 || !s2)) return MOE_ERR_INVALID_ARG;
+    const Experts X{W1q, W3q, W2q, s1, s3, s2, true, true};
     return layer_impl(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, ws_bytes, stream,
                       phase_events);
 }
@@ -378,8 +441,44 @@ moe_status_t moe_expert_ffn_fp8(const uint16_t *x_perm, const int32_t *offsets, 
     if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     int *err = device_error_word();
     if (!err) return cuda_fail(cudaGetLastError());
-    const Experts X{W1q, W3q, W2q, s1, s3, s2, true};
-    return expert_ffn_impl(x_perm, offsets, X, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, err,
+    const Experts X{W1q, W3q, W2q, s1, s3, s2, true, false};
+    return expert_ffn_impl(x_perm, offsets, X, R, H, I, E, static_cast<uint16_t *>(ws), y_perm, ActQ{}, err,
+                           static_cast<cudaStream_t>(stream));
+}
+
+// h [R,I] bf16 (when the caller keeps none), then x_perm's and h's quantized rows and scales.
+size_t moe_expert_ffn_w8a8_ws_bytes(int64_t R, int H, int I)
+{
+    if (R < 0 || R >= (int64_t(1) << 31) || !valid_hidden(H) || !valid_hidden(I)) return 0;
+    return round_up((size_t)R * I * 2) + round_up((size_t)R * H) + round_up((size_t)R * 4) +
+           round_up((size_t)R * I) + round_up((size_t)R * 4);
+}
+
+moe_status_t moe_expert_ffn_w8a8(const uint16_t *x_perm, const int32_t *offsets, const uint8_t *W1q,
+                                 const float *s1, const uint8_t *W3q, const float *s3, const uint8_t *W2q,
+                                 const float *s2, int64_t R, int H, int I, int E, float *y_perm, uint16_t *h,
+                                 void *ws, size_t ws_bytes, void *stream)
+{
+    if (R < 0 || R >= (int64_t(1) << 31) || !valid_hidden(H) || !valid_hidden(I) || E < 1 || E > 256)
+        return MOE_ERR_INVALID_ARG;
+    if (R == 0) return MOE_OK;
+    if (!x_perm || !offsets || !W1q || !W3q || !W2q || !s1 || !s3 || !s2 || !y_perm) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_perm) || !aligned16(W1q) || !aligned16(W3q) || !aligned16(W2q) || !aligned16(y_perm) ||
+        (h && !aligned16(h)))
+        return MOE_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < moe_expert_ffn_w8a8_ws_bytes(R, H, I) || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    int *err = device_error_word();
+    if (!err) return cuda_fail(cudaGetLastError());
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    uint16_t *hb = reinterpret_cast<uint16_t *>(p);
+    p += round_up((size_t)R * I * 2);
+    ActQ Q{};
+    Q.xq = p; p += round_up((size_t)R * H);
+    Q.xsc = reinterpret_cast<float *>(p); p += round_up((size_t)R * 4);
+    Q.hq = p; p += round_up((size_t)R * I);
+    Q.hsc = reinterpret_cast<float *>(p);
+    const Experts X{W1q, W3q, W2q, s1, s3, s2, true, true};
+    return expert_ffn_impl(x_perm, offsets, X, R, H, I, E, h ? h : hb, y_perm, Q, err,
                            static_cast<cudaStream_t>(stream));
 }
 

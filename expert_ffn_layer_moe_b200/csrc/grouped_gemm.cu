@@ -52,6 +52,15 @@
 // W8 runs single-CTA tiles of up to 128 token rows (a pair's MMA would need the other
 // CTA to signal every K step across the cluster, which costs more than the pair saves).
 //
+// fp8 weights and fp8 activations (A8 = true; the same section names activations beside
+// weights): both operands are e4m3 bytes with one fp32 scale per row -- a weight row, or
+// a token row of the activations.  The pipeline is the bf16 one (pairs included): a stage
+// holds 128-byte rows, i.e. 128 K values instead of 64, and the MMA is
+// tcgen05.mma.kind::f8f6f4 (K = 32 per instruction, fp32 accumulation of exact
+// products), so each weight byte costs a quarter of the MMA instructions of the widened
+// path.  The epilogue multiplies the accumulator by the weight row's scale and the token
+// row's scale.
+//
 // Work items are (group, feature tile, K slice, token tile), enumerated on the device
 // from the row offsets with no host synchronisation; empty groups produce no items (no
 // padding to a fixed capacity).  The plain GEMM can split K into `ksplit` slices whose
@@ -77,9 +86,12 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, far above any
 
 constexpr int pow2_at_least(int v, int p = 32) { return p >= v ? p : pow2_at_least(v, p * 2); }
 
-template <int BN, bool SWIGLU, bool PAIR, bool W8>
+template <int BN, bool SWIGLU, bool PAIR, bool W8, bool A8>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "token tile must be 32..256, step 32");
+    static_assert(!(W8 && A8), "fp8 activations use the native fp8 MMA, not the widening path");
+    // K values per pipeline stage: one 128-byte row of the operand tiles (64 bf16 or 128 e4m3)
+    static constexpr int kKStep = A8 ? 2 * kBK : kBK;
     // warps: producer, MMA, 4 epilogue; with W8 also 8 converter warps (fp8 -> bf16)
     // and an activation producer
     static_assert(!(W8 && PAIR), "fp8 weights run single-CTA tiles");
@@ -113,10 +125,11 @@ struct Cfg {
     static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // staging: 4 x [32][33] fp32 (= 2 x [64][33])
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kFStages * kW8Bytes + kBarBytes + 16 +
                                       kTableBytes + kEpiBytes;
-    // tcgen05 instruction descriptor, kind::f16: D=f32 (bit 4), A=B=bf16 (bits 7, 10),
-    // both operands K-major, M>>4 at bit 24 (M = 128 per CTA); N>>3 (bit 17) per tile.
-    static constexpr uint32_t kIdescNoN =
-        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)((kBM * kCtas) >> 4) << 24);
+    // tcgen05 instruction descriptor: D=f32 (bit 4); kind::f16 with A=B=bf16 (format 1 at
+    // bits 7 and 10), or kind::f8f6f4 with A=B=e4m3 (format 0); both operands K-major,
+    // M>>4 at bit 24 (M = 128 per CTA, 256 per pair); N>>3 (bit 17) per tile.
+    static constexpr uint32_t kIdescNoN = (1u << 4) | (A8 ? 0u : (1u << 7) | (1u << 10)) |
+                                          ((uint32_t)((kBM * kCtas) >> 4) << 24);
     static_assert(kStages >= 2, "pipeline needs at least two stages");
     static_assert(!W8 || kFStages >= 2, "fp8 ring needs at least two tiles");
     static_assert(kTmemCols <= 512, "TMEM has 512 columns");
@@ -391,16 +404,31 @@ __device__ __forceinline__ void tmem_dealloc_g(uint32_t taddr, uint32_t ncols)
 }
 
 // One MMA: with PAIR, M = 256 across the pair (each CTA's 128 weight rows), N split
-// between the CTAs' halves of the token tile; issued by the leader CTA only.
-template <bool PAIR>
+// between the CTAs' halves of the token tile; issued by the leader CTA only.  F8: both
+// operands e4m3 (kind::f8f6f4, K = 32), else bf16 (kind::f16, K = 16).
+template <bool PAIR, bool F8>
 __device__ __forceinline__ void umma_g(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate)
 {
-    if (PAIR)
+    if (PAIR && F8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else if (PAIR)
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else if (F8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
             "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
             : "memory");
     else
@@ -424,7 +452,13 @@ __device__ __forceinline__ void umma_commit_g(uint64_t *bar)
     }
 }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+// silu(z) = z / (1 + e^-z) with the hardware exponential and reciprocal: about five
+// instructions instead of about twenty-five for the IEEE forms (whose division also
+// branches to a slow path).  Relative error a few 1e-6, far below the bf16 rounding of h
+// that follows; e^-z overflowing to infinity gives the limit 0.  The SwiGLU epilogue
+// issues almost all of the kernel's instructions on four warps, so at long token
+// tiles this is what keeps it shorter than the main loop.
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // Named barrier for the four epilogue warps (barrier 0 is __syncthreads).
 __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -435,15 +469,16 @@ __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;
 // [n/2 r, n/2 r + n/2) of its n; the leader (r = 0) issues the M=256 MMAs, both CTAs'
 // TMA loads complete on the leader's stage barrier, its commits reach both CTAs'
 // barriers, and each CTA drains its own half of the accumulator.
-template <int BN, bool SWIGLU, bool PAIR, bool W8>
-__global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
+template <int BN, bool SWIGLU, bool PAIR, bool W8, bool A8>
+__global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
                         void *__restrict__ out, int ksplit, int64_t split_stride,
-                        const float *__restrict__ scale_a, const float *__restrict__ scale_b, int *dev_err)
+                        const float *__restrict__ scale_a, const float *__restrict__ scale_b,
+                        const float *__restrict__ scale_act, int *dev_err)
 {
-    using C = Cfg<BN, SWIGLU, PAIR, W8>;
+    using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
     constexpr int kThreads = C::kThreads;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -470,7 +505,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
     const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // work-list walker: one per pair
     const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     const int n_feat = (Nout + C::kFeatTile - 1) / C::kFeatTile;
-    const int KB = (K + kBK - 1) / kBK;
+    const int KB = (K + C::kKStep - 1) / C::kKStep;  // pipeline stages along K
 
     // ---- barriers and TMEM: nothing here reads global memory, so it overlaps the tail
     // of the previous kernel in the stream (programmatic dependent launch)
@@ -609,14 +644,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
                 uint8_t *st = stages + stage * C::kStageBytes;
                 const uint32_t fb = full0 + 8u * stage;
                 if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kCtas * C::kStageBytes);
+                const int kc = kb * C::kKStep;  // K coordinate (elements; bytes for e4m3)
                 if (SWIGLU) {
                     // rows 0-63: W1 features [frow, +64); rows 64-127: the same features of W3
-                    tma_3d<PAIR>(st, &tm_wa, kb * kBK, frow, g, fb);
-                    tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kb * kBK, frow, g, fb);
+                    tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
+                    tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kc, frow, g, fb);
                 } else {
-                    tma_3d<PAIR>(st, &tm_wa, kb * kBK, frow, g, fb);
+                    tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
                 }
-                tma_2d<PAIR>(st + C::kABytes, &tm_act, kb * kBK, trow, fb);
+                tma_2d<PAIR>(st + C::kABytes, &tm_act, kc, trow, fb);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
         }
@@ -653,8 +689,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                         const uint32_t accumulate = (kb != kb0 || kk != 0) ? 1u : 0u;
-                        // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4)
-                        umma_g<PAIR>(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
+                        // +32 bytes of K per step inside the 128-byte swizzled row (encoded >> 4):
+                        // 16 bf16 or 32 e4m3 values, one MMA's K either way
+                        umma_g<PAIR, A8>(d0, da + 2 * kk, db + 2 * kk, idesc, accumulate);
                     }
                 }
                 umma_commit_g<PAIR>(&empty_bar[stage]);  // stage free (in both CTAs) once read
@@ -702,16 +739,22 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
                 const int rr = lane >> 3, j = lane & 7;
                 const int fv = feat * C::kFeatTile + (int)rank * C::kFeat + 8 * j;
                 uint16_t *outh = static_cast<uint16_t *>(out);
-                float sc = 1.0f;  // W8: the scale of this lane's weight row (W1 for g, W3 for u)
-                if (W8) {
+                float sc = 1.0f;  // fp8 weights: the scale of this lane's weight row (W1 for g, W3 for u)
+                if (W8 || A8) {
                     const int row = feat * C::kFeatTile + (int)rank * C::kFeat + fl;
                     sc = row < Nout ? (q < 2 ? scale_a : scale_b)[(int64_t)g * Nout + row] : 0.0f;
                 }
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
+                    // A8: column c is token row row0 + c0 + c, with its own scale (lane c holds it)
+                    const float sa = A8 && c0 + lane < nrows ? scale_act[row0 + c0 + lane] : 0.0f;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) mine[fl][c] = W8 ? a[c] * sc : a[c];
+                    for (int c = 0; c < 32; ++c) {
+                        float v = (W8 || A8) ? a[c] * sc : a[c];
+                        if (A8) v *= __shfl_sync(0xffffffffu, sa, c);
+                        mine[fl][c] = v;
+                    }
                     epilogue_sync();
                     // warp ew stores rows 8*ew .. 8*ew+7 of the chunk: 4 rows x 8 feature octets per step
 #pragma unroll
@@ -734,16 +777,21 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8>::kThreads, 1)
             } else {
                 float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
                 const int fbase = feat * C::kFeatTile + (int)rank * C::kFeat + q * 32;
-                const float sc = W8 ? (fbase + lane < Nout ? scale_a[(int64_t)g * Nout + fbase + lane] : 0.0f) : 1.0f;
+                const float sc =
+                    (W8 || A8) ? (fbase + lane < Nout ? scale_a[(int64_t)g * Nout + fbase + lane] : 0.0f) : 1.0f;
                 // fp32 out through the padded tile: 8 16-byte stores per 32 rows instead of
                 // 32 4-byte ones (store instruction issue, not bytes, limits short-K tiles)
                 float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + ew * 32 * 33);
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
                     float a[32];
                     tmem_ld32(t0 + c0, a);
-                    if (W8) {
+                    if (W8 || A8) {
+                        const float sa = A8 && c0 + lane < nrows ? scale_act[row0 + c0 + lane] : 1.0f;
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) a[c] *= sc;
+                        for (int c = 0; c < 32; ++c) {
+                            a[c] *= sc;
+                            if (A8) a[c] *= __shfl_sync(0xffffffffu, sa, c);
+                        }
                     }
                     if (vec_ok) {
 #pragma unroll
@@ -927,21 +975,37 @@ bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_r
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU, bool PAIR, bool W8>
+// Activations [R, K] e4m3 bytes as a 2-D byte map; box = 128 (K) x box_rows; rows >= R
+// and K values past K read as zero.
+bool encode_act_map_fp8(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)R};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)(2 * kBK), (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWIGLU, bool PAIR, bool W8, bool A8>
 cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
-    using C = Cfg<BN, SWIGLU, PAIR, W8>;
+    using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
     CUtensorMap ma, mb, mact;
     const int box_rows = SWIGLU ? kBM / 2 : kBM;
-    auto enc_w = W8 ? encode_weight_map_fp8 : encode_weight_map;
+    auto enc_w = (W8 || A8) ? encode_weight_map_fp8 : encode_weight_map;
     if (!enc_w(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     if (SWIGLU) {
         if (!enc_w(&mb, a.w_b, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     } else {
         mb = ma;
     }
-    if (!encode_act_map(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
-    auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR, W8>;
+    auto enc_act = A8 ? encode_act_map_fp8 : encode_act_map;
+    if (!enc_act(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
+    auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR, W8, A8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
     const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
@@ -961,7 +1025,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = PAIR ? 2 : 1;
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
-                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.dev_err);
+                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, a.dev_err);
     if (err != cudaSuccess) return err;
     count_launch();
     return cudaGetLastError();
@@ -979,7 +1043,7 @@ int64_t gemm_pair_tiles(int64_t R, int groups, int Nout, bool swiglu, int ksplit
     return active * ((mean + bn - 1) / bn) * ((Nout + feat - 1) / feat) * (ksplit > 1 ? ksplit : 1);
 }
 
-template <bool SWIGLU, bool W8>
+template <bool SWIGLU, bool W8, bool A8>
 cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.groups < 1 || a.groups > kMaxGroups) return cudaErrorInvalidValue;
@@ -989,34 +1053,34 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
     // token tile, and the pair reads each activation tile once per 256 weight rows
     // instead of once per 128.  A tiny batch whose pair tiles would not even cover the
     // SM pairs once runs single-CTA tiles instead (twice the tiles, every SM streaming).
-    if (W8) {
-        // fp8 weights: single-CTA tiles.  A pair's MMA would read converted operands from
+    if (W8 && !A8) {
+        // fp8 weights widened on chip: single-CTA tiles.  A pair's MMA would read converted operands from
         // the other CTA, which then has to signal every K step across the cluster.
         // (token tiles up to 128 rows: two 256-column accumulators and the operand slots
         // would not fit in TMEM's 512 columns)
         switch (bn) {
-            case 32: return launch_impl<32, SWIGLU, false, true>(a, s);
-            case 64: return launch_impl<64, SWIGLU, false, true>(a, s);
+            case 32: return launch_impl<32, SWIGLU, false, true, false>(a, s);
+            case 64: return launch_impl<64, SWIGLU, false, true, false>(a, s);
             case 96:
             case 128:
             case 192:
-            case 256: return launch_impl<128, SWIGLU, false, true>(a, s);
+            case 256: return launch_impl<128, SWIGLU, false, true, false>(a, s);
             default: return cudaErrorInvalidValue;
         }
     } else {
         if (bn <= 64 && gemm_pair_tiles(a.R, a.groups, a.Nout, SWIGLU, a.ksplit) < device_sm_count() / 2) {
             switch (bn) {
-                case 32: return launch_impl<32, SWIGLU, false, false>(a, s);
-                case 64: return launch_impl<64, SWIGLU, false, false>(a, s);
+                case 32: return launch_impl<32, SWIGLU, false, false, A8>(a, s);
+                case 64: return launch_impl<64, SWIGLU, false, false, A8>(a, s);
             }
         }
         switch (bn) {
-            case 32: return launch_impl<32, SWIGLU, true, false>(a, s);
-            case 64: return launch_impl<64, SWIGLU, true, false>(a, s);
-            case 96: return launch_impl<96, SWIGLU, true, false>(a, s);
-            case 128: return launch_impl<128, SWIGLU, true, false>(a, s);
-            case 192: return launch_impl<192, SWIGLU, true, false>(a, s);
-            case 256: return launch_impl<256, SWIGLU, true, false>(a, s);
+            case 32: return launch_impl<32, SWIGLU, true, false, A8>(a, s);
+            case 64: return launch_impl<64, SWIGLU, true, false, A8>(a, s);
+            case 96: return launch_impl<96, SWIGLU, true, false, A8>(a, s);
+            case 128: return launch_impl<128, SWIGLU, true, false, A8>(a, s);
+            case 192: return launch_impl<192, SWIGLU, true, false, A8>(a, s);
+            case 256: return launch_impl<256, SWIGLU, true, false, A8>(a, s);
             default: return cudaErrorInvalidValue;
         }
     }
@@ -1078,13 +1142,17 @@ int gemm2_ksplit(int64_t R, int groups, int K, int Nout)
 cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.w8 && (!a.scale_a || !a.scale_b)) return cudaErrorInvalidValue;
-    return a.w8 ? launch_dispatch<true, true>(a, s) : launch_dispatch<true, false>(a, s);
+    if (a.a8 && (!a.w8 || !a.scale_act)) return cudaErrorInvalidValue;
+    if (a.a8) return launch_dispatch<true, false, true>(a, s);
+    return a.w8 ? launch_dispatch<true, true, false>(a, s) : launch_dispatch<true, false, false>(a, s);
 }
 
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s)
 {
     if (a.w8 && !a.scale_a) return cudaErrorInvalidValue;
-    return a.w8 ? launch_dispatch<false, true>(a, s) : launch_dispatch<false, false>(a, s);
+    if (a.a8 && (!a.w8 || !a.scale_act)) return cudaErrorInvalidValue;
+    if (a.a8) return launch_dispatch<false, false, true>(a, s);
+    return a.w8 ? launch_dispatch<false, true, false>(a, s) : launch_dispatch<false, false, false>(a, s);
 }
 
 }  // namespace moe

@@ -46,21 +46,28 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
 constexpr int kPermuteChunk = 1024;  // assignments per block in the count/rank passes
 inline int64_t permute_blocks(int64_t R) { return (R + kPermuteChunk - 1) / kPermuteChunk; }
 inline int64_t permute_scratch_ints(int64_t R, int E) { return permute_blocks(R) * E; }
+// x_perm == nullptr: dispatch only (counts, offsets, the two row maps), no row copy.
 cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E,
                            int k, int32_t *counts, int32_t *offsets, int32_t *row_to_token,
                            int32_t *token_to_row, uint16_t *x_perm, int32_t *scratch,
                            int *dev_err, cudaStream_t s);
+// x_perm[token_to_row[t,j]] = x[t]: rows of H 16-bit words (H a multiple of 8; e4m3
+// rows of 2H bytes pass as H words); with scale_in, scale_out[token_to_row[t,j]] = scale_in[t].
+cudaError_t launch_scatter_rows(const uint16_t *x, const float *scale_in, const int32_t *token_to_row, int64_t N,
+                                int k, int H, uint16_t *x_perm, float *scale_out, cudaStream_t s);
 
 // Grouped GEMMs on tcgen05.  Weights are [groups, Nout, K]; activations [R, K];
 // rows of group g are offsets[g] .. offsets[g+1]-1 (offsets == nullptr: one group
 // of `rows_single` rows starting at row 0).
 struct GroupedGemmArgs {
-    const uint16_t *act;     // [R, K] bf16
+    const void *act;         // [R, K] bf16, or e4m3 bytes when a8
     const void *w_a;         // [groups, Nout, K] bf16, or e4m3 bytes when w8 (W1, or W2)
     const void *w_b;         // [groups, Nout, K] likewise (W3) -- SwiGLU only
     bool w8;                 // weights are e4m3 with one fp32 scale per row (scale_a, scale_b)
     const float *scale_a;    // [groups, Nout] row scales of w_a (w8 only)
     const float *scale_b;    // [groups, Nout] row scales of w_b (w8, SwiGLU only)
+    bool a8;                 // activations are e4m3 too (needs w8): native fp8 MMA
+    const float *scale_act;  // [R] row scales of act (a8 only)
     const int32_t *offsets;  // [groups + 1] device, or nullptr
     int groups;
     int64_t R;               // rows of `act` (and of `out`)

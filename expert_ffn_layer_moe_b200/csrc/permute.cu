@@ -180,10 +180,13 @@ __global__ void __launch_bounds__(kThreads)
 // x_perm[token_to_row[t,j]] = x[t] for every assignment with a valid row.  A warp's
 // unit of work is 2 KB of one token's row (128 16-byte vectors, four per lane, all in
 // flight at once), read once and written to the token's k rows; units run grid-stride.
+// Rows are H 16-bit words (bf16 values, or pairs of e4m3 bytes); with scale_in the
+// per-row scales move the same way (scale_out[token_to_row[t,j]] = scale_in[t]).
 constexpr int kScatterVec = 128;
 __global__ void __launch_bounds__(kThreads)
     scatter_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ token_to_row, int64_t N, int k,
-                        int H, uint16_t *__restrict__ x_perm)
+                        int H, uint16_t *__restrict__ x_perm, const float *__restrict__ scale_in,
+                        float *__restrict__ scale_out)
 {
     pdl_entry();
     const int nvec = H / 8;
@@ -197,6 +200,10 @@ __global__ void __launch_bounds__(kThreads)
         int rows[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) rows[j] = j < k ? token_to_row[t * k + j] : -1;
+        if (scale_in && v0 == lane && lane < k) {  // first chunk of the row: lane j moves pick j's scale
+            const int r = token_to_row[t * k + lane];
+            if (r >= 0) scale_out[r] = scale_in[t];
+        }
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
         {
             uint4 buf[4];
@@ -216,6 +223,17 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 }  // namespace
+
+cudaError_t launch_scatter_rows(const uint16_t *x, const float *scale_in, const int32_t *token_to_row, int64_t N,
+                                int k, int H, uint16_t *x_perm, float *scale_out, cudaStream_t s)
+{
+    if (N <= 0) return cudaSuccess;
+    const int64_t units = N * ((H / 8 + kScatterVec - 1) / kScatterVec);
+    const int64_t want = (units + kWarps - 1) / kWarps;
+    const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
+    return launch_pdl(scatter_rows_kernel, dim3(gblocks), dim3(kThreads), 0, s, x, token_to_row, N, k, H, x_perm,
+                      scale_in, scale_out);
+}
 
 cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E, int k,
                            int32_t *counts, int32_t *offsets, int32_t *row_to_token, int32_t *token_to_row,
@@ -238,11 +256,8 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
                            E, (const int32_t *)scratch, row_to_token, token_to_row);
         if (e != cudaSuccess) return e;
     }
-    const int64_t units = N * ((H / 8 + kScatterVec - 1) / kScatterVec);
-    const int64_t want = (units + kWarps - 1) / kWarps;
-    const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
-    return launch_pdl(scatter_rows_kernel, dim3(gblocks), dim3(kThreads), 0, s, x, (const int32_t *)token_to_row,
-                      N, k, H, x_perm);
+    if (!x_perm) return cudaSuccess;  // dispatch only: the caller moves the rows itself
+    return launch_scatter_rows(x, nullptr, token_to_row, N, k, H, x_perm, nullptr, s);
 }
 
 }  // namespace moe

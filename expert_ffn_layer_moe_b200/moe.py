@@ -63,9 +63,15 @@ def lib() -> ctypes.CDLL:
         L.moe_quantize_fp8.argtypes = [vp, i64, c_int, vp, vp, vp]
         L.moe_expert_ffn_fp8.argtypes = [vp] * 8 + [i64, c_int, c_int, c_int, vp, vp, sz, vp]
         L.moe_layer_forward_fp8_ex.argtypes = ([vp] * 12 + [i64] + [c_int] * 5 + [vp, vp, vp, sz, vp, vp])
+        L.moe_expert_ffn_w8a8_ws_bytes.argtypes = [i64, c_int, c_int]
+        L.moe_expert_ffn_w8a8_ws_bytes.restype = sz
+        L.moe_expert_ffn_w8a8.argtypes = [vp] * 8 + [i64, c_int, c_int, c_int, vp, vp, vp, sz, vp]
+        L.moe_workspace_bytes_w8a8.argtypes = [i64, c_int, c_int, c_int, c_int, c_int]
+        L.moe_workspace_bytes_w8a8.restype = sz
+        L.moe_layer_forward_w8a8_ex.argtypes = ([vp] * 12 + [i64] + [c_int] * 5 + [vp, vp, vp, sz, vp, vp])
         for fn in ("moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
                    "moe_layer_forward_ex", "moe_get_device_error", "moe_quantize_fp8", "moe_expert_ffn_fp8",
-                   "moe_layer_forward_fp8_ex"):
+                   "moe_layer_forward_fp8_ex", "moe_expert_ffn_w8a8", "moe_layer_forward_w8a8_ex"):
             getattr(L, fn).restype = c_int
         _lib = L
     return _lib
@@ -246,6 +252,48 @@ def moe_layer_forward_fp8_ex(x, W_gate, W1q, s1, W3q, s3, W2q, s2, k, bias=None,
         assert len(phase_events) == len(PHASES) + 1
         ev = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
     _check("moe_layer_forward_fp8_ex", lib().moe_layer_forward_fp8_ex(
+        _p(x), _p(W_gate), _p(bias), _p(W1q), _p(s1), _p(W3q), _p(s3), _p(W2q), _p(s2), _p(Ws1), _p(Ws3),
+        _p(Ws2), N, H, I, E, k, Is, _p(out), _p(logits), _p(ws), ws.numel(), _s(stream), ev))
+    return out
+
+
+def moe_expert_ffn_w8a8_ws_bytes(R: int, H: int, I: int) -> int:
+    return int(lib().moe_expert_ffn_w8a8_ws_bytes(R, H, I))
+
+
+def moe_workspace_bytes_w8a8(N: int, H: int, I: int, E: int, k: int, Is: int = 0) -> int:
+    return int(lib().moe_workspace_bytes_w8a8(N, H, I, E, k, Is))
+
+
+def moe_expert_ffn_w8a8(x_perm, offsets, W1q, s1, W3q, s3, W2q, s2, ws=None, y_perm=None, h=None, stream=None):
+    """moe_expert_ffn with e4m3 weights and e4m3 activations (quantized per row on the
+    device) -> y_perm [R,H] fp32; h [R,I] bf16, when given, receives the SwiGLU output."""
+    R, H = x_perm.shape
+    E, I, _ = W1q.shape
+    y_perm = _empty((R, H), torch.float32, x_perm) if y_perm is None else y_perm
+    if ws is None:
+        ws = _empty((max(16, moe_expert_ffn_w8a8_ws_bytes(R, H, I)),), torch.uint8, x_perm)
+    _check("moe_expert_ffn_w8a8", lib().moe_expert_ffn_w8a8(
+        _p(x_perm), _p(offsets), _p(W1q), _p(s1), _p(W3q), _p(s3), _p(W2q), _p(s2), R, H, I, E, _p(y_perm),
+        _p(h), _p(ws), ws.numel(), _s(stream)))
+    return y_perm
+
+
+def moe_layer_forward_w8a8_ex(x, W_gate, W1q, s1, W3q, s3, W2q, s2, k, bias=None, Ws1=None, Ws3=None, Ws2=None,
+                              ws=None, out=None, logits=None, stream=None,
+                              phase_events: Optional[Sequence] = None):
+    """moe_layer_forward_fp8_ex with the routed experts' activations quantized to e4m3 as well."""
+    N, H = x.shape
+    E, I, _ = W1q.shape
+    Is = 0 if Ws1 is None else Ws1.shape[0]
+    out = _empty((N, H), torch.bfloat16, x) if out is None else out
+    if ws is None:
+        ws = _empty((max(16, moe_workspace_bytes_w8a8(N, H, I, E, k, Is)),), torch.uint8, x)
+    ev = None
+    if phase_events is not None:
+        assert len(phase_events) == len(PHASES) + 1
+        ev = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
+    _check("moe_layer_forward_w8a8_ex", lib().moe_layer_forward_w8a8_ex(
         _p(x), _p(W_gate), _p(bias), _p(W1q), _p(s1), _p(W3q), _p(s3), _p(W2q), _p(s2), _p(Ws1), _p(Ws3),
         _p(Ws2), N, H, I, E, k, Is, _p(out), _p(logits), _p(ws), ws.numel(), _s(stream), ev))
     return out

@@ -267,6 +267,43 @@ MOE_API moe_status_t moe_layer_forward_fp8_ex(const uint16_t *x, const float *W_
                                               void *const *phase_events);
 
 /*
+ * FP8 weights and FP8 activations (the same section names activations beside the
+ * weights).  On top of the e4m3 weights above, every activation row the two routed
+ * GEMMs read is quantized per row exactly as moe_quantize_fp8 does: the permuted
+ * token rows x_perm [R,H] before W1/W3, and the SwiGLU output h [R,I] after its
+ * bf16 rounding, before W2.  Both GEMMs then multiply e4m3 by e4m3 on the tensor
+ * cores (tcgen05 kind::f8f6f4, fp32 accumulation of exact products) and each
+ * output is multiplied by its weight row's scale and its token row's scale.
+ * Routing, combine and the shared experts stay as in the bf16 calls.
+ *
+ * moe_expert_ffn_w8a8: arguments, layouts and errors as moe_expert_ffn_fp8, plus
+ *   h        nullable device bf16 [R,I]: receives h (before its quantization);
+ *   ws       >= moe_expert_ffn_w8a8_ws_bytes(R,H,I) bytes (quantized rows, scales
+ *            and, when h is NULL, h itself).
+ */
+MOE_API size_t moe_expert_ffn_w8a8_ws_bytes(int64_t R, int H, int I);
+MOE_API moe_status_t moe_expert_ffn_w8a8(const uint16_t *x_perm, const int32_t *offsets, const uint8_t *W1q,
+                                         const float *s1, const uint8_t *W3q, const float *s3,
+                                         const uint8_t *W2q, const float *s2, int64_t R, int H, int I, int E,
+                                         float *y_perm, uint16_t *h, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * moe_layer_forward_fp8_ex with the activations quantized as well.  Workspace:
+ * moe_workspace_bytes_w8a8(N,H,I,E,k,Is) bytes (moe_workspace_bytes plus the
+ * quantized rows and their scales).  The x quantization is timed in the permute
+ * phase, the h quantization in the W1/W3 phase.  Other arguments and errors as
+ * moe_layer_forward_fp8_ex.
+ */
+MOE_API size_t moe_workspace_bytes_w8a8(int64_t N, int H, int I, int E, int k, int Is);
+MOE_API moe_status_t moe_layer_forward_w8a8_ex(const uint16_t *x, const float *W_gate, const float *bias,
+                                               const uint8_t *W1q, const float *s1, const uint8_t *W3q,
+                                               const float *s3, const uint8_t *W2q, const float *s2,
+                                               const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2,
+                                               int64_t N, int H, int I, int E, int k, int Is, uint16_t *out,
+                                               float *logits, void *ws, size_t ws_bytes, void *stream,
+                                               void *const *phase_events);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  *code receives a MOE_DEVERR_* value.  Returns MOE_OK, or
  * MOE_ERR_CUDA if the synchronisation itself failed.

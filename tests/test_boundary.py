@@ -42,6 +42,13 @@ def test_workspace_bytes():
     assert f(10, 256, 512, 16, 9) == 0       # k > 8
     assert f(-1, 256, 512, 8, 2) == 0
     assert f(10, 256, 512, 8, 2, 100) == 0   # shared width not a multiple of 64
+    # fp8 activations: the same layout plus the quantized rows (N*k*(H+I) bytes) and their scales
+    g = moe.moe_workspace_bytes_w8a8
+    assert g(156, 6144, 16384, 8, 2) - f(156, 6144, 16384, 8, 2) >= 312 * (6144 + 16384)
+    assert g(10, 100, 512, 8, 2) == 0 and g(10, 256, 512, 4, 5) == 0
+    w = moe.moe_expert_ffn_w8a8_ws_bytes
+    assert w(312, 6144, 16384) >= 312 * 16384 * 2 + 312 * (6144 + 16384) + 2 * 312 * 4
+    assert w(312, 100, 512) == 0 and w(-1, 256, 512) == 0
 
 
 def test_invalid_arguments_are_rejected_before_any_launch():
@@ -66,6 +73,13 @@ def test_invalid_arguments_are_rejected_before_any_launch():
     assert L.moe_expert_ffn_fp8(*([nullp] * 8), 8, 256, 512, 8, nullp, nullp, 0, s) == 1
     assert L.moe_layer_forward_fp8_ex(*([nullp] * 12), 4, 256, 512, 8, 2, 0, nullp, nullp, nullp, 0, s,
                                       nullp) == 1
+    assert L.moe_expert_ffn_w8a8(*([nullp] * 8), 8, 256, 500, 8, nullp, nullp, nullp, 0, s) == 1
+    assert L.moe_expert_ffn_w8a8(*([nullp] * 8), 8, 256, 512, 8, nullp, nullp, nullp, 0, s) == 1
+    assert L.moe_expert_ffn_w8a8(*([nullp] * 8), 0, 256, 512, 8, nullp, nullp, nullp, 0, s) == 0
+    assert L.moe_layer_forward_w8a8_ex(*([nullp] * 12), 4, 256, 512, 8, 2, 0, nullp, nullp, nullp, 0, s,
+                                       nullp) == 1
+    assert L.moe_layer_forward_w8a8_ex(*([nullp] * 12), 4, 256, 512, 8, 9, 0, nullp, nullp, nullp, 0, s,
+                                       nullp) == 1
     assert L.moe_layer_forward(nullp, nullp, nullp, nullp, nullp, 4, 256, 512, 8, 2, nullp) == 1
     assert L.moe_layer_forward_ex(*([nullp] * 9), 4, 256, 512, 8, 2, 64, nullp, nullp, nullp, 0, s,
                                   nullp) == 1
@@ -84,6 +98,10 @@ def test_misaligned_pointers_are_unsupported():
     assert L.moe_combine(fake, ok, ok, None, 4, 256, 2, ok, s) == 2
     assert L.moe_quantize_fp8(fake, 4, 256, ok, ok, s) == 2
     assert L.moe_quantize_fp8(ok, 4, 256, fake, ok, s) == 2
+    # fp8 activations: a misaligned h output is refused before the workspace is looked at
+    assert L.moe_expert_ffn_w8a8(*([ok] * 8), 8, 256, 512, 8, ok, fake, None, 0, s) == 2
+    # and a missing or short workspace is refused
+    assert L.moe_expert_ffn_w8a8(*([ok] * 8), 8, 256, 512, 8, ok, None, None, 0, s) == 3
 
 
 def test_status_strings():
