@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                         int groups, int rows_single, int64_t R, int K, int Nout,
                         void *__restrict__ out, int ksplit, int64_t split_stride,
                         const float *__restrict__ scale_a, const float *__restrict__ scale_b,
-                        const float *__restrict__ scale_act, int *dev_err)
+                        const float *__restrict__ scale_act, int64_t ldo, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
     constexpr int kThreads = C::kThreads;
@@ -714,7 +714,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
         // consecutive features of one row.
         const int q = warp & 3;   // TMEM lane quadrant this warp may read
         const int ew = warp - 2;  // 0..3
-        const bool vec_ok = (Nout & 7) == 0;  // then no 16-byte vector straddles the row end
+        // no 16-byte vector straddles a row end and every one is 16-byte aligned
+        const bool vec_ok = (Nout & 7) == 0 && (ldo & 3) == 0 && (split_stride & 3) == 0;
         const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(&tempty_bar[0]), 0) : 0u;
         int acc = 0;
         uint32_t aphase = 0;
@@ -805,15 +806,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                             if (c0 + r < nrows && fv < Nout) {
                                 const float4 v = make_float4(stage_t[4 * j + 0][r], stage_t[4 * j + 1][r],
                                                              stage_t[4 * j + 2][r], stage_t[4 * j + 3][r]);
-                                *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * Nout + fv) = v;
+                                *reinterpret_cast<float4 *>(outf + (size_t)(row0 + c0 + r) * ldo + fv) = v;
                             }
                         }
                         __syncwarp();
                     } else if (fbase + lane < Nout) {
-                        float *dst = outf + (size_t)(row0 + c0) * Nout + fbase + lane;
+                        float *dst = outf + (size_t)(row0 + c0) * ldo + fbase + lane;
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
-                            if (c0 + c < nrows) dst[(size_t)c * Nout] = a[c];
+                            if (c0 + c < nrows) dst[(size_t)c * ldo] = a[c];
                     }
                 }
             }
@@ -1005,6 +1006,8 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     }
     auto enc_act = A8 ? encode_act_map_fp8 : encode_act_map;
     if (!enc_act(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
+    const int64_t ldo = a.ldo > 0 ? a.ldo : a.Nout;
+    if (ldo < a.Nout) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR, W8, A8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
@@ -1025,7 +1028,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = PAIR ? 2 : 1;
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
-                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, a.dev_err);
+                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, ldo, a.dev_err);
     if (err != cudaSuccess) return err;
     count_launch();
     return cudaGetLastError();
@@ -1068,6 +1071,18 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
             default: return cudaErrorInvalidValue;
         }
     } else {
+        if constexpr (!SWIGLU && !W8 && !A8) {
+            // single-CTA tiles on request: an operand of at most 128 rows (a pair's M = 256
+            // would multiply rows of zeros)
+            if (a.single_cta) {
+                switch (bn) {
+                    case 32: return launch_impl<32, false, false, false, false>(a, s);
+                    case 64: return launch_impl<64, false, false, false, false>(a, s);
+                    case 128: return launch_impl<128, false, false, false, false>(a, s);
+                    default: return cudaErrorInvalidValue;
+                }
+            }
+        }
         if (bn <= 64 && gemm_pair_tiles(a.R, a.groups, a.Nout, SWIGLU, a.ksplit) < device_sm_count() / 2) {
             switch (bn) {
                 case 32: return launch_impl<32, SWIGLU, false, false, A8>(a, s);

@@ -74,11 +74,13 @@ struct GroupedGemmArgs {
     int rows_single;         // rows when offsets == nullptr
     int K;
     int Nout;
-    void *out;               // [R, Nout]: bf16 (SwiGLU GEMM) or fp32 (W2 GEMM)
+    void *out;               // [R, Nout] (row stride ldo): bf16 (SwiGLU GEMM) or fp32 (W2 GEMM)
     int *dev_err;
     int token_tile;          // 0 = choose from the shape
     int ksplit;              // plain GEMM: K slices (0/1 = none); partial sums at out + s*split_stride
     int64_t split_stride;    // elements between the partial-sum buffers
+    int64_t ldo;             // plain GEMM: elements between output rows (0 = Nout)
+    bool single_cta;         // plain bf16 GEMM: single-CTA tiles (token_tile 32, 64 or 128)
 };
 cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s);

@@ -21,8 +21,12 @@
 //  * kTensor (large N x E): the logits are a GEMM on the tcgen05 tensor cores.  W_gate
 //    is split into three bf16 terms hi + mid + lo (each the bf16 rounding of what the
 //    previous terms left; the remainder is below 2^-26 |w|), so x (bf16) times each
-//    term is exact and accumulates in fp32 in TMEM; the grouped GEMM kernel runs once
-//    over the stacked [3E, H] operand and the top-k kernel adds the three partial logits.
+//    term is exact and accumulates in fp32 in TMEM.  The grouped GEMM kernel runs once
+//    over the stacked [3E, H] operand -- on single-CTA tiles of 128 rows where those
+//    pad 3E less than CTA pairs' 256 (E = 128: 384 rows instead of 512), with K split
+//    into S slices so that mid-size batches cover the SMs -- and the top-k kernel adds
+//    the 3 S partial logits (slices interleaved in each output row, so they sit one
+//    stride apart) in a fixed order.
 // All reductions run in a fixed order: the logits' bits do not depend on timing.
 #include "common.cuh"
 #include "internal.h"
@@ -259,7 +263,7 @@ __global__ void __launch_bounds__(kThreads)
 
 // Top-k, one warp per token.  `lin` holds P partial logits of each token: part p of
 // token t, expert e at lin[p * pstride + t * tstride + e] -- the P slices of H of the
-// split path ([P][N][E]) or the hi, mid, lo terms of the tensor path ([N][3E]).  They
+// split path ([P][N][E]) or the 3 S terms and K slices of the tensor path ([N][S][3][E]).  They
 // are added in part order (+ bias), written to `logits` when it is given, then ranked.
 // With P == 1 and no bias `lin` already holds the logits.  P is a template argument so
 // that the loads of one expert's parts, and of consecutive experts, issue together.
@@ -409,6 +413,26 @@ cudaError_t launch_fused_for(const uint16_t *x, const float *W_gate, const float
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+constexpr int kTensorMaxSlices = 4;
+
+// Tensor-core path shape: single-CTA tiles (128 operand rows) where they pad the 3E rows
+// less than pairs (256), the token tile, and the K slices S: double S while the tiles
+// cover fewer than the SMs (or pairs) and each slice keeps at least 8 K blocks.
+void tensor_shape(int64_t N, int H, int E, int *bn, int *S, bool *single)
+{
+    const int64_t sms = device_sm_count();
+    const int rows = 3 * E;
+    *single = (rows + 127) / 128 * 128 < (rows + 255) / 256 * 256;
+    *bn = N >= 2048 ? 128 : 64;
+    const int per_tile = *single ? 128 : 256;
+    const int64_t tiles = ((N + *bn - 1) / *bn) * ((rows + per_tile - 1) / per_tile);
+    const int64_t units = *single ? sms : sms / 2;
+    const int kblocks = H / 64;
+    int sl = 1;
+    while (sl < kTensorMaxSlices && tiles * sl < units && kblocks / (2 * sl) >= 8) sl *= 2;
+    *S = sl;
+}
+
 }  // namespace
 
 RouterPath router_path(int64_t N, int E, bool have_logits_buffer, bool have_ws)
@@ -420,7 +444,8 @@ RouterPath router_path(int64_t N, int E, bool have_logits_buffer, bool have_ws)
 
 size_t router_ws_bytes(int64_t N, int H, int E)
 {
-    return align256((size_t)3 * E * H * 2) + align256((size_t)N * 3 * E * 4) + align256((size_t)N * E * 4);
+    return align256((size_t)3 * E * H * 2) + align256((size_t)kTensorMaxSlices * N * 3 * E * 4) +
+           align256((size_t)N * E * 4);
 }
 
 cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
@@ -432,7 +457,7 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
     const RouterPath path = router_path(N, E, logits != nullptr, have_ws);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     const size_t split_bytes = align256((size_t)3 * E * H * 2);
-    const size_t parts_bytes = align256((size_t)N * 3 * E * 4);
+    const size_t parts_bytes = align256((size_t)kTensorMaxSlices * N * 3 * E * 4);
     float *lbuf = logits ? logits : (have_ws ? reinterpret_cast<float *>(w8 + split_bytes + parts_bytes) : nullptr);
 
     if (path == RouterPath::kTensor) {
@@ -441,12 +466,25 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
         const dim3 sgrid((unsigned)((H + 31) / 32), (unsigned)((E + 31) / 32));
         cudaError_t e = launch_pdl(router_split_kernel, sgrid, dim3(kThreads), 0, s, W_gate, H, E, wsplit);
         if (e != cudaSuccess) return e;
+        int bn, S;
+        bool single;
+        tensor_shape(N, H, E, &bn, &S, &single);
+        // K slice s of token t's three terms lands at parts + t*3ES + s*3E (row stride 3ES,
+        // slices 3E apart): part p = 3s + term of expert e sits at t*3ES + p*E + e
         GroupedGemmArgs g{};
         g.act = x; g.w_a = wsplit; g.w_b = nullptr; g.offsets = nullptr; g.groups = 1; g.R = N;
-        g.rows_single = (int)N; g.K = H; g.Nout = 3 * E; g.out = parts; g.dev_err = dev_err; g.token_tile = 128;
+        g.rows_single = (int)N; g.K = H; g.Nout = 3 * E; g.out = parts; g.dev_err = dev_err;
+        g.token_tile = bn; g.single_cta = single; g.ksplit = S;
+        g.ldo = (int64_t)3 * E * S; g.split_stride = (int64_t)3 * E;
         e = launch_gemm2(g, s);
         if (e != cudaSuccess) return e;
-        return launch_topk<3>(parts, (int64_t)E, (int64_t)3 * E, bias, N, E, k, lbuf, topk_idx, topk_w, s);
+        const int64_t ts = (int64_t)3 * E * S;
+        switch (S) {
+            case 1: return launch_topk<3>(parts, E, ts, bias, N, E, k, lbuf, topk_idx, topk_w, s);
+            case 2: return launch_topk<6>(parts, E, ts, bias, N, E, k, lbuf, topk_idx, topk_w, s);
+            case 4: return launch_topk<12>(parts, E, ts, bias, N, E, k, lbuf, topk_idx, topk_w, s);
+            default: return cudaErrorInvalidValue;
+        }
     }
     if (path == RouterPath::kSplit) {
         // the H-slice partials go to the scratch (its first two regions), else the
