@@ -488,7 +488,11 @@ def run_ours(args, cfg, world, rank, local):
     flops = layer_flops(cfg)
     gemm_flops = 6 * cfg.R * H * I
     lbytes = layer_bytes(cfg, touched, wbytes)
-    floor_s = max(flops / (pk["bf16_tflops"] * 1e12), lbytes / (hbm * 1e9))
+    # tensor floor: the routed experts' FLOPs at their operands' peak (e4m3 x e4m3: the bf16
+    # peak times the nominal 2x), the router's and the shared experts' at the bf16 peak
+    routed_flops = 6 * cfg.R * H * I
+    tensor_s = (routed_flops / (2.0 if a8 else 1.0) + (flops - routed_flops)) / (pk["bf16_tflops"] * 1e12)
+    floor_s = max(tensor_s, lbytes / (hbm * 1e9))
     workload = cfg.name
     # the W1/W3 kernel's bound: weight streaming (HBM) at decode sizes, the tensor cores
     # once the token tiles are long enough (its FLOPs at the tensor peak outlast its
