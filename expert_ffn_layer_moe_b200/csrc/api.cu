@@ -366,6 +366,18 @@ moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, cons
                            static_cast<cudaStream_t>(stream));
 }
 
+moe_status_t moe_scatter_rows(const uint16_t *src, const int32_t *dst_row, int64_t rows, int width, uint16_t *dst,
+                              void *stream)
+{
+    if (rows < 0 || width < 8 || width % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!src || !dst_row || !dst) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(src) || !aligned16(dst)) return MOE_ERR_UNSUPPORTED;
+    MOE_CUDA(moe::launch_scatter_rows(src, nullptr, dst_row, rows, 1, width, dst, nullptr,
+                                      static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
 moe_status_t moe_combine(const float *y_perm, const int32_t *token_to_row, const float *topk_w,
                          const float *shared_out, int64_t N, int H, int k, uint16_t *out, void *stream)
 {

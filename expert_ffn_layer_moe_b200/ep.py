@@ -1,0 +1,165 @@
+"""Expert parallelism: the experts split over G ranks, token rows exchanged all-to-all.
+
+[MoE-latency] "跨 GPU 时,激活要出门": when the experts do not fit one GPU they are
+placed on different GPUs; a token whose chosen expert lives on another GPU sends its
+activation row there and gets the expert's output back, every rank sending to and
+receiving from every other rank at once (all-to-all), in every MoE layer.  Section
+"最慢的 GPU 决定这一步": a step lasts as long as its slowest rank, so the per-rank
+assignment counts and phase times of each step are what to record (``EPStats``).
+
+Layout: rank r holds experts [r*L, (r+1)*L), L = E/G (its slices of W1, W3 and W2).
+Each rank routes and permutes its own token batch with the library's kernels.  Its
+permuted rows x_perm are sorted by expert, so the rows bound for rank r form one
+contiguous range.  Then:
+
+1. all-gather of the per-expert counts [G, E] -- the exchange sizes, read on the host
+   (the one host synchronisation of the step);
+2. all-to-all of the rows: rank r receives, from each source in rank order, that
+   source's rows for r's experts, sorted by expert;
+3. a row scatter into expert-major order (inside an expert: source rank, then the
+   source's order -- stable, so the result is deterministic), the local grouped GEMMs
+   (SwiGLU W1/W3, then W2 with fp32 out);
+4. a row scatter back to the received order and the all-to-all back (fp32 rows);
+5. the combine on the source rank, in pick order: the same sums, in the same order,
+   as the one-device layer computes.
+
+The plan and the exchange are device-independent; the local steps (the expert FFN and
+the row scatter) are passed in.  ``moe_layer_forward_ep`` runs the library's kernels on
+CUDA tensors over an NCCL process group.  The rows cross the wire as raw 32-bit words.
+"""
+from __future__ import annotations
+
+import dataclasses
+import time
+from typing import Callable, List, Optional
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+
+@dataclasses.dataclass
+class ExchangePlan:
+    """Sizes and row maps of one rank's exchange (all rows counted in [R, H] rows)."""
+    send_splits: List[int]      # rows sent to each rank, in rank order (ranges of x_perm)
+    recv_splits: List[int]      # rows received from each rank
+    local_offsets: np.ndarray   # [L+1] int32: row offsets of the local experts, expert-major
+    recv_to_local: np.ndarray   # [sum(recv_splits)] int32: expert-major row of each received row
+    local_to_recv: np.ndarray   # the inverse permutation
+
+
+@dataclasses.dataclass
+class EPStats:
+    """One step on one rank: assignments sent and received, and host-clock phase times
+    (seconds; each phase ends with a device synchronisation)."""
+    rows_sent: int
+    rows_received: int
+    seconds: dict
+
+
+def exchange_plan(counts_all, rank: int) -> ExchangePlan:
+    """The plan of rank `rank` from every rank's per-expert row counts [G, E]."""
+    counts_all = np.asarray(counts_all, dtype=np.int64)
+    G, E = counts_all.shape
+    if E % G != 0:
+        raise ValueError(f"{E} experts do not split evenly over {G} ranks")
+    if not 0 <= rank < G:
+        raise ValueError("rank outside the group")
+    L = E // G
+    per_pair = counts_all.reshape(G, G, L).sum(axis=2)       # [source, destination] rows
+    loc = counts_all[:, rank * L:(rank + 1) * L]              # [source, local expert] rows
+    local_offsets = np.concatenate([[0], np.cumsum(loc.sum(axis=0))]).astype(np.int64)
+    earlier = np.cumsum(loc, axis=0) - loc                    # rows of expert e from earlier sources
+    parts = [np.arange(loc[s, e], dtype=np.int64) + local_offsets[e] + earlier[s, e]
+             for s in range(G) for e in range(L)]
+    recv_to_local = np.concatenate(parts) if parts else np.zeros(0, np.int64)
+    local_to_recv = np.empty_like(recv_to_local)
+    local_to_recv[recv_to_local] = np.arange(recv_to_local.size)
+    return ExchangePlan([int(v) for v in per_pair[rank, :]], [int(v) for v in per_pair[:, rank]],
+                        local_offsets.astype(np.int32), recv_to_local.astype(np.int32),
+                        local_to_recv.astype(np.int32))
+
+
+def _words(t: torch.Tensor) -> torch.Tensor:
+    """A row-major tensor as 32-bit words per row (the wire format of the exchange)."""
+    if t.element_size() == 4:
+        return t if t.dtype in (torch.int32, torch.float32) else t.view(torch.int32)
+    if t.element_size() == 2:
+        return t.view(torch.int32)
+    return t  # 8-byte rows travel as they are
+
+
+def _sync(dev):
+    if dev.type == "cuda":
+        torch.cuda.synchronize(dev)
+
+
+def exchange_ffn(x_perm: torch.Tensor, counts: torch.Tensor, E: int,
+                 local_ffn: Callable[[torch.Tensor, torch.Tensor], torch.Tensor],
+                 scatter_rows: Callable[[torch.Tensor, torch.Tensor, torch.Tensor], torch.Tensor],
+                 group=None, stats: Optional[list] = None):
+    """Steps 1-4: x_perm [R, H] (this rank's rows, sorted by expert) and counts [E] ->
+    y [R, H], row r the output of x_perm[r]'s expert, computed on that expert's rank.
+
+    local_ffn(x_loc, local_offsets) -> y_loc runs the local experts on expert-major rows;
+    scatter_rows(src, dst_row, dst) sets dst[dst_row[i]] = src[i].  Returns (y, plan)."""
+    G = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    dev = x_perm.device
+    t0 = time.perf_counter()
+    gathered = [torch.empty_like(counts) for _ in range(G)]
+    dist.all_gather(gathered, counts.contiguous(), group=group)
+    plan = exchange_plan(torch.stack(gathered).cpu().numpy(), rank)
+    t1 = time.perf_counter()
+    R, H = x_perm.shape
+    recv = torch.empty((sum(plan.recv_splits), H), dtype=x_perm.dtype, device=dev)
+    dist.all_to_all_single(_words(recv), _words(x_perm.contiguous()), plan.recv_splits, plan.send_splits,
+                           group=group)
+    _sync(dev)
+    t2 = time.perf_counter()
+    x_loc = torch.empty_like(recv)
+    scatter_rows(recv, torch.from_numpy(plan.recv_to_local).to(dev), x_loc)
+    y_loc = local_ffn(x_loc, torch.from_numpy(plan.local_offsets).to(dev))
+    y_recv = torch.empty_like(y_loc)
+    scatter_rows(y_loc, torch.from_numpy(plan.local_to_recv).to(dev), y_recv)
+    _sync(dev)
+    t3 = time.perf_counter()
+    y = torch.empty((R, y_loc.shape[1]), dtype=y_loc.dtype, device=dev)
+    dist.all_to_all_single(_words(y), _words(y_recv), plan.send_splits, plan.recv_splits, group=group)
+    _sync(dev)
+    t4 = time.perf_counter()
+    if stats is not None:
+        stats.append(EPStats(R, int(sum(plan.recv_splits)),
+                             {"plan": t1 - t0, "dispatch": t2 - t1, "experts": t3 - t2, "combine_exchange": t4 - t3}))
+    return y, plan
+
+
+def local_experts(W: torch.Tensor, rank: int, G: int) -> torch.Tensor:
+    """This rank's slice [L, ...] of an expert stack [E, ...] (a view)."""
+    E = W.shape[0]
+    if E % G != 0:
+        raise ValueError(f"{E} experts do not split evenly over {G} ranks")
+    L = E // G
+    return W[rank * L:(rank + 1) * L]
+
+
+def moe_layer_forward_ep(x: torch.Tensor, W_gate: torch.Tensor, W1_local: torch.Tensor, W3_local: torch.Tensor,
+                         W2_local: torch.Tensor, k: int, bias: Optional[torch.Tensor] = None, group=None,
+                         stats: Optional[list] = None) -> torch.Tensor:
+    """The MoE layer with the experts split over the ranks of `group` (NCCL, one GPU per
+    rank).  x [N,H] bf16 is this rank's batch; W_gate [H,E] fp32 is the whole router;
+    W1_local, W3_local [L,I,H] and W2_local [L,H,I] bf16 are this rank's experts
+    (``local_experts``).  Returns this rank's out [N,H] bf16."""
+    from expert_ffn_layer_moe_b200 import moe
+    G = dist.get_world_size(group)
+    E = W_gate.shape[1]
+    if W1_local.shape[0] * G != E:
+        raise ValueError("local expert slices do not match E / world size")
+    idx, w, _ = moe.moe_route(x, W_gate, k, bias=bias)
+    p = moe.moe_permute(x, idx, E)
+
+    def ffn(x_loc, offsets_loc):
+        return moe.moe_expert_ffn(x_loc, offsets_loc, W1_local, W3_local, W2_local)
+
+    y, _ = exchange_ffn(p["x_perm"], p["counts"], E, ffn, moe.moe_scatter_rows, group=group, stats=stats)
+    return moe.moe_combine(y, p["token_to_row"], w)

@@ -1,0 +1,131 @@
+"""Expert parallelism on CPU: the exchange plan, and the whole exchange over gloo ranks.
+
+[MoE-latency] "跨 GPU 时,激活要出门": tokens whose experts live on other GPUs send
+their rows there and get the outputs back (all-to-all).  The plan is checked by hand
+on a small case and by its invariants on random counts; the exchange runs as 2 and 4
+gloo ranks (each with its own token batch and E/G experts, the oracle as each rank's
+local expert compute and torch indexing as its row scatter) and must give every rank
+the bit-exact output of the one-device oracle layer on its batch.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+from expert_ffn_layer_moe_b200 import ep
+
+
+def test_plan_by_hand():
+    # G = 2 ranks, E = 4 experts (rank 0: experts 0, 1; rank 1: experts 2, 3)
+    counts = [[1, 2, 0, 3],   # rank 0's rows per expert
+              [2, 0, 1, 1]]   # rank 1's
+    p0 = ep.exchange_plan(counts, 0)
+    assert p0.send_splits == [3, 3] and p0.recv_splits == [3, 2]
+    assert p0.local_offsets.tolist() == [0, 3, 5]
+    # received: (src 0: e0 r0, e1 r0, e1 r1), (src 1: e0 r0, e0 r1); expert-major with
+    # the source order inside an expert: e0 <- s0 r0, s1 r0, s1 r1; e1 <- s0 r0, s0 r1
+    assert p0.recv_to_local.tolist() == [0, 3, 4, 1, 2]
+    assert p0.local_to_recv.tolist() == [0, 3, 4, 1, 2]
+    p1 = ep.exchange_plan(counts, 1)
+    assert p1.send_splits == [2, 2] and p1.recv_splits == [3, 2]
+    assert p1.local_offsets.tolist() == [0, 1, 5]
+    # received: (src 0: e3 x3), (src 1: e2, e3) -> e2 <- s1; e3 <- s0 x3, s1
+    assert p1.recv_to_local.tolist() == [1, 2, 3, 0, 4]
+    with pytest.raises(ValueError):
+        ep.exchange_plan(np.ones((2, 3)), 0)          # 3 experts do not split over 2 ranks
+    with pytest.raises(ValueError):
+        ep.exchange_plan(counts, 2)                   # no rank 2
+
+
+@pytest.mark.parametrize("G,E", [(1, 8), (2, 8), (4, 16), (8, 256)])
+def test_plan_invariants(G, E):
+    rng = np.random.default_rng(G * 100 + E)
+    counts = rng.integers(0, 6, size=(G, E))
+    counts[0, : E // G] = 0                       # a rank whose experts get nothing from rank 0
+    plans = [ep.exchange_plan(counts, r) for r in range(G)]
+    L = E // G
+    for r, p in enumerate(plans):
+        # what r sends to d is what d receives from r; sends cover r's rows, in x_perm order
+        assert sum(p.send_splits) == counts[r].sum()
+        for d in range(G):
+            assert p.send_splits[d] == plans[d].recv_splits[r] == counts[r, d * L:(d + 1) * L].sum()
+        n = sum(p.recv_splits)
+        assert p.local_offsets[-1] == n and np.all(np.diff(p.local_offsets) == counts[:, r * L:(r + 1) * L].sum(0))
+        assert sorted(p.recv_to_local.tolist()) == list(range(n))           # a permutation
+        assert np.array_equal(p.local_to_recv[p.recv_to_local], np.arange(n))
+        # stable: inside each local expert the received rows keep their received order
+        expert_of = np.repeat(np.arange(L), np.diff(p.local_offsets))
+        recv_expert = expert_of[p.recv_to_local]
+        for e in range(L):
+            pos = np.flatnonzero(recv_expert == e)
+            assert np.all(np.diff(p.recv_to_local[pos]) == 1)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from expert_ffn_layer_moe_b200.inputs import MoEConfig, make_inputs
+    from tests._bf16 import to_u16
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    cfg = MoEConfig("ep", N=24, H=64, I=32, E=4 * world, k=3)
+    wts = make_inputs(cfg, seed=0)                               # the same weights on every rank
+    x = to_u16(make_inputs(cfg, seed=10 + rank, weights=False)["x"])   # each rank its own batch
+    W1, W3, W2 = (to_u16(wts[n]) for n in ("W1", "W3", "W2"))
+    Wg = wts["W_gate"].numpy()
+    l32 = oracle.router_logits(x, Wg).astype(np.float32)
+    idx, w = oracle.topk(l32, cfg.k)
+    counts, _, r2t, t2r = oracle.dispatch(idx, cfg.E)
+    xp = oracle.permute_rows(x, r2t)
+    L = cfg.E // world
+    mine = slice(rank * L, (rank + 1) * L)
+
+    def ffn(x_loc, offsets):
+        y = oracle.expert_ffn(x_loc.numpy().view(np.uint16), offsets.numpy(), W1[mine], W3[mine], W2[mine])
+        return torch.from_numpy(y)
+
+    def scatter(src, dst_row, dst):
+        dst[dst_row.long()] = src
+        return dst
+
+    stats = []
+    y, plan = ep.exchange_ffn(torch.from_numpy(xp.view(np.int16)), torch.from_numpy(counts), cfg.E, ffn, scatter,
+                              stats=stats)
+    out = oracle.combine(y.numpy(), t2r, w)
+    ref = oracle.layer_given_logits(x, l32, W1, W3, W2, cfg.k)
+    dist.destroy_process_group()
+    q.put((rank, bool(np.array_equal(out, ref)), stats[0].rows_sent, stats[0].rows_received, plan.recv_splits))
+
+
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_exchange_gives_the_one_device_layer(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=200) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(r[1] for r in res), res
+    assert all(r[2] == 24 * 3 for r in res)                    # every rank sends all its N*k rows
+    assert sum(r[3] for r in res) == world * 24 * 3            # and all of them arrive somewhere
+    assert any(r[4][r[0]] < r[3] for r in res)                 # rows really crossed ranks

@@ -1,0 +1,73 @@
+"""Expert parallelism on one GPU: the row scatter kernel, and the EP layer on a
+one-rank NCCL group (route, permute, the exchange to itself, the local experts, the
+combine) against the oracle given the GPU's logits.
+
+[MoE-latency] "跨 GPU 时,激活要出门".  Runs with more ranks need more GPUs than a
+test here has; the multi-rank exchange is covered on CPU by tests/test_ep_host.py.
+"""
+import datetime
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+import oracle
+from expert_ffn_layer_moe_b200 import ep, moe
+from expert_ffn_layer_moe_b200.inputs import MoEConfig
+from tests._bf16 import dec
+from tests.test_gpu_parity import assert_close, cuda_inputs, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype,cols", [(torch.bfloat16, 64), (torch.bfloat16, 200 * 8), (torch.float32, 64)])
+def test_scatter_rows_bit_exact(dtype, cols):
+    g = torch.Generator().manual_seed(cols)
+    rows = 333
+    src = torch.randn((rows, cols), generator=g).to(dtype)
+    perm = torch.randperm(rows + 20, generator=g)[:rows].to(torch.int32)
+    perm[::7] = -1                                               # skipped rows
+    dst = torch.full((rows + 20, cols), 7.0).to(dtype)
+    got = moe.moe_scatter_rows(src.cuda(), perm.cuda(), dst.cuda())
+    torch.cuda.synchronize()
+    want = dst.clone()
+    keep = perm >= 0
+    want[perm[keep].long()] = src[keep]
+    assert torch.equal(got.cpu().view(torch.int16 if dtype == torch.bfloat16 else torch.int32),
+                       want.view(torch.int16 if dtype == torch.bfloat16 else torch.int32))
+
+
+def _port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+@pytest.mark.parametrize("cfg", [
+    MoEConfig("ep1", N=300, H=256, I=192, E=8, k=2),
+    MoEConfig("ep1_decode", N=7, H=512, I=256, E=16, k=4),       # empty experts, a few rows each
+])
+def test_ep_layer_one_rank_matches_oracle(cfg):
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_port()}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        t = cuda_inputs(cfg, seed=5)
+        stats = []
+        out = ep.moe_layer_forward_ep(t["x"], t["W_gate"], ep.local_experts(t["W1"], 0, 1),
+                                      ep.local_experts(t["W3"], 0, 1), ep.local_experts(t["W2"], 0, 1), cfg.k,
+                                      bias=t["bias"], stats=stats)
+        # the same router call as inside the layer, now keeping its logits (same path, same bits)
+        logits = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device="cuda")
+        moe.moe_route(t["x"], t["W_gate"], cfg.k, bias=t["bias"], logits=logits)
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error() == 0
+        assert stats[0].rows_sent == stats[0].rows_received == cfg.N * cfg.k
+        ref = oracle.layer_given_logits(host(t["x"]), host(logits), host(t["W1"]), host(t["W3"]), host(t["W2"]),
+                                        cfg.k)
+        assert_close(dec(host(out)), dec(ref), f"{cfg.name} ep out")
+    finally:
+        dist.destroy_process_group()
