@@ -242,7 +242,7 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
         MOE_CUDA(moe::launch_quantize_fp8(x, N, H, Q.xqt, Q.xst, s));
         MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
         MOE_CUDA(moe::launch_scatter_rows(reinterpret_cast<const uint16_t *>(Q.xqt), Q.xst, t2r, N, k, H / 2,
-                                          reinterpret_cast<uint16_t *>(Q.xq), Q.xsc, s));
+                                          reinterpret_cast<uint16_t *>(Q.xq), R, Q.xsc, s));
         a.act = Q.xq; a.a8 = true; a.scale_act = Q.xsc;
     } else {
         MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
@@ -367,13 +367,13 @@ moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, cons
 }
 
 moe_status_t moe_scatter_rows(const uint16_t *src, const int32_t *dst_row, int64_t rows, int width, uint16_t *dst,
-                              void *stream)
+                              int64_t dst_rows, void *stream)
 {
-    if (rows < 0 || width < 8 || width % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (rows < 0 || dst_rows < 0 || width < 8 || width % 8 != 0) return MOE_ERR_INVALID_ARG;
     if (rows == 0) return MOE_OK;
     if (!src || !dst_row || !dst) return MOE_ERR_INVALID_ARG;
     if (!aligned16(src) || !aligned16(dst)) return MOE_ERR_UNSUPPORTED;
-    MOE_CUDA(moe::launch_scatter_rows(src, nullptr, dst_row, rows, 1, width, dst, nullptr,
+    MOE_CUDA(moe::launch_scatter_rows(src, nullptr, dst_row, rows, 1, width, dst, dst_rows, nullptr,
                                       static_cast<cudaStream_t>(stream)));
     return MOE_OK;
 }

@@ -53,8 +53,9 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
                            int *dev_err, cudaStream_t s);
 // x_perm[token_to_row[t,j]] = x[t]: rows of H 16-bit words (H a multiple of 8; e4m3
 // rows of 2H bytes pass as H words); with scale_in, scale_out[token_to_row[t,j]] = scale_in[t].
+// Target rows outside [0, out_rows) are skipped.
 cudaError_t launch_scatter_rows(const uint16_t *x, const float *scale_in, const int32_t *token_to_row, int64_t N,
-                                int k, int H, uint16_t *x_perm, float *scale_out, cudaStream_t s);
+                                int k, int H, uint16_t *x_perm, int64_t out_rows, float *scale_out, cudaStream_t s);
 
 // Grouped GEMMs on tcgen05.  Weights are [groups, Nout, K]; activations [R, K];
 // rows of group g are offsets[g] .. offsets[g+1]-1 (offsets == nullptr: one group

@@ -181,11 +181,12 @@ __global__ void __launch_bounds__(kThreads)
 // unit of work is 2 KB of one token's row (128 16-byte vectors, four per lane, all in
 // flight at once), read once and written to the token's k rows; units run grid-stride.
 // Rows are H 16-bit words (bf16 values, or pairs of e4m3 bytes); with scale_in the
-// per-row scales move the same way (scale_out[token_to_row[t,j]] = scale_in[t]).
+// per-row scales move the same way (scale_out[token_to_row[t,j]] = scale_in[t]).  Target
+// rows outside [0, out_rows) are skipped.
 constexpr int kScatterVec = 128;
 __global__ void __launch_bounds__(kThreads)
     scatter_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ token_to_row, int64_t N, int k,
-                        int H, uint16_t *__restrict__ x_perm, const float *__restrict__ scale_in,
+                        int H, uint16_t *__restrict__ x_perm, int64_t out_rows, const float *__restrict__ scale_in,
                         float *__restrict__ scale_out)
 {
     pdl_entry();
@@ -199,10 +200,13 @@ __global__ void __launch_bounds__(kThreads)
         const int v0 = (int)(unit % chunks) * kScatterVec + lane;
         int rows[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) rows[j] = j < k ? token_to_row[t * k + j] : -1;
+        for (int j = 0; j < 8; ++j) {
+            const int r = j < k ? token_to_row[t * k + j] : -1;
+            rows[j] = r < out_rows ? r : -1;  // outside the target: skipped
+        }
         if (scale_in && v0 == lane && lane < k) {  // first chunk of the row: lane j moves pick j's scale
             const int r = token_to_row[t * k + lane];
-            if (r >= 0) scale_out[r] = scale_in[t];
+            if (r >= 0 && r < out_rows) scale_out[r] = scale_in[t];
         }
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
         {
@@ -225,14 +229,14 @@ __global__ void __launch_bounds__(kThreads)
 }  // namespace
 
 cudaError_t launch_scatter_rows(const uint16_t *x, const float *scale_in, const int32_t *token_to_row, int64_t N,
-                                int k, int H, uint16_t *x_perm, float *scale_out, cudaStream_t s)
+                                int k, int H, uint16_t *x_perm, int64_t out_rows, float *scale_out, cudaStream_t s)
 {
     if (N <= 0) return cudaSuccess;
     const int64_t units = N * ((H / 8 + kScatterVec - 1) / kScatterVec);
     const int64_t want = (units + kWarps - 1) / kWarps;
     const int gblocks = (int)(want < 148 * 8 ? want : 148 * 8);
     return launch_pdl(scatter_rows_kernel, dim3(gblocks), dim3(kThreads), 0, s, x, token_to_row, N, k, H, x_perm,
-                      scale_in, scale_out);
+                      out_rows, scale_in, scale_out);
 }
 
 cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E, int k,
@@ -257,7 +261,7 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
         if (e != cudaSuccess) return e;
     }
     if (!x_perm) return cudaSuccess;  // dispatch only: the caller moves the rows itself
-    return launch_scatter_rows(x, nullptr, token_to_row, N, k, H, x_perm, nullptr, s);
+    return launch_scatter_rows(x, nullptr, token_to_row, N, k, H, x_perm, R, nullptr, s);
 }
 
 }  // namespace moe

@@ -69,7 +69,7 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_bytes_w8a8.argtypes = [i64, c_int, c_int, c_int, c_int, c_int]
         L.moe_workspace_bytes_w8a8.restype = sz
         L.moe_layer_forward_w8a8_ex.argtypes = ([vp] * 12 + [i64] + [c_int] * 5 + [vp, vp, vp, sz, vp, vp])
-        L.moe_scatter_rows.argtypes = [vp, vp, i64, c_int, vp, vp]
+        L.moe_scatter_rows.argtypes = [vp, vp, i64, c_int, vp, i64, vp]
         for fn in ("moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
                    "moe_layer_forward_ex", "moe_get_device_error", "moe_quantize_fp8", "moe_expert_ffn_fp8",
                    "moe_layer_forward_fp8_ex", "moe_expert_ffn_w8a8", "moe_layer_forward_w8a8_ex",
@@ -302,11 +302,12 @@ def moe_layer_forward_w8a8_ex(x, W_gate, W1q, s1, W3q, s3, W2q, s2, k, bias=None
 
 
 def moe_scatter_rows(src, dst_row, dst, stream=None):
-    """dst[dst_row[i]] = src[i] for rows with dst_row[i] >= 0 (bf16 or fp32 rows, on the device)."""
+    """dst[dst_row[i]] = src[i] for rows with 0 <= dst_row[i] < len(dst) (bf16 or fp32 rows, on the device)."""
     assert src.dtype == dst.dtype and src.dtype in (torch.bfloat16, torch.float32) and src.shape[1:] == dst.shape[1:]
     rows = src.shape[0]
     width = src.shape[1] * (2 if src.dtype == torch.float32 else 1)
-    _check("moe_scatter_rows", lib().moe_scatter_rows(_p(src), _p(dst_row), rows, width, _p(dst), _s(stream)))
+    _check("moe_scatter_rows", lib().moe_scatter_rows(_p(src), _p(dst_row), rows, width, _p(dst), dst.shape[0],
+                                                      _s(stream)))
     return dst
 
 

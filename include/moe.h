@@ -177,14 +177,15 @@ MOE_API moe_status_t moe_expert_ffn(const uint16_t *x_perm, const int32_t *offse
  * Row scatter, the local reorder steps of expert parallelism ([MoE-latency] "跨 GPU
  * 时,激活要出门": rows received from other ranks are regrouped by local expert, and
  * the expert outputs are put back in the order they travel home in):
- *   dst[dst_row[i]] = src[i] for i in [0, rows) with dst_row[i] >= 0 (rows < 0 skipped)
- *   src, dst: rows of `width` 16-bit words (bf16 values, or fp32 values as word pairs:
- *   width = 2 * columns); width a multiple of 8; src, dst 16-byte aligned device
- *   pointers; dst_row [rows] int32 device, each target row written once (distinct
+ *   dst[dst_row[i]] = src[i] for i in [0, rows) with 0 <= dst_row[i] < dst_rows (other
+ *   target rows are skipped on the device)
+ *   src [rows], dst [dst_rows]: rows of `width` 16-bit words (bf16 values, or fp32 values
+ *   as word pairs: width = 2 * columns); width a multiple of 8; src, dst 16-byte aligned
+ *   device pointers; dst_row [rows] int32 device, each target row written once (distinct
  *   rows; a repeated row is a race).  Asynchronous on `stream`.
  */
 MOE_API moe_status_t moe_scatter_rows(const uint16_t *src, const int32_t *dst_row, int64_t rows, int width,
-                                      uint16_t *dst, void *stream);
+                                      uint16_t *dst, int64_t dst_rows, void *stream);
 
 /*
  * Combine / unpermutation ([MoE-latency] "router 之后还有一串动作": inverse

@@ -82,10 +82,11 @@ def test_invalid_arguments_are_rejected_before_any_launch():
                                        nullp) == 1
     assert L.moe_layer_forward(nullp, nullp, nullp, nullp, nullp, 4, 256, 512, 8, 2, nullp) == 1
     # row scatter: width a positive multiple of 8, rows >= 0, pointers present
-    assert L.moe_scatter_rows(nullp, nullp, 4, 12, nullp, s) == 1
-    assert L.moe_scatter_rows(nullp, nullp, -1, 64, nullp, s) == 1
-    assert L.moe_scatter_rows(nullp, nullp, 4, 64, nullp, s) == 1
-    assert L.moe_scatter_rows(nullp, nullp, 0, 64, nullp, s) == 0
+    assert L.moe_scatter_rows(nullp, nullp, 4, 12, nullp, 4, s) == 1
+    assert L.moe_scatter_rows(nullp, nullp, -1, 64, nullp, 4, s) == 1
+    assert L.moe_scatter_rows(nullp, nullp, 4, 64, nullp, -1, s) == 1
+    assert L.moe_scatter_rows(nullp, nullp, 4, 64, nullp, 4, s) == 1
+    assert L.moe_scatter_rows(nullp, nullp, 0, 64, nullp, 4, s) == 0
     assert L.moe_layer_forward_ex(*([nullp] * 9), 4, 256, 512, 8, 2, 64, nullp, nullp, nullp, 0, s,
                                   nullp) == 1
     # N == 0 is a no-op where no output needs defining
@@ -105,7 +106,7 @@ def test_misaligned_pointers_are_unsupported():
     assert L.moe_quantize_fp8(ok, 4, 256, fake, ok, s) == 2
     # fp8 activations: a misaligned h output is refused before the workspace is looked at
     assert L.moe_expert_ffn_w8a8(*([ok] * 8), 8, 256, 512, 8, ok, fake, None, 0, s) == 2
-    assert L.moe_scatter_rows(fake, ok, 4, 64, ok, s) == 2
+    assert L.moe_scatter_rows(fake, ok, 4, 64, ok, 4, s) == 2
     # and a missing or short workspace is refused
     assert L.moe_expert_ffn_w8a8(*([ok] * 8), 8, 256, 512, 8, ok, None, None, 0, s) == 3
 

@@ -29,11 +29,12 @@ def test_scatter_rows_bit_exact(dtype, cols):
     src = torch.randn((rows, cols), generator=g).to(dtype)
     perm = torch.randperm(rows + 20, generator=g)[:rows].to(torch.int32)
     perm[::7] = -1                                               # skipped rows
+    perm[1::11] = rows + 20 + 5                                  # targets past dst: skipped too
     dst = torch.full((rows + 20, cols), 7.0).to(dtype)
     got = moe.moe_scatter_rows(src.cuda(), perm.cuda(), dst.cuda())
     torch.cuda.synchronize()
     want = dst.clone()
-    keep = perm >= 0
+    keep = (perm >= 0) & (perm < rows + 20)
     want[perm[keep].long()] = src[keep]
     assert torch.equal(got.cpu().view(torch.int16 if dtype == torch.bfloat16 else torch.int32),
                        want.view(torch.int16 if dtype == torch.bfloat16 else torch.int32))
