@@ -129,3 +129,14 @@ def test_gloo_ranks_exchange_gives_the_one_device_layer(world):
     assert all(r[2] == 24 * 3 for r in res)                    # every rank sends all its N*k rows
     assert sum(r[3] for r in res) == world * 24 * 3            # and all of them arrive somewhere
     assert any(r[4][r[0]] < r[3] for r in res)                 # rows really crossed ranks
+
+
+def test_plan_empty_batches_and_slices():
+    p = ep.exchange_plan(np.zeros((4, 8), np.int64), 2)           # nobody routes anything
+    assert p.send_splits == [0] * 4 and p.recv_splits == [0] * 4
+    assert p.local_offsets.tolist() == [0, 0, 0] and p.recv_to_local.size == 0 and p.local_to_recv.size == 0
+    import torch
+    W = torch.arange(8 * 3).reshape(8, 3)
+    assert ep.local_experts(W, 1, 4).tolist() == W[2:4].tolist()
+    with pytest.raises(ValueError):
+        ep.local_experts(W, 0, 3)                                  # 8 experts over 3 ranks
