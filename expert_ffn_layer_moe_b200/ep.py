@@ -112,8 +112,11 @@ def exchange_ffn(x_perm: torch.Tensor, counts: torch.Tensor, E: int,
     plan = exchange_plan(torch.stack(gathered).cpu().numpy(), rank)
     t1 = time.perf_counter()
     R, H = x_perm.shape
+    sent = sum(plan.send_splits)  # rows with a valid expert: the first `sent` rows of x_perm
+    if sent > R:
+        raise ValueError("counts exceed the permuted rows")
     recv = torch.empty((sum(plan.recv_splits), H), dtype=x_perm.dtype, device=dev)
-    dist.all_to_all_single(_words(recv), _words(x_perm.contiguous()), plan.recv_splits, plan.send_splits,
+    dist.all_to_all_single(_words(recv), _words(x_perm[:sent].contiguous()), plan.recv_splits, plan.send_splits,
                            group=group)
     _sync(dev)
     t2 = time.perf_counter()
@@ -124,12 +127,13 @@ def exchange_ffn(x_perm: torch.Tensor, counts: torch.Tensor, E: int,
     scatter_rows(y_loc, torch.from_numpy(plan.local_to_recv).to(dev), y_recv)
     _sync(dev)
     t3 = time.perf_counter()
+    # rows past `sent` (assignments without a valid expert) stay unwritten; the combine skips them
     y = torch.empty((R, y_loc.shape[1]), dtype=y_loc.dtype, device=dev)
-    dist.all_to_all_single(_words(y), _words(y_recv), plan.send_splits, plan.recv_splits, group=group)
+    dist.all_to_all_single(_words(y[:sent]), _words(y_recv), plan.send_splits, plan.recv_splits, group=group)
     _sync(dev)
     t4 = time.perf_counter()
     if stats is not None:
-        stats.append(EPStats(R, int(sum(plan.recv_splits)),
+        stats.append(EPStats(sent, int(sum(plan.recv_splits)),
                              {"plan": t1 - t0, "dispatch": t2 - t1, "experts": t3 - t2, "combine_exchange": t4 - t3}))
     return y, plan
 

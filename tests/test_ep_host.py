@@ -140,3 +140,31 @@ def test_plan_empty_batches_and_slices():
     assert ep.local_experts(W, 1, 4).tolist() == W[2:4].tolist()
     with pytest.raises(ValueError):
         ep.local_experts(W, 0, 3)                                  # 8 experts over 3 ranks
+
+
+def test_exchange_skips_rows_without_an_expert():
+    """Rows past the counted ones (assignments without a valid expert) are neither sent
+    nor written back: a one-rank gloo group, identity experts."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=30))
+    try:
+        x = torch.arange(5 * 4, dtype=torch.int32).reshape(5, 4)
+        counts = torch.tensor([1, 0, 3], dtype=torch.int32)      # 4 counted rows of 5
+
+        def ffn(x_loc, offsets):
+            assert offsets.tolist() == [0, 1, 1, 4]
+            return x_loc.to(torch.float64) * 2
+
+        def scatter(src, dst_row, dst):
+            dst[dst_row.long()] = src
+            return dst
+
+        y, plan = ep.exchange_ffn(x, counts, 3, ffn, scatter)
+        assert plan.send_splits == [4] and plan.recv_splits == [4]
+        assert torch.equal(y[:4], x[:4].to(torch.float64) * 2)
+    finally:
+        dist.destroy_process_group()
