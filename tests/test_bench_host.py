@@ -77,3 +77,10 @@ def test_clock_sampler_region_samples():
         time.sleep(0.05)
     s = c.summary()
     assert s["samples"] >= 5
+
+
+def test_l2_note_says_which_case_the_timing_is():
+    import torch
+    big = bench.l2_note(4.83e9, 8, torch.device("cpu"))
+    small = bench.l2_note(6e6, 8, torch.device("cpu"))
+    assert big.startswith("inputs larger than L2") and small.startswith("no flush")
