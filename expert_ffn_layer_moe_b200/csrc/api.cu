@@ -20,6 +20,22 @@ std::atomic<uint64_t> g_launches{0};
 }  // namespace
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 uint64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
+
+void *current_context()
+{
+    using GetCurrent = int (*)(void **);
+    static GetCurrent fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<GetCurrent>(p);
+    }();
+    void *ctx = nullptr;
+    if (!fn || fn(&ctx) != 0) return nullptr;
+    return ctx;
+}
 }  // namespace moe
 
 namespace {
@@ -42,18 +58,22 @@ moe_status_t cuda_fail(cudaError_t e)
     } while (0)
 
 // Device address of the error word on the current device (host code must not use
-// the symbol itself as a pointer).
+// the symbol itself as a pointer).  Cached per device and looked up again when the
+// thread's current context is not the one the address was taken in.
 int *device_error_word()
 {
     static std::mutex mu;
     static int *addr[64] = {nullptr};
+    static void *ctx_of[64] = {nullptr};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    void *ctx = moe::current_context();
+    if (!addr[dev] || !ctx || ctx != ctx_of[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_moe_device_error) != cudaSuccess) return nullptr;
         addr[dev] = static_cast<int *>(p);
+        ctx_of[dev] = moe::current_context();  // bound now, if the lookup initialised it
     }
     return addr[dev];
 }
@@ -64,7 +84,8 @@ bool valid_hidden(int v) { return v >= 64 && v <= 65536 && v % 64 == 0; }
 
 bool valid_ek(int E, int k) { return E >= 1 && E <= 256 && k >= 1 && k <= 8 && k <= E; }
 
-bool valid_rows(int64_t N, int k) { return N >= 0 && N * (int64_t)k < (int64_t(1) << 31); }
+// N * k < 2^31, checked without forming a product that could overflow
+bool valid_rows(int64_t N, int k) { return k >= 1 && N >= 0 && N < ((int64_t(1) << 31) + k - 1) / k; }
 
 size_t round_up(size_t v) { return (v + 255) & ~size_t(255); }
 

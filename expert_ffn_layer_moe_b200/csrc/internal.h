@@ -12,6 +12,11 @@ namespace moe {
 void count_launch();
 uint64_t launches_so_far();
 
+// The calling thread's current CUDA context (a driver handle), or nullptr when none
+// is bound.  Caches of per-device addresses are keyed on it: after cudaDeviceReset, or
+// under another context on the same device, a cached address would be stale.
+void *current_context();
+
 // Launch with programmatic stream serialization (the kernel calls pdl_entry/pdl_wait
 // before its first global memory access).
 template <typename... KArgs, typename... Args>

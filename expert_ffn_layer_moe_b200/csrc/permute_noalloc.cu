@@ -17,23 +17,27 @@ namespace {
 static __device__ __align__(256) int32_t g_permute_scratch[MOE_PERMUTE_NOALLOC_MAX_SCRATCH_INTS];
 
 // Device address of g_permute_scratch on the current device, looked up once per
-// device.  In host code the symbol itself is only a host-side stand-in: a kernel
-// handed it would fault, or silently touch the wrong memory where the GPU can
+// device and context (again after a device reset, or under another context on the
+// same device).  In host code the symbol itself is only a host-side stand-in: a
+// kernel handed it would fault, or silently touch the wrong memory where the GPU can
 // reach host memory, so kernels get this address instead.
 cudaError_t scratch_address(int32_t **out)
 {
     static std::mutex mu;
     static int32_t *addr[64] = {nullptr};
+    static void *ctx_of[64] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    void *ctx = moe::current_context();
+    if (!addr[dev] || !ctx || ctx != ctx_of[dev]) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_permute_scratch);
         if (e != cudaSuccess) return e;
         addr[dev] = static_cast<int32_t *>(p);
+        ctx_of[dev] = moe::current_context();  // bound now, if the lookup initialised it
     }
     *out = addr[dev];
     return cudaSuccess;
@@ -46,7 +50,8 @@ extern "C" moe_status_t moe_permute_noalloc(const uint16_t *x, const int32_t *to
                                             int32_t *row_to_token, int32_t *token_to_row, uint16_t *x_perm,
                                             void *stream)
 {
-    if (N < 0 || k < 1 || k > 8 || E < 1 || E > 256 || N * (int64_t)k >= (int64_t(1) << 31))
+    // N * k < 2^31, checked before the product is formed (a huge N would overflow it)
+    if (k < 1 || k > 8 || E < 1 || E > 256 || N < 0 || N >= ((int64_t(1) << 31) + k - 1) / k)
         return MOE_ERR_INVALID_ARG;
     if (moe::permute_scratch_ints(N * k, E) > MOE_PERMUTE_NOALLOC_MAX_SCRATCH_INTS) return MOE_ERR_UNSUPPORTED;
     int32_t *scratch = nullptr;

@@ -149,17 +149,23 @@ def local_experts(W: torch.Tensor, rank: int, G: int) -> torch.Tensor:
 
 def moe_layer_forward_ep(x: torch.Tensor, W_gate: torch.Tensor, W1_local: torch.Tensor, W3_local: torch.Tensor,
                          W2_local: torch.Tensor, k: int, bias: Optional[torch.Tensor] = None, group=None,
-                         stats: Optional[list] = None) -> torch.Tensor:
+                         stats: Optional[list] = None, routing=None) -> torch.Tensor:
     """The MoE layer with the experts split over the ranks of `group` (NCCL, one GPU per
     rank).  x [N,H] bf16 is this rank's batch; W_gate [H,E] fp32 is the whole router;
     W1_local, W3_local [L,I,H] and W2_local [L,H,I] bf16 are this rank's experts
-    (``local_experts``).  Returns this rank's out [N,H] bf16."""
+    (``local_experts``).  routing = (topk_idx [N,k] int32, topk_w [N,k] fp32) replaces
+    the router's choice when given; an index outside [0,E) is skipped (its assignment
+    adds nothing) and reported through the device error word.  Returns this rank's
+    out [N,H] bf16."""
     from expert_ffn_layer_moe_b200 import moe
     G = dist.get_world_size(group)
     E = W_gate.shape[1]
     if W1_local.shape[0] * G != E:
         raise ValueError("local expert slices do not match E / world size")
-    idx, w, _ = moe.moe_route(x, W_gate, k, bias=bias)
+    if routing is not None:
+        idx, w = routing
+    else:
+        idx, w, _ = moe.moe_route(x, W_gate, k, bias=bias)
     p = moe.moe_permute(x, idx, E)
 
     def ffn(x_loc, offsets_loc):

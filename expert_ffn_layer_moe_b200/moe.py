@@ -21,6 +21,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
 DEVERR = {0: "MOE_DEVERR_NONE", 1: "MOE_DEVERR_BAD_EXPERT_INDEX", 2: "MOE_DEVERR_PIPELINE_TIMEOUT",
           3: "MOE_DEVERR_BAD_OFFSETS"}
+MOE_DEVERR_NONE, MOE_DEVERR_BAD_EXPERT_INDEX, MOE_DEVERR_PIPELINE_TIMEOUT, MOE_DEVERR_BAD_OFFSETS = 0, 1, 2, 3
 PHASES = ("route", "permute", "gemm13", "gemm2", "shared", "combine")
 
 
@@ -138,11 +139,12 @@ def moe_permute(x, topk_idx, E, ws=None, stream=None, out=None):
     k = topk_idx.shape[1]
     R = N * k
     o = out or {}
-    counts = o.get("counts", _empty((E,), torch.int32, x))
-    offsets = o.get("offsets", _empty((E + 1,), torch.int32, x))
-    r2t = o.get("row_to_token", _empty((R,), torch.int32, x))
-    t2r = o.get("token_to_row", _empty((N, k), torch.int32, x))
-    x_perm = o.get("x_perm", _empty((R, H), torch.bfloat16, x))
+    # only the outputs the caller did not supply are allocated
+    counts = o["counts"] if "counts" in o else _empty((E,), torch.int32, x)
+    offsets = o["offsets"] if "offsets" in o else _empty((E + 1,), torch.int32, x)
+    r2t = o["row_to_token"] if "row_to_token" in o else _empty((R,), torch.int32, x)
+    t2r = o["token_to_row"] if "token_to_row" in o else _empty((N, k), torch.int32, x)
+    x_perm = o["x_perm"] if "x_perm" in o else _empty((R, H), torch.bfloat16, x)
     if ws is None:
         ws = _empty((max(1, moe_workspace_bytes(N, H, 64, E, k, 0)),), torch.uint8, x)
     _check("moe_permute", lib().moe_permute(_p(x), _p(topk_idx), N, H, E, k, _p(counts), _p(offsets),

@@ -145,7 +145,10 @@ MOE_API moe_status_t moe_permute(const uint16_t *x, const int32_t *topk_idx, int
  *
  * The first call on each device looks up the array's device address on that
  * device (the device must be current); make that first call before any stream
- * capture.  All calls share the one array: two calls whose kernels overlap on
+ * capture.  The address is looked up again whenever the calling thread's
+ * current context differs from the one it was taken in (after a device reset,
+ * or under a non-primary context); such a first call under a new context
+ * should likewise come before any capture.  All calls share the one array: two calls whose kernels overlap on
  * the GPU (different streams, or host threads) race on it and must be ordered
  * by the caller.  The array keeps the previous call's contents; the dispatch
  * writes every entry it later reads, so no clearing is needed.

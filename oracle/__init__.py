@@ -33,18 +33,44 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
-_lib = None
+_LIB_MT = os.path.join(_HERE, "libmoe_oracle_mt.so")
+_libs = {}
+_use_mt = False
+
+
+def _compile(path: str, extra) -> None:
+    if not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+        tmp = path + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared",
+                               "-fno-fast-math", "-ffp-contract=off", *extra,
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, path)
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with plain gcc (no vector intrinsics, no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared",
-                               "-fno-fast-math", "-ffp-contract=off",
-                               "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
+    """Compile the oracle with plain gcc (no vector intrinsics, no fast-math): the
+    serial library, and the same source with -fopenmp, whose loops over independent
+    tokens and rows run on several threads (same arithmetic per row, same bits)."""
+    if force:
+        for p in (_LIB, _LIB_MT):
+            if os.path.exists(p):
+                os.utime(p, (0, 0))
+    _compile(_LIB, [])
+    _compile(_LIB_MT, ["-fopenmp"])
     return _LIB
+
+
+def set_threads(n: int) -> int:
+    """n > 1: later calls run on the OpenMP build with n threads; n <= 1: the serial
+    build.  Returns the thread count now in use."""
+    global _use_mt
+    _use_mt = n > 1
+    return int(lib().oracle_threads(n if n > 1 else 0))
+
+
+def threads() -> int:
+    """Threads the oracle's calls use now."""
+    return int(lib().oracle_threads(0))
 
 
 def _P(t):
@@ -52,62 +78,68 @@ def _P(t):
 
 
 def lib():
-    global _lib
-    if _lib is None:
+    path = _LIB_MT if _use_mt else _LIB
+    if path not in _libs:
         build()
-        L = ctypes.CDLL(_LIB)
-        u16, i32, f32, f64, i64 = (ctypes.c_uint16, ctypes.c_int32, ctypes.c_float,
-                                   ctypes.c_double, ctypes.c_int64)
-        c_int = ctypes.c_int
-        L.oracle_bf16_to_double.argtypes = [u16]
-        L.oracle_bf16_to_double.restype = f64
-        L.oracle_round_to_bf16.argtypes = [f64]
-        L.oracle_round_to_bf16.restype = u16
-        L.oracle_router_logits.argtypes = [_P(u16), _P(f32), _P(f32), i64, c_int, c_int, _P(f64)]
-        L.oracle_router_logits.restype = None
-        L.oracle_topk.argtypes = [_P(f32), i64, c_int, c_int, _P(i32), _P(f64)]
-        L.oracle_topk.restype = c_int
-        L.oracle_dispatch.argtypes = [_P(i32), i64, c_int, c_int, _P(i32), _P(i32), _P(i32), _P(i32)]
-        L.oracle_dispatch.restype = c_int
-        L.oracle_permute_rows.argtypes = [_P(u16), _P(i32), i64, c_int, _P(u16)]
-        L.oracle_permute_rows.restype = None
-        L.oracle_swiglu_ffn.argtypes = [_P(u16), _P(u16), _P(u16), _P(u16), c_int, c_int, _P(f64)]
-        L.oracle_swiglu_ffn.restype = None
-        L.oracle_expert_ffn.argtypes = [_P(u16), _P(i32), _P(u16), _P(u16), _P(u16), c_int, c_int,
-                                        c_int, _P(f64)]
-        L.oracle_expert_ffn.restype = None
-        L.oracle_combine.argtypes = [_P(f64), _P(i32), _P(f64), _P(f64), i64, c_int, c_int, _P(u16)]
-        L.oracle_combine.restype = None
-        L.oracle_layer_given_logits.argtypes = (
-            [_P(u16), _P(f32), _P(u16), _P(u16), _P(u16), _P(u16), _P(u16), _P(u16), i64] +
-            [c_int] * 5 + [_P(u16), _P(i32), _P(f64), _P(i32), _P(i32), _P(i32), _P(i32), _P(f64)])
-        L.oracle_layer_given_logits.restype = c_int
-        L.oracle_layer.argtypes = ([_P(u16), _P(f32), _P(f32), _P(u16), _P(u16), _P(u16), _P(u16),
-                                    _P(u16), _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f32)])
-        L.oracle_layer.restype = c_int
-        u8 = ctypes.c_uint8
-        L.oracle_fp8_e4m3_to_double.argtypes = [u8]
-        L.oracle_fp8_e4m3_to_double.restype = f64
-        L.oracle_fp8_e4m3_from_float.argtypes = [f32]
-        L.oracle_fp8_e4m3_from_float.restype = u8
-        L.oracle_quantize_rows_fp8.argtypes = [_P(u16), i64, c_int, _P(u8), _P(f32)]
-        L.oracle_quantize_rows_fp8.restype = None
-        L.oracle_expert_ffn_fp8.argtypes = [_P(u16), _P(i32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8),
-                                            _P(f32), c_int, c_int, c_int, _P(f64)]
-        L.oracle_expert_ffn_fp8.restype = None
-        L.oracle_layer_given_logits_fp8.argtypes = (
-            [_P(u16), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u16), _P(u16),
-             _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f64)])
-        L.oracle_layer_given_logits_fp8.restype = c_int
-        L.oracle_expert_ffn_fp8_ex.argtypes = [_P(u16), _P(i32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8),
-                                               _P(f32), c_int, c_int, c_int, c_int, _P(u16), _P(f64), _P(u16)]
-        L.oracle_expert_ffn_fp8_ex.restype = None
-        L.oracle_layer_given_logits_fp8_ex.argtypes = (
-            [_P(u16), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u16), _P(u16),
-             _P(u16), i64] + [c_int] * 6 + [_P(u16), _P(u16), _P(f64)])
-        L.oracle_layer_given_logits_fp8_ex.restype = c_int
-        _lib = L
-    return _lib
+        _libs[path] = _load(path)
+    return _libs[path]
+
+
+def _load(path):
+    L = ctypes.CDLL(path)
+    u16, i32, f32, f64, i64 = (ctypes.c_uint16, ctypes.c_int32, ctypes.c_float,
+                               ctypes.c_double, ctypes.c_int64)
+    c_int = ctypes.c_int
+    L.oracle_bf16_to_double.argtypes = [u16]
+    L.oracle_bf16_to_double.restype = f64
+    L.oracle_round_to_bf16.argtypes = [f64]
+    L.oracle_round_to_bf16.restype = u16
+    L.oracle_router_logits.argtypes = [_P(u16), _P(f32), _P(f32), i64, c_int, c_int, _P(f64)]
+    L.oracle_router_logits.restype = None
+    L.oracle_topk.argtypes = [_P(f32), i64, c_int, c_int, _P(i32), _P(f64)]
+    L.oracle_topk.restype = c_int
+    L.oracle_dispatch.argtypes = [_P(i32), i64, c_int, c_int, _P(i32), _P(i32), _P(i32), _P(i32)]
+    L.oracle_dispatch.restype = c_int
+    L.oracle_permute_rows.argtypes = [_P(u16), _P(i32), i64, c_int, _P(u16)]
+    L.oracle_permute_rows.restype = None
+    L.oracle_swiglu_ffn.argtypes = [_P(u16), _P(u16), _P(u16), _P(u16), c_int, c_int, _P(f64)]
+    L.oracle_swiglu_ffn.restype = None
+    L.oracle_expert_ffn.argtypes = [_P(u16), _P(i32), _P(u16), _P(u16), _P(u16), c_int, c_int,
+                                    c_int, _P(f64)]
+    L.oracle_expert_ffn.restype = None
+    L.oracle_combine.argtypes = [_P(f64), _P(i32), _P(f64), _P(f64), i64, c_int, c_int, _P(u16)]
+    L.oracle_combine.restype = None
+    L.oracle_layer_given_logits.argtypes = (
+        [_P(u16), _P(f32), _P(u16), _P(u16), _P(u16), _P(u16), _P(u16), _P(u16), i64] +
+        [c_int] * 5 + [_P(u16), _P(i32), _P(f64), _P(i32), _P(i32), _P(i32), _P(i32), _P(f64)])
+    L.oracle_layer_given_logits.restype = c_int
+    L.oracle_layer.argtypes = ([_P(u16), _P(f32), _P(f32), _P(u16), _P(u16), _P(u16), _P(u16),
+                                _P(u16), _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f32)])
+    L.oracle_layer.restype = c_int
+    u8 = ctypes.c_uint8
+    L.oracle_fp8_e4m3_to_double.argtypes = [u8]
+    L.oracle_fp8_e4m3_to_double.restype = f64
+    L.oracle_fp8_e4m3_from_float.argtypes = [f32]
+    L.oracle_fp8_e4m3_from_float.restype = u8
+    L.oracle_quantize_rows_fp8.argtypes = [_P(u16), i64, c_int, _P(u8), _P(f32)]
+    L.oracle_quantize_rows_fp8.restype = None
+    L.oracle_expert_ffn_fp8.argtypes = [_P(u16), _P(i32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8),
+                                        _P(f32), c_int, c_int, c_int, _P(f64)]
+    L.oracle_expert_ffn_fp8.restype = None
+    L.oracle_layer_given_logits_fp8.argtypes = (
+        [_P(u16), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u16), _P(u16),
+         _P(u16), i64] + [c_int] * 5 + [_P(u16), _P(f64)])
+    L.oracle_layer_given_logits_fp8.restype = c_int
+    L.oracle_expert_ffn_fp8_ex.argtypes = [_P(u16), _P(i32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8),
+                                           _P(f32), c_int, c_int, c_int, c_int, _P(u16), _P(f64), _P(u16)]
+    L.oracle_expert_ffn_fp8_ex.restype = None
+    L.oracle_layer_given_logits_fp8_ex.argtypes = (
+        [_P(u16), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u8), _P(f32), _P(u16), _P(u16),
+         _P(u16), i64] + [c_int] * 6 + [_P(u16), _P(u16), _P(f64)])
+    L.oracle_layer_given_logits_fp8_ex.restype = c_int
+    L.oracle_threads.argtypes = [c_int]
+    L.oracle_threads.restype = c_int
+    return L
 
 
 def _ptr(a, ctype):

@@ -67,6 +67,26 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* The same file builds two libraries: a serial one, and (with -fopenmp) one whose
+ * loops over independent tokens or rows run on several host threads.  A row's or a
+ * token's arithmetic is the same in both -- the same operations in the same order on
+ * one thread -- so the two give identical bits; only which thread computes a row
+ * differs.  oracle_threads(n) sets the thread count (n > 0) and returns the count in
+ * use, 1 for the serial build. */
+int oracle_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 /* ---------------------------------------------------------------- bf16 ---- */
 
@@ -170,6 +190,7 @@ void oracle_quantize_rows_fp8(const uint16_t *W, int64_t rows, int K, uint8_t *q
 void oracle_router_logits(const uint16_t *x, const float *W_gate, const float *bias,
                           int64_t N, int H, int E, double *logits)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < N; ++t)
         for (int e = 0; e < E; ++e) {
             double s = 0.0;
@@ -344,11 +365,24 @@ static void expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const ora
                        const oracle_wmat *W3, const oracle_wmat *W2, int E, int H, int I, int qa,
                        const uint16_t *h_given, uint16_t *h_out, double *y_perm)
 {
+    /* every row is independent: row r goes through the expert whose group holds it */
+    const int64_t R = offsets[E] > 0 ? offsets[E] : 0;
+    int32_t *expert_of = (int32_t *)malloc((size_t)(R > 0 ? R : 1) * sizeof(int32_t));
+    if (!expert_of) return;
+    for (int64_t r = 0; r < R; ++r) expert_of[r] = -1; /* rows before offsets[0]: no expert */
     for (int e = 0; e < E; ++e)
         for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r)
-            swiglu_row(x_perm + r * H, W1, W3, W2, (int64_t)e * I, (int64_t)e * H, H, I, qa,
-                       h_given ? h_given + r * I : NULL, h_out ? h_out + r * I : NULL,
-                       y_perm + r * H);
+            if (r >= 0 && r < R) expert_of[r] = e;
+    (void)fp8_val(0); /* fill the e4m3 table before the rows run side by side */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        const int e = expert_of[r];
+        if (e < 0) continue;
+        swiglu_row(x_perm + r * H, W1, W3, W2, (int64_t)e * I, (int64_t)e * H, H, I, qa,
+                   h_given ? h_given + r * I : NULL, h_out ? h_out + r * I : NULL,
+                   y_perm + r * H);
+    }
+    free(expert_of);
 }
 
 void oracle_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W1,
@@ -393,6 +427,7 @@ void oracle_expert_ffn_fp8_ex(const uint16_t *x_perm, const int32_t *offsets, co
 void oracle_combine(const double *y_perm, const int32_t *token_to_row, const double *w,
                     const double *s, int64_t N, int H, int k, uint16_t *out)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < N; ++t)
         for (int o = 0; o < H; ++o) {
             double acc = 0.0;
@@ -446,6 +481,7 @@ static int layer_core(const uint16_t *x, const float *logits, const oracle_wmat 
     if (Is > 0) {
         s = (double *)malloc((size_t)(N ? N : 1) * H * sizeof(double));
         if (!s) goto done;
+#pragma omp parallel for schedule(dynamic, 1)
         for (int64_t t = 0; t < N; ++t) oracle_swiglu_ffn(x + t * H, Ws1, Ws3, Ws2, H, Is, s + t * H);
     }
     oracle_combine(yp, t2r, w, s, N, H, k, out);

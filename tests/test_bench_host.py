@@ -79,8 +79,20 @@ def test_clock_sampler_region_samples():
     assert s["samples"] >= 5
 
 
-def test_l2_note_says_which_case_the_timing_is():
-    import torch
-    big = bench.l2_note(4.83e9, 8, torch.device("cpu"))
-    small = bench.l2_note(6e6, 8, torch.device("cpu"))
-    assert big.startswith("inputs larger than L2") and small.startswith("no flush")
+def test_weight_rotation_covers_twice_l2():
+    l2 = 126 << 20
+    assert bench.rotation_copies(4.83e9, l2) == 1                # streamed from HBM anyway
+    for wb in (6e6, 77e6, 200e6):                                # tiny, Qwen3-30B N=1, just under 2 x L2
+        c = bench.rotation_copies(wb, l2)
+        assert c >= 2 and c * wb >= 2 * l2 and (c - 1) * wb < 2 * l2
+    big = bench.l2_note(4.83e9, 8, l2, 1)
+    small = bench.l2_note(6e6, 8, l2, bench.rotation_copies(6e6, l2))
+    assert big.startswith("inputs larger than L2") and small.startswith("weight rotation")
+
+
+def test_oracle_sample_size():
+    cfg = CONFIGS["qwen3_235b_a22b_skew"]
+    assert bench.sample_size(cfg, 1e6, 15.0, 8) == cfg.N          # the whole batch fits
+    n = bench.sample_size(cfg, 100.0, 15.0, 8)
+    assert n == 1496 and n % 8 == 0                               # whole rounds of the threads
+    assert bench.sample_size(cfg, 0.1, 15.0, 8) == 1

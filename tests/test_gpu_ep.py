@@ -72,3 +72,42 @@ def test_ep_layer_one_rank_matches_oracle(cfg):
         assert_close(dec(host(out)), dec(ref), f"{cfg.name} ep out")
     finally:
         dist.destroy_process_group()
+
+
+def test_ep_layer_skips_an_out_of_range_expert_index():
+    """A caller-supplied choice with an index outside [0, E): that assignment has no
+    row, its slot of the returned y is never written, and the combine must skip it.
+    The output must equal the oracle over the valid picks (the bad pick given weight 0
+    on a valid expert, which adds exactly nothing) and the error word must say
+    MOE_DEVERR_BAD_EXPERT_INDEX."""
+    cfg = MoEConfig("ep1_bad", N=96, H=256, I=128, E=8, k=2)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_port()}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        t = cuda_inputs(cfg, seed=9)
+        idx, w, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k)
+        bad_tokens = [3, 40, 95]
+        idx_bad = idx.clone()
+        for tok in bad_tokens:
+            idx_bad[tok, 1] = cfg.E + 5 if tok != 40 else -2
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error() == 0
+        out = ep.moe_layer_forward_ep(t["x"], t["W_gate"], ep.local_experts(t["W1"], 0, 1),
+                                      ep.local_experts(t["W3"], 0, 1), ep.local_experts(t["W2"], 0, 1), cfg.k,
+                                      routing=(idx_bad, w))
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error() == moe.MOE_DEVERR_BAD_EXPERT_INDEX
+
+        # oracle: the bad pick moved to a valid expert with weight 0
+        idx_ref = host(idx_bad).copy()
+        w_ref = host(w).astype(np.float64)
+        for tok in bad_tokens:
+            idx_ref[tok, 1] = 0 if idx_ref[tok, 0] != 0 else 1
+            w_ref[tok, 1] = 0.0
+        counts, offsets, r2t, t2r = oracle.dispatch(idx_ref, cfg.E)
+        x_perm = oracle.permute_rows(host(t["x"]), r2t)
+        y = oracle.expert_ffn(x_perm, offsets, host(t["W1"]), host(t["W3"]), host(t["W2"]))
+        ref = oracle.combine(y, t2r, w_ref)
+        assert_close(dec(host(out)), dec(ref), "ep out with skipped picks")
+    finally:
+        dist.destroy_process_group()

@@ -536,3 +536,38 @@ def test_fp8_acts_layer_error_against_bf16_is_quantization_sized():
     rel = np.linalg.norm(got - want) / np.linalg.norm(want)
     rel_w8 = np.linalg.norm(w8 - want) / np.linalg.norm(want)
     assert rel_w8 < rel < 8e-2, (rel, rel_w8)
+
+
+def test_threaded_build_gives_the_serial_builds_bits():
+    """The OpenMP build spreads independent tokens and rows over threads; each row's
+    arithmetic is unchanged, so every output (logits, picks, weights, maps, fp64 expert
+    rows, out, with shared experts and fp8 activations too) must be bit-identical to
+    the serial build's."""
+    cfg = MoEConfig("mt", N=37, H=128, I=192, E=16, k=4, Is=128)
+    t = make_inputs(cfg, seed=3)
+    x, Wg = to_u16(t["x"]), t["W_gate"].numpy()
+    W1, W3, W2 = to_u16(t["W1"]), to_u16(t["W3"]), to_u16(t["W2"])
+    Ws = [to_u16(t[n]) for n in ("Ws1", "Ws3", "Ws2")]
+
+    def run():
+        l64 = oracle.router_logits(x, Wg)
+        out, l32 = oracle.layer(x, Wg, W1, W3, W2, cfg.k, Ws1=Ws[0], Ws3=Ws[1], Ws2=Ws[2])
+        ex = oracle.layer_given_logits(x, l32, W1, W3, W2, cfg.k, Ws1=Ws[0], Ws3=Ws[1], Ws2=Ws[2], extras=True)
+        q = [oracle.quantize_rows_fp8(W.reshape(-1, W.shape[-1])) for W in (W1, W3, W2)]
+        qq = [(c.reshape(W.shape), s_.reshape(W.shape[:-1])) for (c, s_), W in zip(q, (W1, W3, W2))]
+        a8 = oracle.expert_ffn_fp8_ex(oracle.permute_rows(x, ex["row_to_token"]), ex["offsets"], *qq[0], *qq[1],
+                                      *qq[2], quantize_acts=1)
+        return [l64, out, l32] + [ex[n] for n in sorted(ex)] + list(a8 if isinstance(a8, tuple) else (a8,))
+
+    try:
+        assert oracle.set_threads(1) == 1
+        serial = run()
+        assert oracle.set_threads(4) == 4
+        threaded = run()
+    finally:
+        oracle.set_threads(1)
+    assert len(serial) == len(threaded)
+    for a, b in zip(serial, threaded):
+        a, b = np.asarray(a), np.asarray(b)
+        assert a.dtype == b.dtype and a.shape == b.shape
+        assert a.tobytes() == b.tobytes()

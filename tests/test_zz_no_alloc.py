@@ -4,8 +4,8 @@ Some callers cannot call cudaMalloc or hand the library a workspace (a serving
 process whose memory pool already owns the device, a plugin inside a framework
 that owns every allocation, code with a hard latency budget).  This entry point
 runs the same dispatch with its scratch in a fixed array inside the library.
-The test calls it through the C ABI twice in a row, on different inputs, and
-checks every output against moe_permute with a caller workspace: all outputs
+The test calls it through the C ABI three times in a row, on inputs of different
+shapes, and checks every output against moe_permute with a caller workspace: all outputs
 are integers or copied bits, so the tolerance is exact equality.  It lives in
 its own file, collected last, and passes alone or after the other tests.
 """
@@ -47,9 +47,18 @@ def _noalloc_via_c_abi(x, idx, E):
     return out
 
 
-@pytest.mark.parametrize("first,second", [((3000, 256, 128, 8), (500, 128, 16, 2))])
-def test_noalloc_permute_matches_workspace_permute_twice(first, second):
-    for seed, (N, H, E, k) in enumerate((first, second)):
+# Every case has more than 2048 assignments, so each call takes the count/scan/rank
+# dispatch whose per-block histograms live in the fixed array (smaller batches run a
+# one-block dispatch that never touches it).  The cases change E and the block count
+# from call to call, so each call starts on an array that still holds the previous
+# call's histograms laid out differently: 24 blocks x 128 experts, then 3 x 16, then
+# 11 x 200.
+CALLS = ((3000, 256, 128, 8), (1500, 128, 16, 2), (2600, 64, 200, 4))
+
+
+def test_noalloc_permute_matches_workspace_permute_on_consecutive_calls():
+    for seed, (N, H, E, k) in enumerate(CALLS):
+        assert N * k > 2048
         x, idx = _inputs(N, H, E, k, seed)
         got = _noalloc_via_c_abi(x, idx, E)
         want = moe.moe_permute(x, idx, E)
