@@ -589,6 +589,9 @@ def other_workloads(args, headline, dev, stream, rank, world, pk):
 
 
 def run_ours(args, cfg, world, rank, local):
+    from expert_ffn_layer_moe_b200 import moe
+    moe.moe_set_gather_mode({"auto": moe.MOE_GATHER_AUTO, "on": moe.MOE_GATHER_ON,
+                             "off": moe.MOE_GATHER_OFF}[args.gather])
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     W = Workload(cfg, args, dev, stream, rank, world)
@@ -707,7 +710,8 @@ def run_ours(args, cfg, world, rank, local):
                                        "timing; " + ("multiplied as e4m3" if a8 else "widened to bf16 on chip")
                                        + ")") if fp8 else "bf16"),
                    "expert_activations": ("e4m3, one fp32 scale per row (x_perm and h quantized on the device "
-                                          "every step)") if a8 else "bf16"},
+                                          "every step)") if a8 else "bf16",
+                   "w13_rows": f"gather mode {args.gather}"},
         "roofline": roofline,
         "layer": layer,
         "grouped_gemm": gg,
@@ -780,6 +784,8 @@ def main():
                     help="routed-expert weight format (fp8: e4m3 with per-channel scales, a separate experiment)")
     ap.add_argument("--acts", choices=["bf16", "fp8"], default="bf16",
                     help="routed-expert activation format (fp8: e4m3 with per-row scales; needs --weights fp8)")
+    ap.add_argument("--gather", choices=["auto", "on", "off"], default="auto",
+                    help="W1/W3 token rows: gathered from x (on), the permuted copy (off), or by shape (auto)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

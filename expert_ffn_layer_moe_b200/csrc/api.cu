@@ -17,9 +17,20 @@
 namespace moe {
 namespace {
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_gather_mode{MOE_GATHER_AUTO};
 }  // namespace
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 uint64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
+
+// Whether the bf16 layer gathers its W1/W3 token rows from x (no permuted copy).
+bool layer_gathers(int64_t N, int k, int H)
+{
+    const int mode = g_gather_mode.load(std::memory_order_relaxed);
+    if (mode == MOE_GATHER_ON) return true;
+    if (mode == MOE_GATHER_OFF) return false;
+    (void)N; (void)k; (void)H;
+    return true;
+}
 
 void *current_context()
 {
@@ -265,6 +276,10 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
         MOE_CUDA(moe::launch_scatter_rows(reinterpret_cast<const uint16_t *>(Q.xqt), Q.xst, t2r, N, k, H / 2,
                                           reinterpret_cast<uint16_t *>(Q.xq), R, Q.xsc, s));
         a.act = Q.xq; a.a8 = true; a.scale_act = Q.xsc;
+    } else if (!X.fp8 && moe::layer_gathers(N, k, H)) {
+        // dispatch only: W1/W3 gathers its rows from x through row_to_token
+        MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
+        a.act = x; a.gather_rows = r2t; a.gather_src_rows = N;
     } else {
         MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, x_perm, perm, err, s));
         a.act = x_perm;
@@ -310,6 +325,12 @@ const char *moe_last_cuda_error(void) { return g_last_cuda_error; }
 int moe_device_sm_count(void) { return moe::device_sm_count(); }
 
 uint64_t moe_kernel_launches(void) { return moe::launches_so_far(); }
+
+int moe_set_gather_mode(int mode)
+{
+    if (mode != MOE_GATHER_AUTO && mode != MOE_GATHER_OFF && mode != MOE_GATHER_ON) return -1;
+    return moe::g_gather_mode.exchange(mode);
+}
 
 size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is)
 {

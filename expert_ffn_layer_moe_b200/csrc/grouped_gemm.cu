@@ -356,6 +356,27 @@ __device__ __forceinline__ void tma_3d(void *dst, const CUtensorMap *m, int c0, 
             : "memory");
 }
 
+// Four rows (r0..r3) of a 2-D map whose box is one row high, K columns [c0, c0 + 64),
+// written as four consecutive 128-byte rows at dst with the map's swizzle: the
+// activation rows of a token tile gathered straight from x.  Never multicast.
+template <bool PAIR>
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *m, int c0, int r0, int r1, int r2, int r3,
+                                            uint32_t bar)
+{
+    if (PAIR)
+        asm volatile(
+            "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+            : "memory");
+    else
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+            : "memory");
+}
+
 template <bool PAIR>
 __device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *m, int c0, int c1, uint32_t bar)
 {
@@ -469,16 +490,24 @@ __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;
 // [n/2 r, n/2 r + n/2) of its n; the leader (r = 0) issues the M=256 MMAs, both CTAs'
 // TMA loads complete on the leader's stage barrier, its commits reach both CTAs'
 // barriers, and each CTA drains its own half of the accumulator.
-template <int BN, bool SWIGLU, bool PAIR, bool W8, bool A8>
+//
+// GATHER = true (bf16 SwiGLU GEMM only): the activation operand is not a permuted copy
+// but x itself; row r of the groups reads x row gather_rows[r] (row_to_token), loaded
+// by tile::gather4 TMA requests -- four rows each, issued by all 32 lanes of warp 0 --
+// so the dispatch never writes x_perm.
+template <int BN, bool SWIGLU, bool PAIR, bool W8, bool A8, bool GATHER>
 __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
                         const __grid_constant__ CUtensorMap tm_act, const int32_t *__restrict__ offsets,
                         int groups, int rows_single, int64_t R, int K, int Nout,
                         void *__restrict__ out, int ksplit, int64_t split_stride,
                         const float *__restrict__ scale_a, const float *__restrict__ scale_b,
-                        const float *__restrict__ scale_act, int64_t ldo, int *dev_err)
+                        const float *__restrict__ scale_act, int64_t ldo, const int32_t *__restrict__ gather_rows,
+                        int *dev_err)
 {
     using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
+    static_assert(!GATHER || (SWIGLU && !W8 && !A8), "gathered activation rows: bf16 SwiGLU GEMM only");
+    static_assert(!GATHER || C::kBRows % 4 == 0, "gather4 loads rows in fours");
     constexpr int kThreads = C::kThreads;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -604,11 +633,14 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
     auto mma_width = [&](int row0, int row_end) { return min(BN, (min(BN, row_end - row0) + 15) & ~15); };
 
     bool failed = false;
-    if (warp == 0 && lane == 0) {
+    if (warp == 0 && (GATHER || lane == 0)) {
         // ------------------------------------------------------ TMA producer
-        tma_prefetch_map(&tm_wa);
-        if (SWIGLU) tma_prefetch_map(&tm_wb);
-        tma_prefetch_map(&tm_act);
+        // (lane 0; with GATHER the whole warp, each lane gathering four activation rows)
+        if (lane == 0) {
+            tma_prefetch_map(&tm_wa);
+            if (SWIGLU) tma_prefetch_map(&tm_wb);
+            tma_prefetch_map(&tm_act);
+        }
         // every load of the pair completes on the leader's stage barrier
         const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&full_bar[0]), 0) : smem_u32(&full_bar[0]);
         int stage = 0;
@@ -639,20 +671,38 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
             kslice(ks, kb0, kb1);
             const int frow = feat * C::kFeatTile + (int)rank * C::kFeat;        // first weight row (W1 / W)
             const int trow = row0 + (PAIR ? (int)rank * (mma_width(row0, row_end) >> 1) : 0);
+            // GATHER: the x rows of this lane's four tile rows, fixed for the whole item.
+            // Tile rows past R (a ragged last tile) read x row 0; like rows of the next
+            // group, their products are never stored.
+            const bool gl = GATHER && 4 * lane < C::kBRows;
+            int xr[4] = {0, 0, 0, 0};
+            if (gl) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t r = (int64_t)trow + 4 * lane + i;
+                    xr[i] = r < R ? gather_rows[r] : 0;
+                }
+            }
             for (int kb = kb0; kb < kb1; ++kb) {
-                if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { failed = true; *abort_flag = 1; break; }
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
+                if (GATHER) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) { failed = true; if (lane == 0) *abort_flag = 1; break; }
                 uint8_t *st = stages + stage * C::kStageBytes;
                 const uint32_t fb = full0 + 8u * stage;
-                if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kCtas * C::kStageBytes);
                 const int kc = kb * C::kKStep;  // K coordinate (elements; bytes for e4m3)
-                if (SWIGLU) {
-                    // rows 0-63: W1 features [frow, +64); rows 64-127: the same features of W3
-                    tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
-                    tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kc, frow, g, fb);
-                } else {
-                    tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
+                if (lane == 0) {
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kCtas * C::kStageBytes);
+                    if (SWIGLU) {
+                        // rows 0-63: W1 features [frow, +64); rows 64-127: the same features of W3
+                        tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
+                        tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kc, frow, g, fb);
+                    } else {
+                        tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
+                    }
+                    if (!GATHER) tma_2d<PAIR>(st + C::kABytes, &tm_act, kc, trow, fb);
                 }
-                tma_2d<PAIR>(st + C::kABytes, &tm_act, kc, trow, fb);
+                if (gl) tma_gather4<PAIR>(st + C::kABytes + lane * 512, &tm_act, kc, xr[0], xr[1], xr[2], xr[3], fb);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
         }
@@ -976,6 +1026,21 @@ bool encode_act_map(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_r
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// x [rows, K] bf16 as a 2-D map whose box is one row high (64 K values): the source of
+// tile::gather4 loads of activation rows in any order.
+bool encode_gather_map(CUtensorMap *m, const void *ptr, int64_t rows, int K)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, 1};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Activations [R, K] e4m3 bytes as a 2-D byte map; box = 128 (K) x box_rows; rows >= R
 // and K values past K read as zero.
 bool encode_act_map_fp8(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_rows)
@@ -991,7 +1056,7 @@ bool encode_act_map_fp8(CUtensorMap *m, const void *ptr, int64_t R, int K, int b
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU, bool PAIR, bool W8, bool A8>
+template <int BN, bool SWIGLU, bool PAIR, bool W8, bool A8, bool GATHER = false>
 cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
     using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
@@ -1004,11 +1069,16 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     } else {
         mb = ma;
     }
-    auto enc_act = A8 ? encode_act_map_fp8 : encode_act_map;
-    if (!enc_act(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
+    if (GATHER) {
+        if (!a.gather_rows || a.gather_src_rows < 1 || !encode_gather_map(&mact, a.act, a.gather_src_rows, a.K))
+            return cudaErrorInvalidValue;
+    } else {
+        auto enc_act = A8 ? encode_act_map_fp8 : encode_act_map;
+        if (!enc_act(&mact, a.act, a.R, a.K, C::kBRows)) return cudaErrorInvalidValue;
+    }
     const int64_t ldo = a.ldo > 0 ? a.ldo : a.Nout;
     if (ldo < a.Nout) return cudaErrorInvalidValue;
-    auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR, W8, A8>;
+    auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR, W8, A8, GATHER>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
     const int ksplit = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
@@ -1028,7 +1098,8 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = PAIR ? 2 : 1;
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
-                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, ldo, a.dev_err);
+                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, ldo, a.gather_rows,
+                             a.dev_err);
     if (err != cudaSuccess) return err;
     count_launch();
     return cudaGetLastError();
@@ -1083,6 +1154,27 @@ cudaError_t launch_dispatch(const GroupedGemmArgs &a, cudaStream_t s)
                 }
             }
         }
+        if constexpr (SWIGLU && !A8) {
+            // activation rows gathered from x through the row map (no permuted copy)
+            if (a.gather_rows) {
+                if (bn <= 64 && gemm_pair_tiles(a.R, a.groups, a.Nout, SWIGLU, a.ksplit) < device_sm_count() / 2) {
+                    switch (bn) {
+                        case 32: return launch_impl<32, true, false, false, false, true>(a, s);
+                        case 64: return launch_impl<64, true, false, false, false, true>(a, s);
+                    }
+                }
+                switch (bn) {
+                    case 32: return launch_impl<32, true, true, false, false, true>(a, s);
+                    case 64: return launch_impl<64, true, true, false, false, true>(a, s);
+                    case 96: return launch_impl<96, true, true, false, false, true>(a, s);
+                    case 128: return launch_impl<128, true, true, false, false, true>(a, s);
+                    case 192: return launch_impl<192, true, true, false, false, true>(a, s);
+                    case 256: return launch_impl<256, true, true, false, false, true>(a, s);
+                    default: return cudaErrorInvalidValue;
+                }
+            }
+        }
+        if (a.gather_rows) return cudaErrorInvalidValue;  // gathering is a bf16 SwiGLU option only
         if (bn <= 64 && gemm_pair_tiles(a.R, a.groups, a.Nout, SWIGLU, a.ksplit) < device_sm_count() / 2) {
             switch (bn) {
                 case 32: return launch_impl<32, SWIGLU, false, false, A8>(a, s);

@@ -17,6 +17,9 @@ uint64_t launches_so_far();
 // under another context on the same device, a cached address would be stale.
 void *current_context();
 
+// Whether the bf16 layer gathers its W1/W3 token rows from x (moe_set_gather_mode).
+bool layer_gathers(int64_t N, int k, int H);
+
 // Launch with programmatic stream serialization (the kernel calls pdl_entry/pdl_wait
 // before its first global memory access).
 template <typename... KArgs, typename... Args>
@@ -87,6 +90,9 @@ struct GroupedGemmArgs {
     int64_t split_stride;    // elements between the partial-sum buffers
     int64_t ldo;             // plain GEMM: elements between output rows (0 = Nout)
     bool single_cta;         // plain bf16 GEMM: single-CTA tiles (token_tile 32, 64 or 128)
+    const int32_t *gather_rows;  // bf16 SwiGLU GEMM: nullptr, or act is x [gather_src_rows, K] and row r
+                                 // of the groups reads x row gather_rows[r] (no permuted copy)
+    int64_t gather_src_rows;
 };
 cudaError_t launch_gemm13_swiglu(const GroupedGemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s);

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_bytes_w8a8.restype = sz
         L.moe_layer_forward_w8a8_ex.argtypes = ([vp] * 12 + [i64] + [c_int] * 5 + [vp, vp, vp, sz, vp, vp])
         L.moe_scatter_rows.argtypes = [vp, vp, i64, c_int, vp, i64, vp]
+        L.moe_set_gather_mode.argtypes = [c_int]
+        L.moe_set_gather_mode.restype = c_int
         for fn in ("moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
                    "moe_layer_forward_ex", "moe_get_device_error", "moe_quantize_fp8", "moe_expert_ffn_fp8",
                    "moe_layer_forward_fp8_ex", "moe_expert_ffn_w8a8", "moe_layer_forward_w8a8_ex",
@@ -108,6 +110,19 @@ def moe_workspace_bytes(N: int, H: int, I: int, E: int, k: int, Is: int = 0) -> 
 
 def moe_device_sm_count() -> int:
     return int(lib().moe_device_sm_count())
+
+
+MOE_GATHER_AUTO, MOE_GATHER_OFF, MOE_GATHER_ON = 0, 1, 2
+
+
+def moe_set_gather_mode(mode: int) -> int:
+    """How the bf16 layer feeds W1/W3 its token rows: MOE_GATHER_AUTO (by shape),
+    MOE_GATHER_OFF (permuted copy x_perm), MOE_GATHER_ON (gathered from x).  Returns
+    the previous mode."""
+    prev = int(lib().moe_set_gather_mode(int(mode)))
+    if prev < 0:
+        raise ValueError(f"gather mode {mode} is not one of MOE_GATHER_AUTO/OFF/ON")
+    return prev
 
 
 def moe_kernel_launches() -> int:

@@ -331,6 +331,24 @@ MOE_API moe_status_t moe_get_device_error(void *stream, int32_t *code);
 MOE_API int moe_device_sm_count(void);
 
 /*
+ * How the bf16 layer calls (moe_layer_forward, moe_layer_forward_ex) feed the
+ * W1/W3 GEMM its token rows.  The pages' dispatch copies every assignment's row
+ * into expert order ([MoE-latency] "router 之后还有一串动作": the permutation, and
+ * the cost of moving token rows it names); with gathering on, the dispatch only
+ * builds the row maps and the GEMM loads each row straight from x through
+ * row_to_token (tile::gather4 TMA), so the permuted copy x_perm is never written.
+ * The results are identical either way.
+ *   mode  MOE_GATHER_AUTO (the default: the library chooses by shape),
+ *         MOE_GATHER_OFF (always the permuted copy), MOE_GATHER_ON (always gather).
+ * Process-wide; takes effect for calls enqueued after it returns.  Returns the
+ * previous mode, or -1 for a mode outside these three.
+ */
+#define MOE_GATHER_AUTO 0
+#define MOE_GATHER_OFF 1
+#define MOE_GATHER_ON 2
+MOE_API int moe_set_gather_mode(int mode);
+
+/*
  * Kernels this library has launched in this process so far, counted on the host
  * at each successful launch (all threads, all devices; never reset).  The
  * difference across a region is the number of the library's kernels it ran.

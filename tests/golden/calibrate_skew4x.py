@@ -13,7 +13,7 @@ Only the oracle computes the routing here (fp64 logits rounded to fp32, then its
 top-k); the CUDA library is not imported.  Needs a CUDA device for the seeded
 inputs (the CUDA generator's stream differs from the CPU one).
 
-    python tests/golden/calibrate_skew4x.py
+    python tests/golden/calibrate_skew4x.py [output path]
 """
 import os
 import sys
@@ -68,7 +68,8 @@ def main():
     rec = float(f"{scale:.4f}")
     r, touched = load_ratio(l64, cfg.E, cfg.k, rec)
     assert LO <= r <= HI, (rec, r)
-    with open(OUT, "w") as f:
+    out = sys.argv[1] if len(sys.argv) > 1 else OUT
+    with open(out, "w") as f:
         f.write("# Router-bias scale of the skew4x workload (the skewed Qwen3-235B-shaped layer, N=16384,\n"
                 "# H=4096, E=128, top-8, bias b_e = scale * 2 ln(rank_e^-1.2)): the scale at which the\n"
                 "# hottest expert's load is 4x the mean (max/mean in [3.9, 4.1]), bisected on the seeded\n"

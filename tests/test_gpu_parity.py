@@ -285,7 +285,7 @@ def test_layer_tiny_matches_oracle():
     check_layer_against_oracle(cfg, t, out, logits)
 
 
-@pytest.mark.parametrize("cfg", [
+LAYER_SHAPES = [
     # several token tiles per expert with a ragged tail, K loop of 5, feature tiles 2.5 and 1.5
     MoEConfig("ragged", N=300, H=320, I=192, E=5, k=2),
     # mean 12 rows per expert -> 32-row token tiles
@@ -306,7 +306,29 @@ def test_layer_tiny_matches_oracle():
     MoEConfig("allexperts", N=96, H=192, I=192, E=4, k=4),
     # the smallest widths (one 64-column K block, one feature half-tile)
     MoEConfig("narrowest", N=40, H=64, I=64, E=3, k=2),
-])
+    # 192-row token tiles on CTA pairs (the widest tile below 256)
+    MoEConfig("tile192", N=1200, H=128, I=128, E=8, k=1),
+]
+
+
+@pytest.mark.parametrize("cfg", LAYER_SHAPES, ids=lambda c: c.name)
+def test_layer_gathered_rows_equal_the_permuted_copy(cfg):
+    """The W1/W3 GEMM either reads the permuted copy x_perm or gathers each row from x
+    through row_to_token (tile::gather4); the two must give the same bits."""
+    t = cuda_inputs(cfg, seed=21)
+    prev = moe.moe_set_gather_mode(moe.MOE_GATHER_OFF)
+    try:
+        copy, lc = run_layer(cfg, t)
+        moe.moe_set_gather_mode(moe.MOE_GATHER_ON)
+        gathered, lg = run_layer(cfg, t)
+    finally:
+        moe.moe_set_gather_mode(prev)
+    torch.cuda.synchronize()
+    assert torch.equal(lc, lg)
+    assert torch.equal(copy.view(torch.int16), gathered.view(torch.int16))
+
+
+@pytest.mark.parametrize("cfg", LAYER_SHAPES, ids=lambda c: c.name)
 def test_layer_shapes_match_oracle(cfg):
     t = cuda_inputs(cfg, seed=1)
     out, logits = run_layer(cfg, t)

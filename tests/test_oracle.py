@@ -571,3 +571,14 @@ def test_threaded_build_gives_the_serial_builds_bits():
         a, b = np.asarray(a), np.asarray(b)
         assert a.dtype == b.dtype and a.shape == b.shape
         assert a.tobytes() == b.tobytes()
+
+
+def test_skew4x_scale_is_the_calibrated_one():
+    """The 4x-mean skew reading's bias scale in the input recipe is the value the
+    calibration script (oracle routing on the seeded inputs) recorded."""
+    from expert_ffn_layer_moe_b200.inputs import SKEW4X_BIAS_SCALE, SKEW4X_LOAD_BAND
+    rec = dict(l.split() for l in (Path(__file__).parent / "golden" / "skew4x_bias_scale.txt").read_text()
+               .splitlines() if l and not l.startswith("#"))
+    assert float(rec["bias_scale"]) == SKEW4X_BIAS_SCALE
+    assert SKEW4X_LOAD_BAND[0] <= float(rec["max_over_mean_load"]) <= SKEW4X_LOAD_BAND[1]
+    assert CONFIGS["qwen3_235b_a22b_skew4x"].bias_scale == SKEW4X_BIAS_SCALE
