@@ -124,11 +124,11 @@ def kernel_source_digest(path):
     return hashlib.sha256(code.encode()).hexdigest()[:12]
 
 
-def kernel_traffic(kernel, workload):
+def kernel_traffic(kernel, workload, path=None, src=None):
     """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.txt,
     valid only while the kernel source is unchanged (its sha256 prefix matches)."""
-    path = os.path.join(ROOT, "profiles", "traffic.txt")
-    src = os.path.join(ROOT, "expert_ffn_layer_moe_b200", "csrc", "grouped_gemm.cu")
+    path = path or os.path.join(ROOT, "profiles", "traffic.txt")
+    src = src or os.path.join(ROOT, "expert_ffn_layer_moe_b200", "csrc", "grouped_gemm.cu")
     if not os.path.exists(path):
         return None
     digest = kernel_source_digest(src)

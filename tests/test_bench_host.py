@@ -38,9 +38,13 @@ def test_traffic_lookup_follows_the_kernel_source(tmp_path):
     assert bench.kernel_source_digest(str(src)) == d0            # comments and blank lines do not count
     src.write_text("int f() { return 2; }\n")
     assert bench.kernel_source_digest(str(src)) != d0
-    # the recorded lines are keyed by the current grouped GEMM source
-    assert bench.kernel_traffic("gemm13", "mixtral_8x22b_decode") is not None
-    assert bench.kernel_traffic("gemm13", "no_such_workload") is None
+    # a recorded line counts only while its digest is the kernel source's current one
+    rec = tmp_path / "traffic.txt"
+    rec.write_text(f"# comment\ngemm13 wl 123.0 {bench.kernel_source_digest(str(src))}\n"
+                   f"gemm13 old 456.0 {d0}\n")
+    assert bench.kernel_traffic("gemm13", "wl", str(rec), str(src)) == 123.0
+    assert bench.kernel_traffic("gemm13", "old", str(rec), str(src)) is None     # source changed since
+    assert bench.kernel_traffic("gemm13", "no_such_workload", str(rec), str(src)) is None
 
 
 FAKE_NVML = r"""
