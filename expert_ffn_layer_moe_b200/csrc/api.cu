@@ -22,14 +22,18 @@ std::atomic<int> g_gather_mode{MOE_GATHER_AUTO};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 uint64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
 
-// Whether the bf16 layer gathers its W1/W3 token rows from x (no permuted copy).
+// Whether the bf16 layer gathers its W1/W3 token rows from x (no permuted copy).  By
+// default it does not: each tile::gather4 request (four 128-byte rows) costs the TMA unit
+// about 85 cycles on B200, so a prefill-sized token tile (128 rows per CTA per K step)
+// takes about 2,700 cycles to gather against about 500 for the MMAs it feeds -- W1/W3
+// ran 3x slower gathered than from the permuted copy on every workload shape measured,
+// more than the copy it saves.
 bool layer_gathers(int64_t N, int k, int H)
 {
     const int mode = g_gather_mode.load(std::memory_order_relaxed);
     if (mode == MOE_GATHER_ON) return true;
-    if (mode == MOE_GATHER_OFF) return false;
     (void)N; (void)k; (void)H;
-    return true;
+    return false;
 }
 
 void *current_context()

@@ -122,7 +122,11 @@ struct Cfg {
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols + kABufs * kACols);
     static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs + 2 * kFStages + kABufs);
     static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
-    static constexpr int kEpiBytes = 4 * 32 * 33 * 4;  // staging: 4 x [32][33] fp32 (= 2 x [64][33])
+    // epilogue staging: one region of 34 x 32 fp32 per epilogue warp (a padded [32][33]
+    // tile, or a dense [32][32] box for bulk stores at its 128-byte-aligned start); the
+    // SwiGLU epilogue uses it as 2 x [64][33]
+    static constexpr int kEpiWarpFloats = 34 * 32;
+    static constexpr int kEpiBytes = 4 * kEpiWarpFloats * 4;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kFStages * kW8Bytes + kBarBytes + 16 +
                                       kTableBytes + kEpiBytes;
     // tcgen05 instruction descriptor: D=f32 (bit 4); kind::f16 with A=B=bf16 (format 1 at
@@ -290,16 +294,15 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar)
                  : "memory");
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane; the wait is inside the
-// same asm statement so no use of the registers can be scheduled before it.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+// 32 consecutive fp32 columns of this thread's TMEM lane (the warp's lane quadrant),
+// without the wait: the registers are valid only after tmem_wait_ld on them (which
+// names them as operands, so no use can be scheduled before it).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32])
 {
-    uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
           "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
@@ -307,8 +310,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+          "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+          "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+          "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+        :
+        : "memory");
+}
+
+// One 32 x 32 fp32 box (32 output rows of 32 consecutive features) from this CTA's
+// shared memory to global memory through the output map, as one bulk group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, int c0, int c1, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(c0), "r"(c1), "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
 // ---------------------------------------------- CTA-pair (cta_group::2) forms --
@@ -481,8 +506,6 @@ __device__ __forceinline__ void umma_commit_g(uint64_t *bar)
 // tiles this is what keeps it shorter than the main loop.
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-// Named barrier for the four epilogue warps (barrier 0 is __syncthreads).
-__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // ------------------------------------------------------------------ kernel --
 // PAIR = true runs as clusters of two CTAs on two SMs: CTA r of a pair holds weight
@@ -503,7 +526,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                         void *__restrict__ out, int ksplit, int64_t split_stride,
                         const float *__restrict__ scale_a, const float *__restrict__ scale_b,
                         const float *__restrict__ scale_act, int64_t ldo, const int32_t *__restrict__ gather_rows,
-                        int *dev_err)
+                        const __grid_constant__ CUtensorMap tm_out, int tma_store, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
     static_assert(!GATHER || (SWIGLU && !W8 && !A8), "gathered activation rows: bf16 SwiGLU GEMM only");
@@ -515,7 +538,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
 
     uint8_t *stages = smem;                                     // TMA ring (W8: activations)
     uint8_t *fring = smem + C::kStages * C::kStageBytes;        // W8: fp8 weight tiles
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(fring + C::kFStages * C::kW8Bytes);
+    // epilogue staging, 1024-byte aligned (every stage and fp8 tile is a multiple of 1 KB)
+    float *epi_stage = reinterpret_cast<float *>(fring + C::kFStages * C::kW8Bytes);
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(epi_stage) + C::kEpiBytes);
     uint64_t *empty_bar = full_bar + C::kStages;
     uint64_t *tfull_bar = empty_bar + C::kStages;
     uint64_t *tempty_bar = tfull_bar + C::kAccBufs;
@@ -524,10 +549,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
     uint64_t *afull_bar = fempty_bar + C::kFStages;             // W8: operand slot written by every converter warp
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(afull_bar + C::kABufs);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
     int *g_tile = g_off + (kMaxGroups + 1);               // [groups+1] work-item prefix
-    float *epi_stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(g_off) + C::kTableBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -657,8 +680,12 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                 const uint32_t fb = smem_u32(&ffull_bar[stage]);
                 mbar_arrive_expect_tx(&ffull_bar[stage], C::kW8Bytes);
                 if (SWIGLU) {
-                    tma_3d<false>(dst, &tm_wa, kb * kBK, frow, g, fb);
-                    tma_3d<false>(dst + C::kW8Bytes / 2, &tm_wb, kb * kBK, frow, g, fb);
+                    // W1 and W3 rows interleaved in 16-row groups, as in the bf16 tiles
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        tma_3d<false>(dst + 32 * i * 128, &tm_wa, kb * kBK, frow + 16 * i, g, fb);
+                        tma_3d<false>(dst + (32 * i + 16) * 128, &tm_wb, kb * kBK, frow + 16 * i, g, fb);
+                    }
                 } else {
                     tma_3d<false>(dst, &tm_wa, kb * kBK, frow, g, fb);
                 }
@@ -694,9 +721,14 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                 if (lane == 0) {
                     if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kCtas * C::kStageBytes);
                     if (SWIGLU) {
-                        // rows 0-63: W1 features [frow, +64); rows 64-127: the same features of W3
-                        tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
-                        tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kc, frow, g, fb);
+                        // rows 32i .. 32i+15: W1 features [frow + 16i, +16); rows 32i+16 ..
+                        // 32i+31: the same features of W3 (each epilogue warp then holds
+                        // g and u of its 16 features)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            tma_3d<PAIR>(st + 32 * i * 128, &tm_wa, kc, frow + 16 * i, g, fb);
+                            tma_3d<PAIR>(st + (32 * i + 16) * 128, &tm_wb, kc, frow + 16 * i, g, fb);
+                        }
                     } else {
                         tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
                     }
@@ -772,70 +804,147 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
         for (int item = unit; item < total; item += nunits) {
             int g, feat, ks, row0, row_end;
             decode(item, g, feat, ks, row0, row_end);
-            // one waiter decides for all four warps, so the named barriers below are
-            // always reached by all of them
-            if (ew == 0 && lane == 0) *epi_ok = mbar_wait(&tfull_bar[acc], aphase, abort_flag) ? 1 : 0;
-            epilogue_sync();
-            const bool ok = *epi_ok != 0;
-            epilogue_sync();  // everyone has read the flag before it can be rewritten
-            if (!ok) { failed = true; *abort_flag = 1; break; }
+            // each warp waits for the accumulator on its own (the warps share no barrier)
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&tfull_bar[acc], aphase, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) { failed = true; if (lane == 0) *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
             const int nrows = min(BN, row_end - row0);
             if (SWIGLU) {
-                float(*Gs)[33] = reinterpret_cast<float(*)[33]>(epi_stage);            // [64][33] g
-                float(*Us)[33] = reinterpret_cast<float(*)[33]>(epi_stage + 64 * 33);  // [64][33] u
-                float(*mine)[33] = q < 2 ? Gs : Us;
-                const int fl = (q & 1) * 32 + lane;  // feature within this CTA's 64
-                const int rr = lane >> 3, j = lane & 7;
-                const int fv = feat * C::kFeatTile + (int)rank * C::kFeat + 8 * j;
+                // The CTA's A tile interleaves W1 and W3 in 16-row groups (the producer's
+                // loads), so warp q's TMEM lanes hold, for the 16 features fq .. fq + 15,
+                // g on lanes 0-15 and u on lanes 16-31.  Per 32-token chunk: shuffles pair
+                // g with u (lane l < 16 then holds h of feature fq + l for tokens 0-15,
+                // lane l + 16 for tokens 16-31), three more exchange rounds turn the
+                // feature-per-lane layout into 16-byte pieces of token rows, and each lane
+                // stores two of them.  No shared memory, no barrier between the warps.
+                const bool hi = lane >= 16;
+                const int l = lane & 15;
+                const int fq = feat * C::kFeatTile + (int)rank * C::kFeat + 16 * q;  // warp's first feature
                 uint16_t *outh = static_cast<uint16_t *>(out);
                 float sc = 1.0f;  // fp8 weights: the scale of this lane's weight row (W1 for g, W3 for u)
-                if (W8 || A8) {
-                    const int row = feat * C::kFeatTile + (int)rank * C::kFeat + fl;
-                    sc = row < Nout ? (q < 2 ? scale_a : scale_b)[(int64_t)g * Nout + row] : 0.0f;
-                }
+                if (W8 || A8) sc = fq + l < Nout ? (hi ? scale_b : scale_a)[(int64_t)g * Nout + fq + l] : 0.0f;
+                // token offsets of this lane's two stored rows inside a chunk, and its features
+                const int tok0 = (hi ? 16 : 0) + 8 * (l & 1) + 4 * ((l >> 1) & 1) + 2 * ((l >> 2) & 1);
+                const int fst = fq + (l & 8);
+                uint32_t cur[32], nxt[32];
+                tmem_ld32_async(t0, cur);
+                tmem_wait_ld(cur);
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
-                    float a[32];
-                    tmem_ld32(t0 + c0, a);
-                    // A8: column c is token row row0 + c0 + c, with its own scale (lane c holds it)
-                    const float sa = A8 && c0 + lane < nrows ? scale_act[row0 + c0 + lane] : 0.0f;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        float v = (W8 || A8) ? a[c] * sc : a[c];
-                        if (A8) v *= __shfl_sync(0xffffffffu, sa, c);
-                        mine[fl][c] = v;
-                    }
-                    epilogue_sync();
-                    // warp ew stores rows 8*ew .. 8*ew+7 of the chunk: 4 rows x 8 feature octets per step
-#pragma unroll
-                    for (int it = 0; it < 2; ++it) {
-                        const int r = 8 * ew + 4 * it + rr;
-                        if (c0 + r < nrows && fv < Nout) {
-                            float h[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) h[i] = silu(Gs[8 * j + i][r]) * Us[8 * j + i][r];
-                            uint4 v;
-                            v.x = pack_bf16x2(h[0], h[1]);
-                            v.y = pack_bf16x2(h[2], h[3]);
-                            v.z = pack_bf16x2(h[4], h[5]);
-                            v.w = pack_bf16x2(h[6], h[7]);
-                            *reinterpret_cast<uint4 *>(outh + (size_t)(row0 + c0 + r) * Nout + fv) = v;
+                    const bool more = c0 + 32 < nrows;
+                    if (more) {
+                        tmem_ld32_async(t0 + c0 + 32, nxt);
+                    } else {
+                        // every column of this accumulator is in registers: release it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * acc);
+                            else mbar_arrive(&tempty_bar[acc]);
                         }
                     }
-                    epilogue_sync();
+                    float a[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) a[c] = __uint_as_float(cur[c]);
+                    if (W8 || A8) {
+                        // A8: column c is token row row0 + c0 + c, with its own scale (lane c holds it)
+                        const float sa = A8 && c0 + lane < nrows ? scale_act[row0 + c0 + lane] : 0.0f;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            a[c] *= sc;
+                            if (A8) a[c] *= __shfl_sync(0xffffffffu, sa, c);
+                        }
+                    }
+                    // g with u: lane l sends g of tokens 16..31, lane l + 16 sends u of 0..15
+                    float h[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float r = __shfl_xor_sync(0xffffffffu, hi ? a[i] : a[16 + i], 16);
+                        const float gv = hi ? r : a[i];
+                        const float uv = hi ? a[16 + i] : r;
+                        h[i] = silu(gv) * uv;  // token (hi ? 16 : 0) + i, feature fq + l
+                    }
+                    // features (l & ~1, l | 1) for 8 tokens: bf16 pairs
+                    const bool p1 = (l & 1) != 0;
+                    uint32_t w[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float r = __shfl_xor_sync(0xffffffffu, p1 ? h[j] : h[8 + j], 1);
+                        w[j] = p1 ? pack_bf16x2(r, h[8 + j]) : pack_bf16x2(h[j], r);
+                    }
+                    // features (l & ~3) .. +3 for 4 tokens: two words each
+                    const bool p2 = (l & 2) != 0;
+                    uint32_t x4[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t r = __shfl_xor_sync(0xffffffffu, p2 ? w[j] : w[4 + j], 2);
+                        x4[2 * j] = p2 ? r : w[j];
+                        x4[2 * j + 1] = p2 ? w[4 + j] : r;
+                    }
+                    // features (l & ~7) .. +7 for 2 tokens: four words each
+                    const bool p4 = (l & 4) != 0;
+                    uint32_t y8[8];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                        for (int wd = 0; wd < 2; ++wd) {
+                            const uint32_t r =
+                                __shfl_xor_sync(0xffffffffu, p4 ? x4[2 * j + wd] : x4[2 * (2 + j) + wd], 4);
+                            y8[4 * j + wd] = p4 ? r : x4[2 * j + wd];
+                            y8[4 * j + 2 + wd] = p4 ? x4[2 * (2 + j) + wd] : r;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int r = c0 + tok0 + j;
+                        if (r < nrows && fst < Nout)
+                            *reinterpret_cast<uint4 *>(outh + (size_t)(row0 + r) * Nout + fst) =
+                                make_uint4(y8[4 * j], y8[4 * j + 1], y8[4 * j + 2], y8[4 * j + 3]);
+                    }
+                    if (more) {
+                        tmem_wait_ld(nxt);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
+                    }
                 }
             } else {
                 float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
                 const int fbase = feat * C::kFeatTile + (int)rank * C::kFeat + q * 32;
                 const float sc =
                     (W8 || A8) ? (fbase + lane < Nout ? scale_a[(int64_t)g * Nout + fbase + lane] : 0.0f) : 1.0f;
-                // fp32 out through the padded tile: 8 16-byte stores per 32 rows instead of
-                // 32 4-byte ones (store instruction issue, not bytes, limits short-K tiles)
-                float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(epi_stage + ew * 32 * 33);
+                // The next chunk's TMEM load is in flight while this one is stored, and the
+                // accumulator goes back to the MMA as soon as its last chunk is in registers.
+                // With tma_store, a chunk of 32 whole rows leaves as one 32 x 32 fp32 box
+                // from this warp's 4 KB staging tile (one bulk store issued by lane 0); a
+                // ragged last chunk, and everything without tma_store, goes through the
+                // padded tile: 8 16-byte stores per 32 rows instead of 32 4-byte ones (store
+                // instruction issue, not bytes, limits short-K tiles).
+                float *wreg = epi_stage + ew * C::kEpiWarpFloats;  // this warp's staging region
+                float(*stage_t)[33] = reinterpret_cast<float(*)[33]>(wreg);
+                float *box = wreg;  // [32 rows][32 features] (tma_store), 128-byte aligned
+                const uint32_t box_s = smem_u32(box);
+                static_assert((C::kEpiWarpFloats * 4) % 128 == 0, "bulk-store boxes start on 128 bytes");
+                uint32_t cur[32], nxt[32];
+                tmem_ld32_async(t0, cur);
+                tmem_wait_ld(cur);
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
+                    const bool more = c0 + 32 < nrows;
+                    if (more) {
+                        tmem_ld32_async(t0 + c0 + 32, nxt);
+                    } else {
+                        // every column of this accumulator is in registers: release it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * acc);
+                            else mbar_arrive(&tempty_bar[acc]);
+                        }
+                    }
                     float a[32];
-                    tmem_ld32(t0 + c0, a);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) a[c] = __uint_as_float(cur[c]);
                     if (W8 || A8) {
                         const float sa = A8 && c0 + lane < nrows ? scale_act[row0 + c0 + lane] : 1.0f;
 #pragma unroll
@@ -844,7 +953,18 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                             if (A8) a[c] *= __shfl_sync(0xffffffffu, sa, c);
                         }
                     }
-                    if (vec_ok) {
+                    if (tma_store) {
+                        // this warp's previous bulk store has finished reading the region
+                        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                        __syncwarp();
+                    }
+                    if (tma_store && c0 + 32 <= nrows && fbase < Nout) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) box[c * 32 + lane] = a[c];
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                        if (lane == 0) tma_store_2d(&tm_out, fbase, (int)((int64_t)ks * R + row0 + c0), box_s);
+                    } else if (vec_ok) {
 #pragma unroll
                         for (int c = 0; c < 32; ++c) stage_t[lane][c] = a[c];
                         __syncwarp();
@@ -866,16 +986,18 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                         for (int c = 0; c < 32; ++c)
                             if (c0 + c < nrows) dst[(size_t)c * ldo] = a[c];
                     }
+                    if (more) {
+                        tmem_wait_ld(nxt);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
+                    }
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * acc);  // the leader's barrier
-                else mbar_arrive(&tempty_bar[acc]);
             }
             if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
         }
+        // bulk stores must have landed before the kernel's writes count as done
+        if (!SWIGLU && tma_store && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
     }
 
     if (W8 && warp >= 6 && warp < 14) {
@@ -1041,6 +1163,21 @@ bool encode_gather_map(CUtensorMap *m, const void *ptr, int64_t rows, int K)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 output rows [rows, Nout] (row stride ldo elements) as a 2-D map for bulk stores:
+// box = 32 features x 32 rows, no swizzle (the staging tile is a dense [32][32]).
+bool encode_out_map_f32(CUtensorMap *m, void *ptr, int64_t rows, int Nout, int64_t ldo)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)Nout, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ldo * 4};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Activations [R, K] e4m3 bytes as a 2-D byte map; box = 128 (K) x box_rows; rows >= R
 // and K values past K read as zero.
 bool encode_act_map_fp8(CUtensorMap *m, const void *ptr, int64_t R, int K, int box_rows)
@@ -1061,7 +1198,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
     using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
     CUtensorMap ma, mb, mact;
-    const int box_rows = SWIGLU ? kBM / 2 : kBM;
+    const int box_rows = SWIGLU ? 16 : kBM;  // SwiGLU: W1 and W3 interleaved in 16-row groups
     auto enc_w = (W8 || A8) ? encode_weight_map_fp8 : encode_weight_map;
     if (!enc_w(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     if (SWIGLU) {
@@ -1078,6 +1215,16 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     }
     const int64_t ldo = a.ldo > 0 ? a.ldo : a.Nout;
     if (ldo < a.Nout) return cudaErrorInvalidValue;
+    const int ks_out = SWIGLU ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
+    // plain GEMM: bulk tensor stores of the fp32 rows when the K slices' buffers sit one
+    // after another (split_stride = R * ldo), the row stride is whole 16-byte units and
+    // every row coordinate fits the map's 32-bit coordinates
+    CUtensorMap mout = ma;
+    int tma_store = 0;
+    if (!SWIGLU && a.out && (ldo & 3) == 0 && (a.Nout & 31) == 0 &&
+        (ks_out == 1 || a.split_stride == a.R * ldo) && (int64_t)ks_out * a.R < (int64_t(1) << 31) &&
+        (reinterpret_cast<uintptr_t>(a.out) & 15) == 0)
+        tma_store = encode_out_map_f32(&mout, a.out, (int64_t)ks_out * a.R, a.Nout, ldo) ? 1 : 0;
     auto kern = grouped_gemm_kernel<BN, SWIGLU, PAIR, W8, A8, GATHER>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
@@ -1098,8 +1245,8 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = PAIR ? 2 : 1;
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
-                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, ldo, a.gather_rows,
-                             a.dev_err);
+                             ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, ldo, a.gather_rows, mout,
+                             tma_store, a.dev_err);
     if (err != cudaSuccess) return err;
     count_launch();
     return cudaGetLastError();

@@ -338,7 +338,8 @@ MOE_API int moe_device_sm_count(void);
  * builds the row maps and the GEMM loads each row straight from x through
  * row_to_token (tile::gather4 TMA), so the permuted copy x_perm is never written.
  * The results are identical either way.
- *   mode  MOE_GATHER_AUTO (the default: the library chooses by shape),
+ *   mode  MOE_GATHER_AUTO (the default: the library chooses; measured on B200,
+ *         gathering was slower on every workload shape, so it picks the copy),
  *         MOE_GATHER_OFF (always the permuted copy), MOE_GATHER_ON (always gather).
  * Process-wide; takes effect for calls enqueued after it returns.  Returns the
  * previous mode, or -1 for a mode outside these three.
