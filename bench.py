@@ -744,6 +744,112 @@ def run_ours(args, cfg, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def ep_local_inputs(cfg, rank, world, device):
+    """Expert-parallel inputs of one rank: its own token batch (seed = rank), the whole
+    router, and its slice [rank*L, (rank+1)*L) of every expert stack (L = E / world)."""
+    from expert_ffn_layer_moe_b200 import ep
+    if cfg.E % world:
+        raise ValueError(f"{cfg.E} experts do not split over {world} ranks")
+    t = make_inputs(cfg, seed=0, device=device)
+    x = make_inputs(cfg, seed=rank, device=device, weights=False)["x"]
+    local = {n: ep.local_experts(t[n], rank, world).contiguous() for n in ("W1", "W3", "W2")}
+    del t["W1"], t["W3"], t["W2"]
+    return x, t["W_gate"], t["bias"], local
+
+
+def ep_line(cfg, world, steps, warmup, step_ms_max, exchange, rows_sent, rows_recv, e2e_ms_max=None):
+    """The expert-parallel JSON line: value = all ranks' tokens / the slowest rank's time."""
+    line = {"metric": METRIC, "value": world * cfg.N / (step_ms_max / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": step_ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "global_batch": world * cfg.N, "tokens_per_gpu": cfg.N,
+                       "parallelism": (f"ep{world}: experts split {cfg.E}/{world} per rank, token rows exchanged "
+                                       f"by {exchange}, one token batch per rank"),
+                       "rows_sent_per_rank": rows_sent, "rows_received_per_rank": rows_recv}}
+    if e2e_ms_max is not None:
+        line["e2e"] = {"value": world * cfg.N / (e2e_ms_max / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": cfg.N * cfg.H * 2, "d2h_bytes_per_step": cfg.N * cfg.H * 2,
+                       "how": "each step's x copied in from pinned host memory and its out read back, synchronous"}
+    return line
+
+
+def run_ep(args, cfg, world, rank, local):
+    """Expert parallelism: every rank holds E/world experts and its own batch; a step is
+    route, permute, the row exchange to the experts' ranks, the local grouped GEMMs,
+    the exchange back and the combine (moe_layer_forward_ep).  One rank works too (the
+    exchange then stays on the GPU)."""
+    import datetime
+    import socket
+    import torch.distributed as dist
+    from expert_ffn_layer_moe_b200 import ep, moe
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    own_group = False
+    if not dist.is_initialized():  # one rank: a group of one
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+        own_group = True
+    try:
+        x, Wg, bias, W = ep_local_inputs(cfg, rank, world, dev)
+        tr = None
+        if args.exchange == "peer_copy":
+            tr = ep.PeerCopyTransport(ep.CudaPeers(device=dev), max_rows=cfg.N * cfg.k, words_in=cfg.H // 2,
+                                      words_out=cfg.H)
+        stats = []
+
+        def step(xx=None, record=None):
+            return ep.moe_layer_forward_ep(x if xx is None else xx, Wg, W["W1"], W["W3"], W["W2"], cfg.k, bias=bias,
+                                           transport=tr, stats=record)
+
+        for _ in range(args.warmup):
+            step()
+        step(record=stats)  # one step with per-phase records (rows moved)
+        torch.cuda.synchronize()
+        if moe.moe_get_device_error() != 0:
+            raise RuntimeError("device error reported during warm-up")
+        s = torch.cuda.current_stream(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(s)
+        for _ in range(args.steps):
+            step()
+        t1.record(s)
+        torch.cuda.synchronize()
+        dist.barrier()
+        ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+        # end to end: x from pinned host memory in, out back to the host, every step
+        xh = x.cpu().pin_memory()
+        oh = torch.empty((cfg.N, cfg.H), dtype=torch.bfloat16).pin_memory()
+        dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(s)
+        for _ in range(args.steps):
+            xd = xh.to(dev, non_blocking=True)
+            oh.copy_(step(xd), non_blocking=True)
+        t1.record(s)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+        if tr is not None:
+            tr.close()
+        if moe.moe_get_device_error() != 0:
+            raise RuntimeError("device error reported during the timed steps")
+        line = ep_line(cfg, world, args.steps, args.warmup, ms, args.exchange, stats[0].rows_sent,
+                       stats[0].rows_received, e2e_ms)
+        line["ep_phase_s"] = stats[0].seconds
+        line["gpu_launches_note"] = "not counted for the expert-parallel step"
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if own_group:
+            dist.destroy_process_group()
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -784,6 +890,10 @@ def main():
                     help="routed-expert weight format (fp8: e4m3 with per-channel scales, a separate experiment)")
     ap.add_argument("--acts", choices=["bf16", "fp8"], default="bf16",
                     help="routed-expert activation format (fp8: e4m3 with per-row scales; needs --weights fp8)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: the experts split over the ranks, token rows exchanged")
+    ap.add_argument("--exchange", choices=["collective", "peer_copy"], default="collective",
+                    help="--ep: rows moved by NCCL all-to-all or by copies into the peers' buffers (CUDA IPC)")
     ap.add_argument("--gather", choices=["auto", "on", "off"], default="auto",
                     help="W1/W3 token rows: gathered from x (on), the permuted copy (off), or by shape (auto)")
     args = ap.parse_args()
@@ -801,6 +911,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, cfg, world, rank)
+        elif args.ep:
+            run_ep(args, cfg, world, rank, local)
         else:
             run_ours(args, cfg, world, rank, local)
     finally:

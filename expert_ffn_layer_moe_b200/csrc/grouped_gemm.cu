@@ -325,6 +325,16 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32])
         : "memory");
 }
 
+// The load and its wait: 32 fp32 columns ready in registers.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    tmem_ld32_async(taddr, r);
+    tmem_wait_ld(r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // One 32 x 32 fp32 box (32 output rows of 32 consecutive features) from this CTA's
 // shared memory to global memory through the output map, as one bulk group.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, int c0, int c1, uint32_t src)
@@ -507,6 +517,9 @@ __device__ __forceinline__ void umma_commit_g(uint64_t *bar)
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 
+// Named barrier for the four epilogue warps (barrier 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 // ------------------------------------------------------------------ kernel --
 // PAIR = true runs as clusters of two CTAs on two SMs: CTA r of a pair holds weight
 // rows [128 r, 128 r + 128) of the work item's 256 and token rows
@@ -549,6 +562,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
     uint64_t *afull_bar = fempty_bar + C::kFStages;             // W8: operand slot written by every converter warp
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(afull_bar + C::kABufs);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
     int *g_tile = g_off + (kMaxGroups + 1);               // [groups+1] work-item prefix
 
@@ -680,12 +694,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                 const uint32_t fb = smem_u32(&ffull_bar[stage]);
                 mbar_arrive_expect_tx(&ffull_bar[stage], C::kW8Bytes);
                 if (SWIGLU) {
-                    // W1 and W3 rows interleaved in 16-row groups, as in the bf16 tiles
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        tma_3d<false>(dst + 32 * i * 128, &tm_wa, kb * kBK, frow + 16 * i, g, fb);
-                        tma_3d<false>(dst + (32 * i + 16) * 128, &tm_wb, kb * kBK, frow + 16 * i, g, fb);
-                    }
+                    tma_3d<false>(dst, &tm_wa, kb * kBK, frow, g, fb);
+                    tma_3d<false>(dst + C::kW8Bytes / 2, &tm_wb, kb * kBK, frow, g, fb);
                 } else {
                     tma_3d<false>(dst, &tm_wa, kb * kBK, frow, g, fb);
                 }
@@ -721,14 +731,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                 if (lane == 0) {
                     if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kCtas * C::kStageBytes);
                     if (SWIGLU) {
-                        // rows 32i .. 32i+15: W1 features [frow + 16i, +16); rows 32i+16 ..
-                        // 32i+31: the same features of W3 (each epilogue warp then holds
-                        // g and u of its 16 features)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            tma_3d<PAIR>(st + 32 * i * 128, &tm_wa, kc, frow + 16 * i, g, fb);
-                            tma_3d<PAIR>(st + (32 * i + 16) * 128, &tm_wb, kc, frow + 16 * i, g, fb);
-                        }
+                        // rows 0-63: W1 features [frow, +64); rows 64-127: the same features of W3
+                        tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
+                        tma_3d<PAIR>(st + C::kABytes / 2, &tm_wb, kc, frow, g, fb);
                     } else {
                         tma_3d<PAIR>(st, &tm_wa, kc, frow, g, fb);
                     }
@@ -804,110 +809,65 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
         for (int item = unit; item < total; item += nunits) {
             int g, feat, ks, row0, row_end;
             decode(item, g, feat, ks, row0, row_end);
-            // each warp waits for the accumulator on its own (the warps share no barrier)
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(&tfull_bar[acc], aphase, abort_flag);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (SWIGLU) {
+                // one waiter decides for all four warps, so the named barriers of the
+                // SwiGLU epilogue are always reached by all of them
+                if (ew == 0 && lane == 0) *epi_ok = mbar_wait(&tfull_bar[acc], aphase, abort_flag) ? 1 : 0;
+                epilogue_sync();
+                ok = *epi_ok != 0;
+                epilogue_sync();  // everyone has read the flag before it can be rewritten
+            } else {
+                // the plain epilogue has no barrier between its warps: each waits on its own
+                if (lane == 0) ok = mbar_wait(&tfull_bar[acc], aphase, abort_flag);
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            }
             if (!ok) { failed = true; if (lane == 0) *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
             const int nrows = min(BN, row_end - row0);
             if (SWIGLU) {
-                // The CTA's A tile interleaves W1 and W3 in 16-row groups (the producer's
-                // loads), so warp q's TMEM lanes hold, for the 16 features fq .. fq + 15,
-                // g on lanes 0-15 and u on lanes 16-31.  Per 32-token chunk: shuffles pair
-                // g with u (lane l < 16 then holds h of feature fq + l for tokens 0-15,
-                // lane l + 16 for tokens 16-31), three more exchange rounds turn the
-                // feature-per-lane layout into 16-byte pieces of token rows, and each lane
-                // stores two of them.  No shared memory, no barrier between the warps.
-                const bool hi = lane >= 16;
-                const int l = lane & 15;
-                const int fq = feat * C::kFeatTile + (int)rank * C::kFeat + 16 * q;  // warp's first feature
+                float(*Gs)[33] = reinterpret_cast<float(*)[33]>(epi_stage);            // [64][33] g
+                float(*Us)[33] = reinterpret_cast<float(*)[33]>(epi_stage + 64 * 33);  // [64][33] u
+                float(*mine)[33] = q < 2 ? Gs : Us;
+                const int fl = (q & 1) * 32 + lane;  // feature within this CTA's 64
+                const int rr = lane >> 3, j = lane & 7;
+                const int fv = feat * C::kFeatTile + (int)rank * C::kFeat + 8 * j;
                 uint16_t *outh = static_cast<uint16_t *>(out);
                 float sc = 1.0f;  // fp8 weights: the scale of this lane's weight row (W1 for g, W3 for u)
-                if (W8 || A8) sc = fq + l < Nout ? (hi ? scale_b : scale_a)[(int64_t)g * Nout + fq + l] : 0.0f;
-                // token offsets of this lane's two stored rows inside a chunk, and its features
-                const int tok0 = (hi ? 16 : 0) + 8 * (l & 1) + 4 * ((l >> 1) & 1) + 2 * ((l >> 2) & 1);
-                const int fst = fq + (l & 8);
-                uint32_t cur[32], nxt[32];
-                tmem_ld32_async(t0, cur);
-                tmem_wait_ld(cur);
+                if (W8 || A8) {
+                    const int row = feat * C::kFeatTile + (int)rank * C::kFeat + fl;
+                    sc = row < Nout ? (q < 2 ? scale_a : scale_b)[(int64_t)g * Nout + row] : 0.0f;
+                }
                 for (int c0 = 0; c0 < nrows; c0 += 32) {
-                    const bool more = c0 + 32 < nrows;
-                    if (more) {
-                        tmem_ld32_async(t0 + c0 + 32, nxt);
-                    } else {
-                        // every column of this accumulator is in registers: release it
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * acc);
-                            else mbar_arrive(&tempty_bar[acc]);
-                        }
-                    }
                     float a[32];
+                    tmem_ld32(t0 + c0, a);
+                    // A8: column c is token row row0 + c0 + c, with its own scale (lane c holds it)
+                    const float sa = A8 && c0 + lane < nrows ? scale_act[row0 + c0 + lane] : 0.0f;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) a[c] = __uint_as_float(cur[c]);
-                    if (W8 || A8) {
-                        // A8: column c is token row row0 + c0 + c, with its own scale (lane c holds it)
-                        const float sa = A8 && c0 + lane < nrows ? scale_act[row0 + c0 + lane] : 0.0f;
+                    for (int c = 0; c < 32; ++c) {
+                        float v = (W8 || A8) ? a[c] * sc : a[c];
+                        if (A8) v *= __shfl_sync(0xffffffffu, sa, c);
+                        mine[fl][c] = v;
+                    }
+                    epilogue_sync();
+                    // warp ew stores rows 8*ew .. 8*ew+7 of the chunk: 4 rows x 8 feature octets per step
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            a[c] *= sc;
-                            if (A8) a[c] *= __shfl_sync(0xffffffffu, sa, c);
+                    for (int it = 0; it < 2; ++it) {
+                        const int r = 8 * ew + 4 * it + rr;
+                        if (c0 + r < nrows && fv < Nout) {
+                            float h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) h[i] = silu(Gs[8 * j + i][r]) * Us[8 * j + i][r];
+                            uint4 v;
+                            v.x = pack_bf16x2(h[0], h[1]);
+                            v.y = pack_bf16x2(h[2], h[3]);
+                            v.z = pack_bf16x2(h[4], h[5]);
+                            v.w = pack_bf16x2(h[6], h[7]);
+                            *reinterpret_cast<uint4 *>(outh + (size_t)(row0 + c0 + r) * Nout + fv) = v;
                         }
                     }
-                    // g with u: lane l sends g of tokens 16..31, lane l + 16 sends u of 0..15
-                    float h[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float r = __shfl_xor_sync(0xffffffffu, hi ? a[i] : a[16 + i], 16);
-                        const float gv = hi ? r : a[i];
-                        const float uv = hi ? a[16 + i] : r;
-                        h[i] = silu(gv) * uv;  // token (hi ? 16 : 0) + i, feature fq + l
-                    }
-                    // features (l & ~1, l | 1) for 8 tokens: bf16 pairs
-                    const bool p1 = (l & 1) != 0;
-                    uint32_t w[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float r = __shfl_xor_sync(0xffffffffu, p1 ? h[j] : h[8 + j], 1);
-                        w[j] = p1 ? pack_bf16x2(r, h[8 + j]) : pack_bf16x2(h[j], r);
-                    }
-                    // features (l & ~3) .. +3 for 4 tokens: two words each
-                    const bool p2 = (l & 2) != 0;
-                    uint32_t x4[8];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t r = __shfl_xor_sync(0xffffffffu, p2 ? w[j] : w[4 + j], 2);
-                        x4[2 * j] = p2 ? r : w[j];
-                        x4[2 * j + 1] = p2 ? w[4 + j] : r;
-                    }
-                    // features (l & ~7) .. +7 for 2 tokens: four words each
-                    const bool p4 = (l & 4) != 0;
-                    uint32_t y8[8];
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                        for (int wd = 0; wd < 2; ++wd) {
-                            const uint32_t r =
-                                __shfl_xor_sync(0xffffffffu, p4 ? x4[2 * j + wd] : x4[2 * (2 + j) + wd], 4);
-                            y8[4 * j + wd] = p4 ? r : x4[2 * j + wd];
-                            y8[4 * j + 2 + wd] = p4 ? x4[2 * (2 + j) + wd] : r;
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int r = c0 + tok0 + j;
-                        if (r < nrows && fst < Nout)
-                            *reinterpret_cast<uint4 *>(outh + (size_t)(row0 + r) * Nout + fst) =
-                                make_uint4(y8[4 * j], y8[4 * j + 1], y8[4 * j + 2], y8[4 * j + 3]);
-                    }
-                    if (more) {
-                        tmem_wait_ld(nxt);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
-                    }
+                    epilogue_sync();
                 }
             } else {
                 float *outf = static_cast<float *>(out) + (int64_t)ks * split_stride;
@@ -991,6 +951,14 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
 #pragma unroll
                         for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
                     }
+                }
+            }
+            if (SWIGLU) {  // (the plain epilogue released the accumulator after its last TMEM load)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * acc);  // the leader's barrier
+                    else mbar_arrive(&tempty_bar[acc]);
                 }
             }
             if (++acc == C::kAccBufs) { acc = 0; aphase ^= 1u; }
@@ -1198,7 +1166,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
 {
     using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
     CUtensorMap ma, mb, mact;
-    const int box_rows = SWIGLU ? 16 : kBM;  // SwiGLU: W1 and W3 interleaved in 16-row groups
+    const int box_rows = SWIGLU ? kBM / 2 : kBM;
     auto enc_w = (W8 || A8) ? encode_weight_map_fp8 : encode_weight_map;
     if (!enc_w(&ma, a.w_a, a.groups, a.Nout, a.K, box_rows)) return cudaErrorInvalidValue;
     if (SWIGLU) {

@@ -26,6 +26,20 @@ contiguous range.  Then:
 The plan and the exchange are device-independent; the local steps (the expert FFN and
 the row scatter) are passed in.  ``moe_layer_forward_ep`` runs the library's kernels on
 CUDA tensors over an NCCL process group.  The rows cross the wire as raw 32-bit words.
+
+Two transports move the rows (steps 2 and 4):
+  * ``CollectiveTransport`` -- torch.distributed all-to-all (NCCL between GPUs, gloo on
+    CPU);
+  * ``PeerCopyTransport`` -- every rank copies its rows straight into the receiving
+    ranks' buffers, one copy per contiguous range, then all ranks meet at a host
+    barrier.  On GPUs the buffers are exported once through CUDA IPC and the copies
+    are the library's moe_copy_async (``CudaPeers``); the receive order is the
+    all-to-all's (source rank, then the source's order), so both transports give the
+    same bits.
+
+Host synchronisations per step: the counts all-gather (the plan is made on the host),
+plus, with peer copies, one per exchange (a rank's copies must have landed before the
+barrier releases the receivers).  Per-phase timing (``stats``) adds one per phase.
 """
 from __future__ import annotations
 
@@ -81,12 +95,11 @@ def exchange_plan(counts_all, rank: int) -> ExchangePlan:
 
 
 def _words(t: torch.Tensor) -> torch.Tensor:
-    """A row-major tensor as 32-bit words per row (the wire format of the exchange)."""
-    if t.element_size() == 4:
-        return t if t.dtype in (torch.int32, torch.float32) else t.view(torch.int32)
-    if t.element_size() == 2:
-        return t.view(torch.int32)
-    return t  # 8-byte rows travel as they are
+    """A row-major tensor as 32-bit words per row (the wire format of the exchange):
+    2-byte values travel in pairs, 8-byte values as two words each."""
+    if t.dtype in (torch.int32, torch.float32):
+        return t
+    return t.view(torch.int32)
 
 
 def _sync(dev):
@@ -94,45 +107,190 @@ def _sync(dev):
         torch.cuda.synchronize(dev)
 
 
+class CollectiveTransport:
+    """Rows exchanged by torch.distributed all-to-all (NCCL between GPUs, gloo on CPU)."""
+    name = "collective"
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def dispatch(self, rows: torch.Tensor, plan: ExchangePlan, counts_all) -> torch.Tensor:
+        recv = torch.empty((sum(plan.recv_splits), rows.shape[1]), dtype=rows.dtype, device=rows.device)
+        dist.all_to_all_single(_words(recv), _words(rows.contiguous()), plan.recv_splits, plan.send_splits,
+                               group=self.group)
+        return recv
+
+    def back(self, y_recv: torch.Tensor, plan: ExchangePlan, counts_all, y: torch.Tensor) -> None:
+        sent = sum(plan.send_splits)
+        dist.all_to_all_single(_words(y[:sent]), _words(y_recv), plan.send_splits, plan.recv_splits,
+                               group=self.group)
+
+
+def peer_offsets(counts_all, rank: int):
+    """Where rank `rank`'s copies go, from every rank's per-expert counts [G, E]:
+    (send, back), each a list over the other ranks d of (source row, destination row,
+    rows).  send: rank's rows for d's experts (a range of its x_perm) land in d's
+    receive buffer after the rows of the sources before it -- the all-to-all's
+    receive order.  back: the outputs of the rows rank received from d go back into
+    d's return buffer at the position of that range in d's own x_perm."""
+    counts_all = np.asarray(counts_all, dtype=np.int64)
+    G, E = counts_all.shape
+    L = E // G
+    per_pair = counts_all.reshape(G, G, L).sum(axis=2)          # [source, destination] rows
+    send_start = np.concatenate([np.zeros((G, 1), np.int64), np.cumsum(per_pair, axis=1)], axis=1)
+    recv_start = np.concatenate([np.zeros((1, G), np.int64), np.cumsum(per_pair, axis=0)], axis=0)
+    send = [(int(send_start[rank, d]), int(recv_start[rank, d]), int(per_pair[rank, d])) for d in range(G)]
+    back = [(int(recv_start[d, rank]), int(send_start[d, rank]), int(per_pair[d, rank])) for d in range(G)]
+    return send, back
+
+
+class PeerCopyTransport:
+    """Rows exchanged by copies into the other ranks' buffers.
+
+    Each rank holds a receive buffer (capacity: every rank's rows, G * max_rows) and a
+    return buffer (its own rows, max_rows), shared with the other ranks once through
+    `peers`.  dispatch: each rank copies its row range for rank d into d's receive
+    buffer at that range's place in the all-to-all order; after `peers.fence()` (this
+    rank's copies have completed, then a barrier) the receive buffer holds what an
+    all-to-all would have delivered.  back: the same, with the outputs into the
+    senders' return buffers.  A rank's buffers are overwritten by the others only
+    after the next fence, by which time its own reads of the previous step have
+    completed (its stream is synchronised before it enters the barrier)."""
+    name = "peer_copy"
+
+    def __init__(self, peers, max_rows: int, words_in: int, words_out: int):
+        self.peers = peers
+        G = peers.world
+        self.max_rows = max_rows
+        self.recv_buf = peers.alloc(G * max_rows, words_in)
+        self.back_buf = peers.alloc(max_rows, words_out)
+        self.recv_peer = peers.share(self.recv_buf)
+        self.back_peer = peers.share(self.back_buf)
+
+    def dispatch(self, rows: torch.Tensor, plan: ExchangePlan, counts_all) -> torch.Tensor:
+        send, _ = peer_offsets(counts_all, self.peers.rank)
+        w = _words(rows.contiguous())
+        if w.shape[0] > self.max_rows or w.shape[1] != self.recv_buf.shape[1]:
+            raise ValueError("rows exceed the peer buffers")
+        for d, (src, dst, n) in enumerate(send):
+            if n:
+                self.peers.copy(self.recv_peer[d], dst, w[src:src + n])
+        self.peers.fence()
+        n_recv = sum(plan.recv_splits)
+        return self.recv_buf[:n_recv].view(rows.dtype)
+
+    def back(self, y_recv: torch.Tensor, plan: ExchangePlan, counts_all, y: torch.Tensor) -> None:
+        _, back = peer_offsets(counts_all, self.peers.rank)
+        w = _words(y_recv.contiguous())
+        if w.shape[1] != self.back_buf.shape[1]:
+            raise ValueError("output rows do not match the return buffer")
+        for d, (src, dst, n) in enumerate(back):
+            if n:
+                self.peers.copy(self.back_peer[d], dst, w[src:src + n])
+        self.peers.fence()
+        sent = sum(plan.send_splits)
+        _words(y)[:sent].copy_(self.back_buf[:sent])
+
+    def close(self):
+        self.peers.close()
+
+
+class CudaPeers:
+    """Peer buffers on the GPUs of one node: buffers exported once through CUDA IPC
+    (moe_ipc_export / moe_ipc_import), rows moved by moe_copy_async on the current
+    stream, and a fence = this rank's stream synchronised, then a barrier of the
+    group.  A rank's own buffer is used directly."""
+
+    def __init__(self, group=None, device=None):
+        from expert_ffn_layer_moe_b200 import moe
+        self.moe = moe
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.device = device or torch.device("cuda", torch.cuda.current_device())
+        self.bases = {}  # (rank, handle) -> the imported allocation's base pointer (one mapping each)
+
+    def alloc(self, rows: int, words: int) -> torch.Tensor:
+        return torch.empty((max(1, rows), words), dtype=torch.int32, device=self.device)
+
+    def share(self, buf: torch.Tensor):
+        """-> for every rank, (pointer, row bytes) of its buffer as this process sees it."""
+        mine = self.moe.moe_ipc_export(buf)
+        allh = [None] * self.world
+        dist.all_gather_object(allh, mine, group=self.group)
+        rb = buf.shape[1] * buf.element_size()
+        out = []
+        for r, (h, off) in enumerate(allh):
+            if r == self.rank:
+                out.append((buf.data_ptr(), rb))
+            else:
+                # two buffers may share one allocation of the other process: map it once
+                if (r, h) not in self.bases:
+                    self.bases[(r, h)] = self.moe.moe_ipc_import(h, 0)
+                out.append((self.bases[(r, h)] + off, rb))
+        return out
+
+    def copy(self, dst, row: int, src: torch.Tensor) -> None:
+        ptr, rb = dst
+        self.moe.moe_copy_async(ptr + row * rb, src.data_ptr(), src.numel() * src.element_size())
+
+    def fence(self) -> None:
+        torch.cuda.current_stream(self.device).synchronize()
+        dist.barrier(group=self.group)
+
+    def close(self) -> None:
+        torch.cuda.current_stream(self.device).synchronize()
+        dist.barrier(group=self.group)  # no rank still copies into a mapping being closed
+        for base in self.bases.values():
+            self.moe.moe_ipc_close(base, 0)
+        self.bases = {}
+
+
 def exchange_ffn(x_perm: torch.Tensor, counts: torch.Tensor, E: int,
                  local_ffn: Callable[[torch.Tensor, torch.Tensor], torch.Tensor],
                  scatter_rows: Callable[[torch.Tensor, torch.Tensor, torch.Tensor], torch.Tensor],
-                 group=None, stats: Optional[list] = None):
+                 group=None, stats: Optional[list] = None, transport=None):
     """Steps 1-4: x_perm [R, H] (this rank's rows, sorted by expert) and counts [E] ->
     y [R, H], row r the output of x_perm[r]'s expert, computed on that expert's rank.
 
     local_ffn(x_loc, local_offsets) -> y_loc runs the local experts on expert-major rows;
-    scatter_rows(src, dst_row, dst) sets dst[dst_row[i]] = src[i].  Returns (y, plan)."""
+    scatter_rows(src, dst_row, dst) sets dst[dst_row[i]] = src[i].  transport moves the
+    rows (default: CollectiveTransport(group)).  With `stats` each phase ends with a
+    device synchronisation and its host time is recorded.  Returns (y, plan)."""
+    transport = transport or CollectiveTransport(group)
     G = dist.get_world_size(group)
     rank = dist.get_rank(group)
     dev = x_perm.device
+    timed = stats is not None
     t0 = time.perf_counter()
     gathered = [torch.empty_like(counts) for _ in range(G)]
     dist.all_gather(gathered, counts.contiguous(), group=group)
-    plan = exchange_plan(torch.stack(gathered).cpu().numpy(), rank)
+    counts_all = torch.stack(gathered).cpu().numpy()   # the step's one host read of device data
+    plan = exchange_plan(counts_all, rank)
     t1 = time.perf_counter()
     R, H = x_perm.shape
     sent = sum(plan.send_splits)  # rows with a valid expert: the first `sent` rows of x_perm
     if sent > R:
         raise ValueError("counts exceed the permuted rows")
-    recv = torch.empty((sum(plan.recv_splits), H), dtype=x_perm.dtype, device=dev)
-    dist.all_to_all_single(_words(recv), _words(x_perm[:sent].contiguous()), plan.recv_splits, plan.send_splits,
-                           group=group)
-    _sync(dev)
+    recv = transport.dispatch(x_perm[:sent], plan, counts_all)
+    if timed:
+        _sync(dev)
     t2 = time.perf_counter()
     x_loc = torch.empty_like(recv)
     scatter_rows(recv, torch.from_numpy(plan.recv_to_local).to(dev), x_loc)
     y_loc = local_ffn(x_loc, torch.from_numpy(plan.local_offsets).to(dev))
     y_recv = torch.empty_like(y_loc)
     scatter_rows(y_loc, torch.from_numpy(plan.local_to_recv).to(dev), y_recv)
-    _sync(dev)
+    if timed:
+        _sync(dev)
     t3 = time.perf_counter()
     # rows past `sent` (assignments without a valid expert) stay unwritten; the combine skips them
     y = torch.empty((R, y_loc.shape[1]), dtype=y_loc.dtype, device=dev)
-    dist.all_to_all_single(_words(y[:sent]), _words(y_recv), plan.send_splits, plan.recv_splits, group=group)
-    _sync(dev)
+    transport.back(y_recv, plan, counts_all, y)
+    if timed:
+        _sync(dev)
     t4 = time.perf_counter()
-    if stats is not None:
+    if timed:
         stats.append(EPStats(sent, int(sum(plan.recv_splits)),
                              {"plan": t1 - t0, "dispatch": t2 - t1, "experts": t3 - t2, "combine_exchange": t4 - t3}))
     return y, plan
@@ -149,11 +307,12 @@ def local_experts(W: torch.Tensor, rank: int, G: int) -> torch.Tensor:
 
 def moe_layer_forward_ep(x: torch.Tensor, W_gate: torch.Tensor, W1_local: torch.Tensor, W3_local: torch.Tensor,
                          W2_local: torch.Tensor, k: int, bias: Optional[torch.Tensor] = None, group=None,
-                         stats: Optional[list] = None, routing=None) -> torch.Tensor:
+                         stats: Optional[list] = None, routing=None, transport=None) -> torch.Tensor:
     """The MoE layer with the experts split over the ranks of `group` (NCCL, one GPU per
     rank).  x [N,H] bf16 is this rank's batch; W_gate [H,E] fp32 is the whole router;
     W1_local, W3_local [L,I,H] and W2_local [L,H,I] bf16 are this rank's experts
-    (``local_experts``).  routing = (topk_idx [N,k] int32, topk_w [N,k] fp32) replaces
+    (``local_experts``).  transport moves the rows (CollectiveTransport by default, or a
+    PeerCopyTransport over CudaPeers).  routing = (topk_idx [N,k] int32, topk_w [N,k] fp32) replaces
     the router's choice when given; an index outside [0,E) is skipped (its assignment
     adds nothing) and reported through the device error word.  Returns this rank's
     out [N,H] bf16."""
@@ -171,5 +330,6 @@ def moe_layer_forward_ep(x: torch.Tensor, W_gate: torch.Tensor, W1_local: torch.
     def ffn(x_loc, offsets_loc):
         return moe.moe_expert_ffn(x_loc, offsets_loc, W1_local, W3_local, W2_local)
 
-    y, _ = exchange_ffn(p["x_perm"], p["counts"], E, ffn, moe.moe_scatter_rows, group=group, stats=stats)
+    y, _ = exchange_ffn(p["x_perm"], p["counts"], E, ffn, moe.moe_scatter_rows, group=group, stats=stats,
+                        transport=transport)
     return moe.moe_combine(y, p["token_to_row"], w)

@@ -73,6 +73,12 @@ def lib() -> ctypes.CDLL:
         L.moe_scatter_rows.argtypes = [vp, vp, i64, c_int, vp, i64, vp]
         L.moe_set_gather_mode.argtypes = [c_int]
         L.moe_set_gather_mode.restype = c_int
+        L.moe_ipc_export.argtypes = [vp, vp, ctypes.POINTER(sz)]
+        L.moe_ipc_import.argtypes = [vp, sz, ctypes.POINTER(vp)]
+        L.moe_ipc_close.argtypes = [vp, sz]
+        L.moe_copy_async.argtypes = [vp, vp, sz, vp]
+        for fn in ("moe_ipc_export", "moe_ipc_import", "moe_ipc_close", "moe_copy_async"):
+            getattr(L, fn).restype = c_int
         for fn in ("moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
                    "moe_layer_forward_ex", "moe_get_device_error", "moe_quantize_fp8", "moe_expert_ffn_fp8",
                    "moe_layer_forward_fp8_ex", "moe_expert_ffn_w8a8", "moe_layer_forward_w8a8_ex",
@@ -110,6 +116,36 @@ def moe_workspace_bytes(N: int, H: int, I: int, E: int, k: int, Is: int = 0) -> 
 
 def moe_device_sm_count() -> int:
     return int(lib().moe_device_sm_count())
+
+
+MOE_IPC_HANDLE_BYTES = 64
+
+
+def moe_ipc_export(t: torch.Tensor):
+    """-> (handle bytes, byte offset) naming the device memory of tensor t for
+    another process (moe_ipc_import)."""
+    h = ctypes.create_string_buffer(MOE_IPC_HANDLE_BYTES)
+    off = ctypes.c_size_t(0)
+    _check("moe_ipc_export", lib().moe_ipc_export(_p(t), h, ctypes.byref(off)))
+    return h.raw, int(off.value)
+
+
+def moe_ipc_import(handle: bytes, offset: int) -> int:
+    """Another process's exported buffer -> a device pointer (int) in this process."""
+    ptr = ctypes.c_void_p(0)
+    _check("moe_ipc_import", lib().moe_ipc_import(ctypes.create_string_buffer(handle, MOE_IPC_HANDLE_BYTES),
+                                                  offset, ctypes.byref(ptr)))
+    return int(ptr.value)
+
+
+def moe_ipc_close(ptr: int, offset: int) -> None:
+    _check("moe_ipc_close", lib().moe_ipc_close(ctypes.c_void_p(ptr), offset))
+
+
+def moe_copy_async(dst_ptr: int, src_ptr: int, nbytes: int, stream=None) -> None:
+    """nbytes from device pointer src_ptr to device pointer dst_ptr (ints), async."""
+    _check("moe_copy_async", lib().moe_copy_async(ctypes.c_void_p(dst_ptr), ctypes.c_void_p(src_ptr), nbytes,
+                                                  _s(stream)))
 
 
 MOE_GATHER_AUTO, MOE_GATHER_OFF, MOE_GATHER_ON = 0, 1, 2

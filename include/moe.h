@@ -331,6 +331,33 @@ MOE_API moe_status_t moe_get_device_error(void *stream, int32_t *code);
 MOE_API int moe_device_sm_count(void);
 
 /*
+ * Buffers shared between processes, and device-to-device copies, for the
+ * expert-parallel layer's own row exchange ([MoE-latency] "跨 GPU 时,激活要出门":
+ * a token whose expert lives on another GPU sends its activation row there and
+ * gets the expert's output back).  A rank exports its receive buffers once; the
+ * other ranks import them and copy rows straight into them, one copy per
+ * contiguous range.  Nothing here waits on another process: the caller orders the
+ * ranks (each rank's copies complete, then a host-side barrier).
+ *
+ * moe_ipc_export: ptr, a device pointer inside an allocation made by cudaMalloc
+ *   (the caching allocator of PyTorch makes such allocations) -> handle, the
+ *   allocation's IPC handle (MOE_IPC_HANDLE_BYTES bytes, caller-owned), and offset,
+ *   the byte offset of ptr inside it.  MOE_ERR_UNSUPPORTED for memory the IPC API
+ *   cannot share (e.g. virtual-memory mappings).
+ * moe_ipc_import: (handle, offset) from another process on the same node -> *ptr,
+ *   this process's pointer to the same bytes (valid until moe_ipc_close).  A handle
+ *   cannot be imported by the process that exported it.  MOE_ERR_CUDA on failure.
+ * moe_ipc_close: releases an imported mapping (ptr and offset as imported).
+ * moe_copy_async: bytes from src to dst, both device pointers (either may be an
+ *   imported peer pointer), asynchronous on stream.
+ */
+#define MOE_IPC_HANDLE_BYTES 64
+MOE_API moe_status_t moe_ipc_export(const void *ptr, void *handle, size_t *offset);
+MOE_API moe_status_t moe_ipc_import(const void *handle, size_t offset, void **ptr);
+MOE_API moe_status_t moe_ipc_close(void *ptr, size_t offset);
+MOE_API moe_status_t moe_copy_async(void *dst, const void *src, size_t bytes, void *stream);
+
+/*
  * How the bf16 layer calls (moe_layer_forward, moe_layer_forward_ex) feed the
  * W1/W3 GEMM its token rows.  The pages' dispatch copies every assignment's row
  * into expert order ([MoE-latency] "router 之后还有一串动作": the permutation, and

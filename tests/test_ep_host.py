@@ -168,3 +168,123 @@ def test_exchange_skips_rows_without_an_expert():
         assert torch.equal(y[:4], x[:4].to(torch.float64) * 2)
     finally:
         dist.destroy_process_group()
+
+
+def test_peer_offsets_follow_the_all_to_all_order():
+    counts = np.array([[1, 2, 0, 3],    # rank 0's rows per expert (rank 0: experts 0,1; rank 1: 2,3)
+                       [2, 0, 1, 1]])   # rank 1's
+    send0, back0 = ep.peer_offsets(counts, 0)
+    send1, back1 = ep.peer_offsets(counts, 1)
+    # rank 0 sends rows [0,3) to itself at row 0 and rows [3,6) to rank 1 at row 0
+    assert send0 == [(0, 0, 3), (3, 0, 3)]
+    # rank 1 sends rows [0,2) to rank 0 after rank 0's own 3 rows, rows [2,4) to itself after rank 0's 3
+    assert send1 == [(0, 3, 2), (2, 3, 2)]
+    # outputs go back to where the rows came from: rank 0 returns rows [3,5) of what it got to rank 1 row 0
+    assert back0 == [(0, 0, 3), (3, 0, 2)]
+    assert back1 == [(0, 3, 3), (3, 2, 2)]
+
+
+class MemmapPeers:
+    """Stand-in for CudaPeers on CPU: each rank's buffers are files mapped by every rank
+    (the 'handle' is the path), copies write into the mapping, and the fence flushes
+    and meets the others at a gloo barrier -- the same protocol without a GPU."""
+
+    def __init__(self, root, tag):
+        import torch.distributed as dist
+        self.dist = dist
+        self.world, self.rank = dist.get_world_size(), dist.get_rank()
+        self.root, self.tag, self.n = root, tag, 0
+        self.maps = {}
+
+    def alloc(self, rows, words):
+        import torch
+        path = os.path.join(self.root, f"{self.tag}_r{self.rank}_b{self.n}.bin")
+        self.n += 1
+        mm = np.memmap(path, dtype=np.int32, mode="w+", shape=(max(1, rows), words))
+        self.maps[path] = mm
+        return torch.from_numpy(mm)
+
+    def share(self, buf):
+        path = next(p for p, m in self.maps.items() if m.ctypes.data == buf.data_ptr())
+        paths = [None] * self.world
+        self.dist.all_gather_object(paths, (path, buf.shape))
+        return paths
+
+    def copy(self, dst, row, src):
+        path, shape = dst
+        if path not in self.maps:
+            self.maps[path] = np.memmap(path, dtype=np.int32, mode="r+", shape=tuple(shape))
+        self.maps[path][row:row + src.shape[0]] = src.numpy()
+
+    def fence(self):
+        for m in self.maps.values():
+            m.flush()
+        self.dist.barrier()
+
+    def close(self):
+        self.dist.barrier()
+
+
+def _rank_main_peer(rank, world, port, root, q):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from expert_ffn_layer_moe_b200.inputs import MoEConfig, make_inputs
+    from tests._bf16 import to_u16
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    cfg = MoEConfig("ep", N=20, H=64, I=32, E=2 * world, k=2)
+    wts = make_inputs(cfg, seed=1)
+    W1, W3, W2 = (to_u16(wts[n]) for n in ("W1", "W3", "W2"))
+    L = cfg.E // world
+    mine = slice(rank * L, (rank + 1) * L)
+
+    def ffn(x_loc, offsets):
+        return torch.from_numpy(oracle.expert_ffn(x_loc.numpy().view(np.uint16), offsets.numpy(), W1[mine],
+                                                  W3[mine], W2[mine]))
+
+    def scatter(src, dst_row, dst):
+        dst[dst_row.long()] = src
+        return dst
+
+    # rows travel as 32-bit words: bf16 x rows are H/2 words, the oracle's fp64 outputs 2H
+    tr = ep.PeerCopyTransport(MemmapPeers(root, "t"), max_rows=cfg.N * cfg.k, words_in=cfg.H // 2,
+                              words_out=2 * cfg.H)
+    ok = True
+    for step in range(3):  # the buffers are reused from step to step
+        x = to_u16(make_inputs(cfg, seed=20 + 7 * rank + step, weights=False)["x"])
+        l32 = oracle.router_logits(x, wts["W_gate"].numpy()).astype(np.float32)
+        idx, w = oracle.topk(l32, cfg.k)
+        counts, _, r2t, t2r = oracle.dispatch(idx, cfg.E)
+        xp = torch.from_numpy(oracle.permute_rows(x, r2t).view(np.int16))   # bf16 rows as their bits
+        y_p, _ = ep.exchange_ffn(xp, torch.from_numpy(counts), cfg.E, ffn, scatter, transport=tr)
+        y_c, _ = ep.exchange_ffn(xp, torch.from_numpy(counts), cfg.E, ffn, scatter)
+        out = oracle.combine(y_p.numpy(), t2r, w)
+        ref = oracle.layer_given_logits(x, l32, W1, W3, W2, cfg.k)
+        ok = ok and bool(np.array_equal(out, ref)) and torch.equal(y_p, y_c)
+    tr.close()
+    dist.destroy_process_group()
+    q.put((rank, ok))
+
+
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("world", [2, 3])
+def test_peer_copy_exchange_equals_the_all_to_all(world, tmp_path):
+    """The peer-copy transport, its buffers reused over three steps on gloo ranks with
+    file-mapped stand-ins for the GPUs' shared buffers: bit-identical expert outputs to
+    the all-to-all, and every rank's layer equals the one-device oracle layer."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_peer, args=(r, world, port, str(tmp_path), q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=200) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(r[1] for r in res), res

@@ -111,3 +111,103 @@ def test_ep_layer_skips_an_out_of_range_expert_index():
         assert_close(dec(host(out)), dec(ref), "ep out with skipped picks")
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("transport", ["collective", "peer_copy"])
+def test_ep_layer_one_rank_both_transports(transport):
+    """A one-rank NCCL group with either transport (the peer copies then go into the
+    rank's own buffers): same bits as each other and the oracle's layer."""
+    cfg = MoEConfig("ep1_tr", N=200, H=256, I=192, E=8, k=2)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_port()}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        t = cuda_inputs(cfg, seed=13)
+        tr = None
+        if transport == "peer_copy":
+            tr = ep.PeerCopyTransport(ep.CudaPeers(), max_rows=cfg.N * cfg.k, words_in=cfg.H // 2, words_out=cfg.H)
+        outs = []
+        for _ in range(2):  # the second step reuses the transport's buffers
+            outs.append(ep.moe_layer_forward_ep(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k,
+                                                transport=tr))
+        if tr is not None:
+            tr.close()
+        logits = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device="cuda")
+        moe.moe_route(t["x"], t["W_gate"], cfg.k, logits=logits)
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error() == 0
+        assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+        ref = oracle.layer_given_logits(host(t["x"]), host(logits), host(t["W1"]), host(t["W3"]), host(t["W2"]),
+                                        cfg.k)
+        assert_close(dec(host(outs[0])), dec(ref), f"ep {transport}")
+    finally:
+        dist.destroy_process_group()
+
+
+def _two_process_rank(rank, port, q):
+    """One of two processes on the same GPU: gloo for the host-side plan and barriers,
+    the rows moved by the library's copies into the other process's IPC-mapped buffers.
+    The processes never wait on each other on the device."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from expert_ffn_layer_moe_b200 import ep, moe
+    from expert_ffn_layer_moe_b200.inputs import MoEConfig, make_inputs
+    from tests._bf16 import to_u16
+    try:
+        torch.cuda.set_device(0)
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=2,
+                                timeout=datetime.timedelta(seconds=60))
+        cfg = MoEConfig("ep2", N=96, H=256, I=128, E=8, k=2)
+        w = make_inputs(cfg, seed=3)
+        x = make_inputs(cfg, seed=40 + rank, weights=False)["x"].cuda()
+        Wg = w["W_gate"].cuda()
+        W1, W3, W2 = (ep.local_experts(w[n], rank, 2).contiguous().cuda() for n in ("W1", "W3", "W2"))
+        idx, wt, _ = moe.moe_route(x, Wg, cfg.k)
+        p = moe.moe_permute(x, idx, cfg.E)
+
+        def ffn(x_loc, offs):
+            return moe.moe_expert_ffn(x_loc, offs, W1, W3, W2)
+
+        tr = ep.PeerCopyTransport(ep.CudaPeers(), max_rows=cfg.N * cfg.k, words_in=cfg.H // 2, words_out=cfg.H)
+        outs = []
+        for _ in range(2):
+            y, _ = ep.exchange_ffn(p["x_perm"], p["counts"].cpu(), cfg.E, ffn, moe.moe_scatter_rows, transport=tr)
+            outs.append(moe.moe_combine(y, p["token_to_row"], wt))
+        tr.close()
+        torch.cuda.synchronize()
+        err = moe.moe_get_device_error()
+        logits = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device="cuda")
+        moe.moe_route(x, Wg, cfg.k, logits=logits)
+        ref = oracle.layer_given_logits(to_u16(x.cpu()), logits.cpu().numpy(), to_u16(w["W1"]), to_u16(w["W3"]),
+                                        to_u16(w["W2"]), cfg.k)
+        same = bool(torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16)))
+        g = to_u16(outs[0].cpu())
+        from tests._bf16 import dec
+        a, b = dec(g), dec(ref)
+        close = bool(np.all(np.abs(a - b) <= 2e-2 * np.abs(b) + 2e-3))
+        dist.destroy_process_group()
+        q.put((rank, err, same, close, None))
+    except Exception as e:  # report instead of hanging the parent
+        q.put((rank, -1, False, False, repr(e)))
+
+
+def test_ep_two_processes_on_one_gpu_peer_copies():
+    """Two ranks as two processes sharing one GPU: the peer-copy transport's buffers
+    are exported and imported through CUDA IPC (a process cannot import its own
+    handle, so this is the only way one GPU exercises the import), rows move by
+    moe_copy_async, and the ranks meet only at host barriers.  Each rank's layer must
+    match the oracle and repeat bit for bit."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_two_process_rank, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert all(r[4] is None for r in res), res
+    assert all(r[1] == 0 and r[2] and r[3] for r in res), res
