@@ -265,13 +265,25 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
     const int64_t R = N * k;
 
     MOE_TRY(record(phase_events, 0, s));
-    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
-    MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
     moe::GroupedGemmArgs a{};
     a.offsets = offsets; a.groups = E; a.R = R;
     a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
     set_weights13(&a, X);
-    if (X.a8) {
+    const bool gather = !X.a8 && !X.fp8 && moe::layer_gathers(N, k, H);
+    // a small batch: router, top-k, dispatch and the row copies in two kernels (the
+    // route phase then holds the permute phase's work too)
+    cudaError_t fused = cudaErrorNotSupported;
+    if (!X.a8 && !gather) {
+        fused = moe::launch_route_dispatch_small(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router,
+                                                 L.router_bytes, counts, offsets, r2t, t2r, x_perm, err, s);
+        if (fused != cudaSuccess && fused != cudaErrorNotSupported) return cuda_fail(fused);
+    }
+    if (fused != cudaSuccess)
+        MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
+    MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
+    if (fused == cudaSuccess) {
+        a.act = x_perm;
+    } else if (X.a8) {
         // each token row is quantized once (N rows, not N*k: a permuted row is a copy of
         // its token's row, so its codes and scale are the same), then the codes and the
         // scales move to the permuted rows
@@ -280,7 +292,7 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
         MOE_CUDA(moe::launch_scatter_rows(reinterpret_cast<const uint16_t *>(Q.xqt), Q.xst, t2r, N, k, H / 2,
                                           reinterpret_cast<uint16_t *>(Q.xq), R, Q.xsc, s));
         a.act = Q.xq; a.a8 = true; a.scale_act = Q.xsc;
-    } else if (!X.fp8 && moe::layer_gathers(N, k, H)) {
+    } else if (gather) {
         // dispatch only: W1/W3 gathers its rows from x through row_to_token
         MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
         a.act = x; a.gather_rows = r2t; a.gather_src_rows = N;

@@ -50,6 +50,15 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
                           int H, int E, int k, float *logits, int32_t *topk_idx, float *topk_w,
                           void *ws, size_t ws_bytes, int *dev_err, cudaStream_t s);
 
+// Router, dispatch and row scatter of a small batch (N*k <= 512) in two kernels: the
+// router's logits (or its one-kernel form with the picks), then top-k, the stable
+// dispatch and the rows in one.  Same outputs as launch_router followed by
+// launch_permute.  cudaErrorNotSupported (nothing launched) for other shapes.
+cudaError_t launch_route_dispatch_small(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H,
+                                        int E, int k, float *logits, int32_t *topk_idx, float *topk_w, void *ws,
+                                        size_t ws_bytes, int32_t *counts, int32_t *offsets, int32_t *row_to_token,
+                                        int32_t *token_to_row, uint16_t *x_perm, int *dev_err, cudaStream_t s);
+
 // Dispatch / permutation.  `scratch` holds permute_scratch_ints(R, E) ints.
 constexpr int kPermuteChunk = 1024;  // assignments per block in the count/rank passes
 inline int64_t permute_blocks(int64_t R) { return (R + kPermuteChunk - 1) / kPermuteChunk; }

@@ -17,14 +17,15 @@
 // Batches of at most kSmallR assignments (decode) do 1-3 in one single-block
 // launch, then the gather: two launches instead of four.
 #include "common.cuh"
+#include "dispatch_block.cuh"
 #include "internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kMaxE = 256;
+constexpr int kThreads = kDispThreads;
+constexpr int kWarps = kDispWarps;
+constexpr int kMaxE = kDispMaxE;
 constexpr int64_t kSmallR = 2048;  // one-block dispatch up to this many assignments
 static_assert(kPermuteChunk % kThreads == 0, "chunk is whole rounds of the block");
 
@@ -81,83 +82,15 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// One round of the stable rank: kThreads consecutive assignments starting at a0,
-// placed after base[e] rows of their expert; advances base.  Block-wide.
-__device__ __forceinline__ void rank_round(const int32_t *__restrict__ idx, int64_t R, int k, int E, int64_t a0,
-                                           int *base, int (*wcnt)[kMaxE], int32_t *__restrict__ row_to_token,
-                                           int32_t *__restrict__ token_to_row)
-{
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int i = threadIdx.x; i < kWarps * E; i += kThreads) wcnt[i / E][i % E] = 0;
-    __syncthreads();
-    const int64_t a = a0 + threadIdx.x;
-    int e = -1;
-    if (a < R) e = idx[a];
-    const bool valid = a < R && e >= 0 && e < E;
-    // lanes with equal keys form one group; invalid lanes get a key of their own
-    const int key = valid ? e : (kMaxE + lane);
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    const int rank_in_warp = __popc(peers & lt_mask);
-    if (valid && rank_in_warp == 0) wcnt[warp][e] = __popc(peers);
-    __syncthreads();
-    if (a < R) {
-        if (valid) {
-            int before = 0;
-            for (int w = 0; w < warp; ++w) before += wcnt[w][e];
-            const int row = base[e] + before + rank_in_warp;
-            row_to_token[row] = (int32_t)(a / k);
-            token_to_row[a] = row;
-        } else {
-            token_to_row[a] = -1;
-        }
-    }
-    __syncthreads();
-    for (int ee = threadIdx.x; ee < E; ee += kThreads) {
-        int add = 0;
-        for (int w = 0; w < kWarps; ++w) add += wcnt[w][ee];
-        base[ee] += add;
-    }
-    __syncthreads();
-}
-
 // Small batches: histogram, exclusive scan and stable ranks in one block.
 __global__ void __launch_bounds__(kThreads)
     dispatch_small_kernel(const int32_t *__restrict__ idx, int64_t R, int k, int E, int32_t *__restrict__ counts,
                           int32_t *__restrict__ offsets, int32_t *__restrict__ row_to_token,
                           int32_t *__restrict__ token_to_row, int *err)
 {
-    __shared__ int base[kMaxE];
-    __shared__ int scan[kThreads];
-    __shared__ int wcnt[kWarps][kMaxE];
+    __shared__ DispatchSmem sm;
     pdl_entry();
-    const int tid = threadIdx.x;
-    if (tid < E) base[tid] = 0;
-    __syncthreads();
-    for (int64_t a = tid; a < R; a += kThreads) {
-        const int e = idx[a];
-        if (e >= 0 && e < E) atomicAdd(&base[e], 1);
-        else set_device_error(err, MOE_DEVERR_BAD_EXPERT_INDEX);
-    }
-    __syncthreads();
-    const int c = tid < E ? base[tid] : 0;
-    scan[tid] = c;
-    __syncthreads();
-    for (int o = 1; o < kThreads; o <<= 1) {  // inclusive scan
-        const int v = tid >= o ? scan[tid - o] : 0;
-        __syncthreads();
-        scan[tid] += v;
-        __syncthreads();
-    }
-    if (tid < E) {
-        counts[tid] = c;
-        offsets[tid] = scan[tid] - c;
-        if (tid == E - 1) offsets[E] = scan[tid];
-        base[tid] = scan[tid] - c;
-    }
-    __syncthreads();
-    for (int64_t a0 = 0; a0 < R; a0 += kThreads)
-        rank_round(idx, R, k, E, a0, base, wcnt, row_to_token, token_to_row);
+    dispatch_block(idx, R, k, E, counts, offsets, row_to_token, token_to_row, err, sm);
 }
 
 __global__ void __launch_bounds__(kThreads)

@@ -29,7 +29,9 @@
 //    stride apart) in a fixed order.
 // All reductions run in a fixed order: the logits' bits do not depend on timing.
 #include "common.cuh"
+#include "dispatch_block.cuh"
 #include "internal.h"
+#include "topk_warp.cuh"
 
 namespace moe {
 namespace {
@@ -129,67 +131,6 @@ __device__ __forceinline__ void warp_sum_store(const float (&acc)[TT][kEC], int 
             const int t = f / kEC, j = f % kEC;
             if (j < ne) out[t * tstride + j] = v[r];
         }
-    }
-}
-
-// Top-k of one token's E logits (in `row`) on one warp; lane 0 writes the picks
-// and their weights.
-__device__ __forceinline__ void topk_warp(const float *row, int E, int k, int lane, int32_t *__restrict__ idx_out,
-                                          float *__restrict__ w_out)
-{
-    constexpr int kPer = kMaxE / 32;
-    float v[kPer];
-    bool taken[kPer];
-#pragma unroll
-    for (int m = 0; m < kPer; ++m) {
-        const int e = lane + 32 * m;
-        v[m] = e < E ? row[e] : 0.f;
-        taken[m] = e >= E;
-    }
-    float pv[kMaxK];
-    int pi[kMaxK];
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-        if (j >= k) break;
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int m = 0; m < kPer; ++m) {
-            const int e = lane + 32 * m;
-            if (!taken[m] && (v[m] > bv || (v[m] == bv && e < bi))) { bv = v[m]; bi = e; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if (bi == 0x7fffffff) {  // only NaN left: take the lowest free index
-            int lo = 0x7fffffff;
-#pragma unroll
-            for (int m = 0; m < kPer; ++m)
-                if (!taken[m]) lo = min(lo, lane + 32 * m);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            bi = lo;
-            bv = row[bi];
-        }
-#pragma unroll
-        for (int m = 0; m < kPer; ++m)
-            if (lane + 32 * m == bi) taken[m] = true;
-        pv[j] = bv;
-        pi[j] = bi;
-    }
-    if (lane == 0) {
-        const float l0 = pv[0];
-        float ex[kMaxK];
-        float den = 0.f;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j < k) { ex[j] = expf(pv[j] - l0); den += ex[j]; }
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j < k) { idx_out[j] = pi[j]; w_out[j] = ex[j] / den; }
     }
 }
 
@@ -300,6 +241,91 @@ cudaError_t launch_topk(const float *lin, int64_t pstride, int64_t tstride, cons
 {
     return launch_pdl(router_topk_kernel<P>, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, lin,
                       pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
+}
+
+// Small batches: the top-k of every token (from P partial logits, summed as the top-k
+// kernel sums them -- or, with P == 0, the picks the router already made), the stable
+// dispatch and the row scatter in one kernel.  Every block ranks and dispatches the
+// whole batch in its own shared memory (a few hundred assignments: repeating that costs
+// less than a launch) and then copies the rows of its share of the tokens; block 0 also
+// writes the routing and dispatch outputs.  No block waits on another.
+constexpr int kFuseMaxR = 512;      // assignments of a batch this kernel takes
+constexpr int kFuseMaxTopkN = 64;   // tokens every block ranks for itself (P > 0)
+template <int P>
+__global__ void __launch_bounds__(kDispThreads)
+    route_dispatch_small_kernel(const float *__restrict__ lin, int64_t pstride, int64_t tstride,
+                                const float *__restrict__ bias, int64_t N, int E, int k, float *__restrict__ logits,
+                                int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                                const uint16_t *__restrict__ x, int H, int32_t *__restrict__ counts,
+                                int32_t *__restrict__ offsets, int32_t *__restrict__ row_to_token,
+                                int32_t *__restrict__ token_to_row, uint16_t *__restrict__ x_perm, int *err)
+{
+    static_assert(kDispThreads == kThreads, "one block size for the ranking and the dispatch");
+    __shared__ DispatchSmem sm;
+    __shared__ int32_t s_idx[kFuseMaxR];
+    __shared__ float s_w[kFuseMaxR];
+    __shared__ int32_t s_t2r[kFuseMaxR];
+    __shared__ float row[P > 0 ? kWarps : 1][kMaxE];
+    pdl_entry();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t R = N * k;
+    const bool lead = blockIdx.x == 0;
+    if (P > 0) {
+        for (int64_t t = warp; t < N; t += kWarps) {
+            for (int e = lane; e < E; e += 32) {
+                const float *p = lin + t * tstride + e;
+                float part[P > 0 ? P : 1];
+#pragma unroll
+                for (int i = 0; i < P; ++i) part[i] = p[i * pstride];
+                float v = part[0];
+#pragma unroll
+                for (int i = 1; i < P; ++i) v += part[i];
+                if (bias) v += bias[e];
+                if (logits && lead) logits[t * E + e] = v;
+                row[warp][e] = v;
+            }
+            __syncwarp();
+            topk_warp(row[warp], E, k, lane, s_idx + t * k, s_w + t * k);
+            __syncwarp();
+        }
+        __syncthreads();
+        if (lead)
+            for (int64_t a = threadIdx.x; a < R; a += kDispThreads) {
+                topk_idx[a] = s_idx[a];
+                topk_w[a] = s_w[a];
+            }
+    } else {
+        for (int64_t a = threadIdx.x; a < R; a += kDispThreads) s_idx[a] = topk_idx[a];
+        __syncthreads();
+    }
+    dispatch_block(s_idx, R, k, E, lead ? counts : nullptr, lead ? offsets : nullptr,
+                   lead ? row_to_token : nullptr, s_t2r, lead ? err : nullptr, sm);
+    if (lead)
+        for (int64_t a = threadIdx.x; a < R; a += kDispThreads) token_to_row[a] = s_t2r[a];
+    // x_perm[token_to_row[t,j]] = x[t] for this block's tokens t (16-byte vectors)
+    const int nvec = H / 8;
+    for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
+        for (int v = threadIdx.x; v < nvec; v += kDispThreads) {
+            const uint4 val = __ldg(src + v);
+            for (int j = 0; j < k; ++j) {
+                const int r = s_t2r[t * k + j];
+                if (r >= 0) reinterpret_cast<uint4 *>(x_perm + (int64_t)r * H)[v] = val;
+            }
+        }
+    }
+}
+
+template <int P>
+cudaError_t launch_route_dispatch(const float *lin, int64_t pstride, int64_t tstride, const float *bias, int64_t N,
+                                  int E, int k, float *logits, int32_t *topk_idx, float *topk_w, const uint16_t *x,
+                                  int H, int32_t *counts, int32_t *offsets, int32_t *r2t, int32_t *t2r,
+                                  uint16_t *x_perm, int *err, cudaStream_t s)
+{
+    const int64_t cap = 2 * (int64_t)device_sm_count();
+    const unsigned grid = (unsigned)(N < cap ? N : cap);
+    return launch_pdl(route_dispatch_small_kernel<P>, dim3(grid), dim3(kDispThreads), 0, s, lin, pstride, tstride,
+                      bias, N, E, k, logits, topk_idx, topk_w, x, H, counts, offsets, r2t, t2r, x_perm, err);
 }
 
 // kTensor: W_gate [H,E] fp32 -> three bf16 terms, stacked K-major as [3E, H]:
@@ -440,6 +466,60 @@ RouterPath router_path(int64_t N, int E, bool have_logits_buffer, bool have_ws)
     if (have_ws && N >= 256 && N * (int64_t)E >= 32768) return RouterPath::kTensor;
     if (have_logits_buffer || have_ws) return RouterPath::kSplit;
     return RouterPath::kFused;
+}
+
+cudaError_t launch_route_dispatch_small(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H,
+                                        int E, int k, float *logits, int32_t *topk_idx, float *topk_w, void *ws,
+                                        size_t ws_bytes, int32_t *counts, int32_t *offsets, int32_t *row_to_token,
+                                        int32_t *token_to_row, uint16_t *x_perm, int *dev_err, cudaStream_t s)
+{
+    if (N <= 0 || N * (int64_t)k > kFuseMaxR) return cudaErrorNotSupported;
+    const bool have_ws = ws != nullptr && ws_bytes >= router_ws_bytes(N, H, E);
+    const RouterPath path = router_path(N, E, logits != nullptr, have_ws);
+    if (path == RouterPath::kTensor) return cudaErrorNotSupported;
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    const size_t split_bytes = align256((size_t)3 * E * H * 2);
+    const size_t parts_bytes = align256((size_t)kTensorMaxSlices * N * 3 * E * 4);
+    float *lbuf = logits ? logits : (have_ws ? reinterpret_cast<float *>(w8 + split_bytes + parts_bytes) : nullptr);
+    if (path == RouterPath::kSplit) {
+        float *part = have_ws ? reinterpret_cast<float *>(w8) : lbuf;
+        const int64_t zcap = have_ws ? (int64_t)((split_bytes + parts_bytes) / ((size_t)N * E * 4)) : 1;
+        int tt, z;
+        split_shape(N, H, E, zcap, &tt, &z);
+        if (!(z == 1 && E <= 2 * kEC)) {
+            if (N > kFuseMaxTopkN) return cudaErrorNotSupported;
+            if (z == 1) part = lbuf;
+            const int hz = (H / z / kChunk) * kChunk;
+            const dim3 grid((unsigned)((N + tt - 1) / tt), (unsigned)((E + kEC - 1) / kEC), (unsigned)z);
+            cudaError_t e;
+            switch (tt) {
+                case 4: e = launch_pdl(router_partial_kernel<4>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H, E,
+                                       hz, part); break;
+                case 2: e = launch_pdl(router_partial_kernel<2>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H, E,
+                                       hz, part); break;
+                default: e = launch_pdl(router_partial_kernel<1>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H,
+                                        E, hz, part); break;
+            }
+            if (e != cudaSuccess) return e;
+            const int64_t ps = N * E;
+            switch (z) {  // z == 1: `part` holds the logits, bias included
+                case 1: return launch_route_dispatch<1>(part, ps, E, nullptr, N, E, k, nullptr, topk_idx, topk_w, x, H,
+                                                        counts, offsets, row_to_token, token_to_row, x_perm, dev_err, s);
+                case 2: return launch_route_dispatch<2>(part, ps, E, bias, N, E, k, lbuf, topk_idx, topk_w, x, H, counts,
+                                                        offsets, row_to_token, token_to_row, x_perm, dev_err, s);
+                case 4: return launch_route_dispatch<4>(part, ps, E, bias, N, E, k, lbuf, topk_idx, topk_w, x, H, counts,
+                                                        offsets, row_to_token, token_to_row, x_perm, dev_err, s);
+                case 8: return launch_route_dispatch<8>(part, ps, E, bias, N, E, k, lbuf, topk_idx, topk_w, x, H, counts,
+                                                        offsets, row_to_token, token_to_row, x_perm, dev_err, s);
+                default: return cudaErrorInvalidValue;
+            }
+        }
+    }
+    // the one-kernel router makes the picks; then the dispatch and the rows
+    cudaError_t e = launch_fused_for(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+    if (e != cudaSuccess) return e;
+    return launch_route_dispatch<0>(nullptr, 0, 0, nullptr, N, E, k, nullptr, topk_idx, topk_w, x, H, counts, offsets,
+                                    row_to_token, token_to_row, x_perm, dev_err, s);
 }
 
 size_t router_ws_bytes(int64_t N, int H, int E)

@@ -102,6 +102,11 @@ def _words(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.int32)
 
 
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    """The same bytes as int32 words per row (so copies between buffers never convert)."""
+    return t if t.dtype == torch.int32 else t.view(torch.int32)
+
+
 def _sync(dev):
     if dev.type == "cuda":
         torch.cuda.synchronize(dev)
@@ -169,7 +174,7 @@ class PeerCopyTransport:
 
     def dispatch(self, rows: torch.Tensor, plan: ExchangePlan, counts_all) -> torch.Tensor:
         send, _ = peer_offsets(counts_all, self.peers.rank)
-        w = _words(rows.contiguous())
+        w = _bits(rows.contiguous())
         if w.shape[0] > self.max_rows or w.shape[1] != self.recv_buf.shape[1]:
             raise ValueError("rows exceed the peer buffers")
         for d, (src, dst, n) in enumerate(send):
@@ -181,7 +186,7 @@ class PeerCopyTransport:
 
     def back(self, y_recv: torch.Tensor, plan: ExchangePlan, counts_all, y: torch.Tensor) -> None:
         _, back = peer_offsets(counts_all, self.peers.rank)
-        w = _words(y_recv.contiguous())
+        w = _bits(y_recv.contiguous())
         if w.shape[1] != self.back_buf.shape[1]:
             raise ValueError("output rows do not match the return buffer")
         for d, (src, dst, n) in enumerate(back):
@@ -189,7 +194,7 @@ class PeerCopyTransport:
                 self.peers.copy(self.back_peer[d], dst, w[src:src + n])
         self.peers.fence()
         sent = sum(plan.send_splits)
-        _words(y)[:sent].copy_(self.back_buf[:sent])
+        _bits(y)[:sent].copy_(self.back_buf[:sent])  # bit copy (both int32 views)
 
     def close(self):
         self.peers.close()

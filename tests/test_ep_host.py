@@ -288,3 +288,31 @@ def test_peer_copy_exchange_equals_the_all_to_all(world, tmp_path):
         p.join(timeout=60)
         assert p.exitcode == 0
     assert all(r[1] for r in res), res
+
+
+def test_peer_copy_moves_bits_of_fp32_rows(tmp_path):
+    """fp32 rows (the GPU path's expert outputs) and bf16 rows travel as raw words: the
+    return copy must not convert values.  One gloo rank, file-mapped buffers."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=30))
+    try:
+        x = torch.randn(6, 8).to(torch.bfloat16)
+        counts = torch.tensor([2, 4], dtype=torch.int32)
+
+        def ffn(x_loc, offsets):
+            return x_loc.float() * 3.0 + 0.25          # fp32 outputs with fractional bits
+
+        def scatter(src, dst_row, dst):
+            dst[dst_row.long()] = src
+            return dst
+
+        tr = ep.PeerCopyTransport(MemmapPeers(str(tmp_path), "f"), max_rows=6, words_in=4, words_out=8)
+        y, _ = ep.exchange_ffn(x, counts, 2, ffn, scatter, transport=tr)
+        tr.close()
+        assert y.dtype == torch.float32 and torch.equal(y, x.float() * 3.0 + 0.25)
+    finally:
+        dist.destroy_process_group()
