@@ -18,7 +18,9 @@ namespace moe {
 namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_gather_mode{MOE_GATHER_AUTO};
+std::atomic<int> g_microbatches{1};
 }  // namespace
+int layer_microbatches() { return g_microbatches.load(std::memory_order_relaxed); }
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 uint64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
 
@@ -141,6 +143,34 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, bool a8, WsLayout 
     L->total = off;
 }
 
+// Rows of the first micro-batch when the layer runs as two (0: it runs in one piece):
+// batches of at least kMicroMinRows assignments, when moe_set_microbatches asked for 2.
+constexpr int64_t kMicroMinRows = 32768;
+int64_t micro_split(int64_t N, int k)
+{
+    if (moe::layer_microbatches() < 2 || N * k < kMicroMinRows || N < 2) return 0;
+    return (N / 2 + 7) & ~int64_t(7);  // a multiple of 8 rows, so the second half starts 16-byte aligned
+}
+
+// Workspace of the layer: enough for the layer in one piece and for two micro-batches.
+size_t layer_ws_bytes(int64_t N, int H, int I, int E, int k, int Is, bool a8)
+{
+    WsLayout L;
+    ws_layout(N, H, I, E, k, Is, a8, &L);
+    size_t total = L.total;
+    if (N >= 2) {
+        const int64_t N0 = (N / 2 + 7) & ~int64_t(7);
+        if (N0 < N) {
+            WsLayout L0, L1;
+            ws_layout(N0, H, I, E, k, Is, a8, &L0);
+            ws_layout(N - N0, H, I, E, k, Is, a8, &L1);
+            const size_t two = round_up(L0.total) + L1.total;
+            if (two > total) total = two;
+        }
+    }
+    return total;
+}
+
 // The routed experts' weights: bf16, or e4m3 bytes with one fp32 scale per row
 // (optionally with e4m3 activations as well).
 struct Experts {
@@ -226,26 +256,16 @@ moe_status_t record(void *const *ev, int i, cudaStream_t s)
         if (st_ != MOE_OK) return st_;           \
     } while (0)
 
-moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bias, const Experts &X,
-                        const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
-                        int E, int k, int Is, uint16_t *out, float *logits, void *ws, size_t ws_bytes,
-                        void *stream, void *const *phase_events)
+// The layer on N rows with a workspace laid out for N rows; after_dispatch (nullable)
+// runs once the permute phase is enqueued on s.
+template <typename Hook>
+moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias, const Experts &X,
+                       const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I, int E,
+                       int k, int Is, uint16_t *out, float *logits, void *ws, int *err, cudaStream_t s,
+                       void *const *phase_events, Hook after_dispatch)
 {
-    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
-    if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return MOE_ERR_INVALID_ARG;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (N == 0) return MOE_OK;
-    if (!x || !W_gate || !X.W1 || !X.W3 || !X.W2 || !out) return MOE_ERR_INVALID_ARG;
-    if (Is > 0 && (!Ws1 || !Ws3 || !Ws2)) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(X.W1) || !aligned16(X.W3) || !aligned16(X.W2) || !aligned16(out))
-        return MOE_ERR_UNSUPPORTED;
-    if (Is > 0 && (!aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2))) return MOE_ERR_UNSUPPORTED;
     WsLayout L;
     ws_layout(N, H, I, E, k, Is, X.a8, &L);
-    if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
-    int *err = device_error_word();
-    if (!err) return cuda_fail(cudaGetLastError());
-
     uint8_t *base = static_cast<uint8_t *>(ws);
     const ActQ Q{base + L.xq, reinterpret_cast<float *>(base + L.xsc), base + L.hq,
                  reinterpret_cast<float *>(base + L.hsc), base + L.xqt, reinterpret_cast<float *>(base + L.xst)};
@@ -301,6 +321,7 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
         a.act = x_perm;
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
+    MOE_TRY(after_dispatch());
     MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     const int ksplit = moe::gemm2_ksplit(R, E, I, H);
     moe::GroupedGemmArgs b{};
@@ -316,6 +337,79 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
     MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r, w, sh, N, H, k, out, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_COMBINE, s));
+    return MOE_OK;
+}
+
+// A second stream and two events per device for the micro-batched layer, created on
+// first use and kept for the process; the mutex makes one layer call's fork and join
+// use them at a time.
+struct MicroStreams {
+    std::mutex mu;
+    cudaStream_t s2 = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    void *ctx = nullptr;
+};
+
+MicroStreams *micro_streams()
+{
+    static MicroStreams per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    return &per_dev[dev];
+}
+
+moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bias, const Experts &X,
+                        const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I,
+                        int E, int k, int Is, uint16_t *out, float *logits, void *ws, size_t ws_bytes,
+                        void *stream, void *const *phase_events)
+{
+    if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return MOE_ERR_INVALID_ARG;
+    if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (N == 0) return MOE_OK;
+    if (!x || !W_gate || !X.W1 || !X.W3 || !X.W2 || !out) return MOE_ERR_INVALID_ARG;
+    if (Is > 0 && (!Ws1 || !Ws3 || !Ws2)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(X.W1) || !aligned16(X.W3) || !aligned16(X.W2) || !aligned16(out))
+        return MOE_ERR_UNSUPPORTED;
+    if (Is > 0 && (!aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2))) return MOE_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < layer_ws_bytes(N, H, I, E, k, Is, X.a8) || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    int *err = device_error_word();
+    if (!err) return cuda_fail(cudaGetLastError());
+    auto none = [] { return MOE_OK; };
+    const int64_t N0 = micro_split(N, k);
+    if (N0 == 0 || phase_events)  // per-phase timing runs the layer in one piece
+        return layer_run(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, err, s,
+                         phase_events, none);
+
+    // Two micro-batches (the pages' ping-pong of micro-batches, inside one GPU): rows
+    // [0, N0) on the caller's stream, rows [N0, N) on a second stream that starts once
+    // the first has dispatched.  The first's grouped GEMMs then run beside the second's
+    // router, dispatch and row copies, and the second's GEMMs beside the first's combine:
+    // HBM-bound kernels fill the room the persistent GEMMs leave on every SM.
+    MicroStreams *ms = micro_streams();
+    if (!ms) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(ms->mu);
+    void *ctx = moe::current_context();
+    if (!ms->s2 || ctx != ms->ctx) {
+        MOE_CUDA(cudaStreamCreateWithFlags(&ms->s2, cudaStreamNonBlocking));
+        MOE_CUDA(cudaEventCreateWithFlags(&ms->fork, cudaEventDisableTiming));
+        MOE_CUDA(cudaEventCreateWithFlags(&ms->join, cudaEventDisableTiming));
+        ms->ctx = moe::current_context();
+    }
+    WsLayout L0;
+    ws_layout(N0, H, I, E, k, Is, X.a8, &L0);
+    uint8_t *ws1 = static_cast<uint8_t *>(ws) + round_up(L0.total);
+    auto fork = [&]() -> moe_status_t {
+        MOE_CUDA(cudaEventRecord(ms->fork, s));
+        MOE_CUDA(cudaStreamWaitEvent(ms->s2, ms->fork, 0));
+        return MOE_OK;
+    };
+    MOE_TRY(layer_run(x, W_gate, bias, X, Ws1, Ws3, Ws2, N0, H, I, E, k, Is, out, logits, ws, err, s, nullptr,
+                      fork));
+    MOE_TRY(layer_run(x + N0 * H, W_gate, bias, X, Ws1, Ws3, Ws2, N - N0, H, I, E, k, Is, out + N0 * H,
+                      logits ? logits + N0 * E : nullptr, ws1, err, ms->s2, nullptr, none));
+    MOE_CUDA(cudaEventRecord(ms->join, ms->s2));
+    MOE_CUDA(cudaStreamWaitEvent(s, ms->join, 0));
     return MOE_OK;
 }
 
@@ -342,6 +436,12 @@ int moe_device_sm_count(void) { return moe::device_sm_count(); }
 
 uint64_t moe_kernel_launches(void) { return moe::launches_so_far(); }
 
+int moe_set_microbatches(int m)
+{
+    if (m < 1 || m > 2) return -1;
+    return moe::g_microbatches.exchange(m);
+}
+
 int moe_set_gather_mode(int mode)
 {
     if (mode != MOE_GATHER_AUTO && mode != MOE_GATHER_OFF && mode != MOE_GATHER_ON) return -1;
@@ -352,18 +452,14 @@ size_t moe_workspace_bytes(int64_t N, int H, int I, int E, int k, int Is)
 {
     if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return 0;
     if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return 0;
-    WsLayout L;
-    ws_layout(N, H, I, E, k, Is, false, &L);
-    return L.total;
+    return layer_ws_bytes(N, H, I, E, k, Is, false);
 }
 
 size_t moe_workspace_bytes_w8a8(int64_t N, int H, int I, int E, int k, int Is)
 {
     if (!valid_rows(N, k) || !valid_hidden(H) || !valid_hidden(I) || !valid_ek(E, k)) return 0;
     if (Is < 0 || (Is > 0 && !valid_hidden(Is))) return 0;
-    WsLayout L;
-    ws_layout(N, H, I, E, k, Is, true, &L);
-    return L.total;
+    return layer_ws_bytes(N, H, I, E, k, Is, true);
 }
 
 moe_status_t moe_route(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,

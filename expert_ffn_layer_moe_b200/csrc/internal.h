@@ -17,6 +17,9 @@ uint64_t launches_so_far();
 // under another context on the same device, a cached address would be stale.
 void *current_context();
 
+// Micro-batches of large layers (moe_set_microbatches): 1 or 2.
+int layer_microbatches();
+
 // Whether the bf16 layer gathers its W1/W3 token rows from x (moe_set_gather_mode).
 bool layer_gathers(int64_t N, int k, int H);
 

@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.moe_scatter_rows.argtypes = [vp, vp, i64, c_int, vp, i64, vp]
         L.moe_set_gather_mode.argtypes = [c_int]
         L.moe_set_gather_mode.restype = c_int
+        L.moe_set_microbatches.argtypes = [c_int]
+        L.moe_set_microbatches.restype = c_int
         L.moe_ipc_export.argtypes = [vp, vp, ctypes.POINTER(sz)]
         L.moe_ipc_import.argtypes = [vp, sz, ctypes.POINTER(vp)]
         L.moe_ipc_close.argtypes = [vp, sz]
@@ -158,6 +160,15 @@ def moe_set_gather_mode(mode: int) -> int:
     prev = int(lib().moe_set_gather_mode(int(mode)))
     if prev < 0:
         raise ValueError(f"gather mode {mode} is not one of MOE_GATHER_AUTO/OFF/ON")
+    return prev
+
+
+def moe_set_microbatches(m: int) -> int:
+    """Run large layer calls as m (1 or 2) micro-batches on two streams; returns the
+    previous value."""
+    prev = int(lib().moe_set_microbatches(int(m)))
+    if prev < 0:
+        raise ValueError(f"micro-batches must be 1 or 2, not {m}")
     return prev
 
 

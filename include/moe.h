@@ -377,6 +377,25 @@ MOE_API moe_status_t moe_copy_async(void *dst, const void *src, size_t bytes, vo
 MOE_API int moe_set_gather_mode(int mode);
 
 /*
+ * Micro-batches of the layer calls (moe_layer_forward_ex and its fp8 forms) on
+ * batches of at least 32768 assignments (N*k).  With m = 2 the batch runs as two
+ * halves: rows [0, N0) on the caller's stream, rows [N0, N) on a second stream of
+ * the library's that starts once the first half has dispatched, joined back
+ * before the call's work ends on the caller's stream.  The first half's grouped
+ * GEMMs then run beside the second half's router, dispatch and row copies, and
+ * the second half's GEMMs beside the first half's combine (MegaScale-Infer
+ * summary page, "核心设计": splitting a batch into micro-batches so that one
+ * micro-batch's work hides another's; here the hidden work is the token-row
+ * movement the MoE-latency article's section "router 之后还有一串动作" names).
+ * Results are identical to m = 1 (every token's arithmetic is unchanged).  The
+ * first such call on a device creates the stream and two events (kept for the
+ * process); it should come before any stream capture.  A call with phase events
+ * runs in one piece.  m = 1 (the default) or 2; returns the previous value, or -1.
+ * Process-wide, like moe_set_gather_mode.
+ */
+MOE_API int moe_set_microbatches(int m);
+
+/*
  * Kernels this library has launched in this process so far, counted on the host
  * at each successful launch (all threads, all devices; never reset).  The
  * difference across a region is the number of the library's kernels it ran.

@@ -147,13 +147,21 @@ def test_route_shapes_and_bias(N, H, E, k, use_ws, with_logits):
 
 
 def test_kernel_launch_counter_counts_a_layer():
-    """The host-side launch count moves by the kernels one layer call runs: the
-    fused router, the single-block dispatch and the row scatter, the two grouped
-    GEMMs and the combine at the tiny shape."""
+    """The host-side launch count moves by the kernels one layer call runs.  At the
+    tiny shape (128 assignments): the one-kernel router, the kernel that dispatches and
+    copies the rows of a small batch, the two grouped GEMMs and the combine.  Through
+    the separate steps the same work is six launches: router, single-block dispatch,
+    row scatter, two GEMMs, combine."""
     cfg = CONFIGS["tiny"]
     t = cuda_inputs(cfg)
     n0 = moe.moe_kernel_launches()
     run_layer(cfg, t)
+    assert moe.moe_kernel_launches() - n0 == 5
+    n0 = moe.moe_kernel_launches()
+    idx, w, _ = moe.moe_route(t["x"], t["W_gate"], cfg.k, use_workspace=False)
+    p = moe.moe_permute(t["x"], idx, cfg.E)
+    y = moe.moe_expert_ffn(p["x_perm"], p["offsets"], t["W1"], t["W3"], t["W2"])
+    moe.moe_combine(y, p["token_to_row"], w)
     assert moe.moe_kernel_launches() - n0 == 6
 
 
@@ -421,3 +429,43 @@ def test_mixtral_decode_full_size_every_token():
         check_layer_against_oracle(cfg, t, out, logits)
     finally:
         oracle.set_threads(1)
+
+
+@pytest.mark.parametrize("cfg", [
+    MoEConfig("micro", N=4100, H=256, I=128, E=64, k=8),             # halves of 2056 and 2044 rows
+    MoEConfig("micro_shared", N=4096, H=128, I=192, E=16, k=8, Is=128),
+])
+def test_layer_in_two_microbatches_gives_the_same_bits(cfg):
+    """The layer run as two micro-batches on two streams (second half started after the
+    first half's dispatch) gives the bits of the one-piece layer, logits included, and
+    replays the same from a CUDA graph (the second stream joins the capture)."""
+    t = cuda_inputs(cfg, seed=31)
+    prev = moe.moe_set_microbatches(1)
+    try:
+        one, l1 = run_layer(cfg, t)
+        moe.moe_set_microbatches(2)
+        two, l2 = run_layer(cfg, t)
+        torch.cuda.synchronize()
+        assert torch.equal(l1, l2)
+        assert torch.equal(one.view(torch.int16), two.view(torch.int16))
+        ws = torch.empty(moe.moe_workspace_bytes(cfg.N, cfg.H, cfg.I, cfg.E, cfg.k, cfg.Is), dtype=torch.uint8,
+                         device="cuda")
+        out = torch.zeros_like(one)
+
+        def step():
+            moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k, Ws1=t.get("Ws1"),
+                                     Ws3=t.get("Ws3"), Ws2=t.get("Ws2"), ws=ws, out=out,
+                                     stream=torch.cuda.current_stream())
+        step()
+        torch.cuda.synchronize()
+        out.zero_()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error() == 0
+        assert torch.equal(out.view(torch.int16), one.view(torch.int16))
+        del g
+    finally:
+        moe.moe_set_microbatches(prev)
