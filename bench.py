@@ -592,6 +592,7 @@ def run_ours(args, cfg, world, rank, local):
     from expert_ffn_layer_moe_b200 import moe
     moe.moe_set_gather_mode({"auto": moe.MOE_GATHER_AUTO, "on": moe.MOE_GATHER_ON,
                              "off": moe.MOE_GATHER_OFF}[args.gather])
+    moe.moe_set_microbatches(args.microbatches)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     W = Workload(cfg, args, dev, stream, rank, world)
@@ -711,7 +712,7 @@ def run_ours(args, cfg, world, rank, local):
                                        + ")") if fp8 else "bf16"),
                    "expert_activations": ("e4m3, one fp32 scale per row (x_perm and h quantized on the device "
                                           "every step)") if a8 else "bf16",
-                   "w13_rows": f"gather mode {args.gather}"},
+                   "w13_rows": f"gather mode {args.gather}", "microbatches": args.microbatches},
         "roofline": roofline,
         "layer": layer,
         "grouped_gemm": gg,
@@ -890,6 +891,8 @@ def main():
                     help="routed-expert weight format (fp8: e4m3 with per-channel scales, a separate experiment)")
     ap.add_argument("--acts", choices=["bf16", "fp8"], default="bf16",
                     help="routed-expert activation format (fp8: e4m3 with per-row scales; needs --weights fp8)")
+    ap.add_argument("--microbatches", type=int, choices=[1, 2], default=1,
+                    help="run large layers as two micro-batches on two streams (moe_set_microbatches)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: the experts split over the ranks, token rows exchanged")
     ap.add_argument("--exchange", choices=["collective", "peer_copy"], default="collective",
