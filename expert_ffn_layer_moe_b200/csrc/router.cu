@@ -235,10 +235,95 @@ __global__ void __launch_bounds__(kThreads)
     topk_warp(row[warp], E, k, lane, topk_idx + t * k, topk_w + t * k);
 }
 
+// Top-k of one token per thread, for large batches: the P partial logits of each expert
+// are added in part order (+ bias) as router_topk_kernel adds them, the experts are
+// visited in index order, and the best k so far are kept in registers, sorted by the
+// picks' order (larger value first, the lower index first on equal values, NaN after
+// every number).  The weights use the same operations, in pick order, as topk_warp:
+// the picks, weights and logits are the ones the warp kernel gives.
+template <int P>
+__global__ void __launch_bounds__(kThreads)
+    router_topk_thread_kernel(const float *__restrict__ lin, int64_t pstride, int64_t tstride,
+                              const float *__restrict__ bias, int64_t N, int E, int k, float *__restrict__ logits,
+                              int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
+{
+    pdl_entry();
+    const int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (t >= N) return;
+    float bv[kMaxK];
+    int bi[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) { bv[j] = NAN; bi[j] = 0x7fffffff; }
+    const float *row = lin + t * tstride;
+    for (int e0 = 0; e0 < E; e0 += 4) {
+        float v[4];
+        if ((E & 3) == 0) {  // four experts' parts as 16-byte loads
+            float4 acc = __ldg(reinterpret_cast<const float4 *>(row + e0));
+#pragma unroll
+            for (int i = 1; i < P; ++i) {
+                const float4 q = __ldg(reinterpret_cast<const float4 *>(row + i * pstride + e0));
+                acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+            }
+            v[0] = acc.x; v[1] = acc.y; v[2] = acc.z; v[3] = acc.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float a = 0.f;
+                if (e0 + u < E) {
+                    a = row[e0 + u];
+#pragma unroll
+                    for (int i = 1; i < P; ++i) a += row[i * pstride + e0 + u];
+                }
+                v[u] = a;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u;
+            if (e >= E) break;
+            float cv = bias ? v[u] + bias[e] : v[u];
+            if (logits) logits[t * E + e] = cv;
+            int ci = e;
+            // bubble (cv, ci) through the list: it takes the first place it beats, and the
+            // entry it displaces moves on.  "Beats" is the picks' total order: the larger
+            // value, on equal values the lower index, NaN after every number (and after the
+            // empty places' index, which no expert reaches).
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j) {
+                if (j < k) {
+                    const bool cn = isnan(cv), bn = isnan(bv[j]);
+                    const bool beats = (!cn && bn) || (!cn && !bn && (cv > bv[j] || (cv == bv[j] && ci < bi[j]))) ||
+                                       (cn && bn && ci < bi[j]);
+                    if (beats) {
+                        const float tv = bv[j]; const int ti = bi[j];
+                        bv[j] = cv; bi[j] = ci; cv = tv; ci = ti;
+                    }
+                }
+            }
+        }
+    }
+    const float l0 = bv[0];
+    float ex[kMaxK];
+    float den = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+        if (j < k) { ex[j] = expf(bv[j] - l0); den += ex[j]; }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+        if (j < k) { topk_idx[t * k + j] = bi[j]; topk_w[t * k + j] = ex[j] / den; }
+}
+
+// Batches from this size on rank with a thread per token (enough threads to fill the
+// SMs); smaller ones with a warp per token.
+constexpr int64_t kTopkThreadMinN = 4096;
+
 template <int P>
 cudaError_t launch_topk(const float *lin, int64_t pstride, int64_t tstride, const float *bias, int64_t N, int E,
                         int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
 {
+    if (N >= kTopkThreadMinN)
+        return launch_pdl(router_topk_thread_kernel<P>, dim3((unsigned)((N + kThreads - 1) / kThreads)),
+                          dim3(kThreads), 0, s, lin, pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
     return launch_pdl(router_topk_kernel<P>, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, lin,
                       pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
 }

@@ -193,6 +193,30 @@ def test_route_ties_lower_index_first():
     assert np.allclose(host(w), 0.25, rtol=0, atol=1e-7)
 
 
+@pytest.mark.parametrize("N", [5, 1500, 5000])
+def test_route_ties_on_every_path(N):
+    """Exact ties at every size, so that each top-k form meets them: the fused and split
+    paths' warp per token (small N) and, on the tensor-core path, the warp per token
+    (N < 4096) and the thread per token (N >= 4096).  x is zero, so every logit is the
+    bias: ties between the picks, a tie straddling the k-th place, and -0 against +0."""
+    H, E, k = 256, 32, 8
+    x = torch.zeros((N, H), dtype=torch.bfloat16, device="cuda")
+    Wg = torch.randn((H, E), device="cuda")
+    b = [0.0] * E
+    for e, v in {3: 2.0, 9: 2.0, 17: 2.0, 30: 1.5, 1: 1.0, 12: 1.0, 20: 1.0, 25: 1.0, 26: 1.0}.items():
+        b[e] = v
+    b[5], b[6] = -0.0, 0.0                      # -0 == +0: the lower index first
+    bias = torch.tensor(b, dtype=torch.float32, device="cuda")
+    logits = torch.empty((N, E), dtype=torch.float32, device="cuda")
+    idx, w, _ = moe.moe_route(x, Wg, k, bias=bias, logits=logits)
+    torch.cuda.synchronize()
+    want = [3, 9, 17, 30, 1, 12, 20, 25]          # 1.0 ties: 1, 12, 20, 25 make it, 26 does not
+    assert host(idx).tolist() == [want] * N
+    ref_idx, ref_w = oracle.topk(host(logits), k)
+    assert np.array_equal(host(idx), ref_idx)
+    assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
+
+
 @pytest.mark.parametrize("N,E,k", [(64, 8, 2), (1000, 160, 6), (3000, 128, 8), (7, 4, 4), (1, 1, 1)])
 def test_permute_bit_exact(N, E, k):
     H = 128
