@@ -593,6 +593,7 @@ def run_ours(args, cfg, world, rank, local):
     moe.moe_set_gather_mode({"auto": moe.MOE_GATHER_AUTO, "on": moe.MOE_GATHER_ON,
                              "off": moe.MOE_GATHER_OFF}[args.gather])
     moe.moe_set_microbatches(args.microbatches)
+    moe.moe_set_shared_stream(bool(args.shared_stream))
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     W = Workload(cfg, args, dev, stream, rank, world)
@@ -712,7 +713,8 @@ def run_ours(args, cfg, world, rank, local):
                                        + ")") if fp8 else "bf16"),
                    "expert_activations": ("e4m3, one fp32 scale per row (x_perm and h quantized on the device "
                                           "every step)") if a8 else "bf16",
-                   "w13_rows": f"gather mode {args.gather}", "microbatches": args.microbatches},
+                   "w13_rows": f"gather mode {args.gather}", "microbatches": args.microbatches,
+                   "shared_experts_stream": "second stream" if args.shared_stream else "caller's stream"},
         "roofline": roofline,
         "layer": layer,
         "grouped_gemm": gg,
@@ -893,6 +895,8 @@ def main():
                     help="routed-expert activation format (fp8: e4m3 with per-row scales; needs --weights fp8)")
     ap.add_argument("--microbatches", type=int, choices=[1, 2], default=1,
                     help="run large layers as two micro-batches on two streams (moe_set_microbatches)")
+    ap.add_argument("--shared-stream", type=int, choices=[0, 1], default=0,
+                    help="run the shared experts on a second stream beside the dispatch (moe_set_shared_stream)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: the experts split over the ranks, token rows exchanged")
     ap.add_argument("--exchange", choices=["collective", "peer_copy"], default="collective",

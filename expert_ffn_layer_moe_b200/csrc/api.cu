@@ -19,8 +19,10 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_gather_mode{MOE_GATHER_AUTO};
 std::atomic<int> g_microbatches{1};
+std::atomic<int> g_shared_side{0};
 }  // namespace
 int layer_microbatches() { return g_microbatches.load(std::memory_order_relaxed); }
+bool layer_shared_side() { return g_shared_side.load(std::memory_order_relaxed) != 0; }
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 uint64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
 
@@ -258,11 +260,17 @@ moe_status_t record(void *const *ev, int i, cudaStream_t s)
 
 // The layer on N rows with a workspace laid out for N rows; after_dispatch (nullable)
 // runs once the permute phase is enqueued on s.
+// A second stream with its fork and join events (the shared experts' side stream).
+struct SideStream {
+    cudaStream_t s2;
+    cudaEvent_t fork, join;
+};
+
 template <typename Hook>
 moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias, const Experts &X,
                        const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2, int64_t N, int H, int I, int E,
                        int k, int Is, uint16_t *out, float *logits, void *ws, int *err, cudaStream_t s,
-                       void *const *phase_events, Hook after_dispatch)
+                       void *const *phase_events, Hook after_dispatch, const SideStream *side = nullptr)
 {
     WsLayout L;
     ws_layout(N, H, I, E, k, Is, X.a8, &L);
@@ -301,6 +309,14 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     if (fused != cudaSuccess)
         MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
+    if (side && Is > 0) {
+        // the shared experts need only x: they start now on the side stream, beside the
+        // dispatch, and are joined before the combine
+        MOE_CUDA(cudaEventRecord(side->fork, s));
+        MOE_CUDA(cudaStreamWaitEvent(side->s2, side->fork, 0));
+        MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, side->s2));
+        MOE_CUDA(cudaEventRecord(side->join, side->s2));
+    }
     if (fused == cudaSuccess) {
         a.act = x_perm;
     } else if (X.a8) {
@@ -333,7 +349,10 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
     MOE_CUDA(moe::launch_gemm2(b, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM2, s));
-    if (Is > 0) MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
+    if (Is > 0) {
+        if (side) MOE_CUDA(cudaStreamWaitEvent(s, side->join, 0));
+        else MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
+    }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_SHARED, s));
     MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r, w, sh, N, H, k, out, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_COMBINE, s));
@@ -349,6 +368,19 @@ struct MicroStreams {
     cudaEvent_t fork = nullptr, join = nullptr;
     void *ctx = nullptr;
 };
+
+// Creates the device's second stream and events on first use (again under a new context).
+moe_status_t ensure_side_stream(MicroStreams *ms)
+{
+    void *ctx = moe::current_context();
+    if (!ms->s2 || ctx != ms->ctx) {
+        MOE_CUDA(cudaStreamCreateWithFlags(&ms->s2, cudaStreamNonBlocking));
+        MOE_CUDA(cudaEventCreateWithFlags(&ms->fork, cudaEventDisableTiming));
+        MOE_CUDA(cudaEventCreateWithFlags(&ms->join, cudaEventDisableTiming));
+        ms->ctx = moe::current_context();
+    }
+    return MOE_OK;
+}
 
 MicroStreams *micro_streams()
 {
@@ -377,6 +409,16 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
     if (!err) return cuda_fail(cudaGetLastError());
     auto none = [] { return MOE_OK; };
     const int64_t N0 = micro_split(N, k);
+    const bool side_shared = Is > 0 && moe::layer_shared_side() && !phase_events && N0 == 0;
+    if (side_shared) {
+        MicroStreams *ms = micro_streams();
+        if (!ms) return MOE_ERR_UNSUPPORTED;
+        std::lock_guard<std::mutex> lock(ms->mu);
+        MOE_TRY(ensure_side_stream(ms));
+        const SideStream side{ms->s2, ms->fork, ms->join};
+        return layer_run(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, err, s, nullptr,
+                         none, &side);
+    }
     if (N0 == 0 || phase_events)  // per-phase timing runs the layer in one piece
         return layer_run(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, err, s,
                          phase_events, none);
@@ -389,13 +431,7 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
     MicroStreams *ms = micro_streams();
     if (!ms) return MOE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(ms->mu);
-    void *ctx = moe::current_context();
-    if (!ms->s2 || ctx != ms->ctx) {
-        MOE_CUDA(cudaStreamCreateWithFlags(&ms->s2, cudaStreamNonBlocking));
-        MOE_CUDA(cudaEventCreateWithFlags(&ms->fork, cudaEventDisableTiming));
-        MOE_CUDA(cudaEventCreateWithFlags(&ms->join, cudaEventDisableTiming));
-        ms->ctx = moe::current_context();
-    }
+    MOE_TRY(ensure_side_stream(ms));
     WsLayout L0;
     ws_layout(N0, H, I, E, k, Is, X.a8, &L0);
     uint8_t *ws1 = static_cast<uint8_t *>(ws) + round_up(L0.total);
@@ -435,6 +471,12 @@ const char *moe_last_cuda_error(void) { return g_last_cuda_error; }
 int moe_device_sm_count(void) { return moe::device_sm_count(); }
 
 uint64_t moe_kernel_launches(void) { return moe::launches_so_far(); }
+
+int moe_set_shared_stream(int on)
+{
+    if (on != 0 && on != 1) return -1;
+    return moe::g_shared_side.exchange(on);
+}
 
 int moe_set_microbatches(int m)
 {

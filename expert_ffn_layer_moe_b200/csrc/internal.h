@@ -19,6 +19,8 @@ void *current_context();
 
 // Micro-batches of large layers (moe_set_microbatches): 1 or 2.
 int layer_microbatches();
+// Whether the shared experts run on a second stream beside the dispatch (moe_set_shared_stream).
+bool layer_shared_side();
 
 // Whether the bf16 layer gathers its W1/W3 token rows from x (moe_set_gather_mode).
 bool layer_gathers(int64_t N, int k, int H);

@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.moe_set_gather_mode.restype = c_int
         L.moe_set_microbatches.argtypes = [c_int]
         L.moe_set_microbatches.restype = c_int
+        L.moe_set_shared_stream.argtypes = [c_int]
+        L.moe_set_shared_stream.restype = c_int
         L.moe_ipc_export.argtypes = [vp, vp, ctypes.POINTER(sz)]
         L.moe_ipc_import.argtypes = [vp, sz, ctypes.POINTER(vp)]
         L.moe_ipc_close.argtypes = [vp, sz]
@@ -170,6 +172,12 @@ def moe_set_microbatches(m: int) -> int:
     if prev < 0:
         raise ValueError(f"micro-batches must be 1 or 2, not {m}")
     return prev
+
+
+def moe_set_shared_stream(on: bool) -> bool:
+    """Run the shared experts on a second stream beside the dispatch; returns the
+    previous setting."""
+    return bool(lib().moe_set_shared_stream(1 if on else 0))
 
 
 def moe_kernel_launches() -> int:

@@ -493,3 +493,39 @@ def test_layer_in_two_microbatches_gives_the_same_bits(cfg):
         del g
     finally:
         moe.moe_set_microbatches(prev)
+
+
+def test_shared_experts_on_the_side_stream_give_the_same_bits():
+    """The shared experts forked onto the library's second stream after the router and
+    joined before the combine: the same bits as on the caller's stream, eager and
+    replayed from a CUDA graph (the second stream joins the capture)."""
+    cfg = MoEConfig("side", N=700, H=256, I=128, E=8, k=2, Is=192)
+    t = cuda_inputs(cfg, seed=17)
+    prev = moe.moe_set_shared_stream(False)
+    try:
+        one, l1 = run_layer(cfg, t)
+        moe.moe_set_shared_stream(True)
+        two, l2 = run_layer(cfg, t)
+        torch.cuda.synchronize()
+        assert torch.equal(l1, l2)
+        assert torch.equal(one.view(torch.int16), two.view(torch.int16))
+        ws = torch.empty(moe.moe_workspace_bytes(cfg.N, cfg.H, cfg.I, cfg.E, cfg.k, cfg.Is), dtype=torch.uint8,
+                         device="cuda")
+        out = torch.zeros_like(one)
+
+        def step():
+            moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k, Ws1=t["Ws1"],
+                                     Ws3=t["Ws3"], Ws2=t["Ws2"], ws=ws, out=out, stream=torch.cuda.current_stream())
+        step()
+        torch.cuda.synchronize()
+        out.zero_()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error() == 0
+        assert torch.equal(out.view(torch.int16), one.view(torch.int16))
+        del g
+    finally:
+        moe.moe_set_shared_stream(prev)
