@@ -241,7 +241,10 @@ __global__ void __launch_bounds__(kThreads)
 // picks' order (larger value first, the lower index first on equal values, NaN after
 // every number).  The weights use the same operations, in pick order, as topk_warp:
 // the picks, weights and logits are the ones the warp kernel gives.
-template <int P>
+// With COLS the partial logits are stored expert-major, [P][E][N] (part p of expert e of
+// token t at lin[(p * E + e) * N + t], the tensor-core router's transposed output):
+// consecutive threads then read consecutive words.
+template <int P, bool COLS>
 __global__ void __launch_bounds__(kThreads)
     router_topk_thread_kernel(const float *__restrict__ lin, int64_t pstride, int64_t tstride,
                               const float *__restrict__ bias, int64_t N, int E, int k, float *__restrict__ logits,
@@ -257,7 +260,19 @@ __global__ void __launch_bounds__(kThreads)
     const float *row = lin + t * tstride;
     for (int e0 = 0; e0 < E; e0 += 4) {
         float v[4];
-        if ((E & 3) == 0) {  // four experts' parts as 16-byte loads
+        if (COLS) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float a = 0.f;
+                if (e0 + u < E) {
+                    const float *q = lin + (int64_t)(e0 + u) * N + t;
+                    a = __ldg(q);
+#pragma unroll
+                    for (int i = 1; i < P; ++i) a += __ldg(q + i * pstride);
+                }
+                v[u] = a;
+            }
+        } else if ((E & 3) == 0) {  // four experts' parts as 16-byte loads
             float4 acc = __ldg(reinterpret_cast<const float4 *>(row + e0));
 #pragma unroll
             for (int i = 1; i < P; ++i) {
@@ -322,7 +337,7 @@ cudaError_t launch_topk(const float *lin, int64_t pstride, int64_t tstride, cons
                         int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
 {
     if (N >= kTopkThreadMinN)
-        return launch_pdl(router_topk_thread_kernel<P>, dim3((unsigned)((N + kThreads - 1) / kThreads)),
+        return launch_pdl(router_topk_thread_kernel<P, false>, dim3((unsigned)((N + kThreads - 1) / kThreads)),
                           dim3(kThreads), 0, s, lin, pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
     return launch_pdl(router_topk_kernel<P>, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, lin,
                       pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
@@ -525,6 +540,9 @@ cudaError_t launch_fused_for(const uint16_t *x, const float *W_gate, const float
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 constexpr int kTensorMaxSlices = 4;
+// Batches from this size on run the tensor-core router transposed (enough 256-token
+// tiles to cover the SM pairs in about one wave).
+constexpr int64_t kTensorTransposedMinN = 8192;
 
 // Tensor-core path shape: single-CTA tiles (128 operand rows) where they pad the 3E rows
 // less than pairs (256), the token tile, and the K slices S: double S while the tiles
@@ -631,6 +649,24 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
         const dim3 sgrid((unsigned)((H + 31) / 32), (unsigned)((E + 31) / 32));
         cudaError_t e = launch_pdl(router_split_kernel, sgrid, dim3(kThreads), 0, s, W_gate, H, E, wsplit);
         if (e != cudaSuccess) return e;
+        if (N >= kTensorTransposedMinN) {
+            // tokens on the MMA's M side (256 per CTA pair), the 3E terms on its N side in
+            // at most 256-row tiles: each operand byte serves more FLOPs than the 128 x 128
+            // tiles below, and the output [3E][N] is expert-major
+            float *parts = reinterpret_cast<float *>(w8 + split_bytes);
+            const int rows = 3 * E;
+            const int ntiles = (rows + 255) / 256;
+            const int bn = ((rows + ntiles - 1) / ntiles + 31) / 32 * 32;
+            GroupedGemmArgs g{};
+            g.w_a = x; g.act = wsplit; g.w_b = nullptr; g.offsets = nullptr; g.groups = 1; g.R = rows;
+            g.rows_single = rows; g.K = H; g.Nout = (int)N; g.out = parts; g.dev_err = dev_err;
+            g.token_tile = bn; g.ldo = N;
+            e = launch_gemm2(g, s);
+            if (e != cudaSuccess) return e;
+            return launch_pdl(router_topk_thread_kernel<3, true>, dim3((unsigned)((N + kThreads - 1) / kThreads)),
+                              dim3(kThreads), 0, s, parts, (int64_t)E * N, (int64_t)0, bias, N, E, k, lbuf,
+                              topk_idx, topk_w);
+        }
         int bn, S;
         bool single;
         tensor_shape(N, H, E, &bn, &S, &single);
