@@ -235,110 +235,51 @@ __global__ void __launch_bounds__(kThreads)
     topk_warp(row[warp], E, k, lane, topk_idx + t * k, topk_w + t * k);
 }
 
-// Top-k of one token per thread, for large batches: the P partial logits of each expert
-// are added in part order (+ bias) as router_topk_kernel adds them, the experts are
-// visited in index order, and the best k so far are kept in registers, sorted by the
-// picks' order (larger value first, the lower index first on equal values, NaN after
-// every number).  The weights use the same operations, in pick order, as topk_warp:
-// the picks, weights and logits are the ones the warp kernel gives.
-// With COLS the partial logits are stored expert-major, [P][E][N] (part p of expert e of
-// token t at lin[(p * E + e) * N + t], the tensor-core router's transposed output):
-// consecutive threads then read consecutive words.
-template <int P, bool COLS>
+// Top-k from the tensor-core router's expert-major partial logits ([P][E][N]: part p of
+// expert e of token t at lin[(p * E + e) * N + t]).  A block takes 32 consecutive
+// tokens: its threads read each expert's parts for the 32 tokens as one 128-byte row
+// (coalesced), add them in part order (+ bias) as router_topk_kernel adds them, and
+// write the logits token-major into shared memory; then each warp ranks its tokens with
+// topk_warp, as router_topk_kernel does.  Same picks, weights and logits.
+constexpr int kColTokens = 32;
+template <int P>
 __global__ void __launch_bounds__(kThreads)
-    router_topk_thread_kernel(const float *__restrict__ lin, int64_t pstride, int64_t tstride,
-                              const float *__restrict__ bias, int64_t N, int E, int k, float *__restrict__ logits,
-                              int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
+    router_topk_cols_kernel(const float *__restrict__ lin, const float *__restrict__ bias, int64_t N, int E, int k,
+                            float *__restrict__ logits, int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
 {
+    __shared__ float row[kColTokens][kMaxE + 1];
     pdl_entry();
-    const int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (t >= N) return;
-    float bv[kMaxK];
-    int bi[kMaxK];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t0 = (int64_t)blockIdx.x * kColTokens;
+    const int64_t t = t0 + lane;
+    for (int e = warp; e < E; e += kWarps) {  // warp w: experts w, w + 8, ...; lane: token
+        float v = 0.f;
+        if (t < N) {
+            const float *q = lin + (int64_t)e * N + t;
+            float part[P];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) { bv[j] = NAN; bi[j] = 0x7fffffff; }
-    const float *row = lin + t * tstride;
-    for (int e0 = 0; e0 < E; e0 += 4) {
-        float v[4];
-        if (COLS) {
+            for (int i = 0; i < P; ++i) part[i] = __ldg(q + (int64_t)i * E * N);
+            v = part[0];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float a = 0.f;
-                if (e0 + u < E) {
-                    const float *q = lin + (int64_t)(e0 + u) * N + t;
-                    a = __ldg(q);
-#pragma unroll
-                    for (int i = 1; i < P; ++i) a += __ldg(q + i * pstride);
-                }
-                v[u] = a;
-            }
-        } else if ((E & 3) == 0) {  // four experts' parts as 16-byte loads
-            float4 acc = __ldg(reinterpret_cast<const float4 *>(row + e0));
-#pragma unroll
-            for (int i = 1; i < P; ++i) {
-                const float4 q = __ldg(reinterpret_cast<const float4 *>(row + i * pstride + e0));
-                acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
-            }
-            v[0] = acc.x; v[1] = acc.y; v[2] = acc.z; v[3] = acc.w;
-        } else {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float a = 0.f;
-                if (e0 + u < E) {
-                    a = row[e0 + u];
-#pragma unroll
-                    for (int i = 1; i < P; ++i) a += row[i * pstride + e0 + u];
-                }
-                v[u] = a;
-            }
+            for (int i = 1; i < P; ++i) v += part[i];
+            if (bias) v += bias[e];
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = e0 + u;
-            if (e >= E) break;
-            float cv = bias ? v[u] + bias[e] : v[u];
-            if (logits) logits[t * E + e] = cv;
-            int ci = e;
-            // bubble (cv, ci) through the list: it takes the first place it beats, and the
-            // entry it displaces moves on.  "Beats" is the picks' total order: the larger
-            // value, on equal values the lower index, NaN after every number (and after the
-            // empty places' index, which no expert reaches).
-#pragma unroll
-            for (int j = 0; j < kMaxK; ++j) {
-                if (j < k) {
-                    const bool cn = isnan(cv), bn = isnan(bv[j]);
-                    const bool beats = (!cn && bn) || (!cn && !bn && (cv > bv[j] || (cv == bv[j] && ci < bi[j]))) ||
-                                       (cn && bn && ci < bi[j]);
-                    if (beats) {
-                        const float tv = bv[j]; const int ti = bi[j];
-                        bv[j] = cv; bi[j] = ci; cv = tv; ci = ti;
-                    }
-                }
-            }
-        }
+        row[lane][e] = v;
     }
-    const float l0 = bv[0];
-    float ex[kMaxK];
-    float den = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-        if (j < k) { ex[j] = expf(bv[j] - l0); den += ex[j]; }
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-        if (j < k) { topk_idx[t * k + j] = bi[j]; topk_w[t * k + j] = ex[j] / den; }
+    __syncthreads();
+    for (int tt = warp; tt < kColTokens; tt += kWarps) {
+        const int64_t tok = t0 + tt;
+        if (tok >= N) break;
+        if (logits)
+            for (int e = lane; e < E; e += 32) logits[tok * E + e] = row[tt][e];
+        topk_warp(row[tt], E, k, lane, topk_idx + tok * k, topk_w + tok * k);
+    }
 }
-
-// Batches from this size on rank with a thread per token (enough threads to fill the
-// SMs); smaller ones with a warp per token.
-constexpr int64_t kTopkThreadMinN = 4096;
 
 template <int P>
 cudaError_t launch_topk(const float *lin, int64_t pstride, int64_t tstride, const float *bias, int64_t N, int E,
                         int k, float *logits, int32_t *topk_idx, float *topk_w, cudaStream_t s)
 {
-    if (N >= kTopkThreadMinN)
-        return launch_pdl(router_topk_thread_kernel<P, false>, dim3((unsigned)((N + kThreads - 1) / kThreads)),
-                          dim3(kThreads), 0, s, lin, pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
     return launch_pdl(router_topk_kernel<P>, dim3((unsigned)((N + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, lin,
                       pstride, tstride, bias, N, E, k, logits, topk_idx, topk_w);
 }
@@ -663,9 +604,9 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
             g.token_tile = bn; g.ldo = N;
             e = launch_gemm2(g, s);
             if (e != cudaSuccess) return e;
-            return launch_pdl(router_topk_thread_kernel<3, true>, dim3((unsigned)((N + kThreads - 1) / kThreads)),
-                              dim3(kThreads), 0, s, parts, (int64_t)E * N, (int64_t)0, bias, N, E, k, lbuf,
-                              topk_idx, topk_w);
+            return launch_pdl(router_topk_cols_kernel<3>,
+                              dim3((unsigned)((N + kColTokens - 1) / kColTokens)), dim3(kThreads), 0, s, parts,
+                              bias, N, E, k, lbuf, topk_idx, topk_w);
         }
         int bn, S;
         bool single;
