@@ -549,10 +549,14 @@ def summarise(cfg, touched, step_s, phase_ms, pk, wbytes, abytes, a8):
 
 
 def other_workload_line(cfg, args, dev, stream, rank, world, graph, pk):
-    """Tokens/s, step time, layer fraction and phase times of one more workload."""
+    """Tokens/s, step time, layer fraction and phase times of one more workload, with
+    the clocks sampled over its timed steps."""
     W = Workload(cfg, args, dev, stream, rank, world)
     try:
-        elapsed_ms, launches, phase_ms = time_steps(W, args.other_steps, args.warmup, world, graph)
+        time.sleep(1.0)  # let the power draw of the previous workload settle
+        clk = ClockSampler(dev.index if dev.index is not None else 0).start()
+        elapsed_ms, launches, phase_ms = time_steps(W, args.other_steps, args.warmup, world, graph, clock=clk)
+        cs = clk.summary()
         elapsed_ms = max_over_ranks(elapsed_ms, world)
         step_s = elapsed_ms / 1e3 / args.other_steps
         layer, gg, roof = summarise(cfg, W.touched, step_s, phase_ms, pk, W.wbytes, W.abytes, W.a8)
@@ -562,7 +566,8 @@ def other_workload_line(cfg, args, dev, stream, rank, world, graph, pk):
                 "gemm13_roofline": {k: roof[k] for k in ("bound", "achieved", "unit", "frac")},
                 "phase_us": {p: 1e3 * v for p, v in phase_ms.items()},
                 "launch_mode": "cuda graph replay" if graph else "stream launches", "gpu_launches": launches,
-                "touched_experts": W.touched, "max_expert_rows": W.max_load, "l2": W.l2_note}
+                "touched_experts": W.touched, "max_expert_rows": W.max_load, "l2": W.l2_note,
+                "clocks": ({k: cs[k] for k in ("sm_mhz", "power_w_max", "reasons", "samples")} if cs else None)}
     finally:
         W.release()
         del W
