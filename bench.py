@@ -900,7 +900,7 @@ def main():
                     help="routed-expert activation format (fp8: e4m3 with per-row scales; needs --weights fp8)")
     ap.add_argument("--microbatches", type=int, choices=[1, 2], default=1,
                     help="run large layers as two micro-batches on two streams (moe_set_microbatches)")
-    ap.add_argument("--shared-stream", type=int, choices=[0, 1], default=0,
+    ap.add_argument("--shared-stream", type=int, choices=[0, 1], default=1,
                     help="run the shared experts on a second stream beside the dispatch (moe_set_shared_stream)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: the experts split over the ranks, token rows exchanged")

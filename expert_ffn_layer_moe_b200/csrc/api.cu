@@ -19,7 +19,7 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_gather_mode{MOE_GATHER_AUTO};
 std::atomic<int> g_microbatches{1};
-std::atomic<int> g_shared_side{0};
+std::atomic<int> g_shared_side{1};
 }  // namespace
 int layer_microbatches() { return g_microbatches.load(std::memory_order_relaxed); }
 bool layer_shared_side() { return g_shared_side.load(std::memory_order_relaxed) != 0; }

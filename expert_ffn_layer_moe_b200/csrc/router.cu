@@ -252,19 +252,28 @@ __global__ void __launch_bounds__(kThreads)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * kColTokens;
     const int64_t t = t0 + lane;
-    for (int e = warp; e < E; e += kWarps) {  // warp w: experts w, w + 8, ...; lane: token
-        float v = 0.f;
-        if (t < N) {
-            const float *q = lin + (int64_t)e * N + t;
-            float part[P];
+    // warp w: experts w, w + 8, ..., eight at a time with all their loads in flight; lane: token
+    constexpr int kBatch = 8;
+    for (int e0 = warp; e0 < E; e0 += kWarps * kBatch) {
+        float part[kBatch][P];
 #pragma unroll
-            for (int i = 0; i < P; ++i) part[i] = __ldg(q + (int64_t)i * E * N);
-            v = part[0];
+        for (int j = 0; j < kBatch; ++j) {
+            const int e = e0 + j * kWarps;
 #pragma unroll
-            for (int i = 1; i < P; ++i) v += part[i];
-            if (bias) v += bias[e];
+            for (int i = 0; i < P; ++i)
+                part[j][i] = (e < E && t < N) ? __ldg(lin + ((int64_t)i * E + e) * N + t) : 0.f;
         }
-        row[lane][e] = v;
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int e = e0 + j * kWarps;
+            if (e < E) {
+                float v = part[j][0];
+#pragma unroll
+                for (int i = 1; i < P; ++i) v += part[j][i];
+                if (bias) v += bias[e];
+                row[lane][e] = v;
+            }
+        }
     }
     __syncthreads();
     for (int tt = warp; tt < kColTokens; tt += kWarps) {
@@ -481,9 +490,10 @@ cudaError_t launch_fused_for(const uint16_t *x, const float *W_gate, const float
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 constexpr int kTensorMaxSlices = 4;
-// Batches from this size on run the tensor-core router transposed (enough 256-token
-// tiles to cover the SM pairs in about one wave).
-constexpr int64_t kTensorTransposedMinN = 8192;
+// Batches from this size on run the tensor-core router transposed (at 8192 tokens the
+// 128 x 128 tiles below measured faster: 64 transposed tiles leave 10 of the 74 SM
+// pairs idle).
+constexpr int64_t kTensorTransposedMinN = 16384;
 
 // Tensor-core path shape: single-CTA tiles (128 operand rows) where they pad the 3E rows
 // less than pairs (256), the token tile, and the K slices S: double S while the tiles

@@ -193,11 +193,11 @@ def test_route_ties_lower_index_first():
     assert np.allclose(host(w), 0.25, rtol=0, atol=1e-7)
 
 
-@pytest.mark.parametrize("N", [5, 1500, 9000])
+@pytest.mark.parametrize("N", [5, 1500, 17000])
 def test_route_ties_on_every_path(N):
     """Exact ties at every size, so that each top-k form meets them: the fused and split
     paths (small N), the tensor-core path with token-major partial logits (N < 8192) and
-    with expert-major ones staged through shared memory (N >= 8192).  x is zero, so
+    with expert-major ones staged through shared memory (N >= 16384).  x is zero, so
     every logit is the bias: ties between the picks, a tie straddling the k-th place, and
     -0 against +0."""
     H, E, k = 256, 32, 8
