@@ -145,32 +145,27 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, bool a8, WsLayout 
     L->total = off;
 }
 
-// Rows of the first micro-batch when the layer runs as two (0: it runs in one piece):
-// batches of at least kMicroMinRows assignments, when moe_set_microbatches asked for 2.
+// Tokens of the first half when the layer runs its expert GEMMs as two micro-batches (0:
+// in one piece): batches of at least kMicroMinRows assignments, when moe_set_microbatches
+// asked for 2.  The first half ends on a block of the dispatch (N0 * k a multiple of
+// kPermuteChunk), whose per-block table then holds where the second half's rows of every
+// expert start.
 constexpr int64_t kMicroMinRows = 32768;
 int64_t micro_split(int64_t N, int k)
 {
-    if (moe::layer_microbatches() < 2 || N * k < kMicroMinRows || N < 2) return 0;
-    return (N / 2 + 7) & ~int64_t(7);  // a multiple of 8 rows, so the second half starts 16-byte aligned
+    if (moe::layer_microbatches() < 2 || N * k < kMicroMinRows) return 0;
+    int64_t g = moe::kPermuteChunk, kk = k;  // step = kPermuteChunk / gcd(k, kPermuteChunk) tokens
+    while (kk) { const int64_t r = g % kk; g = kk; kk = r; }
+    const int64_t step = moe::kPermuteChunk / g;
+    const int64_t N0 = (N / 2) / step * step;
+    return (N0 > 0 && N0 < N) ? N0 : 0;
 }
 
-// Workspace of the layer: enough for the layer in one piece and for two micro-batches.
 size_t layer_ws_bytes(int64_t N, int H, int I, int E, int k, int Is, bool a8)
 {
     WsLayout L;
     ws_layout(N, H, I, E, k, Is, a8, &L);
-    size_t total = L.total;
-    if (N >= 2) {
-        const int64_t N0 = (N / 2 + 7) & ~int64_t(7);
-        if (N0 < N) {
-            WsLayout L0, L1;
-            ws_layout(N0, H, I, E, k, Is, a8, &L0);
-            ws_layout(N - N0, H, I, E, k, Is, a8, &L1);
-            const size_t two = round_up(L0.total) + L1.total;
-            if (two > total) total = two;
-        }
-    }
-    return total;
+    return L.total;
 }
 
 // The routed experts' weights: bf16, or e4m3 bytes with one fp32 scale per row
@@ -365,7 +360,7 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
 struct MicroStreams {
     std::mutex mu;
     cudaStream_t s2 = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr, rows2 = nullptr, half1 = nullptr;
     void *ctx = nullptr;
 };
 
@@ -377,6 +372,8 @@ moe_status_t ensure_side_stream(MicroStreams *ms)
         MOE_CUDA(cudaStreamCreateWithFlags(&ms->s2, cudaStreamNonBlocking));
         MOE_CUDA(cudaEventCreateWithFlags(&ms->fork, cudaEventDisableTiming));
         MOE_CUDA(cudaEventCreateWithFlags(&ms->join, cudaEventDisableTiming));
+        MOE_CUDA(cudaEventCreateWithFlags(&ms->rows2, cudaEventDisableTiming));
+        MOE_CUDA(cudaEventCreateWithFlags(&ms->half1, cudaEventDisableTiming));
         ms->ctx = moe::current_context();
     }
     return MOE_OK;
@@ -388,6 +385,77 @@ MicroStreams *micro_streams()
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     return &per_dev[dev];
+}
+
+// The layer with its expert GEMMs in two micro-batches of tokens, [0, N0) and [N0, N)
+// (the pages' ping-pong of micro-batches, inside one GPU).  The router and the dispatch
+// run once for the whole batch; inside every expert's group the rows of the first half's
+// tokens come first (the dispatch is stable), and the dispatch's per-block table at the
+// block where the second half starts gives, for every expert, the row where its second
+// half starts.  So the two halves' GEMMs are the same grouped kernels on complementary
+// row ranges of each group, writing disjoint rows of h and y.  On the caller's stream s:
+// router, dispatch, the first half's row copies, its GEMMs, then the second half's GEMMs
+// and combine.  On the side stream: the second half's row copies, started after the
+// dispatch, and the first half's combine, started after its GEMMs -- so HBM-bound
+// copies and combines run beside the persistent GEMMs of the other half.  Every token's
+// arithmetic is the one-piece layer's.
+moe_status_t layer_run_micro(const uint16_t *x, const float *W_gate, const float *bias, const Experts &X, int64_t N,
+                             int H, int I, int E, int k, uint16_t *out, float *logits, void *ws, int *err,
+                             cudaStream_t s, MicroStreams *ms, int64_t N0)
+{
+    WsLayout L;
+    ws_layout(N, H, I, E, k, 0, false, &L);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *lg = logits ? logits : reinterpret_cast<float *>(base + L.logits);
+    int32_t *idx = reinterpret_cast<int32_t *>(base + L.idx);
+    float *w = reinterpret_cast<float *>(base + L.w);
+    int32_t *counts = reinterpret_cast<int32_t *>(base + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(base + L.offsets);
+    int32_t *r2t = reinterpret_cast<int32_t *>(base + L.r2t);
+    int32_t *t2r = reinterpret_cast<int32_t *>(base + L.t2r);
+    int32_t *perm = reinterpret_cast<int32_t *>(base + L.perm);
+    uint16_t *x_perm = reinterpret_cast<uint16_t *>(base + L.x_perm);
+    uint16_t *h = reinterpret_cast<uint16_t *>(base + L.h);
+    float *y_perm = reinterpret_cast<float *>(base + L.y_perm);
+    const int64_t R = N * k;
+    const int64_t N1 = N - N0;
+    cudaStream_t s2 = ms->s2;
+
+    MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
+    MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
+    const int32_t *mid = perm + (N0 * k / moe::kPermuteChunk) * E;  // second half's first row, per expert
+    MOE_CUDA(moe::launch_scatter_rows(x, nullptr, t2r, N0, k, H, x_perm, R, nullptr, s));
+    MOE_CUDA(cudaEventRecord(ms->fork, s));
+    MOE_CUDA(cudaStreamWaitEvent(s2, ms->fork, 0));
+    MOE_CUDA(moe::launch_scatter_rows(x + N0 * H, nullptr, t2r + N0 * k, N1, k, H, x_perm, R, nullptr, s2));
+    MOE_CUDA(cudaEventRecord(ms->rows2, s2));
+
+    const int ksplit = moe::gemm2_ksplit(R, E, I, H);
+    auto gemms = [&](const int32_t *starts, const int32_t *ends) -> moe_status_t {
+        moe::GroupedGemmArgs a{};
+        a.act = x_perm; a.offsets = starts; a.ends = ends; a.groups = E; a.R = R;
+        a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
+        set_weights13(&a, X);
+        MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
+        moe::GroupedGemmArgs b{};
+        b.act = h; b.offsets = starts; b.ends = ends; b.groups = E; b.R = R;
+        b.K = I; b.Nout = H; b.out = y_perm; b.dev_err = err;
+        set_weights2(&b, X);
+        b.ksplit = ksplit; b.split_stride = R * (int64_t)H;
+        MOE_CUDA(moe::launch_gemm2(b, s));
+        return MOE_OK;
+    };
+    MOE_TRY(gemms(offsets, mid));                 // first half: [offsets[e], mid[e])
+    MOE_CUDA(cudaEventRecord(ms->half1, s));
+    MOE_CUDA(cudaStreamWaitEvent(s2, ms->half1, 0));
+    MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r, w, nullptr, N0, H, k, out, s2));
+    MOE_CUDA(cudaEventRecord(ms->join, s2));
+    MOE_CUDA(cudaStreamWaitEvent(s, ms->rows2, 0));
+    MOE_TRY(gemms(mid, offsets + 1));             // second half: [mid[e], offsets[e + 1])
+    MOE_CUDA(moe::launch_combine(y_perm, ksplit, R * (int64_t)H, t2r + N0 * k, w + N0 * k, nullptr, N1, H, k,
+                                 out + N0 * H, s));
+    MOE_CUDA(cudaStreamWaitEvent(s, ms->join, 0));
+    return MOE_OK;
 }
 
 moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bias, const Experts &X,
@@ -419,36 +487,16 @@ moe_status_t layer_impl(const uint16_t *x, const float *W_gate, const float *bia
         return layer_run(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, err, s, nullptr,
                          none, &side);
     }
-    if (N0 == 0 || phase_events)  // per-phase timing runs the layer in one piece
+    const bool micro = N0 > 0 && !phase_events && !X.a8 && !X.fp8 && Is == 0 && !moe::layer_gathers(N, k, H);
+    if (!micro)
         return layer_run(x, W_gate, bias, X, Ws1, Ws3, Ws2, N, H, I, E, k, Is, out, logits, ws, err, s,
                          phase_events, none);
-
-    // Two micro-batches (the pages' ping-pong of micro-batches, inside one GPU): rows
-    // [0, N0) on the caller's stream, rows [N0, N) on a second stream that starts once
-    // the first has dispatched.  The first's grouped GEMMs then run beside the second's
-    // router, dispatch and row copies, and the second's GEMMs beside the first's combine:
-    // HBM-bound kernels fill the room the persistent GEMMs leave on every SM.
     MicroStreams *ms = micro_streams();
     if (!ms) return MOE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(ms->mu);
     MOE_TRY(ensure_side_stream(ms));
-    WsLayout L0;
-    ws_layout(N0, H, I, E, k, Is, X.a8, &L0);
-    uint8_t *ws1 = static_cast<uint8_t *>(ws) + round_up(L0.total);
-    auto fork = [&]() -> moe_status_t {
-        MOE_CUDA(cudaEventRecord(ms->fork, s));
-        MOE_CUDA(cudaStreamWaitEvent(ms->s2, ms->fork, 0));
-        return MOE_OK;
-    };
-    MOE_TRY(layer_run(x, W_gate, bias, X, Ws1, Ws3, Ws2, N0, H, I, E, k, Is, out, logits, ws, err, s, nullptr,
-                      fork));
-    MOE_TRY(layer_run(x + N0 * H, W_gate, bias, X, Ws1, Ws3, Ws2, N - N0, H, I, E, k, Is, out + N0 * H,
-                      logits ? logits + N0 * E : nullptr, ws1, err, ms->s2, nullptr, none));
-    MOE_CUDA(cudaEventRecord(ms->join, ms->s2));
-    MOE_CUDA(cudaStreamWaitEvent(s, ms->join, 0));
-    return MOE_OK;
+    return layer_run_micro(x, W_gate, bias, X, N, H, I, E, k, out, logits, ws, err, s, ms, N0);
 }
-
 }  // namespace
 
 extern "C" {

@@ -121,7 +121,7 @@ struct Cfg {
     static constexpr int kASlot0 = kAccBufs * kAccCols;    // W8: first TMEM column of the operand slots
     static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols + kABufs * kACols);
     static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAccBufs + 2 * kFStages + kABufs);
-    static constexpr int kTableBytes = (4 * 2 * (kMaxGroups + 1) + 15) & ~15;
+    static constexpr int kTableBytes = (4 * 3 * (kMaxGroups + 1) + 15) & ~15;  // starts, ends, item prefix
     // epilogue staging: one region of 34 x 32 fp32 per epilogue warp (a padded [32][33]
     // tile, or a dense [32][32] box for bulk stores at its 128-byte-aligned start); the
     // SwiGLU epilogue uses it as 2 x [64][33]
@@ -539,7 +539,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
                         void *__restrict__ out, int ksplit, int64_t split_stride,
                         const float *__restrict__ scale_a, const float *__restrict__ scale_b,
                         const float *__restrict__ scale_act, int64_t ldo, const int32_t *__restrict__ gather_rows,
-                        const __grid_constant__ CUtensorMap tm_out, int tma_store, int *dev_err)
+                        const __grid_constant__ CUtensorMap tm_out, int tma_store,
+                        const int32_t *__restrict__ ends, int *dev_err)
 {
     using C = Cfg<BN, SWIGLU, PAIR, W8, A8>;
     static_assert(!GATHER || (SWIGLU && !W8 && !A8), "gathered activation rows: bf16 SwiGLU GEMM only");
@@ -565,6 +566,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     int *g_off = reinterpret_cast<int *>(tmem_slot + 4);  // [groups+1] row offsets
     int *g_tile = g_off + (kMaxGroups + 1);               // [groups+1] work-item prefix
+    int *g_end = g_tile + (kMaxGroups + 1);               // [groups] end row of each group
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -603,9 +605,11 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
 
     // ---- work list: row offsets and the prefix of (token tiles x feature tiles x K slices) per group
     if (offsets == nullptr) {
-        if (tid == 0) { g_off[0] = 0; g_off[1] = rows_single; }
+        if (tid == 0) { g_off[0] = 0; g_off[1] = rows_single; g_end[0] = rows_single; }
     } else {
+        // group g is rows [offsets[g], ends[g]) when ends is given, else [offsets[g], offsets[g+1])
         for (int i = tid; i <= groups; i += kThreads) g_off[i] = offsets[i];
+        for (int i = tid; i < groups; i += kThreads) g_end[i] = ends ? ends[i] : offsets[i + 1];
     }
     __syncthreads();
     if (warp == 0) {
@@ -615,7 +619,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
             const int gi = base + lane;
             int items = 0;
             if (gi < groups) {
-                const int lo = g_off[gi], hi = g_off[gi + 1];
+                const int lo = g_off[gi], hi = g_end[gi];
                 if (lo < 0 || hi < lo || (int64_t)hi > R) bad = true;
                 else items = ((hi - lo + BN - 1) / BN) * n_feat * ksplit;
             }
@@ -652,7 +656,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWIGLU, PAIR, W8, A8>::kThreads, 1)
         feat = fk / ksplit;
         ks = fk % ksplit;
         row0 = g_off[g] + (local / nfk) * BN;
-        row_end = g_off[g + 1];
+        row_end = g_end[g];
     };
     // W8: slices start and end on 128-wide K blocks (one fp8 load); a last half block
     // past K reads zeros from both tensor maps and adds nothing
@@ -1214,7 +1218,7 @@ cudaError_t launch_impl(const GroupedGemmArgs &a, cudaStream_t s)
     cfg.numAttrs = PAIR ? 2 : 1;
     err = cudaLaunchKernelEx(&cfg, kern, ma, mb, mact, a.offsets, a.groups, a.rows_single, a.R, a.K, a.Nout, a.out,
                              ksplit, a.split_stride, a.scale_a, a.scale_b, a.scale_act, ldo, a.gather_rows, mout,
-                             tma_store, a.dev_err);
+                             tma_store, a.ends, a.dev_err);
     if (err != cudaSuccess) return err;
     count_launch();
     return cudaGetLastError();

@@ -92,6 +92,8 @@ struct GroupedGemmArgs {
     bool a8;                 // activations are e4m3 too (needs w8): native fp8 MMA
     const float *scale_act;  // [R] row scales of act (a8 only)
     const int32_t *offsets;  // [groups + 1] device, or nullptr
+    const int32_t *ends;     // [groups] device, or nullptr: group g is rows [offsets[g], ends[g])
+                             // instead of [offsets[g], offsets[g + 1])
     int groups;
     int64_t R;               // rows of `act` (and of `out`)
     int rows_single;         // rows when offsets == nullptr

@@ -457,13 +457,15 @@ def test_mixtral_decode_full_size_every_token():
 
 
 @pytest.mark.parametrize("cfg", [
-    MoEConfig("micro", N=4100, H=256, I=128, E=64, k=8),             # halves of 2056 and 2044 rows
-    MoEConfig("micro_shared", N=4096, H=128, I=192, E=16, k=8, Is=128),
+    MoEConfig("micro", N=4100, H=256, I=128, E=64, k=8),              # halves of 1920 and 2180 tokens
+    MoEConfig("micro_k6", N=6000, H=128, I=192, E=48, k=6),            # halves of 2816 and 3184 tokens
+    MoEConfig("micro_shared", N=4096, H=128, I=192, E=16, k=8, Is=128),  # shared experts: runs in one piece
 ])
 def test_layer_in_two_microbatches_gives_the_same_bits(cfg):
-    """The layer run as two micro-batches on two streams (second half started after the
-    first half's dispatch) gives the bits of the one-piece layer, logits included, and
-    replays the same from a CUDA graph (the second stream joins the capture)."""
+    """The layer with its expert GEMMs run as two micro-batches of tokens (the second
+    half's row copies and the first half's combine on the library's second stream) gives
+    the bits of the one-piece layer, logits included, and replays the same from a CUDA
+    graph (the second stream joins the capture)."""
     t = cuda_inputs(cfg, seed=31)
     prev = moe.moe_set_microbatches(1)
     try:
