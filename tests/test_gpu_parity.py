@@ -457,8 +457,8 @@ def test_mixtral_decode_full_size_every_token():
 
 
 @pytest.mark.parametrize("cfg", [
-    MoEConfig("micro", N=4100, H=256, I=128, E=64, k=8),              # halves of 1920 and 2180 tokens
-    MoEConfig("micro_k6", N=6000, H=128, I=192, E=48, k=6),            # halves of 2816 and 3184 tokens
+    MoEConfig("micro", N=4100, H=256, I=128, E=64, k=8),              # halves of 2048 and 2052 tokens
+    MoEConfig("micro_k6", N=6000, H=128, I=192, E=48, k=6),            # halves of 2560 and 3440 tokens
     MoEConfig("micro_shared", N=4096, H=128, I=192, E=16, k=8, Is=128),  # shared experts: runs in one piece
 ])
 def test_layer_in_two_microbatches_gives_the_same_bits(cfg):
