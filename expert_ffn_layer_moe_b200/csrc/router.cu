@@ -236,53 +236,126 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // Top-k from the tensor-core router's expert-major partial logits ([P][E][N]: part p of
-// expert e of token t at lin[(p * E + e) * N + t]).  A block takes 32 consecutive
-// tokens: its threads read each expert's parts for the 32 tokens as one 128-byte row
-// (coalesced), add them in part order (+ bias) as router_topk_kernel adds them, and
-// write the logits token-major into shared memory; then each warp ranks its tokens with
-// topk_warp, as router_topk_kernel does.  Same picks, weights and logits.
-constexpr int kColTokens = 32;
+// expert e of token t at lin[(p * E + e) * N + t]).  A block takes 32 tokens, one per
+// lane, and each of its kColSplit warps an equal share of the experts: consecutive lanes read
+// consecutive words.  The parts of each expert are added in part order (+ bias) as
+// router_topk_kernel adds them.  Each candidate becomes one 64-bit key whose unsigned
+// order is the picks' order: the high word maps the value's bits to an increasing
+// integer (-0 counted as +0, NaN below every number), the low word is ~e (a lower index
+// ranks higher on equal values).  The experts go in chunks of eight: a sorting network
+// orders a chunk, and a bitonic merge keeps the best eight of the chunk and of the list
+// so far -- no branches, so the lanes never diverge; the warps' lists then merge in a
+// binary tree.  The weights use the same operations, in pick order, as topk_warp: the picks,
+// weights and logits are the ones the warp kernel gives.
+constexpr int kColSplit = 8;  // warps per block of 32 tokens, each ranking an eighth of the experts
+static_assert((kColSplit & (kColSplit - 1)) == 0, "the lists merge in a binary tree");
+
+__device__ __forceinline__ uint64_t pick_key(float v, int e)
+{
+    const uint32_t u = __float_as_uint(v + 0.0f);  // -0 + 0 = +0
+    const uint32_t hi = isnan(v) ? 0u : ((u & 0x80000000u) ? ~u : (u | 0x80000000u));
+    return ((uint64_t)hi << 32) | (uint32_t)~(uint32_t)e;
+}
+__device__ __forceinline__ float key_value(uint64_t key)
+{
+    const uint32_t hi = (uint32_t)(key >> 32);
+    if (hi == 0u) return __uint_as_float(0x7fc00000u);
+    return __uint_as_float((hi & 0x80000000u) ? (hi & 0x7fffffffu) : ~hi);
+}
+__device__ __forceinline__ int key_index(uint64_t key) { return (int)~(uint32_t)key; }
+// compare-exchange: the larger key to a, the smaller to b
+__device__ __forceinline__ void cx(uint64_t &a, uint64_t &b)
+{
+    const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+    a = hi;
+    b = lo;
+}
+// Batcher's odd-even merge sort of eight, descending (19 compare-exchanges)
+__device__ __forceinline__ void sort8_desc(uint64_t (&c)[8])
+{
+    cx(c[0], c[1]); cx(c[2], c[3]); cx(c[4], c[5]); cx(c[6], c[7]);
+    cx(c[0], c[2]); cx(c[1], c[3]); cx(c[4], c[6]); cx(c[5], c[7]);
+    cx(c[1], c[2]); cx(c[5], c[6]);
+    cx(c[0], c[4]); cx(c[1], c[5]); cx(c[2], c[6]); cx(c[3], c[7]);
+    cx(c[2], c[4]); cx(c[3], c[5]);
+    cx(c[1], c[2]); cx(c[3], c[4]); cx(c[5], c[6]);
+}
+// top := the best eight of two descending lists of eight (top and c).  Pairing one list
+// with the other reversed gives a bitonic sequence holding them, which three
+// half-cleaner rounds sort.
+__device__ __forceinline__ void merge8_desc(uint64_t (&top)[8], const uint64_t (&c)[8])
+{
+#pragma unroll
+    for (int j = 0; j < 8; ++j) top[j] = top[j] > c[7 - j] ? top[j] : c[7 - j];
+    cx(top[0], top[4]); cx(top[1], top[5]); cx(top[2], top[6]); cx(top[3], top[7]);
+    cx(top[0], top[2]); cx(top[1], top[3]); cx(top[4], top[6]); cx(top[5], top[7]);
+    cx(top[0], top[1]); cx(top[2], top[3]); cx(top[4], top[5]); cx(top[6], top[7]);
+}
+
 template <int P>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(32 * kColSplit)
     router_topk_cols_kernel(const float *__restrict__ lin, const float *__restrict__ bias, int64_t N, int E, int k,
                             float *__restrict__ logits, int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
 {
-    __shared__ float row[kColTokens][kMaxE + 1];
+    __shared__ uint64_t lists[kColSplit][8][32];  // each warp's best eight, lane-major
     pdl_entry();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t0 = (int64_t)blockIdx.x * kColTokens;
-    const int64_t t = t0 + lane;
-    // warp w: experts w, w + 8, ..., eight at a time with all their loads in flight; lane: token
-    constexpr int kBatch = 8;
-    for (int e0 = warp; e0 < E; e0 += kWarps * kBatch) {
-        float part[kBatch][P];
+    const int64_t t = (int64_t)blockIdx.x * 32 + lane;
+    const bool live = t < N;
+    // warp w ranks experts [e_lo, e_hi): its share, in whole chunks of eight
+    const int span = ((E + kColSplit - 1) / kColSplit + 7) / 8 * 8;
+    const int e_lo = warp * span, e_hi = min(E, e_lo + span);
+    uint64_t top[8];  // the best eight so far, in descending key order; 0 is below every candidate
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int e = e0 + j * kWarps;
+    for (int j = 0; j < 8; ++j) top[j] = 0;
+    const int64_t pstride = (int64_t)E * N;
+    for (int e0 = e_lo; e0 < e_hi; e0 += 8) {
+        float part[8][P];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
 #pragma unroll
             for (int i = 0; i < P; ++i)
-                part[j][i] = (e < E && t < N) ? __ldg(lin + ((int64_t)i * E + e) * N + t) : 0.f;
+                part[u][i] = live && e0 + u < e_hi ? __ldg(lin + i * pstride + (int64_t)(e0 + u) * N + t) : 0.f;
+        uint64_t c[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u;
+            float v = part[u][0];
+#pragma unroll
+            for (int i = 1; i < P; ++i) v += part[u][i];
+            if (e < e_hi && bias) v += bias[e];
+            if (live && e < e_hi && logits) logits[t * E + e] = v;
+            c[u] = e < e_hi ? pick_key(v, e) : 0;
         }
+        sort8_desc(c);
+        merge8_desc(top, c);
+    }
+    // merge the warps' lists in a tree: at distance d, warp w (a multiple of 2d) takes
+    // warp w + d's list
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int e = e0 + j * kWarps;
-            if (e < E) {
-                float v = part[j][0];
+    for (int j = 0; j < 8; ++j) lists[warp][j][lane] = top[j];
 #pragma unroll
-                for (int i = 1; i < P; ++i) v += part[j][i];
-                if (bias) v += bias[e];
-                row[lane][e] = v;
-            }
+    for (int d = 1; d < kColSplit; d <<= 1) {
+        __syncthreads();
+        if (warp % (2 * d) == 0) {
+            uint64_t c[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) c[j] = lists[warp + d][j][lane];
+            merge8_desc(top, c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) lists[warp][j][lane] = top[j];
         }
     }
-    __syncthreads();
-    for (int tt = warp; tt < kColTokens; tt += kWarps) {
-        const int64_t tok = t0 + tt;
-        if (tok >= N) break;
-        if (logits)
-            for (int e = lane; e < E; e += 32) logits[tok * E + e] = row[tt][e];
-        topk_warp(row[tt], E, k, lane, topk_idx + tok * k, topk_w + tok * k);
-    }
+    if (warp > 0 || !live) return;
+    const float l0 = key_value(top[0]);
+    float ex[kMaxK];
+    float den = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+        if (j < k) { ex[j] = expf(key_value(top[j]) - l0); den += ex[j]; }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+        if (j < k) { topk_idx[t * k + j] = key_index(top[j]); topk_w[t * k + j] = ex[j] / den; }
 }
 
 template <int P>
@@ -614,9 +687,8 @@ cudaError_t launch_router(const uint16_t *x, const float *W_gate, const float *b
             g.token_tile = bn; g.ldo = N;
             e = launch_gemm2(g, s);
             if (e != cudaSuccess) return e;
-            return launch_pdl(router_topk_cols_kernel<3>,
-                              dim3((unsigned)((N + kColTokens - 1) / kColTokens)), dim3(kThreads), 0, s, parts,
-                              bias, N, E, k, lbuf, topk_idx, topk_w);
+            return launch_pdl(router_topk_cols_kernel<3>, dim3((unsigned)((N + 31) / 32)), dim3(32 * kColSplit), 0,
+                              s, parts, bias, N, E, k, lbuf, topk_idx, topk_w);
         }
         int bn, S;
         bool single;

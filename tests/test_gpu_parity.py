@@ -103,6 +103,8 @@ ROUTE_CASES = [
     # tensor cores
     (1000, 512, 128, 8, True, True), (512, 512, 160, 6, True, True), (4096, 512, 8, 2, True, True),
     (300, 512, 256, 8, True, True), (777, 512, 37, 3, True, True), (1024, 2048, 128, 8, True, False),
+    # tensor cores, tokens on the M side, one thread per token ranking expert-major logits
+    (16411, 256, 128, 8, True, True), (16411, 256, 37, 3, True, False), (16384, 512, 256, 8, True, True),
 ]
 
 
@@ -196,8 +198,8 @@ def test_route_ties_lower_index_first():
 @pytest.mark.parametrize("N", [5, 1500, 17000])
 def test_route_ties_on_every_path(N):
     """Exact ties at every size, so that each top-k form meets them: the fused and split
-    paths (small N), the tensor-core path with token-major partial logits (N < 8192) and
-    with expert-major ones staged through shared memory (N >= 16384).  x is zero, so
+    paths (small N), the tensor-core path with token-major partial logits (N < 16384) and
+    with expert-major ones ranked one thread per token (N >= 16384).  x is zero, so
     every logit is the bias: ties between the picks, a tie straddling the k-th place, and
     -0 against +0."""
     H, E, k = 256, 32, 8
@@ -532,3 +534,4 @@ def test_shared_experts_on_the_side_stream_give_the_same_bits():
         del g
     finally:
         moe.moe_set_shared_stream(prev)
+
