@@ -599,6 +599,8 @@ def run_ours(args, cfg, world, rank, local):
                              "off": moe.MOE_GATHER_OFF}[args.gather])
     moe.moe_set_microbatches(args.microbatches)
     moe.moe_set_shared_stream(bool(args.shared_stream))
+    moe.moe_set_decode_gemv({"auto": moe.MOE_DECODE_AUTO, "off": moe.MOE_DECODE_OFF,
+                             "on": moe.MOE_DECODE_ON}[args.decode])
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     W = Workload(cfg, args, dev, stream, rank, world)
@@ -719,7 +721,8 @@ def run_ours(args, cfg, world, rank, local):
                    "expert_activations": ("e4m3, one fp32 scale per row (x_perm and h quantized on the device "
                                           "every step)") if a8 else "bf16",
                    "w13_rows": f"gather mode {args.gather}", "microbatches": args.microbatches,
-                   "shared_experts_stream": "second stream" if args.shared_stream else "caller's stream"},
+                   "shared_experts_stream": "second stream" if args.shared_stream else "caller's stream",
+                   "decode_gemv": args.decode},
         "roofline": roofline,
         "layer": layer,
         "grouped_gemm": gg,
@@ -900,6 +903,9 @@ def main():
                     help="routed-expert activation format (fp8: e4m3 with per-row scales; needs --weights fp8)")
     ap.add_argument("--microbatches", type=int, choices=[1, 2], default=1,
                     help="run large layers as two micro-batches on two streams (moe_set_microbatches)")
+    ap.add_argument("--decode", choices=["auto", "off", "on"], default="auto",
+                    help="decode batches: expert FFN as CUDA-core GEMVs with the combine folded in "
+                         "(moe_set_decode_gemv)")
     ap.add_argument("--shared-stream", type=int, choices=[0, 1], default=1,
                     help="run the shared experts on a second stream beside the dispatch (moe_set_shared_stream)")
     ap.add_argument("--ep", action="store_true",

@@ -20,6 +20,7 @@ std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_gather_mode{MOE_GATHER_AUTO};
 std::atomic<int> g_microbatches{1};
 std::atomic<int> g_shared_side{1};
+std::atomic<int> g_decode_gemv{MOE_DECODE_AUTO};
 }  // namespace
 int layer_microbatches() { return g_microbatches.load(std::memory_order_relaxed); }
 bool layer_shared_side() { return g_shared_side.load(std::memory_order_relaxed) != 0; }
@@ -38,6 +39,24 @@ bool layer_gathers(int64_t N, int k, int H)
     if (mode == MOE_GATHER_ON) return true;
     (void)N; (void)k; (void)H;
     return false;
+}
+
+// Whether the bf16 layer runs its expert FFN as the decode GEMV kernels.  By default for
+// batches of at most a quarter of an assignment per expert on average (4 N*k <= E), with
+// H <= 2048 and I <= 1024, where the grouped GEMM's tiles leave SMs idle and pay their
+// pipeline's setup for a token or two.  Measured (graph replay): at the Qwen3-30B shape
+// (H = 2048, I = 768, E = 128, top-8) N = 1, 2, 4 took 33 / 48 / 77 us against 43 / 62 /
+// 86 us through the grouped GEMMs, N = 8 and 16 128 / 227 against 119 / 166; at the
+// DeepSeek-V2 shape (H = 5120, I = 1536) N = 4 took 283 against 237 us -- a GEMV lane
+// holds its loads in flight in registers, and longer rows need more rounds of them,
+// where the grouped GEMM keeps 200 KB in flight in shared memory.
+bool layer_decode_gemv(int64_t N, int k, int E, int H, int I)
+{
+    const int mode = g_decode_gemv.load(std::memory_order_relaxed);
+    if (mode == MOE_DECODE_OFF) return false;
+    const int64_t R = N * k;
+    if (mode == MOE_DECODE_ON) return R <= MOE_DECODE_MAX_ROWS;
+    return R <= MOE_DECODE_MAX_ROWS && 4 * R <= (int64_t)E && H <= 2048 && I <= 1024;
 }
 
 void *current_context()
@@ -293,12 +312,16 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
     set_weights13(&a, X);
     const bool gather = !X.a8 && !X.fp8 && moe::layer_gathers(N, k, H);
+    // a decode batch in bf16: the expert FFN as GEMVs on CUDA cores, which read x through
+    // the row maps (no row copies) and fold in the combine
+    const bool gemv = !X.a8 && !X.fp8 && !gather && moe::layer_decode_gemv(N, k, E, H, I);
     // a small batch: router, top-k, dispatch and the row copies in two kernels (the
     // route phase then holds the permute phase's work too)
     cudaError_t fused = cudaErrorNotSupported;
     if (!X.a8 && !gather) {
         fused = moe::launch_route_dispatch_small(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router,
-                                                 L.router_bytes, counts, offsets, r2t, t2r, x_perm, err, s);
+                                                 L.router_bytes, counts, offsets, r2t, t2r,
+                                                 gemv ? nullptr : x_perm, err, s);
         if (fused != cudaSuccess && fused != cudaErrorNotSupported) return cuda_fail(fused);
     }
     if (fused != cudaSuccess)
@@ -323,8 +346,8 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
         MOE_CUDA(moe::launch_scatter_rows(reinterpret_cast<const uint16_t *>(Q.xqt), Q.xst, t2r, N, k, H / 2,
                                           reinterpret_cast<uint16_t *>(Q.xq), R, Q.xsc, s));
         a.act = Q.xq; a.a8 = true; a.scale_act = Q.xsc;
-    } else if (gather) {
-        // dispatch only: W1/W3 gathers its rows from x through row_to_token
+    } else if (gather || gemv) {
+        // dispatch only: W1/W3 reads its rows from x through row_to_token
         MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
         a.act = x; a.gather_rows = r2t; a.gather_src_rows = N;
     } else {
@@ -333,6 +356,21 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
     MOE_TRY(after_dispatch());
+    if (gemv) {
+        const auto *W1 = static_cast<const uint16_t *>(X.W1), *W3 = static_cast<const uint16_t *>(X.W3);
+        MOE_CUDA(moe::launch_decode_w13(x, offsets, r2t, N, k, E, H, I, W1, W3, h, err, s));
+        MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
+        // the W2 kernel adds the shared experts' output: it must be complete (with phase
+        // events, the gemm2 phase holds the shared experts and the combine)
+        if (Is > 0) {
+            if (side) MOE_CUDA(cudaStreamWaitEvent(s, side->join, 0));
+            else MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
+        }
+        MOE_CUDA(moe::launch_decode_w2_combine(h, idx, t2r, w, sh, N, E, H, I, k,
+                                               static_cast<const uint16_t *>(X.W2), out, err, s));
+        for (int p : {MOE_PHASE_GEMM2, MOE_PHASE_SHARED, MOE_PHASE_COMBINE}) MOE_TRY(record(phase_events, 1 + p, s));
+        return MOE_OK;
+    }
     MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     const int ksplit = moe::gemm2_ksplit(R, E, I, H);
     moe::GroupedGemmArgs b{};
@@ -524,6 +562,12 @@ int moe_set_shared_stream(int on)
 {
     if (on != 0 && on != 1) return -1;
     return moe::g_shared_side.exchange(on);
+}
+
+int moe_set_decode_gemv(int mode)
+{
+    if (mode != MOE_DECODE_AUTO && mode != MOE_DECODE_OFF && mode != MOE_DECODE_ON) return -1;
+    return moe::g_decode_gemv.exchange(mode);
 }
 
 int moe_set_microbatches(int m)

@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads)
 // so far -- no branches, so the lanes never diverge; the warps' lists then merge in a
 // binary tree.  The weights use the same operations, in pick order, as topk_warp: the picks,
 // weights and logits are the ones the warp kernel gives.
-constexpr int kColSplit = 8;  // warps per block of 32 tokens, each ranking an eighth of the experts
+constexpr int kColSplit = 4;  // warps per block of 32 tokens, each ranking a quarter of the experts
 static_assert((kColSplit & (kColSplit - 1)) == 0, "the lists merge in a binary tree");
 
 __device__ __forceinline__ uint64_t pick_key(float v, int e)
@@ -425,7 +425,9 @@ __global__ void __launch_bounds__(kDispThreads)
                    lead ? row_to_token : nullptr, s_t2r, lead ? err : nullptr, sm);
     if (lead)
         for (int64_t a = threadIdx.x; a < R; a += kDispThreads) token_to_row[a] = s_t2r[a];
-    // x_perm[token_to_row[t,j]] = x[t] for this block's tokens t (16-byte vectors)
+    // x_perm[token_to_row[t,j]] = x[t] for this block's tokens t (16-byte vectors);
+    // no x_perm: dispatch only (the expert kernels read x through the row maps)
+    if (!x_perm) return;
     const int nvec = H / 8;
     for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
@@ -446,7 +448,7 @@ cudaError_t launch_route_dispatch(const float *lin, int64_t pstride, int64_t tst
                                   uint16_t *x_perm, int *err, cudaStream_t s)
 {
     const int64_t cap = 2 * (int64_t)device_sm_count();
-    const unsigned grid = (unsigned)(N < cap ? N : cap);
+    const unsigned grid = x_perm ? (unsigned)(N < cap ? N : cap) : 1u;  // without rows to copy, block 0 alone
     return launch_pdl(route_dispatch_small_kernel<P>, dim3(grid), dim3(kDispThreads), 0, s, lin, pstride, tstride,
                       bias, N, E, k, logits, topk_idx, topk_w, x, H, counts, offsets, r2t, t2r, x_perm, err);
 }

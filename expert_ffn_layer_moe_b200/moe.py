@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.moe_set_microbatches.restype = c_int
         L.moe_set_shared_stream.argtypes = [c_int]
         L.moe_set_shared_stream.restype = c_int
+        L.moe_set_decode_gemv.argtypes = [c_int]
+        L.moe_set_decode_gemv.restype = c_int
         L.moe_ipc_export.argtypes = [vp, vp, ctypes.POINTER(sz)]
         L.moe_ipc_import.argtypes = [vp, sz, ctypes.POINTER(vp)]
         L.moe_ipc_close.argtypes = [vp, sz]
@@ -178,6 +180,21 @@ def moe_set_shared_stream(on: bool) -> bool:
     """Run the shared experts on a second stream beside the dispatch; returns the
     previous setting."""
     return bool(lib().moe_set_shared_stream(1 if on else 0))
+
+
+MOE_DECODE_AUTO, MOE_DECODE_OFF, MOE_DECODE_ON = 0, 1, 2
+MOE_DECODE_MAX_ROWS = 512
+
+
+def moe_set_decode_gemv(mode: int) -> int:
+    """How bf16 layer calls run the expert FFN of decode batches: MOE_DECODE_AUTO (the
+    CUDA-core GEMV kernels for 4*N*k <= E, H <= 2048, I <= 1024), MOE_DECODE_OFF
+    (always the grouped GEMMs), MOE_DECODE_ON (the GEMV kernels whenever N*k <=
+    MOE_DECODE_MAX_ROWS).  Returns the previous mode."""
+    prev = int(lib().moe_set_decode_gemv(int(mode)))
+    if prev < 0:
+        raise ValueError(f"decode mode {mode} is not one of MOE_DECODE_AUTO/OFF/ON")
+    return prev
 
 
 def moe_kernel_launches() -> int:

@@ -409,6 +409,33 @@ MOE_API int moe_set_microbatches(int m);
 MOE_API int moe_set_shared_stream(int on);
 
 /*
+ * How the bf16 layer calls (moe_layer_forward_ex, moe_layer_forward) run the routed
+ * experts' FFN for decode batches (MoE-latency article, section "router 之后还有一串
+ * 动作": at decode, launches, weight reads and row moves are the cost).  With a token or
+ * two per expert every expert GEMM is a GEMV: two CUDA-core kernels deal the touched
+ * experts' weight rows evenly over all SMs -- W1/W3 with the SwiGLU, reading x through
+ * row_to_token (no permuted copy), then W2 with the combine folded in (each token's k
+ * products added in pick order in registers, no fp32 expert outputs in memory) --
+ * instead of the tensor-core grouped GEMMs, the row copies and the combine kernel.
+ * Deterministic; the bits differ from the tensor-core path's (another summation order
+ * inside each dot product), within the same fp32 accuracy.
+ *   mode  MOE_DECODE_AUTO (the default: for 4*N*k <= E, at most a quarter of an
+ *         assignment per expert on average, H <= 2048 and I <= 1024 -- where it
+ *         measured faster: the Qwen3-30B shape at 1, 2 and 4 tokens, 33 / 48 / 77 us
+ *         against 43 / 62 / 86 us through the grouped GEMMs, not at 8 tokens nor with
+ *         DeepSeek-V2's longer rows),
+ *         MOE_DECODE_OFF (always the grouped GEMMs), MOE_DECODE_ON (whenever
+ *         N*k <= MOE_DECODE_MAX_ROWS).
+ * fp8 layers always use the grouped GEMMs.  Process-wide; returns the previous mode,
+ * or -1 for a mode outside these three.
+ */
+#define MOE_DECODE_AUTO 0
+#define MOE_DECODE_OFF 1
+#define MOE_DECODE_ON 2
+#define MOE_DECODE_MAX_ROWS 512
+MOE_API int moe_set_decode_gemv(int mode);
+
+/*
  * Kernels this library has launched in this process so far, counted on the host
  * at each successful launch (all threads, all devices; never reset).  The
  * difference across a region is the number of the library's kernels it ran.

@@ -500,11 +500,18 @@ def test_layer_in_two_microbatches_gives_the_same_bits(cfg):
         moe.moe_set_microbatches(prev)
 
 
-def test_shared_experts_on_the_side_stream_give_the_same_bits():
+SIDE_CASES = [
+    MoEConfig("side", N=700, H=256, I=128, E=8, k=2, Is=192),
+    MoEConfig("side_e32", N=800, H=384, I=192, E=32, k=6, Is=256),
+    MoEConfig("side_ragged", N=300, H=256, I=192, E=16, k=2, Is=320),     # ragged shared feature tiles
+]
+
+
+@pytest.mark.parametrize("cfg", SIDE_CASES, ids=lambda c: c.name)
+def test_shared_experts_on_the_side_stream_give_the_same_bits(cfg):
     """The shared experts forked onto the library's second stream after the router and
     joined before the combine: the same bits as on the caller's stream, eager and
     replayed from a CUDA graph (the second stream joins the capture)."""
-    cfg = MoEConfig("side", N=700, H=256, I=128, E=8, k=2, Is=192)
     t = cuda_inputs(cfg, seed=17)
     prev = moe.moe_set_shared_stream(False)
     try:
@@ -535,3 +542,80 @@ def test_shared_experts_on_the_side_stream_give_the_same_bits():
     finally:
         moe.moe_set_shared_stream(prev)
 
+
+
+DECODE_SHAPES = [
+    # (shape, mode): AUTO takes the GEMV kernels for 4*N*k <= E (H <= 2048, I <= 1024); ON up to 512 rows
+    (MoEConfig("dec_one", N=1, H=512, I=256, E=32, k=8), moe.MOE_DECODE_AUTO),
+    (MoEConfig("dec_qwen_shape", N=4, H=2048, I=768, E=128, k=8), moe.MOE_DECODE_AUTO),
+    (MoEConfig("dec_qwen_8", N=8, H=2048, I=768, E=128, k=8), moe.MOE_DECODE_ON),
+    (MoEConfig("dec_long_rows", N=4, H=5120, I=1536, E=160, k=6), moe.MOE_DECODE_ON),  # several load rounds
+    (MoEConfig("dec_qwen_16", N=16, H=2048, I=768, E=128, k=8), moe.MOE_DECODE_ON),
+    (MoEConfig("dec_ragged", N=5, H=320, I=192, E=160, k=6), moe.MOE_DECODE_AUTO),   # rows and K not multiples of 256
+    (MoEConfig("dec_shared", N=3, H=256, I=128, E=64, k=4, Is=192), moe.MOE_DECODE_AUTO),
+    (MoEConfig("dec_crowded", N=40, H=256, I=128, E=8, k=2), moe.MOE_DECODE_ON),     # ~10 tokens per expert
+    (MoEConfig("dec_max", N=64, H=128, I=64, E=256, k=8), moe.MOE_DECODE_ON),        # 512 rows, every expert
+]
+
+
+@pytest.mark.parametrize("cfg,mode", DECODE_SHAPES, ids=[c.name for c, _ in DECODE_SHAPES])
+def test_decode_gemv_layer_matches_oracle(cfg, mode):
+    """The decode form of the layer (W1/W3 + SwiGLU and W2 + combine as CUDA-core GEMVs,
+    x read through row_to_token) against the oracle on every token, with a router bias;
+    deterministic from call to call and under CUDA-graph replay; the launch count shows
+    the form ran (router, dispatch, two GEMV kernels: four, against five or more for the
+    grouped GEMMs)."""
+    t = cuda_inputs(cfg, seed=37)
+    t["bias"] = torch.linspace(-0.3, 0.3, cfg.E, device="cuda")
+    prev = moe.moe_set_decode_gemv(mode)
+    try:
+        n0 = moe.moe_kernel_launches()
+        out, logits = run_layer(cfg, t)
+        launches = moe.moe_kernel_launches() - n0
+        torch.cuda.synchronize()
+        check_layer_against_oracle(cfg, t, out, logits)
+        if cfg.Is == 0 and cfg.N * cfg.k <= 512:
+            assert launches == 4, launches
+        again, _ = run_layer(cfg, t)
+        torch.cuda.synchronize()
+        assert torch.equal(again.view(torch.int16), out.view(torch.int16))
+        ws = torch.empty(moe.moe_workspace_bytes(cfg.N, cfg.H, cfg.I, cfg.E, cfg.k, cfg.Is), dtype=torch.uint8,
+                         device="cuda")
+        o2 = torch.zeros_like(out)
+
+        def step():
+            moe.moe_layer_forward_ex(t["x"], t["W_gate"], t["W1"], t["W3"], t["W2"], cfg.k, bias=t["bias"],
+                                     Ws1=t.get("Ws1"), Ws3=t.get("Ws3"), Ws2=t.get("Ws2"), ws=ws, out=o2,
+                                     stream=torch.cuda.current_stream())
+        step()
+        torch.cuda.synchronize()
+        o2.zero_()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error() == 0
+        assert torch.equal(o2.view(torch.int16), out.view(torch.int16))
+        del g
+    finally:
+        moe.moe_set_decode_gemv(prev)
+
+
+def test_decode_gemv_and_grouped_gemm_agree():
+    """The same decode batch through the GEMV kernels and through the grouped GEMMs:
+    identical routing, and outputs that differ only by the summation order inside each
+    dot product (a few bf16 ulps at most)."""
+    cfg = MoEConfig("dec_agree", N=8, H=1024, I=512, E=64, k=8)
+    t = cuda_inputs(cfg, seed=41)
+    prev = moe.moe_set_decode_gemv(moe.MOE_DECODE_ON)
+    try:
+        a, la = run_layer(cfg, t)
+        moe.moe_set_decode_gemv(moe.MOE_DECODE_OFF)
+        b, lb = run_layer(cfg, t)
+        torch.cuda.synchronize()
+        assert torch.equal(la, lb)
+        d = (a.float() - b.float()).abs()
+        assert bool((d <= 2.0 ** -6 * b.float().abs() + 1e-3).all()), float(d.max())
+    finally:
+        moe.moe_set_decode_gemv(prev)
