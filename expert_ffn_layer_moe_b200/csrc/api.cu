@@ -42,21 +42,21 @@ bool layer_gathers(int64_t N, int k, int H)
 }
 
 // Whether the bf16 layer runs its expert FFN as the decode GEMV kernels.  By default for
-// batches of at most a quarter of an assignment per expert on average (4 N*k <= E), with
+// batches of at most half an assignment per expert on average (2 N*k <= E), with
 // H <= 2048 and I <= 1024, where the grouped GEMM's tiles leave SMs idle and pay their
-// pipeline's setup for a token or two.  Measured (graph replay): at the Qwen3-30B shape
-// (H = 2048, I = 768, E = 128, top-8) N = 1, 2, 4 took 33 / 48 / 77 us against 43 / 62 /
-// 86 us through the grouped GEMMs, N = 8 and 16 128 / 227 against 119 / 166; at the
-// DeepSeek-V2 shape (H = 5120, I = 1536) N = 4 took 283 against 237 us -- a GEMV lane
-// holds its loads in flight in registers, and longer rows need more rounds of them,
-// where the grouped GEMM keeps 200 KB in flight in shared memory.
+// pipeline's setup for a token or two.  Measured (graph replay) at the Qwen3-30B shape
+// (H = 2048, I = 768, E = 128, top-8): N = 1, 2, 4, 8 took 28 / 41 / 67 / 111 us against
+// 43 / 62 / 86 / 118 us through the grouped GEMMs.  At the DeepSeek-V2 shape (H = 5120,
+// I = 1536) an earlier form lost at N = 4 (283 against 237 us): a GEMV lane holds its
+// loads in flight in registers, and longer rows need more rounds of them, where the
+// grouped GEMM keeps 200 KB in flight in shared memory.
 bool layer_decode_gemv(int64_t N, int k, int E, int H, int I)
 {
     const int mode = g_decode_gemv.load(std::memory_order_relaxed);
-    if (mode == MOE_DECODE_OFF) return false;
     const int64_t R = N * k;
-    if (mode == MOE_DECODE_ON) return R <= MOE_DECODE_MAX_ROWS;
-    return R <= MOE_DECODE_MAX_ROWS && 4 * R <= (int64_t)E && H <= 2048 && I <= 1024;
+    if (mode == MOE_DECODE_OFF || R > MOE_DECODE_MAX_ROWS || N > MOE_DECODE_MAX_TOKENS) return false;
+    if (mode == MOE_DECODE_ON) return true;
+    return 2 * R <= (int64_t)E && H <= 2048 && I <= 1024;
 }
 
 void *current_context()
@@ -312,16 +312,41 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
     set_weights13(&a, X);
     const bool gather = !X.a8 && !X.fp8 && moe::layer_gathers(N, k, H);
-    // a decode batch in bf16: the expert FFN as GEMVs on CUDA cores, which read x through
-    // the row maps (no row copies) and fold in the combine
-    const bool gemv = !X.a8 && !X.fp8 && !gather && moe::layer_decode_gemv(N, k, E, H, I);
+    if (!X.a8 && !X.fp8 && !gather && moe::layer_decode_gemv(N, k, E, H, I)) {
+        // a decode batch in bf16: the router's partial logits, then the expert FFN as two
+        // GEMV kernels on CUDA cores -- the first finishes the top-k, reads x per pick (no
+        // dispatch, no row copies), the second folds in the combine
+        moe::RouterPartials rp{};
+        MOE_CUDA(moe::launch_router_partials(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router,
+                                             L.router_bytes, &rp, s));
+        for (int p : {MOE_PHASE_ROUTE, MOE_PHASE_PERMUTE}) MOE_TRY(record(phase_events, 1 + p, s));
+        if (side && Is > 0) {
+            MOE_CUDA(cudaEventRecord(side->fork, s));
+            MOE_CUDA(cudaStreamWaitEvent(side->s2, side->fork, 0));
+            MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, side->s2));
+            MOE_CUDA(cudaEventRecord(side->join, side->s2));
+        }
+        MOE_TRY(after_dispatch());
+        MOE_CUDA(moe::launch_decode_w13(x, rp, idx, w, N, k, E, H, I, static_cast<const uint16_t *>(X.W1),
+                                        static_cast<const uint16_t *>(X.W3), h, err, s));
+        MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
+        // the W2 kernel adds the shared experts' output: it must be complete (with phase
+        // events, the gemm2 phase holds the shared experts and the combine)
+        if (Is > 0) {
+            if (side) MOE_CUDA(cudaStreamWaitEvent(s, side->join, 0));
+            else MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
+        }
+        MOE_CUDA(moe::launch_decode_w2_combine(h, idx, w, sh, N, E, H, I, k, static_cast<const uint16_t *>(X.W2),
+                                               out, err, s));
+        for (int p : {MOE_PHASE_GEMM2, MOE_PHASE_SHARED, MOE_PHASE_COMBINE}) MOE_TRY(record(phase_events, 1 + p, s));
+        return MOE_OK;
+    }
     // a small batch: router, top-k, dispatch and the row copies in two kernels (the
     // route phase then holds the permute phase's work too)
     cudaError_t fused = cudaErrorNotSupported;
     if (!X.a8 && !gather) {
         fused = moe::launch_route_dispatch_small(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router,
-                                                 L.router_bytes, counts, offsets, r2t, t2r,
-                                                 gemv ? nullptr : x_perm, err, s);
+                                                 L.router_bytes, counts, offsets, r2t, t2r, x_perm, err, s);
         if (fused != cudaSuccess && fused != cudaErrorNotSupported) return cuda_fail(fused);
     }
     if (fused != cudaSuccess)
@@ -346,8 +371,8 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
         MOE_CUDA(moe::launch_scatter_rows(reinterpret_cast<const uint16_t *>(Q.xqt), Q.xst, t2r, N, k, H / 2,
                                           reinterpret_cast<uint16_t *>(Q.xq), R, Q.xsc, s));
         a.act = Q.xq; a.a8 = true; a.scale_act = Q.xsc;
-    } else if (gather || gemv) {
-        // dispatch only: W1/W3 reads its rows from x through row_to_token
+    } else if (gather) {
+        // dispatch only: W1/W3 gathers its rows from x through row_to_token
         MOE_CUDA(moe::launch_permute(x, idx, N, H, E, k, counts, offsets, r2t, t2r, nullptr, perm, err, s));
         a.act = x; a.gather_rows = r2t; a.gather_src_rows = N;
     } else {
@@ -356,21 +381,6 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     }
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_PERMUTE, s));
     MOE_TRY(after_dispatch());
-    if (gemv) {
-        const auto *W1 = static_cast<const uint16_t *>(X.W1), *W3 = static_cast<const uint16_t *>(X.W3);
-        MOE_CUDA(moe::launch_decode_w13(x, offsets, r2t, N, k, E, H, I, W1, W3, h, err, s));
-        MOE_TRY(record(phase_events, 1 + MOE_PHASE_GEMM13, s));
-        // the W2 kernel adds the shared experts' output: it must be complete (with phase
-        // events, the gemm2 phase holds the shared experts and the combine)
-        if (Is > 0) {
-            if (side) MOE_CUDA(cudaStreamWaitEvent(s, side->join, 0));
-            else MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, s));
-        }
-        MOE_CUDA(moe::launch_decode_w2_combine(h, idx, t2r, w, sh, N, E, H, I, k,
-                                               static_cast<const uint16_t *>(X.W2), out, err, s));
-        for (int p : {MOE_PHASE_GEMM2, MOE_PHASE_SHARED, MOE_PHASE_COMBINE}) MOE_TRY(record(phase_events, 1 + p, s));
-        return MOE_OK;
-    }
     MOE_CUDA(moe::launch_gemm13_swiglu(a, s));
     const int ksplit = moe::gemm2_ksplit(R, E, I, H);
     moe::GroupedGemmArgs b{};

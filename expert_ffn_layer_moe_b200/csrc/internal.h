@@ -119,15 +119,30 @@ int device_sm_count();
 // e4m3 weights with one fp32 scale per row: q [rows, K] bytes, scale [rows].
 cudaError_t launch_quantize_fp8(const uint16_t *W, int64_t rows, int K, uint8_t *q, float *scale, cudaStream_t s);
 
-// The expert FFN of a decode batch on CUDA cores (a token or two per expert): W1/W3 with
-// the SwiGLU, h [N*k, I] in row order, x read through row_to_token; then W2 with the
-// combine folded in (out written, no fp32 expert outputs).
-cudaError_t launch_decode_w13(const uint16_t *x, const int32_t *offsets, const int32_t *row_to_token, int64_t N,
-                              int k, int E, int H, int I, const uint16_t *W1, const uint16_t *W3, uint16_t *h,
-                              int *err, cudaStream_t s);
-cudaError_t launch_decode_w2_combine(const uint16_t *h, const int32_t *topk_idx, const int32_t *token_to_row,
-                                     const float *topk_w, const float *shared_out, int64_t N, int E, int H, int I,
-                                     int k, const uint16_t *W2, uint16_t *out, int *err, cudaStream_t s);
+// The router's partial logits of a decode batch, for the first decode kernel to rank:
+// part [P][N][E] (pstride = N*E), summed in slice order (+ bias when bias is given;
+// written to logits when given).  P = 0: the picks are already in topk_idx/topk_w.
+struct RouterPartials {
+    const float *part;
+    int P;
+    int64_t pstride;
+    const float *bias;
+    float *logits;
+};
+cudaError_t launch_router_partials(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
+                                   int k, float *logits, int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes,
+                                   RouterPartials *rp, cudaStream_t s);
+
+// The expert FFN of a decode batch on CUDA cores (a few tokens): W1/W3 with the SwiGLU
+// over (pick, feature) units -- its blocks finish the router's top-k from the partial
+// logits first, and block 0 writes the picks and weights -- h [N*k, I] in pick order
+// (row t*k + j); then W2 with the combine folded in (out written, no fp32 expert outputs).
+cudaError_t launch_decode_w13(const uint16_t *x, const RouterPartials &rp, int32_t *topk_idx, float *topk_w,
+                              int64_t N, int k, int E, int H, int I, const uint16_t *W1, const uint16_t *W3,
+                              uint16_t *h, int *err, cudaStream_t s);
+cudaError_t launch_decode_w2_combine(const uint16_t *h, const int32_t *topk_idx, const float *topk_w,
+                                     const float *shared_out, int64_t N, int E, int H, int I, int k,
+                                     const uint16_t *W2, uint16_t *out, int *err, cudaStream_t s);
 // Whether the layer runs its expert FFN with the kernels above (moe_set_decode_gemv).
 bool layer_decode_gemv(int64_t N, int k, int E, int H, int I);
 

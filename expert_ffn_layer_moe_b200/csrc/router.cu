@@ -651,6 +651,57 @@ cudaError_t launch_route_dispatch_small(const uint16_t *x, const float *W_gate, 
                                     row_to_token, token_to_row, x_perm, dev_err, s);
 }
 
+// Decode batches: the router's partial logits only; the top-k runs in the first decode
+// GEMV kernel (every block ranks the few tokens itself).  With the one-kernel router
+// (one slice of H and E <= 16) the picks are made here instead (rp->P = 0).
+cudaError_t launch_router_partials(const uint16_t *x, const float *W_gate, const float *bias, int64_t N, int H, int E,
+                                   int k, float *logits, int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes,
+                                   RouterPartials *rp, cudaStream_t s)
+{
+    if (N <= 0 || N > kFuseMaxTopkN) return cudaErrorNotSupported;
+    const bool have_ws = ws != nullptr && ws_bytes >= router_ws_bytes(N, H, E);
+    const RouterPath path = router_path(N, E, logits != nullptr, have_ws);
+    if (path == RouterPath::kTensor) return cudaErrorNotSupported;
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    const size_t split_bytes = align256((size_t)3 * E * H * 2);
+    const size_t parts_bytes = align256((size_t)kTensorMaxSlices * N * 3 * E * 4);
+    float *lbuf = logits ? logits : (have_ws ? reinterpret_cast<float *>(w8 + split_bytes + parts_bytes) : nullptr);
+    if (path == RouterPath::kSplit) {
+        float *part = have_ws ? reinterpret_cast<float *>(w8) : lbuf;
+        const int64_t zcap = have_ws ? (int64_t)((split_bytes + parts_bytes) / ((size_t)N * E * 4)) : 1;
+        int tt, z;
+        split_shape(N, H, E, zcap, &tt, &z);
+        if (!(z == 1 && E <= 2 * kEC)) {
+            if (z == 1) part = lbuf;
+            const int hz = (H / z / kChunk) * kChunk;
+            const dim3 grid((unsigned)((N + tt - 1) / tt), (unsigned)((E + kEC - 1) / kEC), (unsigned)z);
+            cudaError_t e;
+            switch (tt) {
+                case 4: e = launch_pdl(router_partial_kernel<4>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H, E,
+                                       hz, part); break;
+                case 2: e = launch_pdl(router_partial_kernel<2>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H, E,
+                                       hz, part); break;
+                default: e = launch_pdl(router_partial_kernel<1>, grid, dim3(kThreads), 0, s, x, W_gate, bias, N, H,
+                                        E, hz, part); break;
+            }
+            if (e != cudaSuccess) return e;
+            // z == 1: `part` holds the logits, bias included
+            rp->part = part;
+            rp->P = z;
+            rp->pstride = N * E;
+            rp->bias = z == 1 ? nullptr : bias;
+            rp->logits = z == 1 ? nullptr : lbuf;
+            return cudaSuccess;
+        }
+    }
+    rp->part = nullptr;
+    rp->P = 0;
+    rp->pstride = 0;
+    rp->bias = nullptr;
+    rp->logits = nullptr;
+    return launch_fused_for(x, W_gate, bias, N, H, E, k, logits, topk_idx, topk_w, s);
+}
+
 size_t router_ws_bytes(int64_t N, int H, int E)
 {
     return align256((size_t)3 * E * H * 2) + align256((size_t)kTensorMaxSlices * N * 3 * E * 4) +

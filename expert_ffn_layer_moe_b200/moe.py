@@ -184,11 +184,12 @@ def moe_set_shared_stream(on: bool) -> bool:
 
 MOE_DECODE_AUTO, MOE_DECODE_OFF, MOE_DECODE_ON = 0, 1, 2
 MOE_DECODE_MAX_ROWS = 512
+MOE_DECODE_MAX_TOKENS = 64
 
 
 def moe_set_decode_gemv(mode: int) -> int:
     """How bf16 layer calls run the expert FFN of decode batches: MOE_DECODE_AUTO (the
-    CUDA-core GEMV kernels for 4*N*k <= E, H <= 2048, I <= 1024), MOE_DECODE_OFF
+    CUDA-core GEMV kernels for 2*N*k <= E, H <= 2048, I <= 1024), MOE_DECODE_OFF
     (always the grouped GEMMs), MOE_DECODE_ON (the GEMV kernels whenever N*k <=
     MOE_DECODE_MAX_ROWS).  Returns the previous mode."""
     prev = int(lib().moe_set_decode_gemv(int(mode)))

@@ -411,28 +411,33 @@ MOE_API int moe_set_shared_stream(int on);
 /*
  * How the bf16 layer calls (moe_layer_forward_ex, moe_layer_forward) run the routed
  * experts' FFN for decode batches (MoE-latency article, section "router 之后还有一串
- * 动作": at decode, launches, weight reads and row moves are the cost).  With a token or
- * two per expert every expert GEMM is a GEMV: two CUDA-core kernels deal the touched
- * experts' weight rows evenly over all SMs -- W1/W3 with the SwiGLU, reading x through
- * row_to_token (no permuted copy), then W2 with the combine folded in (each token's k
- * products added in pick order in registers, no fp32 expert outputs in memory) --
- * instead of the tensor-core grouped GEMMs, the row copies and the combine kernel.
+ * 动作": at decode, launches, weight reads and row moves are the cost).  With a few
+ * tokens every expert GEMM is a GEMV: after the router's partial logits, two CUDA-core
+ * kernels deal the picked experts' weight rows evenly over all SMs -- W1/W3 with the
+ * SwiGLU, per pick (each block first finishes the top-k itself; no dispatch, no row
+ * copies), then W2 with the combine folded in (each token's k products added in pick
+ * order in registers, no fp32 expert outputs in memory) -- instead of the top-k and
+ * dispatch kernel, the tensor-core grouped GEMMs and the combine kernel: three
+ * launches in all.  The picks, weights and logits are the other paths' bits.
  * Deterministic; the bits differ from the tensor-core path's (another summation order
  * inside each dot product), within the same fp32 accuracy.
- *   mode  MOE_DECODE_AUTO (the default: for 4*N*k <= E, at most a quarter of an
- *         assignment per expert on average, H <= 2048 and I <= 1024 -- where it
- *         measured faster: the Qwen3-30B shape at 1, 2 and 4 tokens, 33 / 48 / 77 us
- *         against 43 / 62 / 86 us through the grouped GEMMs, not at 8 tokens nor with
+ * It takes batches of at most MOE_DECODE_MAX_TOKENS tokens and MOE_DECODE_MAX_ROWS
+ * assignments.
+ *   mode  MOE_DECODE_AUTO (the default: for 2*N*k <= E, at most half an assignment
+ *         per expert on average, H <= 2048 and I <= 1024 -- where it measured
+ *         faster: the Qwen3-30B shape at 1, 2, 4 and 8 tokens, 28 / 41 / 67 / 111 us
+ *         against 43 / 62 / 86 / 118 us through the grouped GEMMs; not with
  *         DeepSeek-V2's longer rows),
- *         MOE_DECODE_OFF (always the grouped GEMMs), MOE_DECODE_ON (whenever
- *         N*k <= MOE_DECODE_MAX_ROWS).
+ *         MOE_DECODE_OFF (always the grouped GEMMs), MOE_DECODE_ON (whenever the
+ *         batch is within those limits).
  * fp8 layers always use the grouped GEMMs.  Process-wide; returns the previous mode,
  * or -1 for a mode outside these three.
  */
 #define MOE_DECODE_AUTO 0
 #define MOE_DECODE_OFF 1
 #define MOE_DECODE_ON 2
-#define MOE_DECODE_MAX_ROWS 512
+#define MOE_DECODE_MAX_ROWS 512  /* N*k */
+#define MOE_DECODE_MAX_TOKENS 64 /* N: every block of the first kernel ranks the batch */
 MOE_API int moe_set_decode_gemv(int mode);
 
 /*
