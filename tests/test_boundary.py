@@ -122,3 +122,34 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(moe, "_LIB_PATH", "/nonexistent/libmoe_b200.so")
     with pytest.raises(RuntimeError, match="not built"):
         moe.lib()
+
+
+def test_process_wide_options_round_trip_and_reject_bad_values():
+    """Every option setter returns the previous setting, takes effect for later calls,
+    and refuses values outside its range (-1 from C, ValueError from the binding),
+    all without a GPU."""
+    L = moe.lib()
+    cases = [  # (setter, valid values, default, a rejected value)
+        (L.moe_set_gather_mode, [moe.MOE_GATHER_OFF, moe.MOE_GATHER_ON, moe.MOE_GATHER_AUTO], moe.MOE_GATHER_AUTO, 7),
+        (L.moe_set_microbatches, [2, 1], 1, 3),
+        (L.moe_set_shared_stream, [0, 1], 1, 2),
+        (L.moe_set_decode_gemv, [moe.MOE_DECODE_OFF, moe.MOE_DECODE_ON, moe.MOE_DECODE_AUTO], moe.MOE_DECODE_AUTO, -1),
+    ]
+    for setter, values, default, bad in cases:
+        prev = setter(default)
+        try:
+            assert prev == default          # nothing else in this process changed it
+            last = default
+            for v in values:
+                assert setter(v) == last
+                last = v
+            assert setter(bad) == -1        # refused, and the setting is unchanged
+            assert setter(default) == last
+        finally:
+            setter(default)
+    with pytest.raises(ValueError):
+        moe.moe_set_decode_gemv(5)
+    with pytest.raises(ValueError):
+        moe.moe_set_gather_mode(9)
+    with pytest.raises(ValueError):
+        moe.moe_set_microbatches(0)
