@@ -307,6 +307,14 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     const int64_t R = N * k;
 
     MOE_TRY(record(phase_events, 0, s));
+    if (side && Is > 0) {
+        // the shared experts need only x: they start at once on the side stream, beside the
+        // router and the dispatch, and are joined before whatever adds their output
+        MOE_CUDA(cudaEventRecord(side->fork, s));
+        MOE_CUDA(cudaStreamWaitEvent(side->s2, side->fork, 0));
+        MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, side->s2));
+        MOE_CUDA(cudaEventRecord(side->join, side->s2));
+    }
     moe::GroupedGemmArgs a{};
     a.offsets = offsets; a.groups = E; a.R = R;
     a.K = H; a.Nout = I; a.out = h; a.dev_err = err;
@@ -320,12 +328,6 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
         MOE_CUDA(moe::launch_router_partials(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router,
                                              L.router_bytes, &rp, s));
         for (int p : {MOE_PHASE_ROUTE, MOE_PHASE_PERMUTE}) MOE_TRY(record(phase_events, 1 + p, s));
-        if (side && Is > 0) {
-            MOE_CUDA(cudaEventRecord(side->fork, s));
-            MOE_CUDA(cudaStreamWaitEvent(side->s2, side->fork, 0));
-            MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, side->s2));
-            MOE_CUDA(cudaEventRecord(side->join, side->s2));
-        }
         MOE_TRY(after_dispatch());
         MOE_CUDA(moe::launch_decode_w13(x, rp, idx, w, N, k, E, H, I, static_cast<const uint16_t *>(X.W1),
                                         static_cast<const uint16_t *>(X.W3), h, err, s));
@@ -352,14 +354,6 @@ moe_status_t layer_run(const uint16_t *x, const float *W_gate, const float *bias
     if (fused != cudaSuccess)
         MOE_CUDA(moe::launch_router(x, W_gate, bias, N, H, E, k, lg, idx, w, base + L.router, L.router_bytes, err, s));
     MOE_TRY(record(phase_events, 1 + MOE_PHASE_ROUTE, s));
-    if (side && Is > 0) {
-        // the shared experts need only x: they start now on the side stream, beside the
-        // dispatch, and are joined before the combine
-        MOE_CUDA(cudaEventRecord(side->fork, s));
-        MOE_CUDA(cudaStreamWaitEvent(side->s2, side->fork, 0));
-        MOE_TRY(shared_ffn_impl(x, Ws1, Ws3, Ws2, N, H, Is, hs, sh, err, side->s2));
-        MOE_CUDA(cudaEventRecord(side->join, side->s2));
-    }
     if (fused == cudaSuccess) {
         a.act = x_perm;
     } else if (X.a8) {

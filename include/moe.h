@@ -397,10 +397,11 @@ MOE_API int moe_set_microbatches(int m);
 
 /*
  * Where the layer calls run the always-on shared experts ([FinDEP] "问题定义").
- * on = 1 (the default): on a second stream of the library's, forked right after the
- * router and joined before the combine, so the dispatch and row copies of the routed
- * experts run beside the shared experts' GEMMs (measured 3% faster at the
- * DeepSeek-V2 shape); on = 0: on the caller's stream after the routed experts.  Same
+ * on = 1 (the default): on a second stream of the library's, forked at the start of
+ * the call and joined before the combine, so the router, the dispatch and the row
+ * copies of the routed experts run beside the shared experts' GEMMs (measured 5%
+ * faster at the DeepSeek-V2 shape); on = 0: on the caller's stream after the routed
+ * experts.  Same
  * results either way.  The first call with shared experts on a device creates the
  * stream (and two events) for the process; make it before any stream capture.  A
  * call with phase events runs on the caller's stream.  Process-wide; returns the

@@ -509,8 +509,8 @@ SIDE_CASES = [
 
 @pytest.mark.parametrize("cfg", SIDE_CASES, ids=lambda c: c.name)
 def test_shared_experts_on_the_side_stream_give_the_same_bits(cfg):
-    """The shared experts forked onto the library's second stream after the router and
-    joined before the combine: the same bits as on the caller's stream, eager and
+    """The shared experts forked onto the library's second stream at the start of the
+    call and joined before the combine: the same bits as on the caller's stream, eager and
     replayed from a CUDA graph (the second stream joins the capture)."""
     t = cuda_inputs(cfg, seed=17)
     prev = moe.moe_set_shared_stream(False)
