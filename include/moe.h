@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1, /* a size or pointer is out of the documented range */
-    MOE_ERR_UNSUPPORTED = 2, /* a valid request this build does not handle (alignment, device) */
+    MOE_ERR_UNSUPPORTED = 2, /* a valid request this library does not handle (alignment, device) */
     MOE_ERR_WORKSPACE = 3,   /* workspace pointer NULL or smaller than moe_workspace_bytes() */
     MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed; see moe_last_cuda_error() */
     MOE_ERR_DEVICE = 5       /* a kernel reported a device-side fault (moe_get_device_error) */
