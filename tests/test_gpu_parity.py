@@ -556,6 +556,8 @@ DECODE_SHAPES = [
     (MoEConfig("dec_shared", N=3, H=256, I=128, E=64, k=4, Is=192), moe.MOE_DECODE_AUTO),
     (MoEConfig("dec_crowded", N=40, H=256, I=128, E=8, k=2), moe.MOE_DECODE_ON),     # ~10 tokens per expert
     (MoEConfig("dec_max", N=64, H=128, I=64, E=256, k=8), moe.MOE_DECODE_ON),        # 512 rows, every expert
+    (MoEConfig("dec_dense", N=3, H=256, I=128, E=1, k=1), moe.MOE_DECODE_ON),        # one expert, top-1
+    (MoEConfig("dec_router_fused", N=2, H=192, I=128, E=16, k=2), moe.MOE_DECODE_AUTO),  # the one-kernel router picks
 ]
 
 
