@@ -53,7 +53,19 @@ def fit_multilinear(cols: Sequence[Sequence[float]], t: Sequence[float]) -> Tupl
 
 
 def measure(config: str, tokens: Sequence[int], steps: int = 10, warmup: int = 3) -> List[Dict]:
-    """CUDA-event times of the layer and of its two grouped GEMMs at each N."""
+    """CUDA-event times of the layer and of its two grouped GEMMs at each N (the grouped
+    GEMMs at every N: the decode kernels, which the layer takes for a few tokens, are
+    another model and stay off here)."""
+    from expert_ffn_layer_moe_b200 import moe
+
+    prev = moe.moe_set_decode_gemv(moe.MOE_DECODE_OFF)
+    try:
+        return _measure(config, tokens, steps, warmup)
+    finally:
+        moe.moe_set_decode_gemv(prev)
+
+
+def _measure(config: str, tokens: Sequence[int], steps: int, warmup: int) -> List[Dict]:
     import torch
 
     from expert_ffn_layer_moe_b200 import moe
