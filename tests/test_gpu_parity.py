@@ -220,7 +220,8 @@ def test_route_ties_on_every_path(N):
     assert np.allclose(host(w), ref_w, rtol=4 * 2.0 ** -23, atol=1e-7)
 
 
-@pytest.mark.parametrize("N,E,k", [(64, 8, 2), (1000, 160, 6), (3000, 128, 8), (7, 4, 4), (1, 1, 1)])
+@pytest.mark.parametrize("N,E,k", [(64, 8, 2), (1000, 160, 6), (3000, 128, 8), (7, 4, 4), (1, 1, 1),
+                                   (128, 64, 8), (129, 64, 8), (256, 128, 8)])  # one block up to 1024 rows
 def test_permute_bit_exact(N, E, k):
     H = 128
     g = torch.Generator().manual_seed(N + E)

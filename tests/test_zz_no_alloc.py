@@ -47,7 +47,7 @@ def _noalloc_via_c_abi(x, idx, E):
     return out
 
 
-# Every case has more than 2048 assignments, so each call takes the count/scan/rank
+# Every case has more than 2048 assignments (above the one-block limit), so each call takes the count/scan/rank
 # dispatch whose per-block histograms live in the fixed array (smaller batches run a
 # one-block dispatch that never touches it).  The cases change E and the block count
 # from call to call, so each call starts on an array that still holds the previous
