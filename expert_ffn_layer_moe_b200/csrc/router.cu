@@ -373,11 +373,11 @@ cudaError_t launch_topk(const float *lin, int64_t pstride, int64_t tstride, cons
 // less than a launch) and then copies the rows of its share of the tokens; block 0 also
 // writes the routing and dispatch outputs.  No block waits on another.
 constexpr int kFuseMaxR = 512;      // assignments of a batch this kernel takes
-// Tokens every block ranks for itself (P > 0).  Past 16 the separate top-k, dispatch and
-// scatter kernels win: measured on the Qwen3-30B shape (whole layer, L2 flushed), 24 / 32 /
-// 48 / 64 tokens took 219 / 248 / 256 / 314 us with every block ranking the batch and
-// 216 / 231 / 243 / 257 us with the limit at 16 (16 tokens: 186 us either way).
-constexpr int kFuseMaxTopkN = 16;
+// Tokens every block ranks for itself (P > 0).  Past 8 the separate top-k, dispatch and
+// scatter kernels win: measured on the Qwen3-30B shape (whole layer, L2 flushed), 10 / 12
+// / 16 / 24 / 32 / 48 / 64 tokens took 158 / 164 / 186 / 219 / 248 / 256 / 314 us with
+// every block ranking the batch and 153 / 161 / 181 / 216 / 231 / 243 / 257 us without.
+constexpr int kFuseMaxTopkN = 8;
 template <int P>
 __global__ void __launch_bounds__(kDispThreads)
     route_dispatch_small_kernel(const float *__restrict__ lin, int64_t pstride, int64_t tstride,
