@@ -170,6 +170,7 @@ void ws_layout(int64_t N, int H, int I, int E, int k, int Is, bool a8, WsLayout 
 // kPermuteChunk), whose per-block table then holds where the second half's rows of every
 // expert start.
 constexpr int64_t kMicroMinRows = 32768;
+static_assert(kMicroMinRows >= moe::kPermuteFineMaxR, "the dispatch of such batches runs blocks of kPermuteChunk");
 int64_t micro_split(int64_t N, int k)
 {
     if (moe::layer_microbatches() < 2 || N * k < kMicroMinRows) return 0;

@@ -64,9 +64,16 @@ cudaError_t launch_route_dispatch_small(const uint16_t *x, const float *W_gate, 
                                         size_t ws_bytes, int32_t *counts, int32_t *offsets, int32_t *row_to_token,
                                         int32_t *token_to_row, uint16_t *x_perm, int *dev_err, cudaStream_t s);
 
-// Dispatch / permutation.  `scratch` holds permute_scratch_ints(R, E) ints.
-constexpr int kPermuteChunk = 1024;  // assignments per block in the count/rank passes
-inline int64_t permute_blocks(int64_t R) { return (R + kPermuteChunk - 1) / kPermuteChunk; }
+// Dispatch / permutation.  `scratch` holds permute_scratch_ints(R, E) ints.  The count and
+// rank passes take blocks of permute_chunk(R) assignments: kPermuteFineChunk below
+// kPermuteFineMaxR assignments (more blocks for mid-sized batches; their rank blocks fold
+// the scan in), kPermuteChunk from there on (the scan kernel then leaves every block's
+// starting row per expert in the scratch).
+constexpr int kPermuteChunk = 1024;
+constexpr int kPermuteFineChunk = 256;
+constexpr int64_t kPermuteFineMaxR = 32768;
+inline int64_t permute_chunk(int64_t R) { return R < kPermuteFineMaxR ? kPermuteFineChunk : kPermuteChunk; }
+inline int64_t permute_blocks(int64_t R) { return (R + permute_chunk(R) - 1) / permute_chunk(R); }
 inline int64_t permute_scratch_ints(int64_t R, int E) { return permute_blocks(R) * E; }
 // x_perm == nullptr: dispatch only (counts, offsets, the two row maps), no row copy.
 cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N, int H, int E,

@@ -6,7 +6,7 @@
 // a = t*k + j of expert e lands at row offsets[e] + #{a' < a : e(a') = e}.
 //
 // No atomics decide the row order.  Large batches take four launches:
-//   1. count  : per block of kPermuteChunk assignments, a per-expert histogram;
+//   1. count  : per block of permute_chunk(R) assignments, a per-expert histogram;
 //   2. scan   : one block -- counts[e], offsets = exclusive scan, and every block's
 //               starting row per expert (in place over the histograms);
 //   3. rank   : per block again, the stable rank of each assignment inside its
@@ -15,7 +15,9 @@
 //               its row once (16-byte vectors) and writes its k copies, so x is read
 //               from HBM once however many experts share a token.
 // Batches of at most kSmallR (1024) assignments do 1-3 in one single-block launch,
-// then the gather: two launches instead of four.
+// then the gather: two launches instead of four.  Mid-sized batches (fewer than
+// kPermuteFineMaxR assignments) take blocks of 256 and fold 2 into 3: each rank block
+// sums the (at most 128) histograms itself, which saves the scan's launch.
 #include "common.cuh"
 #include "dispatch_block.cuh"
 #include "internal.h"
@@ -33,14 +35,15 @@ constexpr int64_t kSmallR = 1024;
 static_assert(kPermuteChunk % kThreads == 0, "chunk is whole rounds of the block");
 
 __global__ void __launch_bounds__(kThreads)
-    count_kernel(const int32_t *__restrict__ idx, int64_t R, int E, int32_t *__restrict__ blk_cnt, int *err)
+    count_kernel(const int32_t *__restrict__ idx, int64_t R, int E, int chunk, int32_t *__restrict__ blk_cnt,
+                 int *err)
 {
     __shared__ int hist[kMaxE];
     pdl_entry();
     for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
     __syncthreads();
-    const int64_t a0 = (int64_t)blockIdx.x * kPermuteChunk;
-    for (int i = threadIdx.x; i < kPermuteChunk; i += kThreads) {
+    const int64_t a0 = (int64_t)blockIdx.x * chunk;
+    for (int i = threadIdx.x; i < chunk; i += kThreads) {
         const int64_t a = a0 + i;
         if (a >= R) break;
         const int e = idx[a];
@@ -111,6 +114,54 @@ __global__ void __launch_bounds__(kThreads)
         if (ar >= R) break;  // uniform across the block
         rank_round(idx, R, k, E, ar, base, wcnt, row_to_token, token_to_row);
     }
+}
+
+// Mid-sized batches: the scan and the rank of one block of kPermuteFineChunk (one round of
+// the block) assignments.  Thread e sums expert e's histogram entries over all nblk
+// blocks (the total) and over the blocks before this one; an exclusive scan of the
+// totals gives offsets, and this block's rows of expert e start at offsets[e] plus the
+// earlier blocks' count.  Block 0 writes counts and offsets.  The histograms stay as they
+// are (every block reads all of them).
+__global__ void __launch_bounds__(kThreads)
+    rank_scan_kernel(const int32_t *__restrict__ idx, int64_t R, int k, int E,
+                     const int32_t *__restrict__ blk_cnt, int64_t nblk, int32_t *__restrict__ counts,
+                     int32_t *__restrict__ offsets, int32_t *__restrict__ row_to_token,
+                     int32_t *__restrict__ token_to_row)
+{
+    static_assert(kPermuteFineChunk == kThreads, "one round per block");
+    __shared__ int base[kMaxE];
+    __shared__ int s[kThreads];
+    __shared__ int wcnt[kWarps][kMaxE];
+    pdl_entry();
+    const int e = threadIdx.x;
+    int total = 0, before = 0;
+    if (e < E) {
+#pragma unroll 8
+        for (int64_t b = 0; b < nblk; ++b) {
+            const int c = blk_cnt[b * E + e];
+            total += c;
+            before += b < (int64_t)blockIdx.x ? c : 0;
+        }
+    }
+    s[e] = total;
+    __syncthreads();
+    for (int o = 1; o < kThreads; o <<= 1) {  // inclusive Hillis-Steele scan
+        const int v = e >= o ? s[e - o] : 0;
+        __syncthreads();
+        s[e] += v;
+        __syncthreads();
+    }
+    if (e < E) {
+        const int start = s[e] - total;
+        base[e] = start + before;
+        if (blockIdx.x == 0) {
+            counts[e] = total;
+            offsets[e] = start;
+            if (e == E - 1) offsets[E] = s[e];
+        }
+    }
+    __syncthreads();
+    rank_round(idx, R, k, E, (int64_t)blockIdx.x * kPermuteFineChunk, base, wcnt, row_to_token, token_to_row);
 }
 
 // x_perm[token_to_row[t,j]] = x[t] for every assignment with a valid row.  A warp's
@@ -186,14 +237,19 @@ cudaError_t launch_permute(const uint16_t *x, const int32_t *topk_idx, int64_t N
                                    offsets, row_to_token, token_to_row, dev_err);
         if (e != cudaSuccess) return e;
     } else {
-        const int64_t nblk = permute_blocks(R);
-        cudaError_t e = launch_pdl(count_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s, topk_idx, R, E, scratch,
-                                   dev_err);
-        if (e == cudaSuccess)
-            e = launch_pdl(scan_kernel, dim3(1), dim3(kThreads), 0, s, scratch, nblk, E, counts, offsets);
-        if (e == cudaSuccess)
-            e = launch_pdl(rank_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s, (const int32_t *)topk_idx, R, k,
-                           E, (const int32_t *)scratch, row_to_token, token_to_row);
+        const int64_t chunk = permute_chunk(R), nblk = permute_blocks(R);
+        cudaError_t e = launch_pdl(count_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s, topk_idx, R, E,
+                                   (int)chunk, scratch, dev_err);
+        if (e == cudaSuccess && chunk == kPermuteFineChunk) {
+            e = launch_pdl(rank_scan_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s, (const int32_t *)topk_idx, R,
+                           k, E, (const int32_t *)scratch, nblk, counts, offsets, row_to_token, token_to_row);
+        } else {
+            if (e == cudaSuccess)
+                e = launch_pdl(scan_kernel, dim3(1), dim3(kThreads), 0, s, scratch, nblk, E, counts, offsets);
+            if (e == cudaSuccess)
+                e = launch_pdl(rank_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s, (const int32_t *)topk_idx, R,
+                               k, E, (const int32_t *)scratch, row_to_token, token_to_row);
+        }
         if (e != cudaSuccess) return e;
     }
     if (!x_perm) return cudaSuccess;  // dispatch only: the caller moves the rows itself

@@ -141,7 +141,8 @@ MOE_API moe_status_t moe_permute(const uint16_t *x, const int32_t *topk_idx, int
  *
  * Limit: ceil(N*k / 1024) * E <= MOE_PERMUTE_NOALLOC_MAX_SCRATCH_INTS, i.e.
  * up to 1,048,576 assignments at E = 256 (more at smaller E).  Larger requests
- * return MOE_ERR_UNSUPPORTED before any launch.
+ * return MOE_ERR_UNSUPPORTED before any launch.  (Below 32,768 assignments the
+ * dispatch takes blocks of 256, at most 128 of them: always within the limit.)
  *
  * The first call on each device looks up the array's device address on that
  * device (the device must be current); make that first call before any stream

@@ -221,7 +221,8 @@ def test_route_ties_on_every_path(N):
 
 
 @pytest.mark.parametrize("N,E,k", [(64, 8, 2), (1000, 160, 6), (3000, 128, 8), (7, 4, 4), (1, 1, 1),
-                                   (128, 64, 8), (129, 64, 8), (256, 128, 8)])  # one block up to 1024 rows
+                                   (128, 64, 8), (129, 64, 8), (256, 128, 8),  # one block up to 1024 rows
+                                   (4095, 256, 8), (4096, 256, 8)])  # 128 blocks of 256, then 32 of 1024
 def test_permute_bit_exact(N, E, k):
     H = 128
     g = torch.Generator().manual_seed(N + E)
