@@ -11,8 +11,8 @@
 //               starting row per expert (in place over the histograms);
 //   3. rank   : per block again, the stable rank of each assignment inside its
 //               block (warp match + per-warp counts, warps in order) -> row maps;
-//   4. copy   : x_perm[token_to_row[t,j]] = x[t] for j < k -- one warp per token reads
-//               its row once (16-byte vectors) and writes its k copies, so x is read
+//   4. copy   : x_perm[token_to_row[t,j]] = x[t] for j < k -- a warp reads 2 KB of a
+//               token's row once (16-byte vectors) and writes its k copies, so x is read
 //               from HBM once however many experts share a token.
 // Batches of at most kSmallR (1024) assignments do 1-3 in one single-block launch,
 // then the gather: two launches instead of four.  Mid-sized batches (fewer than
