@@ -47,12 +47,12 @@ def _noalloc_via_c_abi(x, idx, E):
     return out
 
 
-# Every case has more than 2048 assignments (above the one-block limit), so each call takes the count/scan/rank
-# dispatch whose per-block histograms live in the fixed array (smaller batches run a
-# one-block dispatch that never touches it).  The cases change E and the block count
-# from call to call, so each call starts on an array that still holds the previous
-# call's histograms laid out differently: 24 blocks x 128 experts, then 3 x 16, then
-# 11 x 200.
+# Every case has more than 2048 assignments (above the one-block limit of 1024), so each
+# call takes the multi-block dispatch whose per-block histograms live in the fixed array
+# (smaller batches run a one-block dispatch that never touches it).  The cases change E
+# and the block count from call to call, so each call starts on an array that still holds
+# the previous call's histograms laid out differently: 94 blocks of 256 assignments x 128
+# experts, then 12 x 16, then 41 x 200.
 CALLS = ((3000, 256, 128, 8), (1500, 128, 16, 2), (2600, 64, 200, 4))
 
 
